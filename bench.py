@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the LongCat-Flash MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...
+
+One step = one pass of the whole hot path over one batch: router logits + softmax/top-K
++ histogram (moe_route), permutation (moe_permute), grouped SwiGLU FFN on the tensor
+cores with the fused combine epilogue (moe_grouped_ffn), finalize (moe_combine) and the
+PID bias update (moe_pid_bias_update, written to a second bias buffer so every step
+routes the same batch). Workload: the full-shape prefill layer (hidden 6144, 512 SwiGLU
+FFN experts of intermediate 2048 + 256 zero-computation experts, K = 12, 8192 tokens,
+bf16, synthetic seeded inputs). A second timed loop runs the same layer in the decode
+regime (128 tokens) and reports it against the HBM roofline.
+
+Multi-GPU: every rank runs its own replica of the layer on its own batch (no exchange in
+the forward pass: weak scaling); the time is the max over ranks.
+
+--impl reference times the CPU oracle (float64 numpy) on a bounded sample of the same
+workload on the host cores; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_layer_29_b200 import abi  # noqa: E402
+from mixture_experts_layer_29_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1 B200; % of bf16 TC peak (prefill) / HBM BW (decode)"
+UNIT = "tokens/s"
+PID_GAINS = (0.01, 0.001, 0.0, 8 / 12)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+GEMM_SOURCES = [os.path.join(ROOT, "mixture_experts_layer_29_b200", "csrc", f)
+                for f in ("gemm_tc.cu", "common.cuh")]
+
+
+# ------------------------------------------------------------------------------ helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch(workload: str):
+    """DRAM bytes (read + write) per grouped-FFN call from the committed ncu summary, or
+    None when the GEMM source changed since the counters were taken."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("gemm_source_sha") != gemm_source_hash():
+        return None
+    return e.get("dram_bytes_per_call")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clocks not sampled"]}
+        sm = [float(r[1]) for r in self.rows if len(r) > 8 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) > 8 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            if len(r) > 8:
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(self.rows)}
+
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def oracle_sample(cfg, w, x_dev, tokens):
+    """Time the oracle on `tokens` of the workload: logits (float64), routing, and the
+    SwiGLU experts of those tokens. Weights of the experts they hit are copied to the
+    host first (outside the timed region). Returns (seconds, tokens)."""
+    import oracle.moe_oracle as orc
+    x = x_dev[tokens].float().cpu().numpy()
+    wr = w.w_router.cpu().numpy()
+    bias = w.bias.cpu().numpy()
+    # routing decides which experts' weights to stage; staging is not timed
+    L_probe = orc.router_logits(x, wr).astype(np.float32)
+    r = orc.route(L_probe, bias, cfg.n_ffn, cfg.K)
+    experts = sorted({int(e) for e in r.topk_idx.ravel() if e < cfg.n_ffn})
+    wgu = {e: w.w_gate_up[e].float().cpu().numpy() for e in experts}
+    wd = {e: w.w_down[e].float().cpu().numpy() for e in experts}
+    t0 = time.perf_counter()
+    L = orc.router_logits(x, wr).astype(np.float32)
+    orc.moe_layer_forward(x, L, bias, wgu, wd, cfg.n_ffn, cfg.K, cfg.ffn_out_scale)
+    return time.perf_counter() - t0, len(tokens)
+
+
+# ------------------------------------------------------------------------------ our arm
+
+class Stepper:
+    """The layer's ABI steps on one stream, with CUDA events around each call."""
+
+    def __init__(self, cfg, w, x, logits_in, combine, device):
+        self.cfg, self.w, self.x, self.logits_in = cfg, w, x, logits_in
+        self.shape = abi.shape_of(cfg, combine)
+        self.b = abi.StepBuffers.allocate(self.shape, device)
+        self.bias_next = w.bias.clone()
+        self.pid = abi.Pid(*PID_GAINS)
+        self.state = torch.empty(3 * cfg.n_ffn, dtype=torch.float32, device=device)
+        self.stats = torch.zeros(8, dtype=torch.float32, device=device)
+        abi.pid_init(self.shape, w.bias, self.state)
+
+    def step(self, ev=None):
+        s, b, w = self.shape, self.b, self.w
+
+        def mark(i):
+            if ev is not None:
+                ev[i].record()
+        mark(0)
+        abi.route(s, self.x, w.w_router, self.logits_in, w.bias,
+                  None if self.logits_in is not None else b.logits, b.topk_idx, b.topk_gate,
+                  b.counts, b.nffn_hist, b.zgate, b.ws)
+        mark(1)
+        abi.permute(s, b.topk_idx, b.topk_gate, b.zgate, self.x, b.offsets, b.perm_token,
+                    b.row_of, b.row_gate, b.x_perm, b.out_acc, b.ws)
+        mark(2)
+        abi.grouped_ffn(s, b.x_perm, b.offsets, w.w_gate_up, w.w_down, b.perm_token,
+                        b.row_gate, b.h, b.y_perm, b.out_acc, b.ws)
+        mark(3)
+        abi.combine(s, self.x, b.y_perm, b.out_acc, b.topk_gate, b.row_of, b.zgate, b.out)
+        mark(4)
+        abi.pid_bias_update(self.pid, s, b.counts, b.nffn_hist, self.bias_next, self.state,
+                            self.stats)
+        mark(5)
+
+
+PHASES = ["route", "permute", "grouped_ffn", "combine", "pid"]
+
+
+def timed_loop(st: Stepper, steps: int, warmup: int, dist_on: bool):
+    for _ in range(warmup):
+        st.step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    n0 = abi.launch_count()
+    start.record()
+    for k in range(steps):
+        st.step(evs[k])
+    end.record()
+    torch.cuda.synchronize()
+    launches = abi.launch_count() - n0
+    if dist_on:
+        torch.distributed.barrier()
+    total = start.elapsed_time(end)
+    per = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps)]
+           for i, p in enumerate(PHASES)}
+    return total, per, launches
+
+
+def max_over_ranks(v: float, dist_on: bool) -> float:
+    if not dist_on:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    cfg = wl.CONFIGS[args.workload]
+    seed = cfg.seed + rank                 # each replica routes its own batch
+    w = wl.draw_weights(cfg, device, seed=cfg.seed)
+    x = wl.draw_tokens(cfg, device, seed=seed)
+    logits_in = wl.draw_skewed_logits(cfg, device, seed=seed) if cfg.skewed else None
+    st = Stepper(cfg, w, x, logits_in, args.combine, device)
+
+    with ClockSampler(local) as clk:
+        total_ms, per, launches = timed_loop(st, args.steps, args.warmup, dist_on)
+    total_ms = max_over_ranks(total_ms, dist_on)
+    ms_step = total_ms / args.steps
+    tokens = cfg.T * args.steps * world
+    value = tokens / (total_ms / 1e3)
+
+    counts = st.b.counts.cpu().numpy()
+    rows = int(counts[: cfg.n_ffn].sum())
+    flops_ffn = rows * 6.0 * cfg.H * cfg.I
+    ffn_ms = float(np.mean(per["grouped_ffn"]))
+    pk, pk_kind = peaks()
+    achieved = flops_ffn / (ffn_ms / 1e3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    traffic = traffic_per_launch(args.workload)
+    roofline = {"bound": "tensor", "kernel": "grouped_ffn (gate/up + down tcgen05 GEMMs)",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_kind": f"bf16 sustained, {pk_kind}",
+                "frac_of_burst": round(achieved / pk.get("bf16_tflops", peak), 4),
+                "algorithmic_flop_per_call": flops_ffn, "ffn_rows": rows}
+
+    # ---- decode regime: same layer (same weights), 128 tokens ---------------------------
+    decode = None
+    if args.workload == "prefill_bf16" and not args.no_decode:
+        dcfg = wl.CONFIGS["decode_bf16"]
+        dx = wl.draw_tokens(dcfg, device, seed=seed)
+        dst = Stepper(dcfg, w, dx, None, args.combine, device)
+        dsteps = max(args.steps, 20)
+        dms, dper, _ = timed_loop(dst, dsteps, max(args.warmup, 3), dist_on)
+        dms = max_over_ranks(dms, dist_on)
+        dc = dst.b.counts.cpu().numpy()
+        touched = int((dc[: dcfg.n_ffn] > 0).sum())
+        dbytes = (touched * 3.0 * dcfg.H * dcfg.I * 2 + dcfg.E * dcfg.H * 4
+                  + 2 * dcfg.T * dcfg.H * 2)
+        dstep = dms / dsteps
+        dach = dbytes / (dstep / 1e3) / 1e9
+        hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        decode = {"workload": "decode_bf16", "value": round(dcfg.T * dsteps * world / (dms / 1e3), 1),
+                  "unit": UNIT, "ms_per_step": round(dstep, 4),
+                  "breakdown_ms": {p: round(float(np.mean(v)), 4) for p, v in dper.items()},
+                  "roofline": {"bound": "hbm", "scope": "whole layer step",
+                               "achieved": round(dach, 1), "peak": hbm, "unit": "GB/s",
+                               "frac": round(dach / hbm, 4), "frac_of_8TBs": round(dach / 8000, 4),
+                               "traffic": None, "algorithmic_bytes_per_step": dbytes,
+                               "touched_experts": touched, "peak_kind": pk_kind}}
+
+    # ---- end to end through the public API from pinned host memory ----------------------
+    e2e = None
+    if not args.no_e2e:
+        layer = abi.MoELayer(abi.shape_of(cfg, args.combine), w.w_router, w.bias.clone(),
+                             w.w_gate_up, w.w_down)
+        xh = x.cpu().pin_memory()
+        oh = torch.empty(cfg.T, cfg.H, dtype=x.dtype).pin_memory()
+        for _ in range(max(args.warmup, 3)):
+            layer.forward_host(xh, oh, logits_in)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist_on:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        s0.record()
+        for _ in range(args.steps):
+            layer.forward_host(xh, oh, logits_in)
+        s1.record()
+        torch.cuda.synchronize()
+        ems = max_over_ranks(s0.elapsed_time(s1), dist_on)
+        bi = xh.numel() * xh.element_size() + (logits_in.numel() * 4 if logits_in is not None else 0)
+        e2e = {"value": round(cfg.T * args.steps * world / (ems / 1e3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+               "ms_per_step": round(ems / args.steps, 4),
+               "note": "moe_forward via MoELayer.forward_host: pinned x in, out back, each step"}
+        del layer
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rng = np.random.default_rng(0)
+        toks = sorted(rng.choice(cfg.T, size=min(args.cpu_tokens, cfg.T), replace=False).tolist())
+        secs, n = oracle_sample(cfg, w, x, toks)
+        cpu = {"value": round(n / secs, 3), "unit": UNIT, "cores": oracle_threads(),
+               "kind": "oracle",
+               "sample": f"{n} of the {cfg.T} tokens (logits, routing and SwiGLU experts in "
+                         f"float64 numpy), {secs:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal inputs and random-init weights of the layer's shape)",
+        "config": {"workload": args.workload, "tokens": cfg.T, "hidden": cfg.H,
+                   "expert_intermediate": cfg.I, "ffn_experts": cfg.n_ffn,
+                   "zero_experts": cfg.n_zero, "top_k": cfg.K, "combine": args.combine,
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": "no flush: each step streams the touched experts' weights "
+                         f"({roofline['ffn_rows']} FFN rows) and writes x_perm, both far above "
+                         "the 126 MB L2"},
+        "breakdown_ms": {p: round(float(np.mean(v)), 4) for p, v in per.items()},
+        "roofline": roofline,
+        "decode": decode,
+        "e2e": e2e,
+        "gpu_launches": int(launches) * world,
+        "cpu_baseline": cpu,
+        "clocks": clk.summary(),
+        "routing": {"ffn_rows": rows, "ffn_experts_hit": int((counts[: cfg.n_ffn] > 0).sum()),
+                    "max_rows_per_expert": int(counts[: cfg.n_ffn].max())},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+# ------------------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    """The oracle, timed on the host cores on a bounded sample of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = wl.CONFIGS[args.workload]
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    if device == "cpu" and cfg.H * cfg.I * cfg.n_ffn > 2**31:
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "no GPU to draw the full-shape weights of the workload on"}))
+        return 0
+    w = wl.draw_weights(cfg, device)
+    x = wl.draw_tokens(cfg, device)
+    rng = np.random.default_rng(1)
+    times, n_tok = [], 0
+    for k in range(args.warmup + args.steps):
+        toks = sorted(rng.choice(cfg.T, size=args.ref_tokens, replace=False).tolist())
+        secs, n = oracle_sample(cfg, w, x, toks)
+        if k >= args.warmup:
+            times.append(secs)
+            n_tok += n
+    total = sum(times)
+    value = n_tok / total
+    cores = oracle_threads()
+    sample = (f"{args.ref_tokens} random tokens per step of the {cfg.T}-token batch: float64 "
+              f"logits, routing and SwiGLU experts")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "tokens": cfg.T},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_bf16", choices=sorted(wl.CONFIGS))
+    ap.add_argument("--combine", default="fused", choices=["fused", "deterministic"])
+    ap.add_argument("--cpu-tokens", type=int, default=400)
+    ap.add_argument("--ref-tokens", type=int, default=8)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "ours":
+        args.warmup = max(args.warmup, 3)     # timing rule: at least 3 untimed steps
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

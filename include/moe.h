@@ -1,0 +1,213 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) LongCat-Flash Mixture-of-Experts layer forward.
+ *
+ * The layer (LongCat-Flash Technical Report digest, Key claims, report §2.1 / §2.4):
+ * a router scores every token against a pool of n_ffn SwiGLU FFN experts and n_zero
+ * zero-computation (identity) experts and picks K of them per token. Selection uses the
+ * bias-adjusted score p + b, the gate is the unbiased softmax probability p (report
+ * §2.1.1). FFN picks are permuted into expert-contiguous groups and run through a grouped
+ * GEMM; a zero-computation pick adds g * x and costs no GEMM. The per-batch expert
+ * histogram drives a PID update of the FFN experts' biases (report §2.1.1, Fig. 3; the
+ * zero experts are excluded from it, report §2.1.2).
+ *
+ * Conventions for every call
+ *  - Expert indices: FFN experts are [0, n_ffn), zero-computation experts are
+ *    [n_ffn, n_ffn + n_zero). E = n_ffn + n_zero.
+ *  - Pointers marked "device" are CUDA device pointers on the current device; the caller
+ *    owns every buffer. The library never allocates, frees or synchronises, except
+ *    moe_read_device_status, which synchronises the given stream.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream).
+ *  - Layouts are row-major and contiguous. Device pointers must be 16-byte aligned.
+ *  - x, x_perm, h, y_perm and out hold `dtype` elements (bf16 or fp32); logits, gates,
+ *    biases and out_acc are fp32; indices and counts are int32.
+ *  - Return value: MOE_OK (0) or a negative MOE_ERR_* code. Argument checks happen on the
+ *    host before anything is launched, so a call that returns an error has launched
+ *    nothing. Inconsistencies only the device can see (an expert index out of range, a
+ *    bounded wait that ran out) are written to a status word inside the workspace and
+ *    read back with moe_read_device_status; kernels never trap.
+ *  - T = 0 is valid: the call checks its arguments and launches nothing.
+ *  - Limits: 1 <= E <= 1024, 1 <= K <= min(32, E), n_ffn >= 1, n_zero >= 0, T < 2^24,
+ *    T * K < 2^31. bf16: H % 128 == 0 and I % 128 == 0. fp32: H, I >= 1.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------------------- */
+#define MOE_OK                  0
+#define MOE_ERR_INVALID_ARG    -1   /* null pointer, bad size, K > E, ...               */
+#define MOE_ERR_UNSUPPORTED    -2   /* shape outside the limits above                   */
+#define MOE_ERR_ALIGNMENT      -3   /* a device pointer is not 16-byte aligned          */
+#define MOE_ERR_CUDA           -4   /* a CUDA runtime or driver call failed             */
+#define MOE_ERR_WORKSPACE      -5   /* workspace missing or smaller than required       */
+#define MOE_ERR_DEVICE_CHECK   -6   /* device-side consistency check failed (status)    */
+#define MOE_ERR_TIMEOUT        -7   /* a bounded device-side wait ran out (status)      */
+#define MOE_ERR_NO_DEVICE      -8   /* no CUDA device, or not an sm_100 device          */
+
+typedef enum { MOE_BF16 = 0, MOE_FP32 = 1 } moe_dtype_t;
+
+/* MOE_COMBINE_FUSED: the down-projection epilogue adds s * g * y into an fp32 out_acc with
+ * atomic adds (fast; the fp32 summation order, hence the last bits, vary run to run).
+ * MOE_COMBINE_DETERMINISTIC: the down projection stores y per permuted row (y_perm) and
+ * moe_combine sums the K slots of each token in slot order: bit-reproducible. */
+typedef enum { MOE_COMBINE_FUSED = 0, MOE_COMBINE_DETERMINISTIC = 1 } moe_combine_t;
+
+typedef struct {
+  int32_t T;              /* tokens                                                    */
+  int32_t H;              /* hidden width                                              */
+  int32_t I;              /* per-expert FFN intermediate width                         */
+  int32_t n_ffn;          /* SwiGLU FFN experts                                        */
+  int32_t n_zero;         /* zero-computation experts                                  */
+  int32_t K;              /* experts chosen per token                                  */
+  int32_t dtype;          /* moe_dtype_t                                               */
+  int32_t combine;        /* moe_combine_t                                             */
+  float ffn_out_scale;    /* s: factor on the FFN experts' outputs (report §2.3.2,
+                             Eq. 8, "m*n" variance compensation; value not printed;
+                             1.0 leaves the outputs unscaled)                          */
+} moe_shape_t;
+
+/* PID gains and target (report §2.1.1; the equation is not printed). target_ratio is the
+ * wanted mean number of FFN picks per token divided by K. */
+typedef struct {
+  float kp, ki, kd, target_ratio;
+} moe_pid_t;
+
+/* ---- sizes and status ---------------------------------------------------------------- */
+
+/* Bytes of scratch the step calls (moe_route, moe_permute, moe_grouped_ffn) need in `ws`.
+ * Returns MOE_OK and writes *bytes, or an error for an invalid shape. No device access. */
+int moe_scratch_size(const moe_shape_t* shape, size_t* bytes);
+
+/* Bytes moe_forward needs in `ws`: the scratch plus every intermediate of the layer
+ * (logits, zgate, offsets, the permutation, x_perm, h and y_perm or out_acc), sized for
+ * the worst case of T * K FFN rows so that no call ever waits for the device. */
+int moe_workspace_size(const moe_shape_t* shape, size_t* bytes);
+
+/* Synchronises `stream`, writes the device status word of `ws` (0 when no device-side
+ * check failed since the last read, else a MOE_ERR_* code) to *status and clears it. */
+int moe_read_device_status(void* ws, size_t ws_bytes, void* stream, int32_t* status);
+
+/* Static text for a MOE_* code. Never NULL. */
+const char* moe_status_string(int code);
+
+/* Number of kernels this library has launched in this process (all devices, all
+ * threads). A benchmark reads it before and after a timed region. */
+uint64_t moe_launch_count(void);
+
+/* ---- the steps of the layer ------------------------------------------------------------ */
+
+/* Router: logits, softmax over all E experts, bias-adjusted top-K, gates and histograms
+ * (report §2.1, §2.1.1).
+ *   x          device [T, H] dtype            token activations (unused if logits_in)
+ *   w_router   device [E, H] fp32             router weight (unused if logits_in)
+ *   logits_in  device [T, E] fp32 or NULL     given logits; NULL: computed as x . w_r^T
+ *   bias       device [E] fp32                selection bias
+ *   logits_out device [T, E] fp32             receives the logits; may be NULL only when
+ *                                             logits_in is given
+ *   topk_idx   device [T, K] int32            chosen experts, by (p + b) descending,
+ *                                             ties to the lower index
+ *   topk_gate  device [T, K] fp32             gates = softmax probabilities p (not
+ *                                             renormalised; the bias is not in them)
+ *   counts     device [E] int32               tokens per expert (zeroed by the call)
+ *   nffn_hist  device [K + 1] int32           tokens with n FFN picks (zeroed by the call)
+ *   zgate      device [T] fp32                sum of each token's zero-expert gates
+ *   ws         device scratch, >= moe_scratch_size bytes
+ * p is computed in double and rounded once to fp32; p + b is one fp32 add. */
+int moe_route(const moe_shape_t* shape, const void* x, const float* w_router,
+              const float* logits_in, const float* bias, float* logits_out,
+              int32_t* topk_idx, float* topk_gate, int32_t* counts, int32_t* nffn_hist,
+              float* zgate, void* ws, size_t ws_bytes, void* stream);
+
+/* Permutation of the FFN picks into expert-contiguous groups. Group e holds, in ascending
+ * token order, the rows of the tokens that picked e; groups follow in expert order.
+ *   topk_idx   device [T, K] int32            from moe_route
+ *   topk_gate  device [T, K] fp32
+ *   zgate      device [T] fp32                used only when out_acc != NULL
+ *   x          device [T, H] dtype
+ *   offsets    device [n_ffn + 1] int32       exclusive scan of the FFN experts' counts;
+ *                                             offsets[n_ffn] = R, the number of FFN rows
+ *   perm_token device [T * K] int32           token of each row; entries >= R unwritten
+ *   row_of     device [T, K] int32            row of each pick, -1 for zero experts
+ *   row_gate   device [T * K] fp32            gate of each row
+ *   x_perm     device [T * K + 128, H] dtype  x[perm_token[r]] in row r; the 128 extra
+ *                                             rows are read (never written) by the GEMM
+ *   out_acc    device [T, H] fp32 or NULL     if given, set to zgate[t] * x[t]: the
+ *                                             zero-computation experts' term, ready for
+ *                                             the fused combine
+ * Every expert index is checked on the device; one outside [0, E) sets the status word to
+ * MOE_ERR_DEVICE_CHECK and that pick is dropped. Bit-reproducible. */
+int moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* topk_gate,
+                const float* zgate, const void* x, int32_t* offsets, int32_t* perm_token,
+                int32_t* row_of, float* row_gate, void* x_perm, float* out_acc, void* ws,
+                size_t ws_bytes, void* stream);
+
+/* Grouped SwiGLU FFN over the expert groups (report §2.4: intermediate I per expert).
+ *   x_perm     device [T * K + 128, H] dtype  from moe_permute
+ *   offsets    device [n_ffn + 1] int32
+ *   w_gate_up  device [n_ffn, 2I, H] dtype    rows [0, I) gate, rows [I, 2I) up
+ *   w_down     device [n_ffn, H, I] dtype
+ *   perm_token device [T * K] int32           (fused combine only)
+ *   row_gate   device [T * K] fp32            (fused combine only)
+ *   h          device [T * K + 128, I] dtype  receives silu(x W_g^T) * (x W_u^T)
+ *   y_perm     device [T * K + 128, H] dtype  deterministic combine: receives y = h W_d^T
+ *   out_acc    device [T, H] fp32             fused combine: out_acc[perm_token[r]] +=
+ *                                             s * row_gate[r] * y[r] (atomic fp32 adds)
+ * bf16 runs on the tensor cores (tcgen05, fp32 accumulate, h rounded to bf16); fp32 runs
+ * a plain fp32 kernel. The call reads the row counts on the device: it never waits. */
+int moe_grouped_ffn(const moe_shape_t* shape, const void* x_perm, const int32_t* offsets,
+                    const void* w_gate_up, const void* w_down, const int32_t* perm_token,
+                    const float* row_gate, void* h, void* y_perm, float* out_acc, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* Combine (report §2.1: zero-computation experts contribute g * x).
+ * Fused: out = out_acc rounded to dtype. Deterministic: out[t] = sum over the FFN slots k
+ * in slot order of s * g_k * y_perm[row_of[t, k]], then + zgate[t] * x[t], in fp32,
+ * rounded once to dtype. Unused pointers of the other mode may be NULL.
+ *   out        device [T, H] dtype */
+int moe_combine(const moe_shape_t* shape, const void* x, const void* y_perm,
+                const float* out_acc, const float* topk_gate, const int32_t* row_of,
+                const float* zgate, void* out, void* stream);
+
+/* Sets pid_state for a controller that starts from `bias`: b0 = bias[0, n_ffn),
+ * integral = 0, prev_err = 0.
+ *   bias       device [E] fp32
+ *   pid_state  device [3 * n_ffn] fp32: b0, then integral, then prev_err */
+int moe_pid_init(const moe_shape_t* shape, const float* bias, float* pid_state, void* stream);
+
+/* One PID step on the FFN experts' biases from the batch histogram (report §2.1.1,
+ * Fig. 3; zero experts excluded, report §2.1.2). In fp32, in this order, without fused
+ * multiply-add, for i < n_ffn:
+ *   f = counts[i] / T;  tau = (target_ratio * K) / n_ffn;  e = tau - f;
+ *   I += e;  D = e - prev;  b = ((b0 + kp*e) + ki*I) + kd*D;  prev = e;  bias[i] = b.
+ * bias[n_ffn, E) is never written.
+ *   counts     device [E] int32,  nffn_hist device [K + 1] int32
+ *   bias       device [E] fp32, updated in place
+ *   pid_state  device [3 * n_ffn] fp32, updated
+ *   stats_out  device [8] fp32 or NULL: FFN activation ratio, mean and std of FFN picks
+ *              per token, max/mean FFN-expert load, FFN experts hit, zero-expert share of
+ *              all picks, mean |e|, max |e|. */
+int moe_pid_bias_update(const moe_pid_t* pid, const moe_shape_t* shape, const int32_t* counts,
+                        const int32_t* nffn_hist, float* bias, float* pid_state,
+                        float* stats_out, void* stream);
+
+/* The whole layer: moe_route, moe_permute, moe_grouped_ffn and moe_combine on `stream`,
+ * with every intermediate in `ws` (>= moe_workspace_size bytes). topk_idx, topk_gate,
+ * counts and nffn_hist are returned so the caller can chain moe_pid_bias_update.
+ * logits_in may be NULL (then w_router is used) as in moe_route. */
+int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,
+                const float* logits_in, const float* bias, const void* w_gate_up,
+                const void* w_down, void* out, int32_t* topk_idx, float* topk_gate,
+                int32_t* counts, int32_t* nffn_hist, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

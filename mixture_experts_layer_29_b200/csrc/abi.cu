@@ -1,0 +1,363 @@
+// abi.cu - the extern "C" entry points of include/moe.h: host-side argument checks, the
+// workspace layout and the launch order of the layer's kernels. No call here allocates
+// memory or waits for the device, except moe_read_device_status.
+#include <atomic>
+#include <initializer_list>
+#include <mutex>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+int current_device_info(DeviceInfo* info) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  if (dev >= 64) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev].device != dev) {
+    DeviceInfo d;
+    d.device = dev;
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    cache[dev] = d;
+  }
+  *info = cache[dev];
+  // the kernels are built for sm_100a only
+  if (info->cc_major != 10 || info->cc_minor != 0) return MOE_ERR_NO_DEVICE;
+  return MOE_OK;
+}
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+constexpr int kRowPad = 128;    // extra rows of x_perm / h / y_perm read by the GEMM tiles
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  // scratch (all step calls)
+  size_t status, masks, crel, ecount, lpart, scratch_end;
+  // intermediates (moe_forward)
+  size_t logits, zgate, offsets, perm, rowof, rowgate, xperm, h, yperm, outacc, total;
+};
+
+int check_shape(const moe_shape_t* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->n_ffn <= 0 || s->n_zero < 0 || s->K <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (s->dtype != MOE_BF16 && s->dtype != MOE_FP32) return MOE_ERR_INVALID_ARG;
+  if (s->combine != MOE_COMBINE_FUSED && s->combine != MOE_COMBINE_DETERMINISTIC)
+    return MOE_ERR_INVALID_ARG;
+  const long E = (long)s->n_ffn + s->n_zero;
+  if (s->K > E) return MOE_ERR_INVALID_ARG;
+  if (E > 1024 || s->K > 32) return MOE_ERR_UNSUPPORTED;
+  if (s->T >= (1 << 24) || (long)s->T * s->K >= (1L << 31)) return MOE_ERR_UNSUPPORTED;
+  if (s->H % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (s->dtype == MOE_BF16 && (s->H % 128 != 0 || s->I % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (!(s->ffn_out_scale == s->ffn_out_scale)) return MOE_ERR_INVALID_ARG;   // NaN
+  return MOE_OK;
+}
+
+Layout layout_of(const moe_shape_t& s) {
+  Layout L{};
+  const size_t T = s.T, H = s.H, I = s.I, N = s.n_ffn, K = s.K, E = N + s.n_zero;
+  const size_t nchunk = (T + 31) / 32;
+  const size_t esz = s.dtype == MOE_BF16 ? 2 : 4;
+  const size_t rows = T * K + kRowPad;
+  size_t o = 0;
+  L.status = o;  o = align_up(o + 256);
+  L.masks = o;   o = align_up(o + N * nchunk * 4);
+  L.crel = o;    o = align_up(o + N * nchunk * 4);
+  L.ecount = o;  o = align_up(o + N * 4);
+  L.lpart = o;   o = align_up(o + router_partial_bytes(s.T, (int)E, s.H, 0));
+  L.scratch_end = o;
+  L.logits = o;  o = align_up(o + T * E * 4);
+  L.zgate = o;   o = align_up(o + T * 4);
+  L.offsets = o; o = align_up(o + (N + 1) * 4);
+  L.perm = o;    o = align_up(o + T * K * 4);
+  L.rowof = o;   o = align_up(o + T * K * 4);
+  L.rowgate = o; o = align_up(o + T * K * 4);
+  L.xperm = o;   o = align_up(o + rows * H * esz);
+  L.h = o;       o = align_up(o + rows * I * esz);
+  L.yperm = o;
+  if (s.combine == MOE_COMBINE_DETERMINISTIC) o = align_up(o + rows * H * esz);
+  L.outacc = o;
+  if (s.combine == MOE_COMBINE_FUSED) o = align_up(o + T * H * 4);
+  L.total = o;
+  return L;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// all given pointers non-null and 16-byte aligned
+int check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(p)) return MOE_ERR_ALIGNMENT;
+  }
+  return MOE_OK;
+}
+// optional pointers: may be null, else aligned
+int check_opt(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)            \
+  do {                           \
+    const int _rc = (expr);      \
+    if (_rc != MOE_OK) return _rc; \
+  } while (0)
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+int route_impl(const moe_shape_t* s, const void* x, const float* w_router, const float* logits_in,
+               const float* bias, float* logits_out, int32_t* topk_idx, float* topk_gate,
+               int32_t* counts, int32_t* nffn_hist, float* zgate, void* ws, size_t ws_bytes,
+               void* stream) {
+  MOE_TRY(check_shape(s));
+  MOE_TRY(check_ptrs({bias, topk_idx, topk_gate, counts, nffn_hist, zgate, ws}));
+  if (!logits_in) MOE_TRY(check_ptrs({x, w_router, logits_out}));
+  MOE_TRY(check_opt({logits_in, logits_out, x, w_router}));
+  const Layout L = layout_of(*s);
+  if (ws_bytes < L.scratch_end) return MOE_ERR_WORKSPACE;
+  if (s->T == 0) return MOE_OK;
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  const int E = s->n_ffn + s->n_zero;
+  const cudaStream_t st = as_stream(stream);
+  const float* logits = logits_in;
+  if (!logits_in) {
+    const int S = router_splitk(s->T, E, s->H, dev.sm_count);
+    MOE_TRY(cuda_rc(launch_router_logits(x, s->dtype == MOE_BF16, w_router, s->T, E, s->H,
+                                         logits_out, at<float>(ws, L.lpart), S, st)));
+    logits = logits_out;
+  }
+  return cuda_rc(launch_route_topk(logits, bias, s->T, E, s->n_ffn, s->K, topk_idx, topk_gate,
+                                   counts, nffn_hist, zgate, dev.sm_count, st));
+}
+
+int permute_impl(const moe_shape_t* s, const int32_t* topk_idx, const float* topk_gate,
+                 const float* zgate, const void* x, int32_t* offsets, int32_t* perm_token,
+                 int32_t* row_of, float* row_gate, void* x_perm, float* out_acc, void* ws,
+                 size_t ws_bytes, void* stream) {
+  MOE_TRY(check_shape(s));
+  MOE_TRY(check_ptrs({topk_idx, topk_gate, x, offsets, perm_token, row_of, row_gate, x_perm, ws}));
+  if (out_acc) MOE_TRY(check_ptrs({zgate, out_acc}));
+  const Layout L = layout_of(*s);
+  if (ws_bytes < L.scratch_end) return MOE_ERR_WORKSPACE;
+  if (s->T == 0) {
+    return MOE_OK;
+  }
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  return cuda_rc(launch_permute(topk_idx, topk_gate, zgate, x, s->dtype == MOE_BF16, s->T, s->H,
+                                s->n_ffn, s->n_ffn + s->n_zero, s->K, at<uint32_t>(ws, L.masks),
+                                at<int32_t>(ws, L.crel), at<int32_t>(ws, L.ecount), offsets,
+                                perm_token, row_of, row_gate, x_perm, out_acc,
+                                at<int>(ws, L.status), as_stream(stream)));
+}
+
+int grouped_ffn_impl(const moe_shape_t* s, const void* x_perm, const int32_t* offsets,
+                     const void* w_gate_up, const void* w_down, const int32_t* perm_token,
+                     const float* row_gate, void* h, void* y_perm, float* out_acc, void* ws,
+                     size_t ws_bytes, void* stream) {
+  MOE_TRY(check_shape(s));
+  MOE_TRY(check_ptrs({x_perm, offsets, w_gate_up, w_down, h, ws}));
+  const bool fused = s->combine == MOE_COMBINE_FUSED;
+  if (fused) MOE_TRY(check_ptrs({perm_token, row_gate, out_acc}));
+  else MOE_TRY(check_ptrs({y_perm}));
+  const Layout L = layout_of(*s);
+  if (ws_bytes < L.scratch_end) return MOE_ERR_WORKSPACE;
+  if (s->T == 0) return MOE_OK;
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  const cudaStream_t st = as_stream(stream);
+  if (s->dtype == MOE_BF16)
+    return launch_grouped_ffn_tc(x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h, y_perm,
+                                 out_acc, s->T, s->H, s->I, s->n_ffn, s->K, s->ffn_out_scale, fused,
+                                 at<int>(ws, L.status), dev.sm_count, st);
+  return cuda_rc(launch_grouped_ffn_simt(
+      static_cast<const float*>(x_perm), offsets, static_cast<const float*>(w_gate_up),
+      static_cast<const float*>(w_down), perm_token, row_gate, static_cast<float*>(h),
+      static_cast<float*>(y_perm), out_acc, s->T, s->H, s->I, s->n_ffn, s->K, s->ffn_out_scale,
+      fused, st));
+}
+
+int combine_impl(const moe_shape_t* s, const void* x, const void* y_perm, const float* out_acc,
+                 const float* topk_gate, const int32_t* row_of, const float* zgate, void* out,
+                 void* stream) {
+  MOE_TRY(check_shape(s));
+  MOE_TRY(check_ptrs({out}));
+  const bool fused = s->combine == MOE_COMBINE_FUSED;
+  if (fused) MOE_TRY(check_ptrs({out_acc}));
+  else MOE_TRY(check_ptrs({x, y_perm, topk_gate, row_of, zgate}));
+  if (s->T == 0) return MOE_OK;
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  const cudaStream_t st = as_stream(stream);
+  if (fused)
+    return cuda_rc(launch_finalize(out_acc, out, s->dtype == MOE_BF16, (size_t)s->T * s->H, st));
+  return cuda_rc(launch_combine_det(x, y_perm, topk_gate, row_of, zgate, out, s->dtype == MOE_BF16,
+                                    s->T, s->H, s->K, s->ffn_out_scale, st));
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_scratch_size(const moe_shape_t* shape, size_t* bytes) {
+  MOE_TRY(check_shape(shape));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = layout_of(*shape).scratch_end;
+  return MOE_OK;
+}
+
+int moe_workspace_size(const moe_shape_t* shape, size_t* bytes) {
+  MOE_TRY(check_shape(shape));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = layout_of(*shape).total;
+  return MOE_OK;
+}
+
+int moe_read_device_status(void* ws, size_t ws_bytes, void* stream, int32_t* status) {
+  if (!ws || !status) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  const cudaStream_t st = as_stream(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(ws, 0, sizeof(v), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  *status = v;
+  return MOE_OK;
+}
+
+const char* moe_status_string(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_DEVICE_CHECK: return "device-side consistency check failed";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_NO_DEVICE: return "no sm_100 CUDA device";
+    default: return "unknown status";
+  }
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_route(const moe_shape_t* shape, const void* x, const float* w_router,
+              const float* logits_in, const float* bias, float* logits_out, int32_t* topk_idx,
+              float* topk_gate, int32_t* counts, int32_t* nffn_hist, float* zgate, void* ws,
+              size_t ws_bytes, void* stream) {
+  return route_impl(shape, x, w_router, logits_in, bias, logits_out, topk_idx, topk_gate, counts,
+                    nffn_hist, zgate, ws, ws_bytes, stream);
+}
+
+int moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* topk_gate,
+                const float* zgate, const void* x, int32_t* offsets, int32_t* perm_token,
+                int32_t* row_of, float* row_gate, void* x_perm, float* out_acc, void* ws,
+                size_t ws_bytes, void* stream) {
+  return permute_impl(shape, topk_idx, topk_gate, zgate, x, offsets, perm_token, row_of, row_gate,
+                      x_perm, out_acc, ws, ws_bytes, stream);
+}
+
+int moe_grouped_ffn(const moe_shape_t* shape, const void* x_perm, const int32_t* offsets,
+                    const void* w_gate_up, const void* w_down, const int32_t* perm_token,
+                    const float* row_gate, void* h, void* y_perm, float* out_acc, void* ws,
+                    size_t ws_bytes, void* stream) {
+  return grouped_ffn_impl(shape, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h,
+                          y_perm, out_acc, ws, ws_bytes, stream);
+}
+
+int moe_combine(const moe_shape_t* shape, const void* x, const void* y_perm, const float* out_acc,
+                const float* topk_gate, const int32_t* row_of, const float* zgate, void* out,
+                void* stream) {
+  return combine_impl(shape, x, y_perm, out_acc, topk_gate, row_of, zgate, out, stream);
+}
+
+int moe_pid_init(const moe_shape_t* shape, const float* bias, float* pid_state, void* stream) {
+  MOE_TRY(check_shape(shape));
+  MOE_TRY(check_ptrs({bias, pid_state}));
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  return cuda_rc(launch_pid_init(bias, pid_state, shape->n_ffn, as_stream(stream)));
+}
+
+int moe_pid_bias_update(const moe_pid_t* pid, const moe_shape_t* shape, const int32_t* counts,
+                        const int32_t* nffn_hist, float* bias, float* pid_state, float* stats_out,
+                        void* stream) {
+  if (!pid) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_shape(shape));
+  MOE_TRY(check_ptrs({counts, nffn_hist, bias, pid_state}));
+  MOE_TRY(check_opt({stats_out}));
+  if (shape->T == 0) return MOE_ERR_INVALID_ARG;   // frequencies counts / T need T > 0
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  return cuda_rc(launch_pid_update(*pid, counts, nffn_hist, bias, pid_state, stats_out, shape->T,
+                                   shape->K, shape->n_ffn, shape->n_ffn + shape->n_zero,
+                                   as_stream(stream)));
+}
+
+int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,
+                const float* logits_in, const float* bias, const void* w_gate_up,
+                const void* w_down, void* out, int32_t* topk_idx, float* topk_gate,
+                int32_t* counts, int32_t* nffn_hist, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_shape(shape));
+  MOE_TRY(check_ptrs({x, bias, w_gate_up, w_down, out, topk_idx, topk_gate, counts, nffn_hist, ws}));
+  if (!logits_in) MOE_TRY(check_ptrs({w_router}));
+  MOE_TRY(check_opt({logits_in}));
+  const Layout L = layout_of(*shape);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (shape->T == 0) return MOE_OK;
+  const bool fused = shape->combine == MOE_COMBINE_FUSED;
+  float* logits = at<float>(ws, L.logits);
+  float* zgate = at<float>(ws, L.zgate);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* rowof = at<int32_t>(ws, L.rowof);
+  float* rowgate = at<float>(ws, L.rowgate);
+  void* xperm = at<char>(ws, L.xperm);
+  void* h = at<char>(ws, L.h);
+  void* yperm = fused ? nullptr : at<char>(ws, L.yperm);
+  float* outacc = fused ? at<float>(ws, L.outacc) : nullptr;
+  MOE_TRY(route_impl(shape, x, w_router, logits_in, bias, logits, topk_idx, topk_gate, counts,
+                     nffn_hist, zgate, ws, ws_bytes, stream));
+  MOE_TRY(permute_impl(shape, topk_idx, topk_gate, zgate, x, offsets, perm, rowof, rowgate, xperm,
+                       outacc, ws, ws_bytes, stream));
+  MOE_TRY(grouped_ffn_impl(shape, xperm, offsets, w_gate_up, w_down, perm, rowgate, h, yperm,
+                           outacc, ws, ws_bytes, stream));
+  return combine_impl(shape, x, yperm, outacc, topk_gate, rowof, zgate, out, stream);
+}
+
+}  // extern "C"

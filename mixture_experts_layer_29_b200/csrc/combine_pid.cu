@@ -1,0 +1,231 @@
+// combine_pid.cu - the combine step and the PID bias update.
+//
+// Combine (LongCat-Flash Technical Report digest, Key claims, report §2.1: a
+// zero-computation expert is an identity map, so it adds g * x; Method: the MoE combine):
+//   fused mode          out = out_acc rounded to the output type
+//   deterministic mode  out[t] = sum over FFN slots k, in slot order, of s * g_k * y_k,
+//                       then + zgate[t] * x[t]; fp32, rounded once.
+// PID (report §2.1.1, Fig. 3; zero experts excluded, report §2.1.2): one CTA updates the
+// FFN experts' biases from the batch's expert counts and writes the step's statistics.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+template <typename T>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&q);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(b[i]);
+  }
+  __device__ static void store(__nv_bfloat16* p, const float (&v)[8]) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const float* p, float (&v)[4]) {
+    const float4 q = *reinterpret_cast<const float4*>(p);
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+  __device__ static void store(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_finalize(const float* __restrict__ acc, T* __restrict__ out,
+                                                  size_t n) {
+  constexpr int V = Vec<T>::N;
+  const size_t nv = n / V;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nv;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float v[V];
+#pragma unroll
+    for (int j = 0; j < V; j += 4) {
+      const float4 q = reinterpret_cast<const float4*>(acc)[i * (V / 4) + j / 4];
+      v[j] = q.x; v[j + 1] = q.y; v[j + 2] = q.z; v[j + 3] = q.w;
+    }
+    Vec<T>::store(out + i * V, v);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, const T* __restrict__ y_perm,
+                                                     const float* __restrict__ topk_gate,
+                                                     const int32_t* __restrict__ row_of,
+                                                     const float* __restrict__ zgate,
+                                                     T* __restrict__ out, int H, int K, float scale) {
+  constexpr int V = Vec<T>::N;
+  __shared__ int s_row[32];
+  __shared__ float s_g[32];
+  const int t = blockIdx.x;
+  if (threadIdx.x < K) {
+    s_row[threadIdx.x] = row_of[(size_t)t * K + threadIdx.x];
+    s_g[threadIdx.x] = scale * topk_gate[(size_t)t * K + threadIdx.x];
+  }
+  __syncthreads();
+  const float zg = zgate[t];
+  for (int c = threadIdx.x * V; c < H; c += blockDim.x * V) {
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.f;
+    for (int k = 0; k < K; ++k) {
+      const int r = s_row[k];
+      if (r < 0) continue;
+      float y[V];
+      Vec<T>::load(y_perm + (size_t)r * H + c, y);
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] = fmaf(s_g[k], y[i], acc[i]);
+    }
+    float xv[V];
+    Vec<T>::load(x + (size_t)t * H + c, xv);
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = fmaf(zg, xv[i], acc[i]);
+    Vec<T>::store(out + (size_t)t * H + c, acc);
+  }
+}
+
+__global__ void k_pid_init(const float* __restrict__ bias, float* __restrict__ st, int n_ffn) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_ffn; i += gridDim.x * blockDim.x) {
+    st[i] = bias[i];
+    st[n_ffn + i] = 0.f;
+    st[2 * n_ffn + i] = 0.f;
+  }
+}
+
+// block-wide sum / max of doubles (fixed tree: deterministic)
+__device__ double block_sum(double v, double* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double r = 0.0;
+  for (int i = 0; i < nw; ++i) r += red[i];
+  return r;
+}
+__device__ double block_max(double v, double* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double r = red[0];
+  for (int i = 1; i < nw; ++i) r = fmax(r, red[i]);
+  return r;
+}
+
+// One CTA of 1024 threads; expert i = threadIdx.x (n_ffn <= 1024).
+__global__ void __launch_bounds__(1024) k_pid_update(moe_pid_t pid, const int32_t* __restrict__ counts,
+                                                     const int32_t* __restrict__ hist,
+                                                     float* __restrict__ bias, float* __restrict__ st,
+                                                     float* __restrict__ stats, int T, int K,
+                                                     int n_ffn, int E) {
+  __shared__ double red[32];
+  const int i = threadIdx.x;
+  double c_ffn = 0.0, c_hit = 0.0, c_zero = 0.0, abs_e = 0.0;
+  if (i < n_ffn) {
+    const int c = counts[i];
+    const float f = __fdiv_rn((float)c, (float)T);
+    const float tau = __fdiv_rn(__fmul_rn(pid.target_ratio, (float)K), (float)n_ffn);
+    const float e = __fsub_rn(tau, f);
+    const float integ = __fadd_rn(st[n_ffn + i], e);
+    const float deriv = __fsub_rn(e, st[2 * n_ffn + i]);
+    float b = __fadd_rn(st[i], __fmul_rn(pid.kp, e));
+    b = __fadd_rn(b, __fmul_rn(pid.ki, integ));
+    b = __fadd_rn(b, __fmul_rn(pid.kd, deriv));
+    bias[i] = b;
+    st[n_ffn + i] = integ;
+    st[2 * n_ffn + i] = e;
+    c_ffn = (double)c;
+    c_hit = c > 0 ? 1.0 : 0.0;
+    abs_e = fabs((double)e);
+  }
+  for (int j = n_ffn + i; j < E; j += blockDim.x) c_zero += (double)counts[j];
+  double hn = 0.0, hn2 = 0.0;
+  if (i <= K) {
+    hn = (double)hist[i] * i;
+    hn2 = (double)hist[i] * i * i;
+  }
+  const double s_ffn = block_sum(c_ffn, red);
+  const double m_ffn = block_max(c_ffn, red);
+  const double s_hit = block_sum(c_hit, red);
+  const double s_zero = block_sum(c_zero, red);
+  const double s_abs = block_sum(abs_e, red);
+  const double m_abs = block_max(abs_e, red);
+  const double s_hn = block_sum(hn, red);
+  const double s_hn2 = block_sum(hn2, red);
+  if (stats && i == 0) {
+    const double mean = s_hn / T;
+    const double var = fmax(0.0, s_hn2 / T - mean * mean);
+    const double mean_load = s_ffn / n_ffn;
+    stats[0] = (float)(mean / K);
+    stats[1] = (float)mean;
+    stats[2] = (float)sqrt(var);
+    stats[3] = (float)(mean_load > 0.0 ? m_ffn / mean_load : 0.0);
+    stats[4] = (float)s_hit;
+    stats[5] = (float)(s_zero / ((double)T * K));
+    stats[6] = (float)(s_abs / n_ffn);
+    stats[7] = (float)m_abs;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_finalize(const float* out_acc, void* out, int out_is_bf16, size_t n,
+                            cudaStream_t st) {
+  const size_t work = n / 8;
+  int blocks = (int)((work + 255) / 256);
+  if (blocks > 8192) blocks = 8192;
+  if (blocks < 1) blocks = 1;
+  if (out_is_bf16)
+    k_finalize<__nv_bfloat16><<<blocks, 256, 0, st>>>(out_acc, static_cast<__nv_bfloat16*>(out), n);
+  else
+    k_finalize<float><<<blocks, 256, 0, st>>>(out_acc, static_cast<float*>(out), n);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_det(const void* x, const void* y_perm, const float* topk_gate,
+                               const int32_t* row_of, const float* zgate, void* out,
+                               int is_bf16, int T, int H, int K, float scale, cudaStream_t st) {
+  if (is_bf16)
+    k_combine_det<__nv_bfloat16><<<T, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm), topk_gate,
+        row_of, zgate, static_cast<__nv_bfloat16*>(out), H, K, scale);
+  else
+    k_combine_det<float><<<T, 256, 0, st>>>(static_cast<const float*>(x),
+                                            static_cast<const float*>(y_perm), topk_gate, row_of,
+                                            zgate, static_cast<float*>(out), H, K, scale);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pid_init(const float* bias, float* pid_state, int n_ffn, cudaStream_t st) {
+  k_pid_init<<<(n_ffn + 255) / 256, 256, 0, st>>>(bias, pid_state, n_ffn);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pid_update(const moe_pid_t& pid, const int32_t* counts,
+                              const int32_t* nffn_hist, float* bias, float* pid_state,
+                              float* stats, int T, int K, int n_ffn, int E, cudaStream_t st) {
+  k_pid_update<<<1, 1024, 0, st>>>(pid, counts, nffn_hist, bias, pid_state, stats, T, K, n_ffn, E);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

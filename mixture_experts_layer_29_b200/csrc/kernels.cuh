@@ -1,0 +1,66 @@
+// kernels.cuh - host-side launchers of the layer's kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// One launch of one of this library's kernels (counted for moe_launch_count).
+void count_launch(int n = 1);
+
+struct DeviceInfo {
+  int device = -1;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+// Cached per device; returns MOE_OK, MOE_ERR_CUDA or MOE_ERR_NO_DEVICE.
+int current_device_info(DeviceInfo* info);
+
+// ---- router -----------------------------------------------------------------------------
+// Split-K factor of the logits GEMM for this shape (1 = no partial buffer).
+int router_splitk(int T, int E, int H, int sm_count);
+size_t router_partial_bytes(int T, int E, int H, int sm_count_max);
+cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_router, int T,
+                                 int E, int H, float* logits, float* partial, int splitk,
+                                 cudaStream_t st);
+cudaError_t launch_route_topk(const float* logits, const float* bias, int T, int E, int n_ffn,
+                              int K, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                              int32_t* nffn_hist, float* zgate, int sm_count, cudaStream_t st);
+
+// ---- permutation ------------------------------------------------------------------------
+cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, const float* zgate,
+                           const void* x, int x_is_bf16, int T, int H, int n_ffn, int E, int K,
+                           uint32_t* masks, int32_t* crel, int32_t* ecount, int32_t* offsets,
+                           int32_t* perm_token, int32_t* row_of, float* row_gate, void* x_perm,
+                           float* out_acc, int* status, cudaStream_t st);
+
+// ---- grouped FFN --------------------------------------------------------------------------
+// bf16 on tcgen05: gate/up GEMM + SwiGLU -> h, then down GEMM -> y_perm or out_acc.
+int launch_grouped_ffn_tc(const void* x_perm, const int32_t* offsets, const void* w_gate_up,
+                          const void* w_down, const int32_t* perm_token, const float* row_gate,
+                          void* h, void* y_perm, float* out_acc, int T, int H, int I, int n_ffn,
+                          int K, float scale, int fused, int* status, int sm_count,
+                          cudaStream_t st);
+// fp32 on the CUDA cores.
+cudaError_t launch_grouped_ffn_simt(const float* x_perm, const int32_t* offsets,
+                                    const float* w_gate_up, const float* w_down,
+                                    const int32_t* perm_token, const float* row_gate, float* h,
+                                    float* y_perm, float* out_acc, int T, int H, int I,
+                                    int n_ffn, int K, float scale, int fused, cudaStream_t st);
+
+// ---- combine and PID ----------------------------------------------------------------------
+cudaError_t launch_finalize(const float* out_acc, void* out, int out_is_bf16, size_t n,
+                            cudaStream_t st);
+cudaError_t launch_combine_det(const void* x, const void* y_perm, const float* topk_gate,
+                               const int32_t* row_of, const float* zgate, void* out,
+                               int is_bf16, int T, int H, int K, float scale, cudaStream_t st);
+cudaError_t launch_pid_init(const float* bias, float* pid_state, int n_ffn, cudaStream_t st);
+cudaError_t launch_pid_update(const moe_pid_t& pid, const int32_t* counts,
+                              const int32_t* nffn_hist, float* bias, float* pid_state,
+                              float* stats, int T, int K, int n_ffn, int E, cudaStream_t st);
+
+}  // namespace moe

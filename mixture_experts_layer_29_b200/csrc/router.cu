@@ -1,0 +1,352 @@
+// router.cu - router logits (fp32 GEMM on the CUDA cores) and the warp-per-token softmax,
+// bias-adjusted top-K and expert histogram.
+//
+// LongCat-Flash Technical Report digest, Key claims (report §2.1, §2.4): the router picks
+// K experts per token from the combined pool of FFN and zero-computation experts; (report
+// §2.1.1) a per-expert bias steers the selection, the gates stay the softmax values.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------------------
+// logits[t, e] = sum_h x[t, h] * w_router[e, h]   (fp32 FMA, smem-tiled, optional split-K)
+// 128 x 128 output tile per CTA, 16-deep k slices, 256 threads with an 8 x 8 micro-tile.
+// Split-K writes fp32 partials that a second kernel sums in split order, so the logits
+// are bit-reproducible.
+// ---------------------------------------------------------------------------------------
+namespace {
+constexpr int RB = 128, RK = 16, RPAD = 4;
+constexpr int kSmMax = 160;   // sizing bound for the split-K partial buffer
+
+template <bool XBF16>
+__device__ __forceinline__ void load_x_slice(const void* x, int T, int H, int row0, int k0,
+                                             float (&v)[8], int& r, int& kk) {
+  const int tid = threadIdx.x;
+  if (XBF16) {
+    r = tid >> 1;
+    kk = (tid & 1) * 8;
+    const int t = row0 + r;
+    if (t < T) {
+      const uint4 q = *reinterpret_cast<const uint4*>(
+          static_cast<const __nv_bfloat16*>(x) + (size_t)t * H + k0 + kk);
+      const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&q);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(b[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+  } else {
+    // two float4 per thread: rows tid/4 and tid/4 + 64, k quarter tid%4
+    r = tid >> 2;
+    kk = (tid & 3) * 4;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int t = row0 + r + 64 * h;
+      float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < T) q = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * H + k0 + kk);
+      v[4 * h + 0] = q.x; v[4 * h + 1] = q.y; v[4 * h + 2] = q.z; v[4 * h + 3] = q.w;
+    }
+  }
+}
+
+__device__ __forceinline__ void load_w_slice(const float* w, int E, int H, int col0, int k0,
+                                             float (&v)[8]) {
+  const int tid = threadIdx.x;
+  const int r = tid >> 2, kk = (tid & 3) * 4;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int e = col0 + r + 64 * h;
+    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e < E) q = *reinterpret_cast<const float4*>(w + (size_t)e * H + k0 + kk);
+    v[4 * h + 0] = q.x; v[4 * h + 1] = q.y; v[4 * h + 2] = q.z; v[4 * h + 3] = q.w;
+  }
+}
+
+template <bool XBF16>
+__global__ void __launch_bounds__(256, 2) k_router_logits(const void* __restrict__ x,
+                                                       const float* __restrict__ w, int T, int E,
+                                                       int H, int kchunk, float* __restrict__ out,
+                                                       size_t split_stride) {
+  __shared__ __align__(16) float As[2][RK][RB + RPAD];
+  __shared__ __align__(16) float Bs[2][RK][RB + RPAD];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int row0 = blockIdx.y * RB, col0 = blockIdx.x * RB;
+  const int kbeg = blockIdx.z * kchunk;
+  const int kend = min(H, kbeg + kchunk);
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  float xa[8], wb[8];
+  int xr, xk;
+  auto stash = [&](int buf) {
+    if (XBF16) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) As[buf][xk + i][xr] = xa[i];
+    } else {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) As[buf][xk + i][xr + 64 * h] = xa[4 * h + i];
+    }
+    const int wr = tid >> 2, wk = (tid & 3) * 4;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) Bs[buf][wk + i][wr + 64 * h] = wb[4 * h + i];
+  };
+
+  int buf = 0;
+  if (kbeg < kend) {
+    load_x_slice<XBF16>(x, T, H, row0, kbeg, xa, xr, xk);
+    load_w_slice(w, E, H, col0, kbeg, wb);
+    stash(0);
+  }
+  __syncthreads();
+  for (int k0 = kbeg; k0 < kend; k0 += RK) {
+    const bool more = k0 + RK < kend;
+    if (more) {
+      load_x_slice<XBF16>(x, T, H, row0, k0 + RK, xa, xr, xk);
+      load_w_slice(w, E, H, col0, k0 + RK, wb);
+    }
+#pragma unroll
+    for (int kk = 0; kk < RK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    if (more) stash(buf ^ 1);
+    __syncthreads();
+    buf ^= 1;
+  }
+
+  float* dst = out + blockIdx.z * split_stride;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = row0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = col0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+      if (e < E) dst[(size_t)t * E + e] = acc[i][j];
+    }
+  }
+}
+
+// logits = sum over splits s = 0, 1, ... of partial[s] (fixed order)
+__global__ void k_router_splitk_sum(const float* __restrict__ partial, int S, size_t n,
+                                    float* __restrict__ logits) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float a = partial[i];
+    for (int s = 1; s < S; ++s) a += partial[s * n + i];
+    logits[i] = a;
+  }
+}
+}  // namespace
+
+int router_splitk(int T, int E, int H, int sm_count) {
+  if (sm_count > kSmMax) sm_count = kSmMax;
+  const long tiles = (long)((T + RB - 1) / RB) * ((E + RB - 1) / RB);
+  if (tiles <= 0 || tiles >= sm_count) return 1;
+  long s = (2L * sm_count + tiles - 1) / tiles;
+  const long smax = H / 64 > 0 ? H / 64 : 1;     // at least 64 of H per split
+  if (s > smax) s = smax;
+  if (s > 32) s = 32;
+  return s < 1 ? 1 : (int)s;
+}
+
+size_t router_partial_bytes(int T, int E, int H, int sm_count_max) {
+  const int s = router_splitk(T, E, H, sm_count_max > 0 ? sm_count_max : kSmMax);
+  return s > 1 ? (size_t)s * T * E * sizeof(float) : 0;
+}
+
+cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_router, int T,
+                                 int E, int H, float* logits, float* partial, int splitk,
+                                 cudaStream_t st) {
+  int kchunk = (H + splitk - 1) / splitk;
+  kchunk = (kchunk + RK - 1) / RK * RK;
+  const int S = (H + kchunk - 1) / kchunk;
+  dim3 grid((E + RB - 1) / RB, (T + RB - 1) / RB, S);
+  float* dst = S > 1 ? partial : logits;
+  const size_t stride = (size_t)T * E;
+  if (x_is_bf16)
+    k_router_logits<true><<<grid, 256, 0, st>>>(x, w_router, T, E, H, kchunk, dst, stride);
+  else
+    k_router_logits<false><<<grid, 256, 0, st>>>(x, w_router, T, E, H, kchunk, dst, stride);
+  count_launch();
+  if (S > 1) {
+    const size_t n = (size_t)T * E;
+    const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    k_router_splitk_sum<<<blocks, 256, 0, st>>>(partial, S, n, logits);
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------
+// Softmax + bias-adjusted top-K, one warp per token.
+// Lane l holds experts l, l + 32, ... (J groups). p is computed in double and rounded once
+// to fp32; the selection score is the fp32 sum p + b (a zero result stored as +0). K
+// rounds of a warp-wide argmax pick (score descending, expert index ascending). The
+// counts and the FFN-pick histogram go through shared memory, then integer atomics.
+// ---------------------------------------------------------------------------------------
+namespace {
+constexpr int kRouteWarps = 8;
+
+template <int J>
+__global__ void __launch_bounds__(kRouteWarps * 32) k_route_topk(
+    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int n_ffn,
+    int K, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
+    int32_t* __restrict__ counts, int32_t* __restrict__ nffn_hist, float* __restrict__ zgate) {
+  __shared__ int s_counts[1024];
+  __shared__ int s_hist[33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) s_counts[i] = 0;
+  if (threadIdx.x <= K) s_hist[threadIdx.x] = 0;
+  __syncthreads();
+
+  float bia[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    bia[j] = e < E ? bias[e] : 0.f;
+  }
+
+  for (int t = blockIdx.x * kRouteWarps + warp; t < T; t += gridDim.x * kRouteWarps) {
+    const float* Lr = logits + (size_t)t * E;
+    float lv[J];
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int e = lane + 32 * j;
+      lv[j] = e < E ? Lr[e] : -INFINITY;
+      m = fmaxf(m, lv[j]);
+    }
+    m = warp_max(m);
+    double ex[J];
+    double sum = 0.0;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int e = lane + 32 * j;
+      ex[j] = e < E ? exp((double)lv[j] - (double)m) : 0.0;
+      sum += ex[j];
+    }
+    sum = warp_sum(sum);
+    float p[J], s[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int e = lane + 32 * j;
+      p[j] = (float)(ex[j] / sum);
+      float v = __fadd_rn(p[j], bia[j]);
+      if (v == 0.0f) v = 0.0f;          // -0 -> +0
+      s[j] = e < E ? v : -INFINITY;
+    }
+
+    uint32_t taken = 0u;
+    int my_e = 0;
+    float my_g = 0.f;
+    for (int k = 0; k < K; ++k) {
+      float bs = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < J; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && !((taken >> j) & 1u) && (s[j] > bs || be == 0x7fffffff)) {
+          bs = s[j];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (os > bs || (os == bs && oe < be)) {
+          bs = os;
+          be = oe;
+        }
+      }
+      const int owner = be & 31, jw = be >> 5;
+      float g = 0.f;
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+        if (j == jw) g = p[j];
+      if (lane == owner) taken |= 1u << jw;
+      g = __shfl_sync(0xffffffffu, g, owner);
+      if (lane == k) {
+        my_e = be;
+        my_g = g;
+      }
+    }
+    if (lane < K) {
+      topk_idx[(size_t)t * K + lane] = my_e;
+      topk_gate[(size_t)t * K + lane] = my_g;
+      atomicAdd(&s_counts[my_e], 1);
+    }
+    const unsigned ffn = __ballot_sync(0xffffffffu, lane < K && my_e < n_ffn);
+    float z = 0.f;
+    for (int k = 0; k < K; ++k) {
+      const float gk = __shfl_sync(0xffffffffu, my_g, k);
+      const int ek = __shfl_sync(0xffffffffu, my_e, k);
+      if (ek >= n_ffn) z += gk;
+    }
+    if (lane == 0) {
+      atomicAdd(&s_hist[__popc(ffn)], 1);
+      zgate[t] = z;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < E; i += blockDim.x)
+    if (s_counts[i]) atomicAdd(&counts[i], s_counts[i]);
+  if (threadIdx.x <= K && s_hist[threadIdx.x]) atomicAdd(&nffn_hist[threadIdx.x], s_hist[threadIdx.x]);
+}
+
+template <int J>
+void launch_topk_j(dim3 grid, cudaStream_t st, const float* logits, const float* bias, int T,
+                   int E, int n_ffn, int K, int32_t* idx, float* gate, int32_t* counts,
+                   int32_t* hist, float* zgate) {
+  k_route_topk<J><<<grid, kRouteWarps * 32, 0, st>>>(logits, bias, T, E, n_ffn, K, idx, gate,
+                                                     counts, hist, zgate);
+}
+}  // namespace
+
+cudaError_t launch_route_topk(const float* logits, const float* bias, int T, int E, int n_ffn,
+                              int K, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                              int32_t* nffn_hist, float* zgate, int sm_count, cudaStream_t st) {
+  cudaError_t err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st);
+  if (err != cudaSuccess) return err;
+  err = cudaMemsetAsync(nffn_hist, 0, sizeof(int32_t) * (K + 1), st);
+  if (err != cudaSuccess) return err;
+  int blocks = (T + kRouteWarps - 1) / kRouteWarps;
+  if (blocks > 4 * sm_count) blocks = 4 * sm_count;
+  dim3 grid(blocks);
+  const int J = (E + 31) / 32;
+#define MOE_TOPK_CASE(JJ)                                                                      \
+  if (J <= JJ) {                                                                               \
+    launch_topk_j<JJ>(grid, st, logits, bias, T, E, n_ffn, K, topk_idx, topk_gate, counts,     \
+                      nffn_hist, zgate);                                                       \
+  } else
+  MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4) MOE_TOPK_CASE(6)
+  MOE_TOPK_CASE(8) MOE_TOPK_CASE(12) MOE_TOPK_CASE(16) MOE_TOPK_CASE(24) MOE_TOPK_CASE(32) {
+    return cudaErrorInvalidValue;
+  }
+#undef MOE_TOPK_CASE
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -104,8 +104,12 @@ class LayerWeights:
     w_down: torch.Tensor
 
 
-def draw_weights(cfg: MoEConfig, device="cpu", seed: int | None = None) -> LayerWeights:
-    """Draw the layer's parameters: every weight ~ N(0, w_std^2), bias ~ U(bias_lo, bias_hi)."""
+def draw_weights(cfg: MoEConfig, device="cpu", seed: int | None = None,
+                 ffn: bool = True) -> LayerWeights:
+    """Draw the layer's parameters: every weight ~ N(0, w_std^2), bias ~ U(bias_lo, bias_hi).
+
+    ffn=False skips the FFN weights (w_gate_up and w_down are None); the router weight and
+    the bias are the same values either way (they are drawn first)."""
     seed = cfg.seed if seed is None else seed
     g = _gen(device, seed * 7919 + 1)
     dt = torch_dtype(cfg)
@@ -116,6 +120,8 @@ def draw_weights(cfg: MoEConfig, device="cpu", seed: int | None = None) -> Layer
         bias.uniform_(cfg.bias_lo, cfg.bias_hi, generator=g)
     else:
         bias.fill_(cfg.bias_lo)
+    if not ffn:
+        return LayerWeights(w_router, bias, None, None)
     w_gate_up = torch.empty(cfg.n_ffn, 2 * cfg.I, cfg.H, dtype=dt, device=device)
     w_down = torch.empty(cfg.n_ffn, cfg.H, cfg.I, dtype=dt, device=device)
     # one expert at a time keeps the generator's temporaries small on the full shape

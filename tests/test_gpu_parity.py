@@ -1,0 +1,192 @@
+"""GPU parity of every step against the CPU oracle, through the C ABI.
+
+Routing (indices, counts, histograms) and the permutation are bit-exact given the same
+fp32 logits; tokens whose K-th / (K+1)-th score gap is below 1e-6 are reported, not
+asserted. Layer outputs: max per-row relative error <= 2e-2 (bf16) or 1e-5 (fp32), checked
+on (1) each permuted row's expert output y (deterministic combine), (2) the FFN part of
+the output alone (fused combine with a zero-initialised accumulator) and (3) the whole
+output, in both combine modes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.moe_oracle as orc
+from mixture_experts_layer_29_b200 import abi
+from mixture_experts_layer_29_b200 import workloads as wl
+import gpu_harness as gh
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["tiny_fp32", "proxy_bf16"]
+
+
+def _free():
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_logits_and_routing_small(cuda_device, name):
+    case = gh.Case(wl.CONFIGS[name])
+    b = case.buffers()
+    case.route(b)
+    torch.cuda.synchronize()
+    gh.check_logits(case, b)
+    rep = {}
+    gh.check_routing(case, b, rep)
+    assert rep["near_tie_mismatch"] == 0
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_permutation_small(cuda_device, name):
+    case = gh.Case(wl.CONFIGS[name])
+    b = case.buffers()
+    case.route(b)
+    abi.permute(b.shape, b.topk_idx, b.topk_gate, b.zgate, case.x, b.offsets, b.perm_token,
+                b.row_of, b.row_gate, b.x_perm, b.out_acc, b.ws)
+    torch.cuda.synchronize()
+    gh.check_permutation(case, b, zero_init=True)
+    assert abi.read_device_status(b.ws) == 0
+
+
+def _ffn_checks(case, combine):
+    """Run the four steps in `combine` mode and compare with the oracle on all tokens."""
+    cfg = case.cfg
+    tol = gh.TOL[cfg.dtype]
+    b = case.buffers(combine)
+    out = abi.run_steps(b, case.x, case.w.w_router, case.logits_in, case.w.bias,
+                        case.w.w_gate_up, case.w.w_down)
+    torch.cuda.synchronize()
+    L = case.gpu_logits(b)
+    r = gh.check_routing(case, b)
+    toks = list(range(cfg.T))
+    o_out, o_ffn, o_zg, y_rows, rr, _ = gh.oracle_layer(case, L, toks)
+    err_out = gh.row_rel_err(gh.host(out)[: cfg.T], o_out)
+    assert err_out <= tol, ("out", err_out)
+    if combine == "deterministic":
+        row_of = gh.host(b.row_of).reshape(cfg.T, cfg.K)
+        yp = gh.host(b.y_perm)
+        keys = sorted(y_rows)
+        got = np.stack([yp[row_of[t, k]] for (t, k) in keys]) if keys else np.zeros((0, cfg.H))
+        want = np.stack([y_rows[key] for key in keys]) if keys else np.zeros((0, cfg.H))
+        err_y = gh.row_rel_err(got, want)
+        assert err_y <= tol, ("y_perm", err_y)
+    return b, o_ffn, err_out
+
+
+@pytest.mark.parametrize("name", SMALL)
+@pytest.mark.parametrize("combine", ["fused", "deterministic"])
+def test_layer_output_small(cuda_device, name, combine):
+    case = gh.Case(wl.CONFIGS[name])
+    _ffn_checks(case, combine)
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_ffn_part_alone_fused(cuda_device, name):
+    """Fused epilogue with out_acc starting at zero: out_acc is the FFN part alone."""
+    case = gh.Case(wl.CONFIGS[name])
+    cfg = case.cfg
+    b = case.buffers("fused")
+    case.route(b)
+    abi.permute(b.shape, b.topk_idx, b.topk_gate, b.zgate, case.x, b.offsets, b.perm_token,
+                b.row_of, b.row_gate, b.x_perm, None, b.ws)
+    b.out_acc.zero_()
+    abi.grouped_ffn(b.shape, b.x_perm, b.offsets, case.w.w_gate_up, case.w.w_down,
+                    b.perm_token, b.row_gate, b.h, None, b.out_acc, b.ws)
+    torch.cuda.synchronize()
+    L = case.gpu_logits(b)
+    gh.check_routing(case, b)
+    _, o_ffn, _, _, _, _ = gh.oracle_layer(case, L, list(range(cfg.T)))
+    has_ffn = np.abs(o_ffn).max(axis=1) > 0
+    err = gh.row_rel_err(gh.host(b.out_acc)[: cfg.T][has_ffn], o_ffn[has_ffn])
+    assert err <= gh.TOL[cfg.dtype], err
+    assert (gh.host(b.out_acc)[: cfg.T][~has_ffn] == 0).all()
+
+
+def test_deterministic_mode_is_bit_reproducible(cuda_device):
+    case = gh.Case(wl.CONFIGS["proxy_bf16"])
+    outs = []
+    for _ in range(2):
+        b = case.buffers("deterministic")
+        abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up,
+                      case.w.w_down)
+        torch.cuda.synchronize()
+        R = int(b.offsets[-1])          # entries past R of the row buffers are unwritten
+        outs.append([t.clone() for t in (b.logits, b.topk_idx, b.topk_gate, b.offsets,
+                                         b.perm_token[:R], b.row_of, b.x_perm[:R], b.h[:R],
+                                         b.y_perm[:R], b.out)])
+    for a, c in zip(*outs):
+        assert torch.equal(a, c)
+
+
+def test_forward_entry_point_matches_steps(cuda_device):
+    case = gh.Case(wl.CONFIGS["proxy_bf16"])
+    for combine in ("fused", "deterministic"):
+        s = case.shape(combine)
+        layer = abi.MoELayer(s, case.w.w_router, case.w.bias, case.w.w_gate_up, case.w.w_down)
+        out, idx, gate, counts, hist = layer.forward(case.x)
+        b = case.buffers(combine)
+        ref = abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up,
+                            case.w.w_down)
+        torch.cuda.synchronize()
+        assert torch.equal(idx, b.topk_idx) and torch.equal(counts, b.counts)
+        err = gh.row_rel_err(gh.host(out), gh.host(ref))
+        assert err <= (1e-6 if combine == "deterministic" else 1e-2)
+        if combine == "deterministic":
+            assert torch.equal(out, ref)
+
+
+# ------------------------------------------------------------------------- edge cases
+
+@pytest.mark.parametrize("T", [1, 31, 33, 129, 1000])
+def test_ragged_token_counts(cuda_device, T):
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=T)
+    case = gh.Case(cfg, seed=3)
+    _ffn_checks(case, "fused")
+    _ffn_checks(case, "deterministic")
+
+
+def test_zero_only_tokens_output_gate_sum_times_x(cuda_device):
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=256, bias_lo=0.0, bias_hi=0.0)
+    zero_tok = [0, 5, 31, 32, 200, 255]
+    logits = wl.draw_forced_logits(cfg.T, cfg.n_ffn, cfg.n_zero, zero_tok, "cuda", seed=1)
+    case = gh.Case(cfg, logits=logits)
+    for combine in ("fused", "deterministic"):
+        b, _, _ = _ffn_checks(case, combine)
+        idx = gh.host(b.topk_idx)
+        row_of = gh.host(b.row_of).reshape(cfg.T, cfg.K)
+        out = gh.host(b.out)
+        x = gh.host(case.x)
+        zg = gh.host(b.zgate)
+        for t in zero_tok:
+            assert (idx[t] >= cfg.n_ffn).all() and (row_of[t] == -1).all()
+            want = torch.tensor(zg[t] * x[t].astype(np.float32)).to(torch.bfloat16).float().numpy()
+            np.testing.assert_array_equal(out[t], want)
+
+
+def test_every_token_on_one_expert_and_empty_experts(cuda_device):
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=700)
+    case = gh.Case(cfg, seed=5)
+    case.w.bias.zero_()
+    case.w.bias[7] = 5.0            # expert 7 is picked by every token
+    case.w.bias[20:40] = -5.0       # experts 20..39 by none
+    for combine in ("fused", "deterministic"):
+        b, _, _ = _ffn_checks(case, combine)
+        counts = gh.host(b.counts)
+        assert counts[7] == cfg.T and (counts[: cfg.n_ffn] == 0).sum() > 0
+
+
+def test_all_experts_chosen_k_equals_e(cuda_device):
+    cfg = wl.CONFIGS["tiny_fp32"].with_(K=24, T=50)
+    case = gh.Case(cfg, seed=2)
+    for combine in ("fused", "deterministic"):
+        b, _, _ = _ffn_checks(case, combine)
+        assert (gh.host(b.counts) == cfg.T).all()
+
+
+def test_ffn_out_scale(cuda_device):
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=300, ffn_out_scale=2.5)
+    case = gh.Case(cfg, seed=4)
+    _ffn_checks(case, "fused")
+    _ffn_checks(case, "deterministic")
