@@ -235,6 +235,18 @@ def max_over_ranks(v: float, dist_on: bool) -> float:
     return float(t.item())
 
 
+def workload(args):
+    cfg = wl.CONFIGS[args.workload]
+    kw = {}
+    if args.tokens is not None:
+        kw["T"] = args.tokens
+    if args.ffn_experts is not None:
+        kw["n_ffn"] = args.ffn_experts
+    if args.zero_experts is not None:
+        kw["n_zero"] = args.zero_experts
+    return cfg.with_(**kw) if kw else cfg
+
+
 def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -246,7 +258,7 @@ def run_ours(args):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
-    cfg = wl.CONFIGS[args.workload]
+    cfg = workload(args)
     seed = cfg.seed + rank                 # each replica routes its own batch
     w = wl.draw_weights(cfg, device, seed=cfg.seed)
     x = wl.draw_tokens(cfg, device, seed=seed)
@@ -278,7 +290,7 @@ def run_ours(args):
     # ---- decode regime: same layer (same weights), 128 tokens ---------------------------
     decode = None
     if args.workload == "prefill_bf16" and not args.no_decode:
-        dcfg = wl.CONFIGS["decode_bf16"]
+        dcfg = cfg.with_(T=wl.CONFIGS["decode_bf16"].T)
         dx = wl.draw_tokens(dcfg, device, seed=seed)
         dst = Stepper(dcfg, w, dx, None, args.combine, device)
         dsteps = max(args.steps, 20)
@@ -341,7 +353,9 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded normal inputs and random-init weights of the layer's shape)",
-        "config": {"workload": args.workload, "tokens": cfg.T, "hidden": cfg.H,
+        "config": {"workload": args.workload if cfg == wl.CONFIGS[args.workload] else
+                   f"{args.workload} (overridden: T={cfg.T}, n_ffn={cfg.n_ffn}, n_zero={cfg.n_zero})",
+                   "tokens": cfg.T, "hidden": cfg.H,
                    "expert_intermediate": cfg.I, "ffn_experts": cfg.n_ffn,
                    "zero_experts": cfg.n_zero, "top_k": cfg.K, "combine": args.combine,
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
@@ -373,7 +387,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cfg = wl.CONFIGS[args.workload]
+    cfg = workload(args)
     device = "cuda" if torch.cuda.is_available() else "cpu"
     if device == "cpu" and cfg.H * cfg.I * cfg.n_ffn > 2**31:
         print(json.dumps({"impl": "reference", "unavailable":
@@ -417,6 +431,9 @@ def main(argv=None):
     ap.add_argument("--combine", default="fused", choices=["fused", "deterministic"])
     ap.add_argument("--cpu-tokens", type=int, default=400)
     ap.add_argument("--ref-tokens", type=int, default=8)
+    ap.add_argument("--tokens", type=int, default=None, help="override the workload's T")
+    ap.add_argument("--ffn-experts", type=int, default=None, help="override n_ffn (profiling)")
+    ap.add_argument("--zero-experts", type=int, default=None, help="override n_zero (profiling)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

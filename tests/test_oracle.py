@@ -94,6 +94,14 @@ def test_topk_ties_go_to_lower_index():
     assert list(orc.select_topk(s, 3)[0]) == [0, 1, 2]
 
 
+def test_near_tie_gap_by_hand():
+    s = np.array([[0.5, 0.3, 0.3, 0.125], [0.25, 0.75, 0.0, 0.5]], dtype=np.float32)
+    np.testing.assert_array_equal(orc.near_tie_gap(s, 1), [0.5 - np.float32(0.3), 0.25])
+    np.testing.assert_array_equal(orc.near_tie_gap(s, 2), [0.0, 0.25])
+    np.testing.assert_array_equal(orc.near_tie_gap(s, 3), [np.float32(0.3) - 0.125, 0.25])
+    assert np.isinf(orc.near_tie_gap(s, 4)).all()
+
+
 def test_bias_moves_selection_not_gates():
     r = rng(7)
     L = r.standard_normal((300, 24)).astype(np.float32)
