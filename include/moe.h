@@ -206,6 +206,32 @@ int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,
                 const void* w_down, void* out, int32_t* topk_idx, float* topk_gate,
                 int32_t* counts, int32_t* nffn_hist, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- allocation-free variant ------------------------------------------------------------
+ * The pages have no counterpart to this call: it is moe_permute for callers that cannot
+ * give the library a device workspace. Such callers include code running while its
+ * stream is captured into a CUDA graph in a capture mode where cudaMalloc is an error,
+ * plugins inside a host framework that owns all device memory and only passes tensors
+ * in and out, and latency-bound paths that cannot afford a cudaMalloc, which may
+ * synchronise the whole device.
+ *
+ * Arguments and results are exactly those of moe_permute without ws and ws_bytes. The
+ * scratch is a fixed 4 MiB array in the library's own device memory; each GPU that loads
+ * the library keeps it until the process exits. A call needs
+ * 1024 + 2 * round_up_1024(n_ffn * ceil(T / 32) * 4) + 4 * n_ffn bytes of it and returns
+ * MOE_ERR_WORKSPACE, launching nothing, when the shape needs more (with n_ffn = 512:
+ * T <= 32736). The call never calls cudaMalloc, cudaFree or any allocating routine.
+ * The first call on a device looks up the array's device address and caches it: make
+ * that first call before any stream capture on that device.
+ * Every call uses the same array, which keeps what the last call left there. Calls whose
+ * GPU work can overlap (unordered streams, several host threads) race on it and give
+ * wrong results: order them on one stream. Each call clears the array's status word;
+ * that word cannot be read back, so an invalid expert index is dropped (row_of = -1)
+ * as in moe_permute but not reported: use moe_permute to get the report. */
+int moe_permute_static_scratch(const moe_shape_t* shape, const int32_t* topk_idx,
+                               const float* topk_gate, const float* zgate, const void* x,
+                               int32_t* offsets, int32_t* perm_token, int32_t* row_of,
+                               float* row_gate, void* x_perm, float* out_acc, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

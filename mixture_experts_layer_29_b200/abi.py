@@ -79,6 +79,7 @@ _SIGS = {
     "moe_pid_bias_update": (ctypes.c_int, [ctypes.POINTER(Pid), ctypes.POINTER(Shape)]
                             + [_P] * 6),
     "moe_forward": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 12 + [_SZ, _P]),
+    "moe_permute_static_scratch": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 10 + [_P]),
 }
 
 _lib = None
@@ -182,6 +183,16 @@ def permute(shape, topk_idx, topk_gate, zgate, x, offsets, perm_token, row_of, r
                              ptr(x), ptr(offsets), ptr(perm_token), ptr(row_of), ptr(row_gate),
                              ptr(x_perm), ptr(out_acc), ptr(ws), _nbytes(ws), _stream(stream)),
            "moe_permute")
+
+
+def permute_static_scratch(shape, topk_idx, topk_gate, zgate, x, offsets, perm_token, row_of,
+                           row_gate, x_perm, out_acc, stream=None):
+    """moe_permute without a workspace argument: its scratch is the library's own fixed
+    device array (for callers that cannot allocate device memory; see include/moe.h)."""
+    _check(lib().moe_permute_static_scratch(ctypes.byref(shape), ptr(topk_idx), ptr(topk_gate),
+                                            ptr(zgate), ptr(x), ptr(offsets), ptr(perm_token),
+                                            ptr(row_of), ptr(row_gate), ptr(x_perm), ptr(out_acc),
+                                            _stream(stream)), "moe_permute_static_scratch")
 
 
 def grouped_ffn(shape, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h, y_perm,
