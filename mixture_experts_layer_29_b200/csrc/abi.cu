@@ -83,7 +83,9 @@ Layout layout_of(const moe_shape_t& s) {
   L.masks = o;   o = align_up(o + N * nchunk * 4);
   L.crel = o;    o = align_up(o + N * nchunk * 4);
   L.ecount = o;  o = align_up(o + N * 4);
-  L.lpart = o;   o = align_up(o + router_partial_bytes(s.T, (int)E, s.H, 0));
+  L.lpart = o;   // router scratch: split weight + partials (bf16) or SIMT partials (fp32)
+  o = align_up(o + (s.dtype == MOE_BF16 ? router_tc_scratch_bytes(s.T, (int)E, s.H)
+                                        : router_partial_bytes(s.T, (int)E, s.H, 0)));
   L.scratch_end = o;
   L.logits = o;  o = align_up(o + T * E * 4);
   L.zgate = o;   o = align_up(o + T * 4);
@@ -149,9 +151,14 @@ int route_impl(const moe_shape_t* s, const void* x, const float* w_router, const
   const cudaStream_t st = as_stream(stream);
   const float* logits = logits_in;
   if (!logits_in) {
-    const int S = router_splitk(s->T, E, s->H, dev.sm_count);
-    MOE_TRY(cuda_rc(launch_router_logits(x, s->dtype == MOE_BF16, w_router, s->T, E, s->H,
-                                         logits_out, at<float>(ws, L.lpart), S, st)));
+    if (s->dtype == MOE_BF16) {
+      MOE_TRY(launch_router_logits_tc(x, w_router, s->T, E, s->H, logits_out,
+                                      at<char>(ws, L.lpart), dev.sm_count, st));
+    } else {
+      const int S = router_splitk(s->T, E, s->H, dev.sm_count);
+      MOE_TRY(cuda_rc(launch_router_logits(x, 0, w_router, s->T, E, s->H, logits_out,
+                                           at<float>(ws, L.lpart), S, st)));
+    }
     logits = logits_out;
   }
   return cuda_rc(launch_route_topk(logits, bias, s->T, E, s->n_ffn, s->K, topk_idx, topk_gate,

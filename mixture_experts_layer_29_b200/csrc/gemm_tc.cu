@@ -35,24 +35,34 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
-constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 48 KB
 constexpr int kThreads = 192;
 constexpr int kMaxExperts = 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
 
-enum Mode : int { kGateUp = 0, kDownStore = 1, kDownAtomic = 2 };
+// Per N-tile width: 256 for the expert GEMMs, 128 for the router (whose epilogue keeps a
+// 128-column running sum per row in registers).
+template <int BN_>
+struct Cfg {
+  static constexpr int BN = BN_;
+  static constexpr int B_BYTES = BN_ * BK * 2;                 // 32 KB / 16 KB
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 48 KB / 32 KB
+  static constexpr int STAGES = BN_ == 256 ? 4 : 6;            // 192 KB of ring either way
+  static constexpr int NACC = 512 / BN_;                       // TMEM accumulators
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN_);
+};
 
+enum Mode : int { kGateUp = 0, kDownStore = 1, kDownAtomic = 2, kLogits = 3 };
+
+template <int BN_>
 struct alignas(1024) SharedStorage {
-  uint8_t a[STAGES][A_BYTES];
-  uint8_t b[STAGES][B_BYTES];
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint8_t a[Cfg<BN_>::STAGES][A_BYTES];
+  uint8_t b[Cfg<BN_>::STAGES][Cfg<BN_>::B_BYTES];
+  uint64_t full[Cfg<BN_>::STAGES];
+  uint64_t empty[Cfg<BN_>::STAGES];
+  uint64_t tfull[Cfg<BN_>::NACC];
+  uint64_t tempty[Cfg<BN_>::NACC];
   uint32_t tmem_base;
   int abort_flag;
   int offs[kMaxExperts + 1];
@@ -66,26 +76,38 @@ struct GemmArgs {
   int n_tiles;        // N tiles per M tile
   int b_rows;         // B rows per expert: 2I (gate/up) or H (down)
   int b_second;       // row offset of the second 128-row B box: I (gate/up) or 128 (down)
-  int n_valid;        // valid output columns: I (h) or H (y)
+  int n_valid;        // valid output columns: I (h), H (y) or E (logits)
   int ld_out;         // output row length in elements
-  int col_step;       // output columns per N tile: 128 (h) or 256 (y)
   const int32_t* offsets;
   void* out;
   const int32_t* perm_token;
   const float* row_gate;
   float scale;
   int* status;
+  int a_kwrap;              // A's K coordinate wraps every a_kwrap k-blocks (0: no wrap)
+  int dense_rows;           // > 0: one dense group of this many rows, offsets unused
+  int ksplit;               // K splits per output tile (each writes its own fp32 slice)
+  int kb_per_split;         // k-blocks per split
+  int kchunk;               // k-blocks per tensor-core accumulation (0: the whole split)
+  long long split_stride;   // elements between the outputs of consecutive splits
 };
 
 struct Tile {
-  int e, row0, row_end, nt;
+  int e, row0, row_end, nt, kb0, kb1, split;
 };
 
-__device__ __forceinline__ Tile decode_tile(const SharedStorage& s, const GemmArgs& g, int tile) {
+template <int BN_>
+__device__ __forceinline__ Tile decode_tile(const SharedStorage<BN_>& s, const GemmArgs& g,
+                                            int tile) {
   Tile t;
+  const int per_split = s.toff[g.n_ffn] * g.n_tiles;
+  t.split = tile / per_split;
+  tile -= t.split * per_split;
+  t.kb0 = t.split * g.kb_per_split;
+  t.kb1 = min(g.kblocks, t.kb0 + g.kb_per_split);
   const int mt = tile / g.n_tiles;
   t.nt = tile - mt * g.n_tiles;
-  // largest e with toff[e] <= mt
+  // largest e with toff[e] <= mt (empty groups share the next group's toff and are skipped)
   int lo = 0, hi = g.n_ffn - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -97,23 +119,98 @@ __device__ __forceinline__ Tile decode_tile(const SharedStorage& s, const GemmAr
   return t;
 }
 
+__device__ __forceinline__ int chunk_len(const GemmArgs& g, const Tile& t) {
+  return g.kchunk > 0 ? g.kchunk : (t.kb1 - t.kb0);
+}
+
 __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
+// Epilogue of one 128 x 256 accumulator of the expert GEMMs (modes gate-up / down).
+__device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                                int row) {
+  const bool valid = row < t.row_end;
+  if (g.mode == kGateUp) {
+    __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(g.out);
+#pragma unroll 1
+    for (int c = 0; c < BM; c += 32) {
+      uint32_t gr[32], ur[32];
+      tmem_ld_32x32b_x32(tbase + c, gr);
+      tmem_ld_32x32b_x32(tbase + BM + c, ur);
+      tmem_ld_wait();
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(hout + (size_t)row * g.ld_out + t.nt * BM + c);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int j = v * 8 + i * 2;
+            const float h0 = silu_f(__uint_as_float(gr[j])) * __uint_as_float(ur[j]);
+            const float h1 = silu_f(__uint_as_float(gr[j + 1])) * __uint_as_float(ur[j + 1]);
+            w[i] = pack_bf16x2(h0, h1);
+          }
+          dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    return;
+  }
+  int tok = 0;
+  float sc = 0.f;
+  if (g.mode == kDownAtomic && valid) {
+    tok = g.perm_token[row];
+    sc = g.scale * g.row_gate[row];
+  }
+#pragma unroll 1
+  for (int c = 0; c < 256; c += 32) {
+    uint32_t yr[32];
+    tmem_ld_32x32b_x32(tbase + c, yr);
+    tmem_ld_wait();
+    const int col = t.nt * 256 + c;
+    if (!valid || col >= g.n_valid) continue;
+    if (g.mode == kDownStore) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                            (size_t)row * g.ld_out + col);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = v * 8 + i * 2;
+          w[i] = pack_bf16x2(__uint_as_float(yr[j]), __uint_as_float(yr[j + 1]));
+        }
+        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) +
+                                              (size_t)tok * g.ld_out + col);
+#pragma unroll
+      for (int v = 0; v < 8; ++v)
+        atomicAdd(dst + v, make_float4(sc * __uint_as_float(yr[4 * v + 0]),
+                                       sc * __uint_as_float(yr[4 * v + 1]),
+                                       sc * __uint_as_float(yr[4 * v + 2]),
+                                       sc * __uint_as_float(yr[4 * v + 3])));
+    }
+  }
+}
+
+template <int BN_>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+  using C = Cfg<BN_>;
   extern __shared__ uint8_t smem_raw[];
-  SharedStorage& s = *reinterpret_cast<SharedStorage*>(
+  SharedStorage<BN_>& s = *reinterpret_cast<SharedStorage<BN_>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- set-up -------------------------------------------------------------------------
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
+    for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NACC; ++i) {
       mbar_init(&s.tfull[i], 1);
       mbar_init(&s.tempty[i], 128);
     }
@@ -127,7 +224,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   // tile table: toff[e] = sum_{e' < e} ceil(count_e' / 128)
-  for (int i = threadIdx.x; i <= g.n_ffn; i += kThreads) s.offs[i] = g.offsets[i];
+  if (g.dense_rows > 0) {
+    if (threadIdx.x == 0) {
+      s.offs[0] = 0;
+      s.offs[1] = g.dense_rows;
+    }
+  } else {
+    for (int i = threadIdx.x; i <= g.n_ffn; i += kThreads) s.offs[i] = g.offsets[i];
+  }
   __syncthreads();
   if (warp == 2) {
     const int per = (g.n_ffn + 31) / 32;
@@ -148,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = s.tmem_base;
-  const int total_tiles = s.toff[g.n_ffn] * g.n_tiles;
+  const int total_tiles = s.toff[g.n_ffn] * g.n_tiles * g.ksplit;
   volatile int* abort_flag = &s.abort_flag;
 
   if (warp == 0) {
@@ -158,15 +262,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
         const Tile t = decode_tile(s, g, tile);
-        const int brow0 = t.e * g.b_rows + t.nt * (g.mode == kGateUp ? BM : BN);
+        const int brow0 = t.e * g.b_rows + t.nt * (g.mode == kGateUp ? BM : BN_);
         const int brow1 = brow0 + g.b_second;
-        for (int kb = 0; kb < g.kblocks; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
-          mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
-          tma_load_2d(s.a[stage], &tmA, kb * BK, t.row0, &s.full[stage]);
+          mbar_arrive_expect_tx(&s.full[stage], C::STAGE_BYTES);
+          const int ka = g.a_kwrap > 0 ? kb % g.a_kwrap : kb;
+          tma_load_2d(s.a[stage], &tmA, ka * BK, t.row0, &s.full[stage]);
           tma_load_2d(s.b[stage], &tmB, kb * BK, brow0, &s.full[stage]);
-          tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
-          if (++stage == STAGES) {
+          if (BN_ == 256) tma_load_2d(s.b[stage] + C::B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -174,40 +279,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer ----------------------------------------------------------------------
+    // ---- MMA issuer: one TMEM accumulator per chunk of k-blocks -------------------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
-        if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        bool ok = true;
-        for (int kb = 0; kb < g.kblocks; ++kb) {
-          if (!mbar_wait(&s.full[stage], phase, abort_flag)) {
-            ok = false;
-            break;
-          }
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles && !*abort_flag; tile += gridDim.x) {
+        const Tile t = decode_tile(s, g, tile);
+        const int cl = chunk_len(g, t);
+        for (int c0 = t.kb0; ok && c0 < t.kb1; c0 += cl) {
+          const int c1 = min(c0 + cl, t.kb1);
+          if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(s.a[stage]);
-          const uint32_t b0 = smem_u32(s.b[stage]);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN_);
+          for (int kb = c0; kb < c1; ++kb) {
+            if (!mbar_wait(&s.full[stage], phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(s.a[stage]);
+            const uint32_t b0 = smem_u32(s.b[stage]);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            umma_bf16(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
-                      kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
+                        C::IDESC, (kb > c0 || k > 0) ? 1u : 0u);
+            umma_commit(&s.empty[stage]);
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          umma_commit(&s.empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+          if (!ok) break;
+          umma_commit(&s.tfull[acc]);
+          if (++acc == C::NACC) {
+            acc = 0;
+            acc_phase ^= 1u;
           }
         }
-        if (!ok) break;
-        umma_commit(&s.tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
       }
     }
   } else {
@@ -216,87 +324,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_in_tile = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       const Tile t = decode_tile(s, g, tile);
-      // one lane waits, the warp follows it: tcgen05.ld below needs all 32 lanes
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(&s.tfull[acc], acc_phase, abort_flag) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
       const int row = t.row0 + row_in_tile;
-      const bool valid = row < t.row_end;
-      if (g.mode == kGateUp) {
-        __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(g.out);
-#pragma unroll 1
-        for (int c = 0; c < BM; c += 32) {
-          uint32_t gr[32], ur[32];
-          tmem_ld_32x32b_x32(tbase + c, gr);
-          tmem_ld_32x32b_x32(tbase + BM + c, ur);
-          tmem_ld_wait();
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(hout + (size_t)row * g.ld_out + t.nt * BM + c);
+      const int cl = chunk_len(g, t);
+      float sum[BN_ == 128 ? 128 : 1];
+      if constexpr (BN_ == 128) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint32_t w[4];
+        for (int i = 0; i < 128; ++i) sum[i] = 0.f;
+      }
+      for (int c0 = t.kb0; c0 < t.kb1; c0 += cl) {
+        // one lane waits, the warp follows it: tcgen05.ld below needs all 32 lanes
+        int w_ok = 1;
+        if (lane == 0) w_ok = mbar_wait(&s.tfull[acc], acc_phase, abort_flag) ? 1 : 0;
+        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+        if (!w_ok) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(acc * BN_);
+        if constexpr (BN_ == 128) {
+          // router logits: add this chunk to the fp32 running sum (round to nearest)
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int j = v * 8 + i * 2;
-                const float h0 = silu_f(__uint_as_float(gr[j])) * __uint_as_float(ur[j]);
-                const float h1 = silu_f(__uint_as_float(gr[j + 1])) * __uint_as_float(ur[j + 1]);
-                w[i] = pack_bf16x2(h0, h1);
-              }
-              dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tbase + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum[c + i] = __fadd_rn(sum[c + i], __uint_as_float(v[i]));
           }
+        } else {
+          epilogue_expert(g, t, tbase, row);
         }
-      } else {
-        int tok = 0;
-        float sc = 0.f;
-        if (g.mode == kDownAtomic && valid) {
-          tok = g.perm_token[row];
-          sc = g.scale * g.row_gate[row];
+        tc_fence_before();
+        mbar_arrive(&s.tempty[acc]);
+        if (++acc == C::NACC) {
+          acc = 0;
+          acc_phase ^= 1u;
         }
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t yr[32];
-          tmem_ld_32x32b_x32(tbase + c, yr);
-          tmem_ld_wait();
-          const int col = t.nt * BN + c;
-          if (valid && col < g.n_valid) {
-            if (g.mode == kDownStore) {
-              uint4* dst = reinterpret_cast<uint4*>(
-                  static_cast<__nv_bfloat16*>(g.out) + (size_t)row * g.ld_out + col);
+      }
+      if constexpr (BN_ == 128) {
+        if (ok && row < t.row_end) {
+          const int col0 = t.nt * 128;
+          float* dst = static_cast<float*>(g.out) + t.split * g.split_stride +
+                       (size_t)row * g.ld_out + col0;
+          if (col0 + 128 <= g.n_valid && (g.ld_out & 3) == 0) {
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                uint32_t w[4];
+            for (int v = 0; v < 32; ++v)
+              reinterpret_cast<float4*>(dst)[v] =
+                  make_float4(sum[4 * v], sum[4 * v + 1], sum[4 * v + 2], sum[4 * v + 3]);
+          } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int j = v * 8 + i * 2;
-                  w[i] = pack_bf16x2(__uint_as_float(yr[j]), __uint_as_float(yr[j + 1]));
-                }
-                dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-              }
-            } else {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) +
-                                                      (size_t)tok * g.ld_out + col);
-#pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                atomicAdd(dst + v, make_float4(sc * __uint_as_float(yr[4 * v + 0]),
-                                               sc * __uint_as_float(yr[4 * v + 1]),
-                                               sc * __uint_as_float(yr[4 * v + 2]),
-                                               sc * __uint_as_float(yr[4 * v + 3])));
-              }
-            }
+            for (int v = 0; v < 128; ++v)
+              if (col0 + v < g.n_valid) dst[v] = sum[v];
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&s.tempty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
     }
   }
 
@@ -344,26 +427,126 @@ int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-constexpr size_t kSmemBytes = sizeof(SharedStorage) + 1024;
-
+template <int BN_>
 int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int sm_count,
                cudaStream_t st) {
-  if (cudaFuncSetAttribute(k_grouped_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSmemBytes) != cudaSuccess)
+  constexpr size_t smem = sizeof(SharedStorage<BN_>) + 1024;
+  static_assert(smem <= 227 * 1024, "shared memory budget");
+  if (cudaFuncSetAttribute(k_grouped_gemm_tc<BN_>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
-  k_grouped_gemm_tc<<<sm_count, kThreads, kSmemBytes, st>>>(ma, mb, g);
+  k_grouped_gemm_tc<BN_><<<sm_count, kThreads, smem, st>>>(ma, mb, g);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// W_r fp32 [E, H] -> bf16 [E, 3H] = [hi | mid | lo] with hi + mid + lo == w exactly:
+// hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid); each difference is exact in
+// fp32 (the significands shrink by 8 bits per step), and so is every product x * part
+// for bf16 x, so the three-part GEMM forms the same products as the fp32 one.
+__global__ void __launch_bounds__(256) k_split_router_weight(const float4* __restrict__ w,
+                                                             __nv_bfloat16* __restrict__ out,
+                                                             int E, int H) {
+  const int H4 = H / 4;                       // four weights per thread step
+  const size_t n = (size_t)E * H4;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t e = i / H4, k = (i - e * H4) * 4;
+    const float4 v4 = w[i];
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    float hi[4], mid[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      hi[j] = __bfloat162float(__float2bfloat16_rn(v[j]));
+      const float r1 = __fsub_rn(v[j], hi[j]);
+      mid[j] = __bfloat162float(__float2bfloat16_rn(r1));
+      lo[j] = __fsub_rn(r1, mid[j]);             // exact in bf16: at most 8 significant bits
+    }
+    __nv_bfloat16* row = out + e * 3 * (size_t)H + k;
+    *reinterpret_cast<uint2*>(row) = make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
+    *reinterpret_cast<uint2*>(row + H) =
+        make_uint2(pack_bf16x2(mid[0], mid[1]), pack_bf16x2(mid[2], mid[3]));
+    *reinterpret_cast<uint2*>(row + 2 * (size_t)H) =
+        make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
+  }
+}
+
 }  // namespace
+
+// Router logits: 128 x 128 tiles, K = 3H (the three weight parts); the tensor cores
+// accumulate kRouterChunk k-blocks at a time and the epilogue sums the chunks in fp32.
+constexpr int kRouterChunk = 6;
+constexpr int kRouterMinSplit = 12;   // k-blocks per split at least (two chunks)
+
+int router_tc_splitk(int T, int E, int H, int sm_count) {
+  if (sm_count > 160) sm_count = 160;
+  const long tiles = (long)((T + BM - 1) / BM) * ((E + 127) / 128);
+  const int kblocks = 3 * H / BK;
+  if (tiles <= 0) return 1;
+  long s = (2L * sm_count + tiles - 1) / tiles;
+  long smax = kblocks / kRouterMinSplit;
+  if (smax > 64) smax = 64;
+  if (s > smax) s = smax;
+  if (s < 1) s = 1;
+  const int kbp = (kblocks + (int)s - 1) / (int)s;      // no empty split
+  return (kblocks + kbp - 1) / kbp;
+}
+
+size_t router_tc_scratch_bytes(int T, int E, int H) {
+  const int S = router_tc_splitk(T, E, H, 160);
+  size_t b = (size_t)E * 3 * H * 2;                  // split weight
+  b = (b + 1023) / 1024 * 1024;
+  if (S > 1) b += (size_t)S * T * E * sizeof(float); // per-split partial logits
+  return b;
+}
+
+int launch_router_logits_tc(const void* x, const float* w_router, int T, int E, int H,
+                            float* logits, void* scratch, int sm_count, cudaStream_t st) {
+  if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
+  __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(scratch);
+  size_t off = ((size_t)E * 3 * H * 2 + 1023) / 1024 * 1024;
+  float* partial = reinterpret_cast<float*>(static_cast<char*>(scratch) + off);
+  {
+    const size_t n = (size_t)E * H / 4;
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 8 * sm_count) blocks = 8 * sm_count;
+    k_split_router_weight<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(w_router),
+                                                  wsplit, E, H);
+    count_launch();
+  }
+  CUtensorMap mx, mw;
+  int rc;
+  if ((rc = make_map(&mx, x, (uint64_t)T, H)) != MOE_OK) return rc;
+  if ((rc = make_map(&mw, wsplit, (uint64_t)E, 3ull * H)) != MOE_OK) return rc;
+  const int S = router_tc_splitk(T, E, H, sm_count);
+  GemmArgs g{};
+  g.mode = kLogits;
+  g.n_ffn = 1;
+  g.dense_rows = T;
+  g.kblocks = 3 * H / BK;
+  g.a_kwrap = H / BK;
+  g.ksplit = S;
+  g.kb_per_split = (g.kblocks + S - 1) / S;
+  g.kchunk = kRouterChunk;
+  g.n_tiles = (E + 127) / 128;
+  g.b_rows = 0;
+  g.b_second = 0;
+  g.n_valid = E;
+  g.ld_out = E;
+  g.out = S > 1 ? static_cast<void*>(partial) : static_cast<void*>(logits);
+  g.split_stride = (long long)T * E;
+  if ((rc = launch_one<128>(mx, mw, g, sm_count, st)) != MOE_OK) return rc;
+  if (S > 1) {
+    if (launch_splitk_sum(partial, S, (size_t)T * E, logits, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
 
 int launch_grouped_ffn_tc(const void* x_perm, const int32_t* offsets, const void* w_gate_up,
                           const void* w_down, const int32_t* perm_token, const float* row_gate,
                           void* h, void* y_perm, float* out_acc, int T, int H, int I, int n_ffn,
                           int K, float scale, int fused, int* status, int sm_count,
                           cudaStream_t st) {
-  static_assert(sizeof(SharedStorage) + 1024 <= 227 * 1024, "shared memory budget");
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   const uint64_t rows = (uint64_t)T * K + BM;   // x_perm / h / y_perm allocation rows
   CUtensorMap mx, mwgu, mh, mwd;
@@ -382,29 +565,31 @@ int launch_grouped_ffn_tc(const void* x_perm, const int32_t* offsets, const void
   g1.b_second = I;
   g1.n_valid = I;
   g1.ld_out = I;
-  g1.col_step = BM;
   g1.offsets = offsets;
   g1.out = h;
   g1.status = status;
-  if ((rc = launch_one(mx, mwgu, g1, sm_count, st)) != MOE_OK) return rc;
+  g1.ksplit = 1;
+  g1.kb_per_split = g1.kblocks;
+  if ((rc = launch_one<256>(mx, mwgu, g1, sm_count, st)) != MOE_OK) return rc;
 
   GemmArgs g2{};
   g2.mode = fused ? kDownAtomic : kDownStore;
   g2.n_ffn = n_ffn;
   g2.kblocks = I / BK;
-  g2.n_tiles = (H + BN - 1) / BN;
+  g2.n_tiles = (H + 255) / 256;
   g2.b_rows = H;
   g2.b_second = BM;
   g2.n_valid = H;
   g2.ld_out = H;
-  g2.col_step = BN;
   g2.offsets = offsets;
   g2.out = fused ? static_cast<void*>(out_acc) : y_perm;
   g2.perm_token = perm_token;
   g2.row_gate = row_gate;
   g2.scale = scale;
   g2.status = status;
-  return launch_one(mh, mwd, g2, sm_count, st);
+  g2.ksplit = 1;
+  g2.kb_per_split = g2.kblocks;
+  return launch_one<256>(mh, mwd, g2, sm_count, st);
 }
 
 }  // namespace moe

@@ -27,6 +27,12 @@ size_t router_partial_bytes(int T, int E, int H, int sm_count_max);
 cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_router, int T,
                                  int E, int H, float* logits, float* partial, int splitk,
                                  cudaStream_t st);
+cudaError_t launch_splitk_sum(const float* partial, int S, size_t n, float* out, cudaStream_t st);
+// bf16 x: logits on the tensor cores with W_r split into three exact bf16 parts.
+int router_tc_splitk(int T, int E, int H, int sm_count);
+size_t router_tc_scratch_bytes(int T, int E, int H);
+int launch_router_logits_tc(const void* x, const float* w_router, int T, int E, int H,
+                            float* logits, void* scratch, int sm_count, cudaStream_t st);
 cudaError_t launch_route_topk(const float* logits, const float* bias, int T, int E, int n_ffn,
                               int K, int32_t* topk_idx, float* topk_gate, int32_t* counts,
                               int32_t* nffn_hist, float* zgate, int sm_count, cudaStream_t st);

@@ -159,6 +159,13 @@ __global__ void k_router_splitk_sum(const float* __restrict__ partial, int S, si
 }
 }  // namespace
 
+cudaError_t launch_splitk_sum(const float* partial, int S, size_t n, float* out, cudaStream_t st) {
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  k_router_splitk_sum<<<blocks, 256, 0, st>>>(partial, S, n, out);
+  count_launch();
+  return cudaGetLastError();
+}
+
 int router_splitk(int T, int E, int H, int sm_count) {
   if (sm_count > kSmMax) sm_count = kSmMax;
   const long tiles = (long)((T + RB - 1) / RB) * ((E + RB - 1) / RB);
