@@ -188,10 +188,11 @@ class Stepper:
                   None if self.logits_in is not None else b.logits, b.topk_idx, b.topk_gate,
                   b.counts, b.nffn_hist, b.zgate, b.ws)
         mark(1)
+        xp = b.x_perm
         abi.permute(s, b.topk_idx, b.topk_gate, b.zgate, self.x, b.offsets, b.perm_token,
-                    b.row_of, b.row_gate, b.x_perm, b.out_acc, b.ws)
+                    b.row_of, b.row_gate, xp, b.out_acc, b.ws)
         mark(2)
-        abi.grouped_ffn(s, b.x_perm, b.offsets, w.w_gate_up, w.w_down, b.perm_token,
+        abi.grouped_ffn(s, self.x, xp, b.offsets, w.w_gate_up, w.w_down, b.perm_token,
                         b.row_gate, b.h, b.y_perm, b.out_acc, b.ws)
         mark(3)
         abi.combine(s, self.x, b.y_perm, b.out_acc, b.topk_gate, b.row_of, b.zgate, b.out)
@@ -428,7 +429,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_bf16", choices=sorted(wl.CONFIGS))
-    ap.add_argument("--combine", default="fused", choices=["fused", "deterministic"])
+    ap.add_argument("--combine", default="deterministic", choices=["fused", "deterministic"])
     ap.add_argument("--cpu-tokens", type=int, default=400)
     ap.add_argument("--ref-tokens", type=int, default=8)
     ap.add_argument("--tokens", type=int, default=None, help="override the workload's T")

@@ -136,8 +136,12 @@ int moe_route(const moe_shape_t* shape, const void* x, const float* w_router,
  *   perm_token device [T * K] int32           token of each row; entries >= R unwritten
  *   row_of     device [T, K] int32            row of each pick, -1 for zero experts
  *   row_gate   device [T * K] fp32            gate of each row
- *   x_perm     device [T * K + 128, H] dtype  x[perm_token[r]] in row r; the 128 extra
- *                                             rows are read (never written) by the GEMM
+ *   x_perm     device [T * K + 128, H] dtype  x[perm_token[r]] in row r, or NULL: no copy
+ *              or NULL                        (bf16 layers can let moe_grouped_ffn gather
+ *                                             the rows from x instead, which saves this
+ *                                             buffer but makes the gate/up GEMM slower);
+ *                                             the 128 extra rows are read (never written)
+ *                                             by the GEMM
  *   out_acc    device [T, H] fp32 or NULL     if given, set to zgate[t] * x[t]: the
  *                                             zero-computation experts' term, ready for
  *                                             the fused combine
@@ -149,11 +153,16 @@ int moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* 
                 size_t ws_bytes, void* stream);
 
 /* Grouped SwiGLU FFN over the expert groups (report §2.4: intermediate I per expert).
- *   x_perm     device [T * K + 128, H] dtype  from moe_permute
+ *   x          device [T, H] dtype            token activations; read when x_perm is NULL
+ *   x_perm     device [T * K + 128, H] dtype  from moe_permute, or NULL (bf16 only): the
+ *              or NULL                        gate/up GEMM then gathers row r from
+ *                                             x[perm_token[r]] with TMA four-row gathers
+ *                                             (no x_perm buffer, but about 3x slower gate/up
+ *                                             GEMM on B200: 32 gathers per k-block)
  *   offsets    device [n_ffn + 1] int32
  *   w_gate_up  device [n_ffn, 2I, H] dtype    rows [0, I) gate, rows [I, 2I) up
  *   w_down     device [n_ffn, H, I] dtype
- *   perm_token device [T * K] int32           (fused combine only)
+ *   perm_token device [T * K] int32           (fused combine, or x_perm NULL)
  *   row_gate   device [T * K] fp32            (fused combine only)
  *   h          device [T * K + 128, I] dtype  receives silu(x W_g^T) * (x W_u^T)
  *   y_perm     device [T * K + 128, H] dtype  deterministic combine: receives y = h W_d^T
@@ -161,10 +170,10 @@ int moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* 
  *                                             s * row_gate[r] * y[r] (atomic fp32 adds)
  * bf16 runs on the tensor cores (tcgen05, fp32 accumulate, h rounded to bf16); fp32 runs
  * a plain fp32 kernel. The call reads the row counts on the device: it never waits. */
-int moe_grouped_ffn(const moe_shape_t* shape, const void* x_perm, const int32_t* offsets,
-                    const void* w_gate_up, const void* w_down, const int32_t* perm_token,
-                    const float* row_gate, void* h, void* y_perm, float* out_acc, void* ws,
-                    size_t ws_bytes, void* stream);
+int moe_grouped_ffn(const moe_shape_t* shape, const void* x, const void* x_perm,
+                    const int32_t* offsets, const void* w_gate_up, const void* w_down,
+                    const int32_t* perm_token, const float* row_gate, void* h, void* y_perm,
+                    float* out_acc, void* ws, size_t ws_bytes, void* stream);
 
 /* Combine (report §2.1: zero-computation experts contribute g * x).
  * Fused: out = out_acc rounded to dtype. Deterministic: out[t] = sum over the FFN slots k

@@ -73,7 +73,7 @@ _SIGS = {
     "moe_launch_count": (ctypes.c_uint64, []),
     "moe_route": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 11 + [_SZ, _P]),
     "moe_permute": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 11 + [_SZ, _P]),
-    "moe_grouped_ffn": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 10 + [_SZ, _P]),
+    "moe_grouped_ffn": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 11 + [_SZ, _P]),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 7 + [_P]),
     "moe_pid_init": (ctypes.c_int, [ctypes.POINTER(Shape), _P, _P, _P]),
     "moe_pid_bias_update": (ctypes.c_int, [ctypes.POINTER(Pid), ctypes.POINTER(Shape)]
@@ -195,12 +195,13 @@ def permute_static_scratch(shape, topk_idx, topk_gate, zgate, x, offsets, perm_t
                                             _stream(stream)), "moe_permute_static_scratch")
 
 
-def grouped_ffn(shape, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h, y_perm,
+def grouped_ffn(shape, x, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h, y_perm,
                 out_acc, ws, stream=None):
-    _check(lib().moe_grouped_ffn(ctypes.byref(shape), ptr(x_perm), ptr(offsets), ptr(w_gate_up),
-                                 ptr(w_down), ptr(perm_token), ptr(row_gate), ptr(h), ptr(y_perm),
-                                 ptr(out_acc), ptr(ws), _nbytes(ws), _stream(stream)),
-           "moe_grouped_ffn")
+    """x_perm None (bf16): the gate/up GEMM gathers the token rows of x via perm_token."""
+    _check(lib().moe_grouped_ffn(ctypes.byref(shape), ptr(x), ptr(x_perm), ptr(offsets),
+                                 ptr(w_gate_up), ptr(w_down), ptr(perm_token), ptr(row_gate),
+                                 ptr(h), ptr(y_perm), ptr(out_acc), ptr(ws), _nbytes(ws),
+                                 _stream(stream)), "moe_grouped_ffn")
 
 
 def combine(shape, x, y_perm, out_acc, topk_gate, row_of, zgate, out, stream=None):
@@ -280,15 +281,21 @@ class StepBuffers:
         )
 
 
-def run_steps(b: StepBuffers, x, w_router, logits_in, bias, w_gate_up, w_down, stream=None):
+def run_steps(b: StepBuffers, x, w_router, logits_in, bias, w_gate_up, w_down, stream=None,
+              gather=None):
     """The layer as its four ABI steps on one stream (moe_route, moe_permute,
-    moe_grouped_ffn, moe_combine); returns b.out."""
+    moe_grouped_ffn, moe_combine); returns b.out. gather=True (bf16 only) skips the
+    permuted copy of x and lets the gate/up GEMM gather the token rows (less memory,
+    slower GEMM)."""
     s = b.shape
+    if gather is None:
+        gather = False
+    xp = None if gather else b.x_perm
     route(s, x, w_router, logits_in, bias, None if logits_in is not None else b.logits,
           b.topk_idx, b.topk_gate, b.counts, b.nffn_hist, b.zgate, b.ws, stream)
     permute(s, b.topk_idx, b.topk_gate, b.zgate, x, b.offsets, b.perm_token, b.row_of,
-            b.row_gate, b.x_perm, b.out_acc, b.ws, stream)
-    grouped_ffn(s, b.x_perm, b.offsets, w_gate_up, w_down, b.perm_token, b.row_gate, b.h,
+            b.row_gate, xp, b.out_acc, b.ws, stream)
+    grouped_ffn(s, x, xp, b.offsets, w_gate_up, w_down, b.perm_token, b.row_gate, b.h,
                 b.y_perm, b.out_acc, b.ws, stream)
     combine(s, x, b.y_perm, b.out_acc, b.topk_gate, b.row_of, b.zgate, b.out, stream)
     return b.out

@@ -149,20 +149,28 @@ int route_impl(const moe_shape_t* s, const void* x, const float* w_router, const
   MOE_TRY(current_device_info(&dev));
   const int E = s->n_ffn + s->n_zero;
   const cudaStream_t st = as_stream(stream);
-  const float* logits = logits_in;
+  const float* src = logits_in;      // logits, or S split-K slices of them
+  int S = 1;
   if (!logits_in) {
     if (s->dtype == MOE_BF16) {
       MOE_TRY(launch_router_logits_tc(x, w_router, s->T, E, s->H, logits_out,
-                                      at<char>(ws, L.lpart), dev.sm_count, st));
+                                      at<char>(ws, L.lpart), dev.sm_count, st, &src, &S));
     } else {
-      const int S = router_splitk(s->T, E, s->H, dev.sm_count);
-      MOE_TRY(cuda_rc(launch_router_logits(x, 0, w_router, s->T, E, s->H, logits_out,
-                                           at<float>(ws, L.lpart), S, st)));
+      S = router_splitk(s->T, E, s->H, dev.sm_count);
+      float* part = at<float>(ws, L.lpart);
+      MOE_TRY(cuda_rc(launch_router_logits(x, 0, w_router, s->T, E, s->H, logits_out, part, S,
+                                           st)));
+      src = S > 1 ? part : logits_out;
     }
-    logits = logits_out;
   }
-  return cuda_rc(launch_route_topk(logits, bias, s->T, E, s->n_ffn, s->K, topk_idx, topk_gate,
-                                   counts, nffn_hist, zgate, dev.sm_count, st));
+  if (S > 4) {
+    // many slices: one wide reduction kernel beats summing them inside the top-K warps
+    MOE_TRY(cuda_rc(launch_splitk_sum(src, S, (size_t)s->T * E, logits_out, st)));
+    src = logits_out;
+    S = 1;
+  }
+  return cuda_rc(launch_route_topk(src, S, logits_out, bias, s->T, E, s->n_ffn, s->K, topk_idx,
+                                   topk_gate, counts, nffn_hist, zgate, dev.sm_count, st));
 }
 
 int permute_impl(const moe_shape_t* s, const int32_t* topk_idx, const float* topk_gate,
@@ -170,7 +178,8 @@ int permute_impl(const moe_shape_t* s, const int32_t* topk_idx, const float* top
                  int32_t* row_of, float* row_gate, void* x_perm, float* out_acc, void* ws,
                  size_t ws_bytes, void* stream) {
   MOE_TRY(check_shape(s));
-  MOE_TRY(check_ptrs({topk_idx, topk_gate, x, offsets, perm_token, row_of, row_gate, x_perm, ws}));
+  MOE_TRY(check_ptrs({topk_idx, topk_gate, x, offsets, perm_token, row_of, row_gate, ws}));
+  MOE_TRY(check_opt({x_perm}));
   if (out_acc) MOE_TRY(check_ptrs({zgate, out_acc}));
   const Layout L = layout_of(*s);
   if (ws_bytes < L.scratch_end) return MOE_ERR_WORKSPACE;
@@ -186,12 +195,15 @@ int permute_impl(const moe_shape_t* s, const int32_t* topk_idx, const float* top
                                 at<int>(ws, L.status), as_stream(stream)));
 }
 
-int grouped_ffn_impl(const moe_shape_t* s, const void* x_perm, const int32_t* offsets,
-                     const void* w_gate_up, const void* w_down, const int32_t* perm_token,
-                     const float* row_gate, void* h, void* y_perm, float* out_acc, void* ws,
-                     size_t ws_bytes, void* stream) {
+int grouped_ffn_impl(const moe_shape_t* s, const void* x, const void* x_perm,
+                     const int32_t* offsets, const void* w_gate_up, const void* w_down,
+                     const int32_t* perm_token, const float* row_gate, void* h, void* y_perm,
+                     float* out_acc, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(check_shape(s));
-  MOE_TRY(check_ptrs({x_perm, offsets, w_gate_up, w_down, h, ws}));
+  MOE_TRY(check_ptrs({offsets, w_gate_up, w_down, h, ws}));
+  if (x_perm) MOE_TRY(check_ptrs({x_perm}));
+  else if (s->dtype == MOE_BF16) MOE_TRY(check_ptrs({x, perm_token}));   // gathered rows
+  else return MOE_ERR_INVALID_ARG;                                      // fp32 needs x_perm
   const bool fused = s->combine == MOE_COMBINE_FUSED;
   if (fused) MOE_TRY(check_ptrs({perm_token, row_gate, out_acc}));
   else MOE_TRY(check_ptrs({y_perm}));
@@ -202,7 +214,7 @@ int grouped_ffn_impl(const moe_shape_t* s, const void* x_perm, const int32_t* of
   MOE_TRY(current_device_info(&dev));
   const cudaStream_t st = as_stream(stream);
   if (s->dtype == MOE_BF16)
-    return launch_grouped_ffn_tc(x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h, y_perm,
+    return launch_grouped_ffn_tc(x, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h, y_perm,
                                  out_acc, s->T, s->H, s->I, s->n_ffn, s->K, s->ffn_out_scale, fused,
                                  at<int>(ws, L.status), dev.sm_count, st);
   return cuda_rc(launch_grouped_ffn_simt(
@@ -299,11 +311,11 @@ int moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* 
                       x_perm, out_acc, ws, ws_bytes, stream);
 }
 
-int moe_grouped_ffn(const moe_shape_t* shape, const void* x_perm, const int32_t* offsets,
-                    const void* w_gate_up, const void* w_down, const int32_t* perm_token,
-                    const float* row_gate, void* h, void* y_perm, float* out_acc, void* ws,
-                    size_t ws_bytes, void* stream) {
-  return grouped_ffn_impl(shape, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h,
+int moe_grouped_ffn(const moe_shape_t* shape, const void* x, const void* x_perm,
+                    const int32_t* offsets, const void* w_gate_up, const void* w_down,
+                    const int32_t* perm_token, const float* row_gate, void* h, void* y_perm,
+                    float* out_acc, void* ws, size_t ws_bytes, void* stream) {
+  return grouped_ffn_impl(shape, x, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h,
                           y_perm, out_acc, ws, ws_bytes, stream);
 }
 
@@ -362,7 +374,7 @@ int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,
                      nffn_hist, zgate, ws, ws_bytes, stream));
   MOE_TRY(permute_impl(shape, topk_idx, topk_gate, zgate, x, offsets, perm, rowof, rowgate, xperm,
                        outacc, ws, ws_bytes, stream));
-  MOE_TRY(grouped_ffn_impl(shape, xperm, offsets, w_gate_up, w_down, perm, rowgate, h, yperm,
+  MOE_TRY(grouped_ffn_impl(shape, x, xperm, offsets, w_gate_up, w_down, perm, rowgate, h, yperm,
                            outacc, ws, ws_bytes, stream));
   return combine_impl(shape, x, yperm, outacc, topk_gate, rowof, zgate, out, stream);
 }

@@ -76,7 +76,11 @@ __global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, co
   }
   __syncthreads();
   const float zg = zgate[t];
-  for (int c = threadIdx.x * V; c < H; c += blockDim.x * V) {
+  // blockIdx.y picks a contiguous slice of the columns (several blocks per token when T
+  // is small)
+  const int per = (H / V + gridDim.y - 1) / gridDim.y * V;
+  const int c_end = min(H, (int)(blockIdx.y + 1) * per);
+  for (int c = blockIdx.y * per + threadIdx.x * V; c < c_end; c += blockDim.x * V) {
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
@@ -104,39 +108,18 @@ __global__ void k_pid_init(const float* __restrict__ bias, float* __restrict__ s
   }
 }
 
-// block-wide sum / max of doubles (fixed tree: deterministic)
-__device__ double block_sum(double v, double* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  double r = 0.0;
-  for (int i = 0; i < nw; ++i) r += red[i];
-  return r;
-}
-__device__ double block_max(double v, double* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  double r = red[0];
-  for (int i = 1; i < nw; ++i) r = fmax(r, red[i]);
-  return r;
-}
-
-// One CTA of 1024 threads; expert i = threadIdx.x (n_ffn <= 1024).
+// One CTA of 1024 threads; expert i = threadIdx.x (n_ffn <= 1024). The statistics are
+// reduced in one pass: warp butterflies, then thread 0 over the warps (fixed order).
 __global__ void __launch_bounds__(1024) k_pid_update(moe_pid_t pid, const int32_t* __restrict__ counts,
                                                      const int32_t* __restrict__ hist,
                                                      float* __restrict__ bias, float* __restrict__ st,
                                                      float* __restrict__ stats, int T, int K,
                                                      int n_ffn, int E) {
-  __shared__ double red[32];
-  const int i = threadIdx.x;
-  double c_ffn = 0.0, c_hit = 0.0, c_zero = 0.0, abs_e = 0.0;
+  __shared__ double red[32][8];
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  // v: [0] FFN count, [1] max FFN count, [2] FFN experts hit, [3] zero-expert count,
+  //    [4] |e|, [5] max |e|, [6] n * hist[n], [7] n^2 * hist[n]
+  double v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (i < n_ffn) {
     const int c = counts[i];
     const float f = __fdiv_rn((float)c, (float)T);
@@ -150,36 +133,43 @@ __global__ void __launch_bounds__(1024) k_pid_update(moe_pid_t pid, const int32_
     bias[i] = b;
     st[n_ffn + i] = integ;
     st[2 * n_ffn + i] = e;
-    c_ffn = (double)c;
-    c_hit = c > 0 ? 1.0 : 0.0;
-    abs_e = fabs((double)e);
+    v[0] = v[1] = (double)c;
+    v[2] = c > 0 ? 1.0 : 0.0;
+    v[4] = v[5] = fabs((double)e);
   }
-  for (int j = n_ffn + i; j < E; j += blockDim.x) c_zero += (double)counts[j];
-  double hn = 0.0, hn2 = 0.0;
+  for (int j = n_ffn + i; j < E; j += blockDim.x) v[3] += (double)counts[j];
   if (i <= K) {
-    hn = (double)hist[i] * i;
-    hn2 = (double)hist[i] * i * i;
+    v[6] = (double)hist[i] * i;
+    v[7] = (double)hist[i] * i * i;
   }
-  const double s_ffn = block_sum(c_ffn, red);
-  const double m_ffn = block_max(c_ffn, red);
-  const double s_hit = block_sum(c_hit, red);
-  const double s_zero = block_sum(c_zero, red);
-  const double s_abs = block_sum(abs_e, red);
-  const double m_abs = block_max(abs_e, red);
-  const double s_hn = block_sum(hn, red);
-  const double s_hn2 = block_sum(hn2, red);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const double u = __shfl_xor_sync(0xffffffffu, v[k], o);
+      v[k] = (k == 1 || k == 5) ? fmax(v[k], u) : v[k] + u;
+    }
+  }
+  if (lane == 0)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) red[warp][k] = v[k];
+  __syncthreads();
   if (stats && i == 0) {
-    const double mean = s_hn / T;
-    const double var = fmax(0.0, s_hn2 / T - mean * mean);
-    const double mean_load = s_ffn / n_ffn;
+    double r[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) r[k] = (k == 1 || k == 5) ? fmax(r[k], red[w][k]) : r[k] + red[w][k];
+    const double mean = r[6] / T;
+    const double var = fmax(0.0, r[7] / T - mean * mean);
+    const double mean_load = r[0] / n_ffn;
     stats[0] = (float)(mean / K);
     stats[1] = (float)mean;
     stats[2] = (float)sqrt(var);
-    stats[3] = (float)(mean_load > 0.0 ? m_ffn / mean_load : 0.0);
-    stats[4] = (float)s_hit;
-    stats[5] = (float)(s_zero / ((double)T * K));
-    stats[6] = (float)(s_abs / n_ffn);
-    stats[7] = (float)m_abs;
+    stats[3] = (float)(mean_load > 0.0 ? r[1] / mean_load : 0.0);
+    stats[4] = (float)r[2];
+    stats[5] = (float)(r[3] / ((double)T * K));
+    stats[6] = (float)(r[4] / n_ffn);
+    stats[7] = (float)r[5];
   }
 }
 
@@ -202,12 +192,19 @@ cudaError_t launch_finalize(const float* out_acc, void* out, int out_is_bf16, si
 cudaError_t launch_combine_det(const void* x, const void* y_perm, const float* topk_gate,
                                const int32_t* row_of, const float* zgate, void* out,
                                int is_bf16, int T, int H, int K, float scale, cudaStream_t st) {
+  // enough blocks for every SM even at small T (one CTA per token and column slice)
+  const int V = is_bf16 ? 8 : 4;
+  int nseg = (2 * 148 + T - 1) / T;
+  const int max_seg = (H / V + 255) / 256;
+  if (nseg > max_seg) nseg = max_seg;
+  if (nseg < 1) nseg = 1;
+  const dim3 grid(T, nseg);
   if (is_bf16)
-    k_combine_det<__nv_bfloat16><<<T, 256, 0, st>>>(
+    k_combine_det<__nv_bfloat16><<<grid, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm), topk_gate,
         row_of, zgate, static_cast<__nv_bfloat16*>(out), H, K, scale);
   else
-    k_combine_det<float><<<T, 256, 0, st>>>(static_cast<const float*>(x),
+    k_combine_det<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x),
                                             static_cast<const float*>(y_perm), topk_gate, row_of,
                                             zgate, static_cast<float*>(out), H, K, scale);
   count_launch();

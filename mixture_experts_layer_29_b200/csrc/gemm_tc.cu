@@ -35,34 +35,26 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BK = 64;
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
-constexpr int kThreads = 192;
+constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 48 KB
+constexpr int kEpiWarps = 8;                         // two per TMEM lane quarter
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = 64 + kEpiThreads;           // producer, MMA, epilogue
 constexpr int kMaxExperts = 1024;
-constexpr uint32_t kTmemCols = 512;
-
-// Per N-tile width: 256 for the expert GEMMs, 128 for the router (whose epilogue keeps a
-// 128-column running sum per row in registers).
-template <int BN_>
-struct Cfg {
-  static constexpr int BN = BN_;
-  static constexpr int B_BYTES = BN_ * BK * 2;                 // 32 KB / 16 KB
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 48 KB / 32 KB
-  static constexpr int STAGES = BN_ == 256 ? 4 : 6;            // 192 KB of ring either way
-  static constexpr int NACC = 512 / BN_;                       // TMEM accumulators
-  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN_);
-};
+constexpr uint32_t kTmemCols = 512;                  // two 256-column fp32 accumulators
+constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
 
 enum Mode : int { kGateUp = 0, kDownStore = 1, kDownAtomic = 2, kLogits = 3 };
 
-template <int BN_>
 struct alignas(1024) SharedStorage {
-  uint8_t a[Cfg<BN_>::STAGES][A_BYTES];
-  uint8_t b[Cfg<BN_>::STAGES][Cfg<BN_>::B_BYTES];
-  uint64_t full[Cfg<BN_>::STAGES];
-  uint64_t empty[Cfg<BN_>::STAGES];
-  uint64_t tfull[Cfg<BN_>::NACC];
-  uint64_t tempty[Cfg<BN_>::NACC];
+  uint8_t a[STAGES][A_BYTES];
+  uint8_t b[STAGES][B_BYTES];
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
   uint32_t tmem_base;
   int abort_flag;
   int offs[kMaxExperts + 1];
@@ -74,8 +66,8 @@ struct GemmArgs {
   int n_ffn;
   int kblocks;        // K / 64
   int n_tiles;        // N tiles per M tile
-  int b_rows;         // B rows per expert: 2I (gate/up) or H (down)
-  int b_second;       // row offset of the second 128-row B box: I (gate/up) or 128 (down)
+  int b_rows;         // B rows per expert: 2I (gate/up) or H (down); 0 for the router
+  int b_second;       // row offset of the second 128-row B box: I (gate/up) or 128
   int n_valid;        // valid output columns: I (h), H (y) or E (logits)
   int ld_out;         // output row length in elements
   const int32_t* offsets;
@@ -90,15 +82,14 @@ struct GemmArgs {
   int kb_per_split;         // k-blocks per split
   int kchunk;               // k-blocks per tensor-core accumulation (0: the whole split)
   long long split_stride;   // elements between the outputs of consecutive splits
+  const int32_t* gather_tok;  // non-null: A row r is row gather_tok[r] of A's tensor
 };
 
 struct Tile {
   int e, row0, row_end, nt, kb0, kb1, split;
 };
 
-template <int BN_>
-__device__ __forceinline__ Tile decode_tile(const SharedStorage<BN_>& s, const GemmArgs& g,
-                                            int tile) {
+__device__ __forceinline__ Tile decode_tile(const SharedStorage& s, const GemmArgs& g, int tile) {
   Tile t;
   const int per_split = s.toff[g.n_ffn] * g.n_tiles;
   t.split = tile / per_split;
@@ -125,14 +116,16 @@ __device__ __forceinline__ int chunk_len(const GemmArgs& g, const Tile& t) {
 
 __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
-// Epilogue of one 128 x 256 accumulator of the expert GEMMs (modes gate-up / down).
+// Epilogue of one 128 x 256 accumulator of the expert GEMMs for one thread: its TMEM lane
+// (row) and its half of the columns (gate/up: gate columns [64h, 64h+64) with the matching
+// up columns; down: columns [128h, 128h+128)).
 __device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t, uint32_t tbase,
-                                                int row) {
+                                                int row, int half) {
   const bool valid = row < t.row_end;
   if (g.mode == kGateUp) {
     __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(g.out);
 #pragma unroll 1
-    for (int c = 0; c < BM; c += 32) {
+    for (int c = 64 * half; c < 64 * half + 64; c += 32) {
       uint32_t gr[32], ur[32];
       tmem_ld_32x32b_x32(tbase + c, gr);
       tmem_ld_32x32b_x32(tbase + BM + c, ur);
@@ -162,11 +155,11 @@ __device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t
     sc = g.scale * g.row_gate[row];
   }
 #pragma unroll 1
-  for (int c = 0; c < 256; c += 32) {
+  for (int c = 128 * half; c < 128 * half + 128; c += 32) {
     uint32_t yr[32];
     tmem_ld_32x32b_x32(tbase + c, yr);
     tmem_ld_wait();
-    const int col = t.nt * 256 + c;
+    const int col = t.nt * BN + c;
     if (!valid || col >= g.n_valid) continue;
     if (g.mode == kDownStore) {
       uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
@@ -194,25 +187,26 @@ __device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t
   }
 }
 
-template <int BN_>
+// LOGITS: the router instantiation (mode kLogits, running sums in the epilogue); the
+// expert GEMMs use the other one.
+template <bool LOGITS>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
-  using C = Cfg<BN_>;
   extern __shared__ uint8_t smem_raw[];
-  SharedStorage<BN_>& s = *reinterpret_cast<SharedStorage<BN_>*>(
+  SharedStorage& s = *reinterpret_cast<SharedStorage*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- set-up -------------------------------------------------------------------------
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::STAGES; ++i) {
+    for (int i = 0; i < STAGES; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    for (int i = 0; i < C::NACC; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], 128);
+      mbar_init(&s.tempty[i], kEpiThreads);
     }
     s.abort_flag = 0;
     fence_barrier_init();
@@ -255,23 +249,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total_tiles = s.toff[g.n_ffn] * g.n_tiles * g.ksplit;
   volatile int* abort_flag = &s.abort_flag;
 
-  if (warp == 0) {
+  if (warp == 0 && g.gather_tok != nullptr) {
+    // ---- TMA producer, gathered A: lane i fetches rows 4i..4i+3 of the A tile ----------
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles && !*abort_flag; tile += gridDim.x) {
+      const Tile t = decode_tile(s, g, tile);
+      int r[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)   // rows past the group repeat its last token (never stored)
+        r[j] = g.gather_tok[min(t.row0 + 4 * lane + j, t.row_end - 1)];
+      const int brow0 = t.e * g.b_rows + t.nt * (g.mode == kGateUp ? BM : BN);
+      const int brow1 = brow0 + g.b_second;
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        int w_ok = 1;
+        if (lane == 0) {
+          w_ok = mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag) ? 1 : 0;
+          if (w_ok) mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
+        }
+        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+        if (!w_ok) {
+          ok = false;
+          break;
+        }
+        const int ka = g.a_kwrap > 0 ? kb % g.a_kwrap : kb;
+        tma_gather4(s.a[stage] + lane * 4 * (BK * 2), &tmA, ka * BK, r[0], r[1], r[2], r[3],
+                    &s.full[stage]);
+        if (lane == 0) {
+          tma_load_2d(s.b[stage], &tmB, kb * BK, brow0, &s.full[stage]);
+          tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 0) {
     // ---- TMA producer ------------------------------------------------------------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
         const Tile t = decode_tile(s, g, tile);
-        const int brow0 = t.e * g.b_rows + t.nt * (g.mode == kGateUp ? BM : BN_);
+        const int brow0 = t.e * g.b_rows + t.nt * (g.mode == kGateUp ? BM : BN);
         const int brow1 = brow0 + g.b_second;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
-          mbar_arrive_expect_tx(&s.full[stage], C::STAGE_BYTES);
+          mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
           const int ka = g.a_kwrap > 0 ? kb % g.a_kwrap : kb;
           tma_load_2d(s.a[stage], &tmA, ka * BK, t.row0, &s.full[stage]);
           tma_load_2d(s.b[stage], &tmB, kb * BK, brow0, &s.full[stage]);
-          if (BN_ == 256) tma_load_2d(s.b[stage] + C::B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
-          if (++stage == C::STAGES) {
+          tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -293,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c1 = min(c0 + cl, t.kb1);
           if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN_);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
           for (int kb = c0; kb < c1; ++kb) {
             if (!mbar_wait(&s.full[stage], phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
@@ -302,25 +333,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
               umma_bf16(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
-                        C::IDESC, (kb > c0 || k > 0) ? 1u : 0u);
+                        kIdesc, (kb > c0 || k > 0) ? 1u : 0u);
             umma_commit(&s.empty[stage]);
-            if (++stage == C::STAGES) {
+            if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
             }
           }
           if (!ok) break;
           umma_commit(&s.tfull[acc]);
-          if (++acc == C::NACC) {
-            acc = 0;
-            acc_phase ^= 1u;
-          }
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
         }
       }
     }
   } else {
-    // ---- epilogue (warps 2..5: TMEM lane quarter = warp % 4) -----------------------------
+    // ---- epilogue (warps 2..9): TMEM lane quarter = warp % 4, column half = (warp-2) / 4
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row_in_tile = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -329,8 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile t = decode_tile(s, g, tile);
       const int row = t.row0 + row_in_tile;
       const int cl = chunk_len(g, t);
-      float sum[BN_ == 128 ? 128 : 1];
-      if constexpr (BN_ == 128) {
+      constexpr bool logits = LOGITS;
+      float sum[LOGITS ? 128 : 1];   // router logits: running fp32 sum of this half-row
+      if constexpr (LOGITS) {
 #pragma unroll
         for (int i = 0; i < 128; ++i) sum[i] = 0.f;
       }
@@ -342,43 +373,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!w_ok) { ok = false; break; }
         tc_fence_after();
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(acc * BN_);
-        if constexpr (BN_ == 128) {
-          // router logits: add this chunk to the fp32 running sum (round to nearest)
+                               static_cast<uint32_t>(acc * BN);
+        if constexpr (LOGITS) {
+          // add this chunk to the running sum (fp32, round to nearest)
 #pragma unroll
           for (int c = 0; c < 128; c += 32) {
             uint32_t v[32];
-            tmem_ld_32x32b_x32(tbase + c, v);
+            tmem_ld_32x32b_x32(tbase + 128 * half + c, v);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) sum[c + i] = __fadd_rn(sum[c + i], __uint_as_float(v[i]));
           }
         } else {
-          epilogue_expert(g, t, tbase, row);
+          epilogue_expert(g, t, tbase, row, half);
         }
         tc_fence_before();
         mbar_arrive(&s.tempty[acc]);
-        if (++acc == C::NACC) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
       }
-      if constexpr (BN_ == 128) {
-        if (ok && row < t.row_end) {
-          const int col0 = t.nt * 128;
-          float* dst = static_cast<float*>(g.out) + t.split * g.split_stride +
-                       (size_t)row * g.ld_out + col0;
-          if (col0 + 128 <= g.n_valid && (g.ld_out & 3) == 0) {
+      if constexpr (LOGITS) {
+       if (ok && row < t.row_end) {
+        const int col0 = t.nt * BN + 128 * half;
+        float* dst = static_cast<float*>(g.out) + t.split * g.split_stride +
+                     (size_t)row * g.ld_out + col0;
+        if (col0 + 128 <= g.n_valid && (g.ld_out & 3) == 0) {
 #pragma unroll
-            for (int v = 0; v < 32; ++v)
-              reinterpret_cast<float4*>(dst)[v] =
-                  make_float4(sum[4 * v], sum[4 * v + 1], sum[4 * v + 2], sum[4 * v + 3]);
-          } else {
+          for (int v = 0; v < 32; ++v)
+            reinterpret_cast<float4*>(dst)[v] =
+                make_float4(sum[4 * v], sum[4 * v + 1], sum[4 * v + 2], sum[4 * v + 3]);
+        } else {
 #pragma unroll
-            for (int v = 0; v < 128; ++v)
-              if (col0 + v < g.n_valid) dst[v] = sum[v];
-          }
+          for (int v = 0; v < 128; ++v)
+            if (col0 + v < g.n_valid) dst[v] = sum[v];
         }
+       }
       }
     }
   }
@@ -414,11 +443,13 @@ int get_encoder() {
   return g_encode ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// rows x cols bf16 matrix, row-major; box = 64 columns x 128 rows, 128-byte swizzle.
-int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+// rows x cols bf16 matrix, row-major; box = 64 columns x box_rows rows (128 for tiled
+// loads, 1 for four-row gathers), 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+             uint32_t box_rows = BM) {
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t box[2] = {BK, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -427,15 +458,15 @@ int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-template <int BN_>
 int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int sm_count,
                cudaStream_t st) {
-  constexpr size_t smem = sizeof(SharedStorage<BN_>) + 1024;
+  constexpr size_t smem = sizeof(SharedStorage) + 1024;
   static_assert(smem <= 227 * 1024, "shared memory budget");
-  if (cudaFuncSetAttribute(k_grouped_gemm_tc<BN_>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  auto kern = g.mode == kLogits ? k_grouped_gemm_tc<true> : k_grouped_gemm_tc<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
-  k_grouped_gemm_tc<BN_><<<sm_count, kThreads, smem, st>>>(ma, mb, g);
+  kern<<<sm_count, kThreads, smem, st>>>(ma, mb, g);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -473,16 +504,16 @@ __global__ void __launch_bounds__(256) k_split_router_weight(const float4* __res
 
 }  // namespace
 
-// Router logits: 128 x 128 tiles, K = 3H (the three weight parts); the tensor cores
+// Router logits: 128 x 256 tiles, K = 3H (the three weight parts); the tensor cores
 // accumulate kRouterChunk k-blocks at a time and the epilogue sums the chunks in fp32.
 constexpr int kRouterChunk = 6;
 constexpr int kRouterMinSplit = 12;   // k-blocks per split at least (two chunks)
 
 int router_tc_splitk(int T, int E, int H, int sm_count) {
   if (sm_count > 160) sm_count = 160;
-  const long tiles = (long)((T + BM - 1) / BM) * ((E + 127) / 128);
+  const long tiles = (long)((T + BM - 1) / BM) * ((E + BN - 1) / BN);
   const int kblocks = 3 * H / BK;
-  if (tiles <= 0) return 1;
+  if (tiles <= 0 || tiles >= sm_count) return 1;   // a full wave already: no partial slices
   long s = (2L * sm_count + tiles - 1) / tiles;
   long smax = kblocks / kRouterMinSplit;
   if (smax > 64) smax = 64;
@@ -501,7 +532,8 @@ size_t router_tc_scratch_bytes(int T, int E, int H) {
 }
 
 int launch_router_logits_tc(const void* x, const float* w_router, int T, int E, int H,
-                            float* logits, void* scratch, int sm_count, cudaStream_t st) {
+                            float* logits, void* scratch, int sm_count, cudaStream_t st,
+                            const float** src_out, int* splits_out) {
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(scratch);
   size_t off = ((size_t)E * 3 * H * 2 + 1023) / 1024 * 1024;
@@ -528,21 +560,22 @@ int launch_router_logits_tc(const void* x, const float* w_router, int T, int E, 
   g.ksplit = S;
   g.kb_per_split = (g.kblocks + S - 1) / S;
   g.kchunk = kRouterChunk;
-  g.n_tiles = (E + 127) / 128;
+  g.n_tiles = (E + BN - 1) / BN;
   g.b_rows = 0;
-  g.b_second = 0;
+  g.b_second = BM;
   g.n_valid = E;
   g.ld_out = E;
   g.out = S > 1 ? static_cast<void*>(partial) : static_cast<void*>(logits);
   g.split_stride = (long long)T * E;
-  if ((rc = launch_one<128>(mx, mw, g, sm_count, st)) != MOE_OK) return rc;
-  if (S > 1) {
-    if (launch_splitk_sum(partial, S, (size_t)T * E, logits, st) != cudaSuccess) return MOE_ERR_CUDA;
-  }
+  if ((rc = launch_one(mx, mw, g, sm_count, st)) != MOE_OK) return rc;
+  // with S > 1 the top-K kernel sums the partial slices in split order
+  *src_out = S > 1 ? partial : logits;
+  *splits_out = S;
   return MOE_OK;
 }
 
-int launch_grouped_ffn_tc(const void* x_perm, const int32_t* offsets, const void* w_gate_up,
+int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offsets,
+                          const void* w_gate_up,
                           const void* w_down, const int32_t* perm_token, const float* row_gate,
                           void* h, void* y_perm, float* out_acc, int T, int H, int I, int n_ffn,
                           int K, float scale, int fused, int* status, int sm_count,
@@ -551,7 +584,12 @@ int launch_grouped_ffn_tc(const void* x_perm, const int32_t* offsets, const void
   const uint64_t rows = (uint64_t)T * K + BM;   // x_perm / h / y_perm allocation rows
   CUtensorMap mx, mwgu, mh, mwd;
   int rc;
-  if ((rc = make_map(&mx, x_perm, rows, H)) != MOE_OK) return rc;
+  // A of the gate/up GEMM: the permuted rows, or the token rows gathered through perm_token
+  if (x_perm) {
+    if ((rc = make_map(&mx, x_perm, rows, H)) != MOE_OK) return rc;
+  } else {
+    if ((rc = make_map(&mx, x, (uint64_t)T, H, 1)) != MOE_OK) return rc;
+  }
   if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H)) != MOE_OK) return rc;
   if ((rc = make_map(&mh, h, rows, I)) != MOE_OK) return rc;
   if ((rc = make_map(&mwd, w_down, (uint64_t)n_ffn * H, I)) != MOE_OK) return rc;
@@ -566,11 +604,12 @@ int launch_grouped_ffn_tc(const void* x_perm, const int32_t* offsets, const void
   g1.n_valid = I;
   g1.ld_out = I;
   g1.offsets = offsets;
+  g1.gather_tok = x_perm ? nullptr : perm_token;
   g1.out = h;
   g1.status = status;
   g1.ksplit = 1;
   g1.kb_per_split = g1.kblocks;
-  if ((rc = launch_one<256>(mx, mwgu, g1, sm_count, st)) != MOE_OK) return rc;
+  if ((rc = launch_one(mx, mwgu, g1, sm_count, st)) != MOE_OK) return rc;
 
   GemmArgs g2{};
   g2.mode = fused ? kDownAtomic : kDownStore;
@@ -589,7 +628,7 @@ int launch_grouped_ffn_tc(const void* x_perm, const int32_t* offsets, const void
   g2.status = status;
   g2.ksplit = 1;
   g2.kb_per_split = g2.kblocks;
-  return launch_one<256>(mh, mwd, g2, sm_count, st);
+  return launch_one(mh, mwd, g2, sm_count, st);
 }
 
 }  // namespace moe

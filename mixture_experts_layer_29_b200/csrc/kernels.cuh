@@ -31,11 +31,17 @@ cudaError_t launch_splitk_sum(const float* partial, int S, size_t n, float* out,
 // bf16 x: logits on the tensor cores with W_r split into three exact bf16 parts.
 int router_tc_splitk(int T, int E, int H, int sm_count);
 size_t router_tc_scratch_bytes(int T, int E, int H);
+// Writes the logits (S == 1) or S partial slices; *src_out / *splits_out tell the top-K
+// kernel where to read them.
 int launch_router_logits_tc(const void* x, const float* w_router, int T, int E, int H,
-                            float* logits, void* scratch, int sm_count, cudaStream_t st);
-cudaError_t launch_route_topk(const float* logits, const float* bias, int T, int E, int n_ffn,
-                              int K, int32_t* topk_idx, float* topk_gate, int32_t* counts,
-                              int32_t* nffn_hist, float* zgate, int sm_count, cudaStream_t st);
+                            float* logits, void* scratch, int sm_count, cudaStream_t st,
+                            const float** src_out, int* splits_out);
+// Softmax / top-K / histograms from S logit slices of T x E (summed in order; S > 1 also
+// writes the sum to logits_out).
+cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const float* bias,
+                              int T, int E, int n_ffn, int K, int32_t* topk_idx,
+                              float* topk_gate, int32_t* counts, int32_t* nffn_hist,
+                              float* zgate, int sm_count, cudaStream_t st);
 
 // ---- permutation ------------------------------------------------------------------------
 cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, const float* zgate,
@@ -46,7 +52,9 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, cons
 
 // ---- grouped FFN --------------------------------------------------------------------------
 // bf16 on tcgen05: gate/up GEMM + SwiGLU -> h, then down GEMM -> y_perm or out_acc.
-int launch_grouped_ffn_tc(const void* x_perm, const int32_t* offsets, const void* w_gate_up,
+// x_perm == nullptr: the gate/up GEMM gathers the rows of x through perm_token (TMA gather4).
+int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offsets,
+                          const void* w_gate_up,
                           const void* w_down, const int32_t* perm_token, const float* row_gate,
                           void* h, void* y_perm, float* out_acc, int T, int H, int I, int n_ffn,
                           int K, float scale, int fused, int* status, int sm_count,

@@ -148,12 +148,15 @@ __global__ void __launch_bounds__(256) k_perm_scatter(
   constexpr int esz = XBF16 ? 2 : 4;
   const int nvec = H * esz / 16;
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + (size_t)t * H * esz);
+  if (!x_perm && !out_acc) return;
   for (int v = lane; v < nvec; v += 32) {
     const uint4 q = __ldg(src + v);
-    for (int k = 0; k < K; ++k) {
-      const int r = s_rows[warp][k];
-      if (r >= 0)
-        reinterpret_cast<uint4*>(static_cast<char*>(x_perm) + (size_t)r * H * esz)[v] = q;
+    if (x_perm) {
+      for (int k = 0; k < K; ++k) {
+        const int r = s_rows[warp][k];
+        if (r >= 0)
+          reinterpret_cast<uint4*>(static_cast<char*>(x_perm) + (size_t)r * H * esz)[v] = q;
+      }
     }
     if (out_acc) {
       float* o = out_acc + (size_t)t * H + (size_t)v * (16 / esz);

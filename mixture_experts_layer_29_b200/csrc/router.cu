@@ -174,7 +174,11 @@ int router_splitk(int T, int E, int H, int sm_count) {
   const long smax = H / 64 > 0 ? H / 64 : 1;     // at least 64 of H per split
   if (s > smax) s = smax;
   if (s > 32) s = 32;
-  return s < 1 ? 1 : (int)s;
+  if (s < 1) s = 1;
+  // the effective split count: slices of a multiple of RK, none empty
+  int kchunk = (H + (int)s - 1) / (int)s;
+  kchunk = (kchunk + RK - 1) / RK * RK;
+  return (H + kchunk - 1) / kchunk;
 }
 
 size_t router_partial_bytes(int T, int E, int H, int sm_count_max) {
@@ -196,30 +200,39 @@ cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_ro
   else
     k_router_logits<false><<<grid, 256, 0, st>>>(x, w_router, T, E, H, kchunk, dst, stride);
   count_launch();
-  if (S > 1) {
-    const size_t n = (size_t)T * E;
-    const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-    k_router_splitk_sum<<<blocks, 256, 0, st>>>(partial, S, n, logits);
-    count_launch();
-  }
+  // with S > 1 the partials are summed (in split order) by the top-K kernel
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------------------
 // Softmax + bias-adjusted top-K, one warp per token.
-// Lane l holds experts l, l + 32, ... (J groups). p is computed in double and rounded once
-// to fp32; the selection score is the fp32 sum p + b (a zero result stored as +0). K
-// rounds of a warp-wide argmax pick (score descending, expert index ascending). The
-// counts and the FFN-pick histogram go through shared memory, then integer atomics.
+// Lane l holds experts l, l + 32, ... (J groups). The logits are read from S split-K
+// slices summed in slice order (S = 1: the logits themselves; S > 1: the sum is also
+// written out). exp(L - max) is evaluated in fp32 on the exactly split argument
+// (hi + lo, exp(hi) * (1 + lo)), summed in double, and normalised with a double
+// reciprocal, so p is within a few fp32 ulps of the float64 softmax. The selection score
+// is the fp32 sum p + b (a zero result stored as +0); K rounds of a warp-wide argmax pick
+// (score descending, expert index ascending). Counts and the FFN-pick histogram go
+// through shared memory, then integer atomics.
 // ---------------------------------------------------------------------------------------
 namespace {
 constexpr int kRouteWarps = 8;
 
+// exp(d) for d = L - max given exactly in double, evaluated as exp(hi) * (1 + lo)
+__device__ __forceinline__ float exp_split(float L, double dm) {
+  const double d = (double)L - dm;
+  const float dh = (float)d;
+  const float dl = (float)(d - (double)dh);
+  const float v = expf(dh);
+  return fmaf(v, dl, v);
+}
+
 template <int J>
 __global__ void __launch_bounds__(kRouteWarps * 32) k_route_topk(
-    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int n_ffn,
-    int K, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
-    int32_t* __restrict__ counts, int32_t* __restrict__ nffn_hist, float* __restrict__ zgate) {
+    const float* __restrict__ src, int S, size_t slice, float* __restrict__ logits_out,
+    const float* __restrict__ bias, int T, int E, int n_ffn, int K,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ counts,
+    int32_t* __restrict__ nffn_hist, float* __restrict__ zgate) {
   __shared__ int s_counts[1024];
   __shared__ int s_hist[33];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -235,35 +248,43 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route_topk(
   }
 
   for (int t = blockIdx.x * kRouteWarps + warp; t < T; t += gridDim.x * kRouteWarps) {
-    const float* Lr = logits + (size_t)t * E;
+    const float* Lr = src + (size_t)t * E;
     float lv[J];
     float m = -INFINITY;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
       const int e = lane + 32 * j;
-      lv[j] = e < E ? Lr[e] : -INFINITY;
-      m = fmaxf(m, lv[j]);
+      float v = -INFINITY;
+      if (e < E) {
+        v = Lr[e];
+        for (int sp = 1; sp < S; ++sp) v += Lr[sp * slice + e];
+        if (S > 1) logits_out[(size_t)t * E + e] = v;
+      }
+      lv[j] = v;
+      m = fmaxf(m, v);
     }
     m = warp_max(m);
-    double ex[J];
+    const double dm = (double)m;
     double sum = 0.0;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
       const int e = lane + 32 * j;
-      ex[j] = e < E ? exp((double)lv[j] - (double)m) : 0.0;
-      sum += ex[j];
+      const float v = e < E ? exp_split(lv[j], dm) : 0.f;
+      lv[j] = v;                                       // lv now holds exp(L - max)
+      sum += (double)v;
     }
     sum = warp_sum(sum);
-    float p[J], s[J];
+    const double inv = 1.0 / sum;
+    float p[J], sc[J];
 #pragma unroll
     for (int j = 0; j < J; ++j) {
       const int e = lane + 32 * j;
-      p[j] = (float)(ex[j] / sum);
+      p[j] = (float)((double)lv[j] * inv);
       float v = __fadd_rn(p[j], bia[j]);
-      if (v == 0.0f) v = 0.0f;          // -0 -> +0
-      s[j] = e < E ? v : -INFINITY;
+      if (v == 0.0f) v = 0.0f;                          // -0 -> +0
+      sc[j] = e < E ? v : -INFINITY;
     }
-
+    // K rounds of a warp argmax on (score descending, expert index ascending)
     uint32_t taken = 0u;
     int my_e = 0;
     float my_g = 0.f;
@@ -273,8 +294,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route_topk(
 #pragma unroll
       for (int j = 0; j < J; ++j) {
         const int e = lane + 32 * j;
-        if (e < E && !((taken >> j) & 1u) && (s[j] > bs || be == 0x7fffffff)) {
-          bs = s[j];
+        if (e < E && !((taken >> j) & 1u) && (sc[j] > bs || be == 0x7fffffff)) {
+          bs = sc[j];
           be = e;
         }
       }
@@ -323,29 +344,31 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route_topk(
 }
 
 template <int J>
-void launch_topk_j(dim3 grid, cudaStream_t st, const float* logits, const float* bias, int T,
-                   int E, int n_ffn, int K, int32_t* idx, float* gate, int32_t* counts,
-                   int32_t* hist, float* zgate) {
-  k_route_topk<J><<<grid, kRouteWarps * 32, 0, st>>>(logits, bias, T, E, n_ffn, K, idx, gate,
-                                                     counts, hist, zgate);
+void launch_topk_j(dim3 grid, cudaStream_t st, const float* src, int S, size_t slice,
+                   float* logits_out, const float* bias, int T, int E, int n_ffn, int K,
+                   int32_t* idx, float* gate, int32_t* counts, int32_t* hist, float* zgate) {
+  k_route_topk<J><<<grid, kRouteWarps * 32, 0, st>>>(src, S, slice, logits_out, bias, T, E,
+                                                     n_ffn, K, idx, gate, counts, hist, zgate);
 }
 }  // namespace
 
-cudaError_t launch_route_topk(const float* logits, const float* bias, int T, int E, int n_ffn,
-                              int K, int32_t* topk_idx, float* topk_gate, int32_t* counts,
-                              int32_t* nffn_hist, float* zgate, int sm_count, cudaStream_t st) {
+cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const float* bias,
+                              int T, int E, int n_ffn, int K, int32_t* topk_idx,
+                              float* topk_gate, int32_t* counts, int32_t* nffn_hist,
+                              float* zgate, int sm_count, cudaStream_t st) {
   cudaError_t err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st);
   if (err != cudaSuccess) return err;
   err = cudaMemsetAsync(nffn_hist, 0, sizeof(int32_t) * (K + 1), st);
   if (err != cudaSuccess) return err;
   int blocks = (T + kRouteWarps - 1) / kRouteWarps;
-  if (blocks > 4 * sm_count) blocks = 4 * sm_count;
+  if (blocks > 8 * sm_count) blocks = 8 * sm_count;
   dim3 grid(blocks);
   const int J = (E + 31) / 32;
+  const size_t slice = (size_t)T * E;
 #define MOE_TOPK_CASE(JJ)                                                                      \
   if (J <= JJ) {                                                                               \
-    launch_topk_j<JJ>(grid, st, logits, bias, T, E, n_ffn, K, topk_idx, topk_gate, counts,     \
-                      nffn_hist, zgate);                                                       \
+    launch_topk_j<JJ>(grid, st, src, S, slice, logits_out, bias, T, E, n_ffn, K, topk_idx,     \
+                      topk_gate, counts, nffn_hist, zgate);                                    \
   } else
   MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4) MOE_TOPK_CASE(6)
   MOE_TOPK_CASE(8) MOE_TOPK_CASE(12) MOE_TOPK_CASE(16) MOE_TOPK_CASE(24) MOE_TOPK_CASE(32) {

@@ -88,7 +88,7 @@ def test_host_checks_run_before_any_device_access(L):
     assert L.moe_route(ctypes.byref(s), *args, ws_n - 1, None) == -5
     # permute / grouped_ffn / forward with a workspace that is too small
     assert L.moe_permute(ctypes.byref(s), *([good] * 11), 16, None) == -5
-    assert L.moe_grouped_ffn(ctypes.byref(s), *([good] * 10), 16, None) == -5
+    assert L.moe_grouped_ffn(ctypes.byref(s), *([good] * 11), 16, None) == -5
     assert L.moe_forward(ctypes.byref(s), *([good] * 12), abi.workspace_size(s) - 1, None) == -5
     # combine: fused mode needs out_acc
     assert L.moe_combine(ctypes.byref(s), good, None, None, None, None, None, good, None) == -1
@@ -107,7 +107,7 @@ def test_empty_batch_is_a_no_op(L):
     ws_n = abi.scratch_size(s)
     assert L.moe_route(ctypes.byref(s), *([p] * 11), ws_n, None) == 0
     assert L.moe_permute(ctypes.byref(s), *([p] * 11), ws_n, None) == 0
-    assert L.moe_grouped_ffn(ctypes.byref(s), *([p] * 10), ws_n, None) == 0
+    assert L.moe_grouped_ffn(ctypes.byref(s), *([p] * 11), ws_n, None) == 0
     assert L.moe_combine(ctypes.byref(s), *([p] * 7), None) == 0
     assert L.moe_forward(ctypes.byref(s), *([p] * 12), abi.workspace_size(s), None) == 0
 

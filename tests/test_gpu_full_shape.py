@@ -70,9 +70,9 @@ def test_full_shape_ffn_part_alone(full_case):
     b = case.buffers("fused")
     case.route(b)
     abi.permute(b.shape, b.topk_idx, b.topk_gate, b.zgate, case.x, b.offsets, b.perm_token,
-                b.row_of, b.row_gate, b.x_perm, None, b.ws)
+                b.row_of, b.row_gate, None, None, b.ws)
     b.out_acc.zero_()
-    abi.grouped_ffn(b.shape, b.x_perm, b.offsets, case.w.w_gate_up, case.w.w_down,
+    abi.grouped_ffn(b.shape, case.x, None, b.offsets, case.w.w_gate_up, case.w.w_down,
                     b.perm_token, b.row_gate, b.h, None, b.out_acc, b.ws)
     torch.cuda.synchronize()
     toks = _sample(cfg, 8)
