@@ -28,6 +28,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -427,6 +428,206 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---- CTA-pair variant of the expert GEMMs (tcgen05 cta_group::2) -------------------------
+// A cluster of two CTAs computes a 256 x 256 tile: CTA r loads rows [128r, 128r+128) of the
+// A tile and B rows [128r, 128r+128) of the N tile (gate/up: CTA 0 the gate rows, CTA 1
+// the up rows), so each CTA moves 32 KB per k-block instead of 48 KB. Both CTAs' TMA loads
+// count on the leader's (rank 0) full barrier; the leader's single thread issues
+// tcgen05.mma.cta_group::2 (M = 256) and commits to the empty / accumulator-full barriers
+// of both CTAs (two commits, one per CTA); both CTAs' epilogues read their own TMEM rows
+// and release the accumulator on the leader's barrier.
+constexpr int BMP = 256;                             // M rows per CTA pair
+constexpr int PSTAGES = 6;                           // 32 KB per stage per CTA
+constexpr int P_B_BYTES = 128 * BK * 2;              // 16 KB: this CTA's half of B
+constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES;   // 32 KB
+constexpr uint32_t kIdescPair = idesc_bf16_f32(BMP, BN);
+
+struct alignas(1024) PairStorage {
+  uint8_t a[PSTAGES][A_BYTES];
+  uint8_t b[PSTAGES][P_B_BYTES];
+  uint64_t full[PSTAGES];       // leader: both CTAs' bytes; peer: unused
+  uint64_t empty[PSTAGES];      // both: the leader's MMA commit
+  uint64_t tfull[2];            // both: the leader's MMA commit
+  uint64_t tempty[2];           // leader: one arrival per epilogue warp of both CTAs
+  uint32_t tmem_base;
+  int abort_flag;
+  int offs[kMaxExperts + 1];
+  int toff[kMaxExperts + 1];    // prefix of ceil(count / 256)
+};
+
+__device__ __forceinline__ Tile decode_pair_tile(const PairStorage& s, const GemmArgs& g, int tile) {
+  Tile t;
+  t.split = 0;
+  t.kb0 = 0;
+  t.kb1 = g.kblocks;
+  const int mt = tile / g.n_tiles;
+  t.nt = tile - mt * g.n_tiles;
+  int lo = 0, hi = g.n_ffn - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.toff[mid] <= mt) lo = mid; else hi = mid - 1;
+  }
+  t.e = lo;
+  t.row0 = s.offs[lo] + (mt - s.toff[lo]) * BMP;
+  t.row_end = s.offs[lo + 1];
+  return t;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  PairStorage& s = *reinterpret_cast<PairStorage*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();            // 0: leader, 1: peer
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+  // ---- set-up -------------------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < PSTAGES; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 2 * kEpiWarps);
+    }
+    s.abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  for (int i = threadIdx.x; i <= g.n_ffn; i += kThreads) s.offs[i] = g.offsets[i];
+  __syncthreads();
+  cluster_sync();                                     // both CTAs' barriers initialised
+  if (warp == 1) {
+    tmem_alloc_pair(&s.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == 2) {
+    const int per = (g.n_ffn + 31) / 32;
+    const int b = lane * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i)
+      if (b + i < g.n_ffn) local += (s.offs[b + i + 1] - s.offs[b + i] + BMP - 1) / BMP;
+    const int inc = warp_inclusive_scan(local);
+    int run = inc - local;
+    for (int i = 0; i < per; ++i)
+      if (b + i < g.n_ffn) {
+        s.toff[b + i] = run;
+        run += (s.offs[b + i + 1] - s.offs[b + i] + BMP - 1) / BMP;
+      }
+    if (lane == 31) s.toff[g.n_ffn] = inc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s.tmem_base;
+  const int total_tiles = s.toff[g.n_ffn] * g.n_tiles;
+  volatile int* abort_flag = &s.abort_flag;
+
+  if (warp == 0) {
+    // ---- TMA producer (both CTAs): this CTA's A rows and B half, counted on the leader --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = cluster; tile < total_tiles && !*abort_flag; tile += nclusters) {
+        const Tile t = decode_pair_tile(s, g, tile);
+        const int arow = t.row0 + 128 * (int)rank;
+        const int brow = g.mode == kGateUp
+                             ? t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM
+                             : t.e * g.b_rows + t.nt * BN + 128 * (int)rank;
+        for (int kb = 0; kb < g.kblocks; ++kb) {
+          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
+          const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * P_STAGE_BYTES);
+          tma_load_2d_pair(s.a[stage], &tmA, kb * BK, arow, full_leader);
+          tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
+          if (++stage == PSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer (leader only) ---------------------------------------------------------
+    if (rank == 0 && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
+        if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < g.kblocks; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(s.a[stage]);
+          const uint32_t b0 = smem_u32(s.b[stage]);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
+                           kIdescPair, (kb > 0 || k > 0) ? 1u : 0u);
+          const uint32_t e_local = smem_u32(&s.empty[stage]);
+          umma_commit_pair(mapa_shared(e_local, 0));
+          umma_commit_pair(mapa_shared(e_local, 1));
+          if (++stage == PSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        const uint32_t f_local = smem_u32(&s.tfull[acc]);
+        umma_commit_pair(mapa_shared(f_local, 0));
+        umma_commit_pair(mapa_shared(f_local, 1));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ---- epilogue (both CTAs, warps 2..9): this CTA's 128 rows of the 256-row tile ------
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row_in_tile = 128 * (int)rank + q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster; tile < total_tiles; tile += nclusters) {
+      const Tile t = decode_pair_tile(s, g, tile);
+      int w_ok = 1;
+      if (lane == 0) w_ok = mbar_wait(&s.tfull[acc], acc_phase, abort_flag) ? 1 : 0;
+      w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+      if (!w_ok) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      epilogue_expert(g, t, tbase, t.row0 + row_in_tile, half);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  // ---- tear-down ------------------------------------------------------------------------
+  if (*abort_flag) {
+    set_status(g.status, MOE_ERR_TIMEOUT);
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();            // neither CTA leaves while the other may still signal it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // ---- host side ------------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -469,6 +670,63 @@ int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, 
   kern<<<sm_count, kThreads, smem, st>>>(ma, mb, g);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Cluster-of-two launch of the CTA-pair kernel: as many clusters as fit at once (cached
+// per device), so the persistent tile loop never waits for a cluster slot.
+int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int sm_count,
+                cudaStream_t st) {
+  constexpr size_t smem = sizeof(PairStorage) + 1024;
+  static_assert(smem <= 227 * 1024, "shared memory budget");
+  static std::mutex mu;
+  static int clusters_of[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return MOE_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_grouped_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int nclusters;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (clusters_of[dev] == 0) {
+      cfg.gridDim = dim3(sm_count & ~1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k_grouped_gemm_pair, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      clusters_of[dev] = n;
+    }
+    nclusters = clusters_of[dev];
+  }
+  if (nclusters > sm_count / 2) nclusters = sm_count / 2;
+  cfg.gridDim = dim3(2 * nclusters);
+  if (cudaLaunchKernelEx(&cfg, k_grouped_gemm_pair, ma, mb, g) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  count_launch();
+  return MOE_OK;
+}
+
+// The CTA-pair kernel pays off once groups are tall (256-row tiles); small batches keep
+// the one-CTA kernel. MOE_B200_GEMM_PAIR=0 / 1 forces either (for measurements).
+bool use_pair_kernel(int T) {
+  static const char* env = getenv("MOE_B200_GEMM_PAIR");
+  if (env && env[0] == '0') return false;
+  if (env && env[0] == '1') return true;
+  return T >= 1024;
 }
 
 // W_r fp32 [E, H] -> bf16 [E, 3H] = [hi | mid | lo] with hi + mid + lo == w exactly:
@@ -609,7 +867,10 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g1.status = status;
   g1.ksplit = 1;
   g1.kb_per_split = g1.kblocks;
-  if ((rc = launch_one(mx, mwgu, g1, sm_count, st)) != MOE_OK) return rc;
+  const bool pair = use_pair_kernel(T) && !g1.gather_tok;
+  if ((rc = pair ? launch_pair(mx, mwgu, g1, sm_count, st) : launch_one(mx, mwgu, g1, sm_count, st)) !=
+      MOE_OK)
+    return rc;
 
   GemmArgs g2{};
   g2.mode = fused ? kDownAtomic : kDownStore;
@@ -628,7 +889,7 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g2.status = status;
   g2.ksplit = 1;
   g2.kb_per_split = g2.kblocks;
-  return launch_one(mh, mwd, g2, sm_count, st);
+  return pair ? launch_pair(mh, mwd, g2, sm_count, st) : launch_one(mh, mwd, g2, sm_count, st);
 }
 
 }  // namespace moe

@@ -150,8 +150,9 @@ def test_forward_entry_point_matches_steps(cuda_device):
 
 # ------------------------------------------------------------------------- edge cases
 
-@pytest.mark.parametrize("T", [1, 31, 33, 129, 1000])
+@pytest.mark.parametrize("T", [1, 31, 33, 129, 1000, 1025, 3001])
 def test_ragged_token_counts(cuda_device, T):
+    # T >= 1024 runs the expert GEMMs on CTA pairs (256-row tiles), smaller T on single CTAs
     cfg = wl.CONFIGS["proxy_bf16"].with_(T=T)
     case = gh.Case(cfg, seed=3)
     _ffn_checks(case, "fused")
