@@ -5,7 +5,8 @@
     python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...
 
 One step = one pass of the whole hot path over one batch: router logits + softmax/top-K
-+ histogram (moe_route), permutation (moe_permute), grouped SwiGLU FFN on the tensor
++ histogram (moe_route_packed, with the router weight packed once at set-up), permutation
+(moe_permute), grouped SwiGLU FFN on the tensor
 cores with the fused combine epilogue (moe_grouped_ffn), finalize (moe_combine) and the
 PID bias update (moe_pid_bias_update, written to a second bias buffer so every step
 routes the same batch). Workload: the full-shape prefill layer (hidden 6144, 512 SwiGLU
@@ -171,6 +172,12 @@ class Stepper:
         self.cfg, self.w, self.x, self.logits_in = cfg, w, x, logits_in
         self.shape = abi.shape_of(cfg, combine)
         self.b = abi.StepBuffers.allocate(self.shape, device)
+        # the router weight in the tensor cores' three-part bf16 form, packed once like any
+        # weight layout (model-load time), not per step
+        self.w_packed = None
+        if self.shape.dtype == abi.MOE_BF16 and logits_in is None:
+            self.w_packed = torch.empty(cfg.E, 3 * cfg.H, dtype=torch.bfloat16, device=device)
+            abi.router_pack(self.shape, w.w_router, self.w_packed)
         self.bias_next = w.bias.clone()
         self.pid = abi.Pid(*PID_GAINS)
         self.state = torch.empty(3 * cfg.n_ffn, dtype=torch.float32, device=device)
@@ -184,9 +191,13 @@ class Stepper:
             if ev is not None:
                 ev[i].record()
         mark(0)
-        abi.route(s, self.x, w.w_router, self.logits_in, w.bias,
-                  None if self.logits_in is not None else b.logits, b.topk_idx, b.topk_gate,
-                  b.counts, b.nffn_hist, b.zgate, b.ws)
+        if self.w_packed is not None:
+            abi.route_packed(s, self.x, self.w_packed, w.bias, b.logits, b.topk_idx,
+                             b.topk_gate, b.counts, b.nffn_hist, b.zgate, b.ws)
+        else:
+            abi.route(s, self.x, w.w_router, self.logits_in, w.bias,
+                      None if self.logits_in is not None else b.logits, b.topk_idx,
+                      b.topk_gate, b.counts, b.nffn_hist, b.zgate, b.ws)
         mark(1)
         xp = b.x_perm
         abi.permute(s, b.topk_idx, b.topk_gate, b.zgate, self.x, b.offsets, b.perm_token,

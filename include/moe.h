@@ -125,6 +125,23 @@ int moe_route(const moe_shape_t* shape, const void* x, const float* w_router,
               int32_t* topk_idx, float* topk_gate, int32_t* counts, int32_t* nffn_hist,
               float* zgate, void* ws, size_t ws_bytes, void* stream);
 
+/* The router weight in the tensor cores' format, once, at load time (bf16 layers):
+ * w_packed = [hi | mid | lo] per expert row, three bf16 parts with hi + mid + lo == w
+ * exactly (hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid)). moe_route splits
+ * w_router like this on every call; moe_route_packed takes the packed weight instead.
+ *   w_router   device [E, H] fp32
+ *   w_packed   device [E, 3H] bf16, written
+ * MOE_ERR_UNSUPPORTED for fp32 layers (their router runs on the CUDA cores). */
+int moe_router_pack(const moe_shape_t* shape, const float* w_router, void* w_packed,
+                    void* stream);
+
+/* moe_route with the router weight from moe_router_pack (bf16 layers; the logits are
+ * computed, there is no logits_in). Same outputs, bit for bit. */
+int moe_route_packed(const moe_shape_t* shape, const void* x, const void* w_packed,
+                     const float* bias, float* logits_out, int32_t* topk_idx, float* topk_gate,
+                     int32_t* counts, int32_t* nffn_hist, float* zgate, void* ws, size_t ws_bytes,
+                     void* stream);
+
 /* Permutation of the FFN picks into expert-contiguous groups. Group e holds, in ascending
  * token order, the rows of the tokens that picked e; groups follow in expert order.
  *   topk_idx   device [T, K] int32            from moe_route

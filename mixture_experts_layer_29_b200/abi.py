@@ -80,6 +80,8 @@ _SIGS = {
                             + [_P] * 6),
     "moe_forward": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 12 + [_SZ, _P]),
     "moe_permute_static_scratch": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 10 + [_P]),
+    "moe_router_pack": (ctypes.c_int, [ctypes.POINTER(Shape), _P, _P, _P]),
+    "moe_route_packed": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 10 + [_SZ, _P]),
 }
 
 _lib = None
@@ -175,6 +177,20 @@ def route(shape, x, w_router, logits_in, bias, logits_out, topk_idx, topk_gate, 
                            ptr(logits_out), ptr(topk_idx), ptr(topk_gate), ptr(counts),
                            ptr(nffn_hist), ptr(zgate), ptr(ws), _nbytes(ws), _stream(stream)),
            "moe_route")
+
+
+def router_pack(shape, w_router, w_packed, stream=None):
+    """Pack the fp32 router weight [E, H] into the exact three-part bf16 form [E, 3H]."""
+    _check(lib().moe_router_pack(ctypes.byref(shape), ptr(w_router), ptr(w_packed),
+                                 _stream(stream)), "moe_router_pack")
+
+
+def route_packed(shape, x, w_packed, bias, logits_out, topk_idx, topk_gate, counts, nffn_hist,
+                 zgate, ws, stream=None):
+    _check(lib().moe_route_packed(ctypes.byref(shape), ptr(x), ptr(w_packed), ptr(bias),
+                                  ptr(logits_out), ptr(topk_idx), ptr(topk_gate), ptr(counts),
+                                  ptr(nffn_hist), ptr(zgate), ptr(ws), _nbytes(ws),
+                                  _stream(stream)), "moe_route_packed")
 
 
 def permute(shape, topk_idx, topk_gate, zgate, x, offsets, perm_token, row_of, row_gate, x_perm,

@@ -134,13 +134,14 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
 
-int route_impl(const moe_shape_t* s, const void* x, const float* w_router, const float* logits_in,
-               const float* bias, float* logits_out, int32_t* topk_idx, float* topk_gate,
-               int32_t* counts, int32_t* nffn_hist, float* zgate, void* ws, size_t ws_bytes,
-               void* stream) {
+int route_impl(const moe_shape_t* s, const void* x, const float* w_router, const void* w_packed,
+               const float* logits_in, const float* bias, float* logits_out, int32_t* topk_idx,
+               float* topk_gate, int32_t* counts, int32_t* nffn_hist, float* zgate, void* ws,
+               size_t ws_bytes, void* stream) {
   MOE_TRY(check_shape(s));
   MOE_TRY(check_ptrs({bias, topk_idx, topk_gate, counts, nffn_hist, zgate, ws}));
-  if (!logits_in) MOE_TRY(check_ptrs({x, w_router, logits_out}));
+  if (!logits_in) MOE_TRY(check_ptrs({x, w_packed ? w_packed : w_router, logits_out}));
+  if (w_packed && s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   MOE_TRY(check_opt({logits_in, logits_out, x, w_router}));
   const Layout L = layout_of(*s);
   if (ws_bytes < L.scratch_end) return MOE_ERR_WORKSPACE;
@@ -153,7 +154,7 @@ int route_impl(const moe_shape_t* s, const void* x, const float* w_router, const
   int S = 1;
   if (!logits_in) {
     if (s->dtype == MOE_BF16) {
-      MOE_TRY(launch_router_logits_tc(x, w_router, s->T, E, s->H, logits_out,
+      MOE_TRY(launch_router_logits_tc(x, w_router, w_packed, s->T, E, s->H, logits_out,
                                       at<char>(ws, L.lpart), dev.sm_count, st, &src, &S));
     } else {
       S = router_splitk(s->T, E, s->H, dev.sm_count);
@@ -299,8 +300,28 @@ int moe_route(const moe_shape_t* shape, const void* x, const float* w_router,
               const float* logits_in, const float* bias, float* logits_out, int32_t* topk_idx,
               float* topk_gate, int32_t* counts, int32_t* nffn_hist, float* zgate, void* ws,
               size_t ws_bytes, void* stream) {
-  return route_impl(shape, x, w_router, logits_in, bias, logits_out, topk_idx, topk_gate, counts,
-                    nffn_hist, zgate, ws, ws_bytes, stream);
+  return route_impl(shape, x, w_router, nullptr, logits_in, bias, logits_out, topk_idx, topk_gate,
+                    counts, nffn_hist, zgate, ws, ws_bytes, stream);
+}
+
+int moe_router_pack(const moe_shape_t* shape, const float* w_router, void* w_packed,
+                    void* stream) {
+  MOE_TRY(check_shape(shape));
+  MOE_TRY(check_ptrs({w_router, w_packed}));
+  if (shape->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  return launch_router_pack(w_router, w_packed, shape->n_ffn + shape->n_zero, shape->H,
+                            dev.sm_count, as_stream(stream));
+}
+
+int moe_route_packed(const moe_shape_t* shape, const void* x, const void* w_packed,
+                     const float* bias, float* logits_out, int32_t* topk_idx, float* topk_gate,
+                     int32_t* counts, int32_t* nffn_hist, float* zgate, void* ws, size_t ws_bytes,
+                     void* stream) {
+  if (!w_packed) return MOE_ERR_INVALID_ARG;
+  return route_impl(shape, x, nullptr, w_packed, nullptr, bias, logits_out, topk_idx, topk_gate,
+                    counts, nffn_hist, zgate, ws, ws_bytes, stream);
 }
 
 int moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* topk_gate,
@@ -370,8 +391,8 @@ int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,
   void* h = at<char>(ws, L.h);
   void* yperm = fused ? nullptr : at<char>(ws, L.yperm);
   float* outacc = fused ? at<float>(ws, L.outacc) : nullptr;
-  MOE_TRY(route_impl(shape, x, w_router, logits_in, bias, logits, topk_idx, topk_gate, counts,
-                     nffn_hist, zgate, ws, ws_bytes, stream));
+  MOE_TRY(route_impl(shape, x, w_router, nullptr, logits_in, bias, logits, topk_idx, topk_gate,
+                     counts, nffn_hist, zgate, ws, ws_bytes, stream));
   MOE_TRY(permute_impl(shape, topk_idx, topk_gate, zgate, x, offsets, perm, rowof, rowgate, xperm,
                        outacc, ws, ws_bytes, stream));
   MOE_TRY(grouped_ffn_impl(shape, x, xperm, offsets, w_gate_up, w_down, perm, rowgate, h, yperm,

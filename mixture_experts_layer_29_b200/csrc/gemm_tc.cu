@@ -789,14 +789,27 @@ size_t router_tc_scratch_bytes(int T, int E, int H) {
   return b;
 }
 
-int launch_router_logits_tc(const void* x, const float* w_router, int T, int E, int H,
-                            float* logits, void* scratch, int sm_count, cudaStream_t st,
-                            const float** src_out, int* splits_out) {
+int launch_router_pack(const float* w_router, void* w_packed, int E, int H, int sm_count,
+                       cudaStream_t st) {
+  const size_t n = (size_t)E * H / 4;
+  int blocks = (int)((n + 255) / 256);
+  if (blocks > 8 * sm_count) blocks = 8 * sm_count;
+  k_split_router_weight<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(w_router),
+                                                static_cast<__nv_bfloat16*>(w_packed), E, H);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_router_logits_tc(const void* x, const float* w_router, const void* w_packed, int T,
+                            int E, int H, float* logits, void* scratch, int sm_count,
+                            cudaStream_t st, const float** src_out, int* splits_out) {
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(scratch);
   size_t off = ((size_t)E * 3 * H * 2 + 1023) / 1024 * 1024;
   float* partial = reinterpret_cast<float*>(static_cast<char*>(scratch) + off);
-  {
+  if (w_packed) {
+    wsplit = static_cast<__nv_bfloat16*>(const_cast<void*>(w_packed));
+  } else {
     const size_t n = (size_t)E * H / 4;
     int blocks = (int)((n + 255) / 256);
     if (blocks > 8 * sm_count) blocks = 8 * sm_count;

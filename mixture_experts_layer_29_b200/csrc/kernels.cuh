@@ -33,9 +33,12 @@ int router_tc_splitk(int T, int E, int H, int sm_count);
 size_t router_tc_scratch_bytes(int T, int E, int H);
 // Writes the logits (S == 1) or S partial slices; *src_out / *splits_out tell the top-K
 // kernel where to read them.
-int launch_router_logits_tc(const void* x, const float* w_router, int T, int E, int H,
-                            float* logits, void* scratch, int sm_count, cudaStream_t st,
-                            const float** src_out, int* splits_out);
+// w_packed (bf16 [E, 3H] from launch_router_pack) or nullptr: split w_router here.
+int launch_router_logits_tc(const void* x, const float* w_router, const void* w_packed, int T,
+                            int E, int H, float* logits, void* scratch, int sm_count,
+                            cudaStream_t st, const float** src_out, int* splits_out);
+int launch_router_pack(const float* w_router, void* w_packed, int E, int H, int sm_count,
+                       cudaStream_t st);
 // Softmax / top-K / histograms from S logit slices of T x E (summed in order; S > 1 also
 // writes the sum to logits_out).
 cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const float* bias,

@@ -174,6 +174,159 @@ __global__ void __launch_bounds__(256) k_perm_scatter(
   }
 }
 
+// ---- small batches (T <= 512): all index work in one CTA, then a wide copy kernel -------
+constexpr int kSmallT = 512;
+constexpr int kSmallChunks = kSmallT / 32;
+
+// One CTA of 512 threads: bitmasks [n_ffn][16] and their per-expert prefixes in shared
+// memory, the expert counts, the offsets (block scan), then every pick's row. The same
+// ranking as the three-kernel path, so the same rows.
+__global__ void __launch_bounds__(512) k_perm_index_small(
+    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_gate, int T, int n_ffn,
+    int E, int K, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+    int32_t* __restrict__ row_of, float* __restrict__ row_gate, int* status) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* masks = sm;                                          // [n_ffn][16]
+  int32_t* crel = reinterpret_cast<int32_t*>(sm + n_ffn * kSmallChunks);   // [n_ffn][16]
+  int32_t* offs = crel + n_ffn * kSmallChunks;                   // [n_ffn + 1]
+  __shared__ int32_t s_wsum[16];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < n_ffn * kSmallChunks; i += blockDim.x) masks[i] = 0u;
+  __syncthreads();
+  const int t = tid;
+  // keep[k]: slot k is in range and the first slot of its expert (a repeated expert shows
+  // as its bit already set: a token's own slots run in order, other tokens use other bits)
+  uint32_t keep = 0u;
+  int ek[32];
+  if (t < T) {
+    const int32_t* row = topk_idx + (size_t)t * K;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) ek[k] = k < K ? row[k] : -1;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      if (k >= K) break;
+      const int e = ek[k];
+      if (e < 0 || e >= E) {
+        set_status(status, MOE_ERR_DEVICE_CHECK);
+        continue;
+      }
+      if (e < n_ffn) {
+        const uint32_t bit = 1u << (t & 31);
+        if (atomicOr(&masks[e * kSmallChunks + (t >> 5)], bit) & bit) {
+          set_status(status, MOE_ERR_DEVICE_CHECK);
+          continue;
+        }
+      } else {
+        // zero experts have no mask: repeated zero experts are checked directly
+        bool dup = false;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < k && ek[j] == e) dup = true;
+        if (dup) {
+          set_status(status, MOE_ERR_DEVICE_CHECK);
+          continue;
+        }
+      }
+      keep |= 1u << k;
+    }
+  }
+  __syncthreads();
+  // per expert: exclusive prefix of the chunk popcounts, and the count
+  int local = 0;
+  for (int e = tid; e < n_ffn; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < kSmallChunks; ++c) {
+      crel[e * kSmallChunks + c] = run;
+      run += __popc(masks[e * kSmallChunks + c]);
+    }
+    offs[e] = run;          // count for now
+  }
+  __syncthreads();
+  // offsets: exclusive scan of the counts (each thread a contiguous run of experts)
+  const int per = (n_ffn + blockDim.x - 1) / blockDim.x;
+  const int b = tid * per;
+  for (int i = 0; i < per; ++i)
+    if (b + i < n_ffn) local += offs[b + i];
+  const int inc = warp_inclusive_scan(local);
+  if (lane == 31) s_wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < 16 ? s_wsum[lane] : 0;
+    const int wi = warp_inclusive_scan(v);
+    if (lane < 16) s_wsum[lane] = wi - v;
+  }
+  __syncthreads();
+  int run = s_wsum[warp] + inc - local;
+  int cnt[4];
+  for (int i = 0; i < per && i < 4; ++i) cnt[i] = (b + i < n_ffn) ? offs[b + i] : 0;
+  __syncthreads();
+  for (int i = 0; i < per && i < 4; ++i)
+    if (b + i < n_ffn) {
+      offs[b + i] = run;
+      run += cnt[i];
+    }
+  if (tid == blockDim.x - 1) offs[n_ffn] = run;
+  __syncthreads();
+  for (int i = tid; i <= n_ffn; i += blockDim.x) offsets[i] = offs[i];
+  if (t < T) {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      if (k >= K) break;
+      int r = -1;
+      const int e = ek[k];
+      if (((keep >> k) & 1u) && e < n_ffn) {
+        const int c = t >> 5;
+        r = offs[e] + crel[e * kSmallChunks + c] +
+            __popc(masks[e * kSmallChunks + c] & ((1u << (t & 31)) - 1u));
+        perm_token[r] = t;
+        row_gate[r] = topk_gate[(size_t)t * K + k];
+      }
+      row_of[(size_t)t * K + k] = r;
+    }
+  }
+}
+
+// Copy x[t] into the rows of its FFN picks (and out_acc = zgate * x): block (t, seg) takes
+// one contiguous slice of the row, 16 bytes per thread per step.
+template <bool XBF16>
+__global__ void __launch_bounds__(128) k_perm_copy(const int32_t* __restrict__ row_of,
+                                                   const float* __restrict__ zgate,
+                                                   const void* __restrict__ x, int H, int K,
+                                                   void* __restrict__ x_perm,
+                                                   float* __restrict__ out_acc) {
+  __shared__ int32_t s_rows[32];
+  const int t = blockIdx.x;
+  if (threadIdx.x < K) s_rows[threadIdx.x] = row_of[(size_t)t * K + threadIdx.x];
+  __syncthreads();
+  constexpr int esz = XBF16 ? 2 : 4;
+  const int nvec = H * esz / 16;
+  const int per = (nvec + gridDim.y - 1) / gridDim.y;
+  const int v_end = min(nvec, (int)(blockIdx.y + 1) * per);
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + (size_t)t * H * esz);
+  const float zg = out_acc ? zgate[t] : 0.f;
+  for (int v = blockIdx.y * per + threadIdx.x; v < v_end; v += blockDim.x) {
+    const uint4 q = __ldg(src + v);
+    if (x_perm)
+      for (int k = 0; k < K; ++k) {
+        const int r = s_rows[k];
+        if (r >= 0) reinterpret_cast<uint4*>(static_cast<char*>(x_perm) + (size_t)r * H * esz)[v] = q;
+      }
+    if (out_acc) {
+      float* o = out_acc + (size_t)t * H + (size_t)v * (16 / esz);
+      if (XBF16) {
+        const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&q);
+        reinterpret_cast<float4*>(o)[0] =
+            make_float4(zg * to_f32(b[0]), zg * to_f32(b[1]), zg * to_f32(b[2]), zg * to_f32(b[3]));
+        reinterpret_cast<float4*>(o)[1] =
+            make_float4(zg * to_f32(b[4]), zg * to_f32(b[5]), zg * to_f32(b[6]), zg * to_f32(b[7]));
+      } else {
+        const float* f = reinterpret_cast<const float*>(&q);
+        reinterpret_cast<float4*>(o)[0] = make_float4(zg * f[0], zg * f[1], zg * f[2], zg * f[3]);
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, const float* zgate,
@@ -181,6 +334,32 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, cons
                            uint32_t* masks, int32_t* crel, int32_t* ecount, int32_t* offsets,
                            int32_t* perm_token, int32_t* row_of, float* row_gate, void* x_perm,
                            float* out_acc, int* status, cudaStream_t st) {
+  if (T <= kSmallT && n_ffn <= 1024) {
+    // one CTA for the indices, then a wide copy (short chain for small batches)
+    const size_t smem = sizeof(uint32_t) * (size_t)n_ffn * kSmallChunks * 2 + sizeof(int32_t) * (n_ffn + 1);
+    if (smem > 48 * 1024) {
+      const cudaError_t e = cudaFuncSetAttribute(k_perm_index_small,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    k_perm_index_small<<<1, 512, smem, st>>>(topk_idx, topk_gate, T, n_ffn, E, K, offsets,
+                                             perm_token, row_of, row_gate, status);
+    count_launch();
+    if (x_perm || out_acc) {
+      const int nvec = H * (x_is_bf16 ? 2 : 4) / 16;
+      int nseg = (4 * 148 + T - 1) / T;                 // about four CTAs per SM in total
+      const int max_seg = (nvec + 127) / 128;
+      if (nseg > max_seg) nseg = max_seg;
+      if (nseg < 1) nseg = 1;
+      const dim3 grid(T, nseg);
+      if (x_is_bf16)
+        k_perm_copy<true><<<grid, 128, 0, st>>>(row_of, zgate, x, H, K, x_perm, out_acc);
+      else
+        k_perm_copy<false><<<grid, 128, 0, st>>>(row_of, zgate, x, H, K, x_perm, out_acc);
+      count_launch();
+    }
+    return cudaGetLastError();
+  }
   const int nchunk = (T + 31) / 32;
   const int g1 = (nchunk + kChunksPerBlock - 1) / kChunksPerBlock;
   const size_t sm1 = sizeof(uint32_t) * kChunksPerBlock * n_ffn;

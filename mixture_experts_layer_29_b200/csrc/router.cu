@@ -216,7 +216,6 @@ cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_ro
 // through shared memory, then integer atomics.
 // ---------------------------------------------------------------------------------------
 namespace {
-constexpr int kRouteWarps = 8;
 
 // exp(d) for d = L - max given exactly in double, evaluated as exp(hi) * (1 + lo)
 __device__ __forceinline__ float exp_split(float L, double dm) {
@@ -227,8 +226,10 @@ __device__ __forceinline__ float exp_split(float L, double dm) {
   return fmaf(v, dl, v);
 }
 
-template <int J>
-__global__ void __launch_bounds__(kRouteWarps * 32) k_route_topk(
+// WARPS tokens per CTA at a time: 8 for large batches, 1 for small ones (each token's
+// dependent chain then has an SM to itself).
+template <int J, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1) k_route_topk(
     const float* __restrict__ src, int S, size_t slice, float* __restrict__ logits_out,
     const float* __restrict__ bias, int T, int E, int n_ffn, int K,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ counts,
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route_topk(
     bia[j] = e < E ? bias[e] : 0.f;
   }
 
-  for (int t = blockIdx.x * kRouteWarps + warp; t < T; t += gridDim.x * kRouteWarps) {
+  for (int t = blockIdx.x * WARPS + warp; t < T; t += gridDim.x * WARPS) {
     const float* Lr = src + (size_t)t * E;
     float lv[J];
     float m = -INFINITY;
@@ -344,11 +345,18 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route_topk(
 }
 
 template <int J>
-void launch_topk_j(dim3 grid, cudaStream_t st, const float* src, int S, size_t slice,
-                   float* logits_out, const float* bias, int T, int E, int n_ffn, int K,
-                   int32_t* idx, float* gate, int32_t* counts, int32_t* hist, float* zgate) {
-  k_route_topk<J><<<grid, kRouteWarps * 32, 0, st>>>(src, S, slice, logits_out, bias, T, E,
-                                                     n_ffn, K, idx, gate, counts, hist, zgate);
+void launch_topk_j(int T, int sm_count, cudaStream_t st, const float* src, int S, size_t slice,
+                   float* logits_out, const float* bias, int E, int n_ffn, int K, int32_t* idx,
+                   float* gate, int32_t* counts, int32_t* hist, float* zgate) {
+  if (T < 8 * sm_count) {
+    k_route_topk<J, 1><<<T, 32, 0, st>>>(src, S, slice, logits_out, bias, T, E, n_ffn, K, idx,
+                                         gate, counts, hist, zgate);
+  } else {
+    int blocks = (T + 7) / 8;
+    if (blocks > 8 * sm_count) blocks = 8 * sm_count;
+    k_route_topk<J, 8><<<blocks, 256, 0, st>>>(src, S, slice, logits_out, bias, T, E, n_ffn, K,
+                                               idx, gate, counts, hist, zgate);
+  }
 }
 }  // namespace
 
@@ -360,14 +368,11 @@ cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const 
   if (err != cudaSuccess) return err;
   err = cudaMemsetAsync(nffn_hist, 0, sizeof(int32_t) * (K + 1), st);
   if (err != cudaSuccess) return err;
-  int blocks = (T + kRouteWarps - 1) / kRouteWarps;
-  if (blocks > 8 * sm_count) blocks = 8 * sm_count;
-  dim3 grid(blocks);
-  const int J = (E + 31) / 32;
   const size_t slice = (size_t)T * E;
+  const int J = (E + 31) / 32;
 #define MOE_TOPK_CASE(JJ)                                                                      \
   if (J <= JJ) {                                                                               \
-    launch_topk_j<JJ>(grid, st, src, S, slice, logits_out, bias, T, E, n_ffn, K, topk_idx,     \
+    launch_topk_j<JJ>(T, sm_count, st, src, S, slice, logits_out, bias, E, n_ffn, K, topk_idx, \
                       topk_gate, counts, nffn_hist, zgate);                                    \
   } else
   MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4) MOE_TOPK_CASE(6)

@@ -202,3 +202,26 @@ def test_ffn_out_scale(cuda_device):
     case = gh.Case(cfg, seed=4)
     _ffn_checks(case, "fused")
     _ffn_checks(case, "deterministic")
+
+
+@pytest.mark.parametrize("name,T", [("proxy_bf16", 4096), ("prefill_bf16", 8192),
+                                    ("decode_bf16", 128)])
+def test_packed_router_weight_gives_the_same_routing(cuda_device, name, T):
+    """moe_router_pack once + moe_route_packed == moe_route, bit for bit."""
+    cfg = wl.CONFIGS[name].with_(T=T)
+    case = gh.Case(cfg, ffn=False)
+    b = case.buffers()
+    case.route(b)
+    ref = [t.clone() for t in (b.logits, b.topk_idx, b.topk_gate, b.counts, b.nffn_hist, b.zgate)]
+    packed = torch.empty(cfg.E, 3 * cfg.H, dtype=torch.bfloat16, device="cuda")
+    abi.router_pack(b.shape, case.w.w_router, packed)
+    # hi + mid + lo reproduces the fp32 weight exactly
+    hi, mid, lo = packed.view(cfg.E, 3, cfg.H).float().unbind(1)
+    assert torch.equal((hi + mid) + lo, case.w.w_router)
+    for t in (b.logits, b.topk_idx, b.topk_gate, b.counts, b.nffn_hist, b.zgate):
+        t.zero_()
+    abi.route_packed(b.shape, case.x, packed, case.w.bias, b.logits, b.topk_idx, b.topk_gate,
+                     b.counts, b.nffn_hist, b.zgate, b.ws)
+    torch.cuda.synchronize()
+    for a, c in zip(ref, (b.logits, b.topk_idx, b.topk_gate, b.counts, b.nffn_hist, b.zgate)):
+        assert torch.equal(a, c)
