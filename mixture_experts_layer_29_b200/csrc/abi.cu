@@ -4,15 +4,25 @@
 #include <atomic>
 #include <initializer_list>
 #include <mutex>
+#include <stdlib.h>
 #include <string.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_B200_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 
 int current_device_info(DeviceInfo* info) {
   static std::mutex mu;
@@ -152,20 +162,28 @@ int route_impl(const moe_shape_t* s, const void* x, const float* w_router, const
   const cudaStream_t st = as_stream(stream);
   const float* src = logits_in;      // logits, or S split-K slices of them
   int S = 1;
+  // the router kernel clears the counts and the histogram the top-K kernel adds to
+  ZeroSpec zero;
+  zero.a = counts;
+  zero.na = E;
+  zero.b = nffn_hist;
+  zero.nb = s->K + 1;
   if (!logits_in) {
     if (s->dtype == MOE_BF16) {
       MOE_TRY(launch_router_logits_tc(x, w_router, w_packed, s->T, E, s->H, logits_out,
-                                      at<char>(ws, L.lpart), dev.sm_count, st, &src, &S));
+                                      at<char>(ws, L.lpart), dev.sm_count, zero, st, &src, &S));
     } else {
       S = router_splitk(s->T, E, s->H, dev.sm_count);
       float* part = at<float>(ws, L.lpart);
       MOE_TRY(cuda_rc(launch_router_logits(x, 0, w_router, s->T, E, s->H, logits_out, part, S,
-                                           st)));
+                                           zero, st)));
       src = S > 1 ? part : logits_out;
     }
+  } else {
+    MOE_TRY(cuda_rc(launch_zero_counts(counts, E, nffn_hist, s->K, st)));
   }
-  if (S > 4) {
-    // many slices: one wide reduction kernel beats summing them inside the top-K warps
+  if (!route_topk_sums_slices(s->T, S, dev.sm_count)) {
+    // many slices and many tokens: one wide reduction kernel first
     MOE_TRY(cuda_rc(launch_splitk_sum(src, S, (size_t)s->T * E, logits_out, st)));
     src = logits_out;
     S = 1;

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 namespace {
@@ -46,6 +47,8 @@ struct Vec<float> {
 template <typename T>
 __global__ void __launch_bounds__(256) k_finalize(const float* __restrict__ acc, T* __restrict__ out,
                                                   size_t n) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int V = Vec<T>::N;
   const size_t nv = n / V;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nv;
@@ -60,19 +63,24 @@ __global__ void __launch_bounds__(256) k_finalize(const float* __restrict__ acc,
   }
 }
 
-template <typename T>
+// G rows are loaded before they are summed: G = 4 for small batches (more loads in
+// flight per thread), 1 for large ones (fewer registers, more CTAs per SM).
+template <typename T, int G>
 __global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, const T* __restrict__ y_perm,
                                                      const float* __restrict__ topk_gate,
                                                      const int32_t* __restrict__ row_of,
                                                      const float* __restrict__ zgate,
                                                      T* __restrict__ out, int H, int K, float scale) {
   constexpr int V = Vec<T>::N;
-  __shared__ int s_row[32];
-  __shared__ float s_g[32];
+  __shared__ int s_row[32 + G];
+  __shared__ float s_g[32 + G];
+  pdl_launch_dependents();
+  pdl_wait();
   const int t = blockIdx.x;
-  if (threadIdx.x < K) {
-    s_row[threadIdx.x] = row_of[(size_t)t * K + threadIdx.x];
-    s_g[threadIdx.x] = scale * topk_gate[(size_t)t * K + threadIdx.x];
+  if (threadIdx.x < 32 + G) {
+    const bool in = threadIdx.x < K;
+    s_row[threadIdx.x] = in ? row_of[(size_t)t * K + threadIdx.x] : -1;
+    s_g[threadIdx.x] = in ? scale * topk_gate[(size_t)t * K + threadIdx.x] : 0.f;
   }
   __syncthreads();
   const float zg = zgate[t];
@@ -84,13 +92,20 @@ __global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, co
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
-    for (int k = 0; k < K; ++k) {
-      const int r = s_row[k];
-      if (r < 0) continue;
-      float y[V];
-      Vec<T>::load(y_perm + (size_t)r * H + c, y);
+    // slots in order
+    for (int k0 = 0; k0 < K; k0 += G) {
+      float y[G][V];
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] = fmaf(s_g[k], y[i], acc[i]);
+      for (int u = 0; u < G; ++u) {
+        const int r = s_row[k0 + u];
+        if (r >= 0) Vec<T>::load(y_perm + (size_t)r * H + c, y[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < G; ++u) {
+        if (s_row[k0 + u] < 0) continue;
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(s_g[k0 + u], y[u][i], acc[i]);
+      }
     }
     float xv[V];
     Vec<T>::load(x + (size_t)t * H + c, xv);
@@ -101,6 +116,8 @@ __global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, co
 }
 
 __global__ void k_pid_init(const float* __restrict__ bias, float* __restrict__ st, int n_ffn) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_ffn; i += gridDim.x * blockDim.x) {
     st[i] = bias[i];
     st[n_ffn + i] = 0.f;
@@ -116,6 +133,8 @@ __global__ void __launch_bounds__(1024) k_pid_update(moe_pid_t pid, const int32_
                                                      float* __restrict__ stats, int T, int K,
                                                      int n_ffn, int E) {
   __shared__ double red[32][8];
+  pdl_launch_dependents();
+  pdl_wait();
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
   // v: [0] FFN count, [1] max FFN count, [2] FFN experts hit, [3] zero-expert count,
   //    [4] |e|, [5] max |e|, [6] n * hist[n], [7] n^2 * hist[n]
@@ -181,12 +200,13 @@ cudaError_t launch_finalize(const float* out_acc, void* out, int out_is_bf16, si
   int blocks = (int)((work + 255) / 256);
   if (blocks > 8192) blocks = 8192;
   if (blocks < 1) blocks = 1;
-  if (out_is_bf16)
-    k_finalize<__nv_bfloat16><<<blocks, 256, 0, st>>>(out_acc, static_cast<__nv_bfloat16*>(out), n);
-  else
-    k_finalize<float><<<blocks, 256, 0, st>>>(out_acc, static_cast<float*>(out), n);
+  const cudaError_t e =
+      out_is_bf16 ? launch_kernel(k_finalize<__nv_bfloat16>, blocks, 256, 0, st, 1, out_acc,
+                                  static_cast<__nv_bfloat16*>(out), n)
+                  : launch_kernel(k_finalize<float>, blocks, 256, 0, st, 1, out_acc,
+                                  static_cast<float*>(out), n);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_combine_det(const void* x, const void* y_perm, const float* topk_gate,
@@ -199,30 +219,34 @@ cudaError_t launch_combine_det(const void* x, const void* y_perm, const float* t
   if (nseg > max_seg) nseg = max_seg;
   if (nseg < 1) nseg = 1;
   const dim3 grid(T, nseg);
-  if (is_bf16)
-    k_combine_det<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm), topk_gate,
-        row_of, zgate, static_cast<__nv_bfloat16*>(out), H, K, scale);
-  else
-    k_combine_det<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x),
-                                            static_cast<const float*>(y_perm), topk_gate, row_of,
-                                            zgate, static_cast<float*>(out), H, K, scale);
+  const bool small = T < 1024;
+  const cudaError_t e =
+      is_bf16 ? launch_kernel(small ? k_combine_det<__nv_bfloat16, 4> : k_combine_det<__nv_bfloat16, 1>,
+                              grid, 256, 0, st, 1, static_cast<const __nv_bfloat16*>(x),
+                              static_cast<const __nv_bfloat16*>(y_perm), topk_gate, row_of, zgate,
+                              static_cast<__nv_bfloat16*>(out), H, K, scale)
+              : launch_kernel(small ? k_combine_det<float, 4> : k_combine_det<float, 1>, grid, 256,
+                              0, st, 1, static_cast<const float*>(x),
+                              static_cast<const float*>(y_perm), topk_gate, row_of, zgate,
+                              static_cast<float*>(out), H, K, scale);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_pid_init(const float* bias, float* pid_state, int n_ffn, cudaStream_t st) {
-  k_pid_init<<<(n_ffn + 255) / 256, 256, 0, st>>>(bias, pid_state, n_ffn);
+  const cudaError_t e = launch_kernel(k_pid_init, (n_ffn + 255) / 256, 256, 0, st, 1, bias,
+                                      pid_state, n_ffn);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_pid_update(const moe_pid_t& pid, const int32_t* counts,
                               const int32_t* nffn_hist, float* bias, float* pid_state,
                               float* stats, int T, int K, int n_ffn, int E, cudaStream_t st) {
-  k_pid_update<<<1, 1024, 0, st>>>(pid, counts, nffn_hist, bias, pid_state, stats, T, K, n_ffn, E);
+  const cudaError_t e = launch_kernel(k_pid_update, 1, 1024, 0, st, 1, pid, counts, nffn_hist,
+                                      bias, pid_state, stats, T, K, n_ffn, E);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace moe

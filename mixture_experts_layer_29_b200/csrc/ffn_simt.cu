@@ -8,6 +8,7 @@
 // LongCat-Flash Technical Report digest, Key claims (report §2.4): per-expert intermediate.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 namespace {
@@ -25,6 +26,8 @@ __global__ void __launch_bounds__(128) k_ffn_up_simt(const float* __restrict__ x
                                                      const int32_t* __restrict__ offsets,
                                                      const float* __restrict__ wgu, float* __restrict__ h,
                                                      int H, int I, int n_ffn) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int R = offsets[n_ffn];
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= I) return;
@@ -51,6 +54,8 @@ __global__ void __launch_bounds__(128) k_ffn_down_simt(const float* __restrict__
                                                        float* __restrict__ y_perm,
                                                        float* __restrict__ out_acc, int H, int I,
                                                        int n_ffn, float scale, int fused) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int R = offsets[n_ffn];
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= H) return;
@@ -76,13 +81,15 @@ cudaError_t launch_grouped_ffn_simt(const float* x_perm, const int32_t* offsets,
                                     int n_ffn, int K, float scale, int fused, cudaStream_t st) {
   const int rows = T * K < 65535 ? T * K : 65535;   // rows beyond: grid-stride loop
   dim3 g1((I + 127) / 128, rows);
-  k_ffn_up_simt<<<g1, 128, 0, st>>>(x_perm, offsets, w_gate_up, h, H, I, n_ffn);
+  cudaError_t e = launch_kernel(k_ffn_up_simt, g1, 128, 0, st, 1, x_perm, offsets, w_gate_up, h,
+                                H, I, n_ffn);
   count_launch();
+  if (e != cudaSuccess) return e;
   dim3 g2((H + 127) / 128, rows);
-  k_ffn_down_simt<<<g2, 128, 0, st>>>(h, offsets, w_down, perm_token, row_gate, y_perm, out_acc,
-                                       H, I, n_ffn, scale, fused);
+  e = launch_kernel(k_ffn_down_simt, g2, 128, 0, st, 1, h, offsets, w_down, perm_token, row_gate,
+                    y_perm, out_acc, H, I, n_ffn, scale, fused);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace moe

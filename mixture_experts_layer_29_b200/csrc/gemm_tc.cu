@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 namespace {
@@ -84,6 +85,7 @@ struct GemmArgs {
   int kchunk;               // k-blocks per tensor-core accumulation (0: the whole split)
   long long split_stride;   // elements between the outputs of consecutive splits
   const int32_t* gather_tok;  // non-null: A row r is row gather_tok[r] of A's tensor
+  ZeroSpec zero;              // buffers cleared after the dependency wait
 };
 
 struct Tile {
@@ -198,8 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   SharedStorage& s = *reinterpret_cast<SharedStorage*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
 
-  // ---- set-up -------------------------------------------------------------------------
+  // ---- set-up (no global memory before the dependency wait) ----------------------------
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&s.full[i], 1);
@@ -218,6 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  pdl_wait();
+  g.zero.run(blockIdx.x, gridDim.x, threadIdx.x, kThreads);
   // tile table: toff[e] = sum_{e' < e} ceil(count_e' / 128)
   if (g.dense_rows > 0) {
     if (threadIdx.x == 0) {
@@ -482,8 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();            // 0: leader, 1: peer
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  pdl_launch_dependents();
 
-  // ---- set-up -------------------------------------------------------------------------
+  // ---- set-up (no global memory before the dependency wait) ----------------------------
   if (threadIdx.x == 0) {
     for (int i = 0; i < PSTAGES; ++i) {
       mbar_init(&s.full[i], 1);
@@ -498,6 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
   }
+  pdl_wait();
   for (int i = threadIdx.x; i <= g.n_ffn; i += kThreads) s.offs[i] = g.offsets[i];
   __syncthreads();
   cluster_sync();                                     // both CTAs' barriers initialised
@@ -667,9 +674,9 @@ int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, 
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  kern<<<sm_count, kThreads, smem, st>>>(ma, mb, g);
+  const cudaError_t e = launch_kernel(kern, sm_count, kThreads, smem, st, 1, ma, mb, g);
   count_launch();
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // Cluster-of-two launch of the CTA-pair kernel: as many clusters as fit at once (cached
@@ -711,8 +718,8 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
     nclusters = clusters_of[dev];
   }
   if (nclusters > sm_count / 2) nclusters = sm_count / 2;
-  cfg.gridDim = dim3(2 * nclusters);
-  if (cudaLaunchKernelEx(&cfg, k_grouped_gemm_pair, ma, mb, g) != cudaSuccess) {
+  if (launch_kernel(k_grouped_gemm_pair, 2 * nclusters, kThreads, smem, st, 2, ma, mb, g) !=
+      cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
@@ -736,6 +743,8 @@ bool use_pair_kernel(int T) {
 __global__ void __launch_bounds__(256) k_split_router_weight(const float4* __restrict__ w,
                                                              __nv_bfloat16* __restrict__ out,
                                                              int E, int H) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int H4 = H / 4;                       // four weights per thread step
   const size_t n = (size_t)E * H4;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
@@ -794,15 +803,17 @@ int launch_router_pack(const float* w_router, void* w_packed, int E, int H, int 
   const size_t n = (size_t)E * H / 4;
   int blocks = (int)((n + 255) / 256);
   if (blocks > 8 * sm_count) blocks = 8 * sm_count;
-  k_split_router_weight<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(w_router),
-                                                static_cast<__nv_bfloat16*>(w_packed), E, H);
+  const cudaError_t e = launch_kernel(k_split_router_weight, blocks, 256, 0, st, 1,
+                                      reinterpret_cast<const float4*>(w_router),
+                                      static_cast<__nv_bfloat16*>(w_packed), E, H);
   count_launch();
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_router_logits_tc(const void* x, const float* w_router, const void* w_packed, int T,
                             int E, int H, float* logits, void* scratch, int sm_count,
-                            cudaStream_t st, const float** src_out, int* splits_out) {
+                            ZeroSpec zero, cudaStream_t st, const float** src_out,
+                            int* splits_out) {
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(scratch);
   size_t off = ((size_t)E * 3 * H * 2 + 1023) / 1024 * 1024;
@@ -813,9 +824,10 @@ int launch_router_logits_tc(const void* x, const float* w_router, const void* w_
     const size_t n = (size_t)E * H / 4;
     int blocks = (int)((n + 255) / 256);
     if (blocks > 8 * sm_count) blocks = 8 * sm_count;
-    k_split_router_weight<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(w_router),
-                                                  wsplit, E, H);
+    const cudaError_t e = launch_kernel(k_split_router_weight, blocks, 256, 0, st, 1,
+                                        reinterpret_cast<const float4*>(w_router), wsplit, E, H);
     count_launch();
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   CUtensorMap mx, mw;
   int rc;
@@ -838,6 +850,7 @@ int launch_router_logits_tc(const void* x, const float* w_router, const void* w_
   g.ld_out = E;
   g.out = S > 1 ? static_cast<void*>(partial) : static_cast<void*>(logits);
   g.split_stride = (long long)T * E;
+  g.zero = zero;
   if ((rc = launch_one(mx, mw, g, sm_count, st)) != MOE_OK) return rc;
   // with S > 1 the top-K kernel sums the partial slices in split order
   *src_out = S > 1 ? partial : logits;

@@ -20,13 +20,30 @@ struct DeviceInfo {
 // Cached per device; returns MOE_OK, MOE_ERR_CUDA or MOE_ERR_NO_DEVICE.
 int current_device_info(DeviceInfo* info);
 
+// Two int32 buffers that a kernel clears (after its dependency wait) for the kernels
+// after it: the router kernels clear the expert counts and the FFN-pick histogram that
+// the top-K kernel then accumulates into.
+struct ZeroSpec {
+  int32_t* a = nullptr;
+  int na = 0;
+  int32_t* b = nullptr;
+  int nb = 0;
+#ifdef __CUDACC__
+  __device__ __forceinline__ void run(int block, int nblocks, int tid, int nthreads) const {
+    const int stride = nblocks * nthreads;
+    for (int i = block * nthreads + tid; i < na; i += stride) a[i] = 0;
+    for (int i = block * nthreads + tid; i < nb; i += stride) b[i] = 0;
+  }
+#endif
+};
+
 // ---- router -----------------------------------------------------------------------------
 // Split-K factor of the logits GEMM for this shape (1 = no partial buffer).
 int router_splitk(int T, int E, int H, int sm_count);
 size_t router_partial_bytes(int T, int E, int H, int sm_count_max);
 cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_router, int T,
                                  int E, int H, float* logits, float* partial, int splitk,
-                                 cudaStream_t st);
+                                 ZeroSpec zero, cudaStream_t st);
 cudaError_t launch_splitk_sum(const float* partial, int S, size_t n, float* out, cudaStream_t st);
 // bf16 x: logits on the tensor cores with W_r split into three exact bf16 parts.
 int router_tc_splitk(int T, int E, int H, int sm_count);
@@ -36,15 +53,22 @@ size_t router_tc_scratch_bytes(int T, int E, int H);
 // w_packed (bf16 [E, 3H] from launch_router_pack) or nullptr: split w_router here.
 int launch_router_logits_tc(const void* x, const float* w_router, const void* w_packed, int T,
                             int E, int H, float* logits, void* scratch, int sm_count,
-                            cudaStream_t st, const float** src_out, int* splits_out);
+                            ZeroSpec zero, cudaStream_t st, const float** src_out,
+                            int* splits_out);
 int launch_router_pack(const float* w_router, void* w_packed, int E, int H, int sm_count,
                        cudaStream_t st);
 // Softmax / top-K / histograms from S logit slices of T x E (summed in order; S > 1 also
 // writes the sum to logits_out).
+// counts [E] and nffn_hist [K + 1] must be zero when it runs (a router kernel's ZeroSpec,
+// or launch_zero_counts).
 cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const float* bias,
                               int T, int E, int n_ffn, int K, int32_t* topk_idx,
                               float* topk_gate, int32_t* counts, int32_t* nffn_hist,
                               float* zgate, int sm_count, cudaStream_t st);
+// Whether launch_route_topk reads S slices itself (else sum them first with
+// launch_splitk_sum).
+bool route_topk_sums_slices(int T, int S, int sm_count);
+cudaError_t launch_zero_counts(int32_t* counts, int E, int32_t* nffn_hist, int K, cudaStream_t st);
 
 // ---- permutation ------------------------------------------------------------------------
 cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, const float* zgate,

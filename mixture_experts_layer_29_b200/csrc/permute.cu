@@ -15,6 +15,7 @@
 //                        §2.1: a zero-computation expert is an identity map).
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 namespace {
@@ -42,7 +43,9 @@ __global__ void __launch_bounds__(256) k_perm_masks(const int32_t* __restrict__ 
                                                     uint32_t* __restrict__ masks, int* status) {
   extern __shared__ uint32_t sm_masks[];   // [8][n_ffn]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_launch_dependents();
   for (int i = threadIdx.x; i < kChunksPerBlock * n_ffn; i += blockDim.x) sm_masks[i] = 0u;
+  pdl_wait();
   __syncthreads();
   const int c = blockIdx.x * kChunksPerBlock + warp;
   const int t = c * 32 + lane;
@@ -66,6 +69,8 @@ __global__ void __launch_bounds__(256) k_perm_masks(const int32_t* __restrict__ 
 __global__ void __launch_bounds__(256) k_perm_scan(const uint32_t* __restrict__ masks, int n_ffn,
                                                    int nchunk, int32_t* __restrict__ crel,
                                                    int32_t* __restrict__ ecount) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (e >= n_ffn) return;
@@ -94,6 +99,8 @@ __global__ void __launch_bounds__(256) k_perm_scatter(
   __shared__ int32_t s_off[1025];
   __shared__ int32_t s_wsum[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_launch_dependents();
+  pdl_wait();
 
   // offsets = exclusive scan of ecount[0, n_ffn): each thread owns ceil(n_ffn/256) entries
   {
@@ -191,7 +198,9 @@ __global__ void __launch_bounds__(512) k_perm_index_small(
   int32_t* offs = crel + n_ffn * kSmallChunks;                   // [n_ffn + 1]
   __shared__ int32_t s_wsum[16];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_launch_dependents();
   for (int i = tid; i < n_ffn * kSmallChunks; i += blockDim.x) masks[i] = 0u;
+  pdl_wait();
   __syncthreads();
   const int t = tid;
   // keep[k]: slot k is in range and the first slot of its expert (a repeated expert shows
@@ -295,6 +304,8 @@ __global__ void __launch_bounds__(128) k_perm_copy(const int32_t* __restrict__ r
                                                    void* __restrict__ x_perm,
                                                    float* __restrict__ out_acc) {
   __shared__ int32_t s_rows[32];
+  pdl_launch_dependents();
+  pdl_wait();
   const int t = blockIdx.x;
   if (threadIdx.x < K) s_rows[threadIdx.x] = row_of[(size_t)t * K + threadIdx.x];
   __syncthreads();
@@ -342,9 +353,10 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, cons
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    k_perm_index_small<<<1, 512, smem, st>>>(topk_idx, topk_gate, T, n_ffn, E, K, offsets,
-                                             perm_token, row_of, row_gate, status);
+    cudaError_t e = launch_kernel(k_perm_index_small, 1, 512, smem, st, 1, topk_idx, topk_gate, T,
+                                  n_ffn, E, K, offsets, perm_token, row_of, row_gate, status);
     count_launch();
+    if (e != cudaSuccess) return e;
     if (x_perm || out_acc) {
       const int nvec = H * (x_is_bf16 ? 2 : 4) / 16;
       int nseg = (4 * 148 + T - 1) / T;                 // about four CTAs per SM in total
@@ -352,13 +364,11 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, cons
       if (nseg > max_seg) nseg = max_seg;
       if (nseg < 1) nseg = 1;
       const dim3 grid(T, nseg);
-      if (x_is_bf16)
-        k_perm_copy<true><<<grid, 128, 0, st>>>(row_of, zgate, x, H, K, x_perm, out_acc);
-      else
-        k_perm_copy<false><<<grid, 128, 0, st>>>(row_of, zgate, x, H, K, x_perm, out_acc);
+      e = launch_kernel(x_is_bf16 ? k_perm_copy<true> : k_perm_copy<false>, grid, 128, 0, st, 1,
+                        row_of, zgate, x, H, K, x_perm, out_acc);
       count_launch();
     }
-    return cudaGetLastError();
+    return e;
   }
   const int nchunk = (T + 31) / 32;
   const int g1 = (nchunk + kChunksPerBlock - 1) / kChunksPerBlock;
@@ -367,21 +377,20 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, cons
     cudaError_t e = cudaFuncSetAttribute(k_perm_masks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
     if (e != cudaSuccess) return e;
   }
-  k_perm_masks<<<g1, 256, sm1, st>>>(topk_idx, T, n_ffn, E, K, nchunk, masks, status);
+  cudaError_t e = launch_kernel(k_perm_masks, g1, 256, sm1, st, 1, topk_idx, T, n_ffn, E, K,
+                                nchunk, masks, status);
   count_launch();
-  k_perm_scan<<<(n_ffn + 7) / 8, 256, 0, st>>>(masks, n_ffn, nchunk, crel, ecount);
+  if (e != cudaSuccess) return e;
+  e = launch_kernel(k_perm_scan, (n_ffn + 7) / 8, 256, 0, st, 1, masks, n_ffn, nchunk, crel,
+                    ecount);
   count_launch();
+  if (e != cudaSuccess) return e;
   const int g3 = (T + 7) / 8;
-  if (x_is_bf16)
-    k_perm_scatter<true><<<g3, 256, 0, st>>>(topk_idx, topk_gate, zgate, x, T, H, n_ffn, E, K,
-                                              nchunk, masks, crel, ecount, offsets, perm_token,
-                                              row_of, row_gate, x_perm, out_acc, status);
-  else
-    k_perm_scatter<false><<<g3, 256, 0, st>>>(topk_idx, topk_gate, zgate, x, T, H, n_ffn, E, K,
-                                               nchunk, masks, crel, ecount, offsets, perm_token,
-                                               row_of, row_gate, x_perm, out_acc, status);
+  e = launch_kernel(x_is_bf16 ? k_perm_scatter<true> : k_perm_scatter<false>, g3, 256, 0, st, 1,
+                    topk_idx, topk_gate, zgate, x, T, H, n_ffn, E, K, nchunk, masks, crel, ecount,
+                    offsets, perm_token, row_of, row_gate, x_perm, out_acc, status);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace moe

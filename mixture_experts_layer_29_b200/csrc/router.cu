@@ -6,8 +6,11 @@
 // §2.1.1) a per-expert bias steers the selection, the gates stay the softmax values.
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -70,9 +73,13 @@ template <bool XBF16>
 __global__ void __launch_bounds__(256, 2) k_router_logits(const void* __restrict__ x,
                                                        const float* __restrict__ w, int T, int E,
                                                        int H, int kchunk, float* __restrict__ out,
-                                                       size_t split_stride) {
+                                                       size_t split_stride, ZeroSpec zero) {
   __shared__ __align__(16) float As[2][RK][RB + RPAD];
   __shared__ __align__(16) float Bs[2][RK][RB + RPAD];
+  pdl_launch_dependents();
+  pdl_wait();
+  zero.run(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z),
+           gridDim.x * gridDim.y * gridDim.z, threadIdx.x, blockDim.x);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int row0 = blockIdx.y * RB, col0 = blockIdx.x * RB;
   const int kbeg = blockIdx.z * kchunk;
@@ -150,6 +157,8 @@ __global__ void __launch_bounds__(256, 2) k_router_logits(const void* __restrict
 // logits = sum over splits s = 0, 1, ... of partial[s] (fixed order)
 __global__ void k_router_splitk_sum(const float* __restrict__ partial, int S, size_t n,
                                     float* __restrict__ logits) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
     float a = partial[i];
@@ -161,9 +170,9 @@ __global__ void k_router_splitk_sum(const float* __restrict__ partial, int S, si
 
 cudaError_t launch_splitk_sum(const float* partial, int S, size_t n, float* out, cudaStream_t st) {
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  k_router_splitk_sum<<<blocks, 256, 0, st>>>(partial, S, n, out);
+  const cudaError_t e = launch_kernel(k_router_splitk_sum, blocks, 256, 0, st, 1, partial, S, n, out);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 int router_splitk(int T, int E, int H, int sm_count) {
@@ -188,32 +197,36 @@ size_t router_partial_bytes(int T, int E, int H, int sm_count_max) {
 
 cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_router, int T,
                                  int E, int H, float* logits, float* partial, int splitk,
-                                 cudaStream_t st) {
+                                 ZeroSpec zero, cudaStream_t st) {
   int kchunk = (H + splitk - 1) / splitk;
   kchunk = (kchunk + RK - 1) / RK * RK;
   const int S = (H + kchunk - 1) / kchunk;
   dim3 grid((E + RB - 1) / RB, (T + RB - 1) / RB, S);
   float* dst = S > 1 ? partial : logits;
   const size_t stride = (size_t)T * E;
-  if (x_is_bf16)
-    k_router_logits<true><<<grid, 256, 0, st>>>(x, w_router, T, E, H, kchunk, dst, stride);
-  else
-    k_router_logits<false><<<grid, 256, 0, st>>>(x, w_router, T, E, H, kchunk, dst, stride);
+  const cudaError_t e = launch_kernel(x_is_bf16 ? k_router_logits<true> : k_router_logits<false>,
+                                      grid, 256, 0, st, 1, x, w_router, T, E, H, kchunk, dst,
+                                      stride, zero);
   count_launch();
-  // with S > 1 the partials are summed (in split order) by the top-K kernel
-  return cudaGetLastError();
+  // with S > 1 the partials are summed in split order (by the top-K kernel or a sum kernel)
+  return e;
 }
 
 // ---------------------------------------------------------------------------------------
 // Softmax + bias-adjusted top-K, one warp per token.
-// Lane l holds experts l, l + 32, ... (J groups). The logits are read from S split-K
-// slices summed in slice order (S = 1: the logits themselves; S > 1: the sum is also
-// written out). exp(L - max) is evaluated in fp32 on the exactly split argument
-// (hi + lo, exp(hi) * (1 + lo)), summed in double, and normalised with a double
-// reciprocal, so p is within a few fp32 ulps of the float64 softmax. The selection score
-// is the fp32 sum p + b (a zero result stored as +0); K rounds of a warp-wide argmax pick
-// (score descending, expert index ascending). Counts and the FFN-pick histogram go
-// through shared memory, then integer atomics.
+// Lane l holds experts l, l + 32, ... (J groups). exp(L - max) is evaluated in fp32 on
+// the exactly split argument (hi + lo, exp(hi) * (1 + lo)), summed in double, and
+// normalised with a double reciprocal, so p is within a few fp32 ulps of the float64
+// softmax. The selection score is the fp32 sum p + b (a zero result stored as +0); the K
+// picks are the first K experts in the order (score descending, expert index ascending).
+//
+// Selection: theta = the K-th largest of the 32 lane maxima. At least K scores are >=
+// theta, so every pick has a score >= theta; the candidates (scores >= theta, typically
+// 12 to 25 of 768) are packed into shared memory and each candidate's rank in the order
+// above is counted directly. Should more than 32 candidates pass (many equal scores),
+// K rounds of a warp-wide argmax over all experts take over. Both give the same picks.
+// Counts and the FFN-pick histogram go through shared memory (8-warp CTAs) or straight
+// to global integer atomics (one-warp CTAs), with the token's zero-expert gate sum.
 // ---------------------------------------------------------------------------------------
 namespace {
 
@@ -226,69 +239,104 @@ __device__ __forceinline__ float exp_split(float L, double dm) {
   return fmaf(v, dl, v);
 }
 
-// WARPS tokens per CTA at a time: 8 for large batches, 1 for small ones (each token's
-// dependent chain then has an SM to itself).
-template <int J, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1) k_route_topk(
-    const float* __restrict__ src, int S, size_t slice, float* __restrict__ logits_out,
-    const float* __restrict__ bias, int T, int E, int n_ffn, int K,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ counts,
-    int32_t* __restrict__ nffn_hist, float* __restrict__ zgate) {
-  __shared__ int s_counts[1024];
-  __shared__ int s_hist[33];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < E; i += blockDim.x) s_counts[i] = 0;
-  if (threadIdx.x <= K) s_hist[threadIdx.x] = 0;
-  __syncthreads();
+struct WarpScratch {        // per warp, in shared memory
+  float cs[32];             // candidate scores
+  int ce[32];               // candidate experts
+  float cp[32];             // candidate gates
+  int se[32];               // picks by rank
+  float sp[32];
+};
 
-  float bia[J];
+// lv[j] holds the logit of expert lane + 32 j (-inf past E). Writes the picks of token t
+// and adds them to cnt / hist (shared or global memory).
+template <int J>
+__device__ __forceinline__ void route_token(float (&lv)[J], const float (&bia)[J], int lane, int t,
+                                            int E, int n_ffn, int K, WarpScratch& ws,
+                                            int32_t* __restrict__ topk_idx,
+                                            float* __restrict__ topk_gate,
+                                            float* __restrict__ zgate, int* cnt, int* hist) {
+  constexpr unsigned kFull = 0xffffffffu;
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < J; ++j) m = fmaxf(m, lv[j]);
+  m = warp_max(m);
+  const double dm = (double)m;
+  double sum = 0.0;
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int e = lane + 32 * j;
-    bia[j] = e < E ? bias[e] : 0.f;
+    const float v = e < E ? exp_split(lv[j], dm) : 0.f;
+    lv[j] = v;                                       // lv now holds exp(L - max)
+    sum += (double)v;
   }
-
-  for (int t = blockIdx.x * WARPS + warp; t < T; t += gridDim.x * WARPS) {
-    const float* Lr = src + (size_t)t * E;
-    float lv[J];
-    float m = -INFINITY;
+  sum = warp_sum(sum);
+  const double inv = 1.0 / sum;
+  float p[J], sc[J];
+  float lm = -INFINITY;                              // this lane's largest score
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int e = lane + 32 * j;
-      float v = -INFINITY;
-      if (e < E) {
-        v = Lr[e];
-        for (int sp = 1; sp < S; ++sp) v += Lr[sp * slice + e];
-        if (S > 1) logits_out[(size_t)t * E + e] = v;
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    p[j] = (float)((double)lv[j] * inv);
+    float v = __fadd_rn(p[j], bia[j]);
+    if (v == 0.0f) v = 0.0f;                          // -0 -> +0
+    sc[j] = e < E ? v : -INFINITY;
+    lm = fmaxf(lm, sc[j]);
+  }
+  // theta: the K-th largest lane maximum (rank by value descending, lane ascending)
+  int rk = 0;
+#pragma unroll
+  for (int i = 1; i < 32; ++i) {
+    const int src = (lane + i) & 31;
+    const float o = __shfl_sync(kFull, lm, src);
+    rk += (o > lm || (o == lm && src < lane)) ? 1 : 0;
+  }
+  const float theta = __shfl_sync(kFull, lm, __ffs(__ballot_sync(kFull, rk == K - 1)) - 1);
+  uint32_t cm = 0u;
+#pragma unroll
+  for (int j = 0; j < J; ++j)
+    if (sc[j] >= theta) cm |= 1u << j;
+  const int cnt_l = __popc(cm);
+  const int incl = warp_inclusive_scan(cnt_l);
+  const int total = __shfl_sync(kFull, incl, 31);
+  int my_e = 0;
+  float my_g = 0.f;
+  if (total <= 32) {
+    int pos = incl - cnt_l;
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+      if ((cm >> j) & 1u) {
+        ws.cs[pos] = sc[j];
+        ws.ce[pos] = lane + 32 * j;
+        ws.cp[pos] = p[j];
+        ++pos;
       }
-      lv[j] = v;
-      m = fmaxf(m, v);
+    __syncwarp();
+    float cs = 0.f;
+    int ce = 0;
+    int r = 0;
+    if (lane < total) {
+      cs = ws.cs[lane];
+      ce = ws.ce[lane];
+#pragma unroll 4
+      for (int i = 0; i < total; ++i) {
+        const float os = ws.cs[i];
+        const int oe = ws.ce[i];
+        r += (os > cs || (os == cs && oe < ce)) ? 1 : 0;
+      }
+      if (r < K) {
+        ws.se[r] = ce;
+        ws.sp[r] = ws.cp[lane];
+      }
     }
-    m = warp_max(m);
-    const double dm = (double)m;
-    double sum = 0.0;
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int e = lane + 32 * j;
-      const float v = e < E ? exp_split(lv[j], dm) : 0.f;
-      lv[j] = v;                                       // lv now holds exp(L - max)
-      sum += (double)v;
+    __syncwarp();
+    if (lane < K) {
+      my_e = ws.se[lane];
+      my_g = ws.sp[lane];
     }
-    sum = warp_sum(sum);
-    const double inv = 1.0 / sum;
-    float p[J], sc[J];
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int e = lane + 32 * j;
-      p[j] = (float)((double)lv[j] * inv);
-      float v = __fadd_rn(p[j], bia[j]);
-      if (v == 0.0f) v = 0.0f;                          // -0 -> +0
-      sc[j] = e < E ? v : -INFINITY;
-    }
+    __syncwarp();
+  } else {
     // K rounds of a warp argmax on (score descending, expert index ascending)
     uint32_t taken = 0u;
-    int my_e = 0;
-    float my_g = 0.f;
     for (int k = 0; k < K; ++k) {
       float bs = -INFINITY;
       int be = 0x7fffffff;
@@ -302,8 +350,8 @@ __global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1) k_route_topk(
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        const float os = __shfl_xor_sync(kFull, bs, o);
+        const int oe = __shfl_xor_sync(kFull, be, o);
         if (os > bs || (os == bs && oe < be)) {
           bs = os;
           be = oe;
@@ -315,65 +363,217 @@ __global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1) k_route_topk(
       for (int j = 0; j < J; ++j)
         if (j == jw) g = p[j];
       if (lane == owner) taken |= 1u << jw;
-      g = __shfl_sync(0xffffffffu, g, owner);
+      g = __shfl_sync(kFull, g, owner);
       if (lane == k) {
         my_e = be;
         my_g = g;
       }
     }
-    if (lane < K) {
-      topk_idx[(size_t)t * K + lane] = my_e;
-      topk_gate[(size_t)t * K + lane] = my_g;
-      atomicAdd(&s_counts[my_e], 1);
-    }
-    const unsigned ffn = __ballot_sync(0xffffffffu, lane < K && my_e < n_ffn);
-    float z = 0.f;
-    for (int k = 0; k < K; ++k) {
-      const float gk = __shfl_sync(0xffffffffu, my_g, k);
-      const int ek = __shfl_sync(0xffffffffu, my_e, k);
-      if (ek >= n_ffn) z += gk;
-    }
-    if (lane == 0) {
-      atomicAdd(&s_hist[__popc(ffn)], 1);
-      zgate[t] = z;
-    }
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < E; i += blockDim.x)
-    if (s_counts[i]) atomicAdd(&counts[i], s_counts[i]);
-  if (threadIdx.x <= K && s_hist[threadIdx.x]) atomicAdd(&nffn_hist[threadIdx.x], s_hist[threadIdx.x]);
+  if (lane < K) {
+    topk_idx[(size_t)t * K + lane] = my_e;
+    topk_gate[(size_t)t * K + lane] = my_g;
+    atomicAdd(&cnt[my_e], 1);
+  }
+  const unsigned ffn = __ballot_sync(kFull, lane < K && my_e < n_ffn);
+  float z = 0.f;
+  for (int k = 0; k < K; ++k) {
+    const float gk = __shfl_sync(kFull, my_g, k);
+    const int ek = __shfl_sync(kFull, my_e, k);
+    if (ek >= n_ffn) z += gk;
+  }
+  if (lane == 0) {
+    atomicAdd(&hist[__popc(ffn)], 1);
+    zgate[t] = z;
+  }
 }
 
 template <int J>
-void launch_topk_j(int T, int sm_count, cudaStream_t st, const float* src, int S, size_t slice,
-                   float* logits_out, const float* bias, int E, int n_ffn, int K, int32_t* idx,
-                   float* gate, int32_t* counts, int32_t* hist, float* zgate) {
-  if (T < 8 * sm_count) {
-    k_route_topk<J, 1><<<T, 32, 0, st>>>(src, S, slice, logits_out, bias, T, E, n_ffn, K, idx,
-                                         gate, counts, hist, zgate);
-  } else {
-    int blocks = (T + 7) / 8;
-    if (blocks > 8 * sm_count) blocks = 8 * sm_count;
-    k_route_topk<J, 8><<<blocks, 256, 0, st>>>(src, S, slice, logits_out, bias, T, E, n_ffn, K,
-                                               idx, gate, counts, hist, zgate);
+__device__ __forceinline__ void load_bias(const float* __restrict__ bias, int E, int lane,
+                                          float (&bia)[J]) {
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    bia[j] = e < E ? bias[e] : 0.f;
   }
 }
+
+// WARPS tokens per CTA at a time: 8 for large batches, 1 for small ones (each token's
+// dependent chain then has an SM to itself). The logits come from S split-K slices summed
+// in slice order (S = 1: the logits themselves; S > 1: the sum is also written out).
+template <int J, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1) k_route_topk(
+    const float* __restrict__ src, int S, size_t slice, float* __restrict__ logits_out,
+    const float* __restrict__ bias, int T, int E, int n_ffn, int K,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ counts,
+    int32_t* __restrict__ nffn_hist, float* __restrict__ zgate) {
+  __shared__ int s_counts[WARPS > 1 ? 1024 : 1];
+  __shared__ int s_hist[33];
+  __shared__ WarpScratch s_ws[WARPS];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_launch_dependents();
+  if constexpr (WARPS > 1) {
+    for (int i = threadIdx.x; i < E; i += blockDim.x) s_counts[i] = 0;
+    if (threadIdx.x <= K) s_hist[threadIdx.x] = 0;
+  }
+  pdl_wait();
+  __syncthreads();
+  int* cnt = WARPS > 1 ? s_counts : counts;
+  int* hist = WARPS > 1 ? s_hist : nffn_hist;
+
+  float bia[J];
+  load_bias<J>(bias, E, lane, bia);
+  for (int t = blockIdx.x * WARPS + warp; t < T; t += gridDim.x * WARPS) {
+    const float* Lr = src + (size_t)t * E;
+    float lv[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int e = lane + 32 * j;
+      float v = -INFINITY;
+      if (e < E) {
+        v = Lr[e];
+        for (int sp = 1; sp < S; ++sp) v += Lr[sp * slice + e];
+        if (S > 1) logits_out[(size_t)t * E + e] = v;
+      }
+      lv[j] = v;
+    }
+    route_token<J>(lv, bia, lane, t, E, n_ffn, K, s_ws[warp], topk_idx, topk_gate, zgate, cnt,
+                   hist);
+  }
+  if constexpr (WARPS > 1) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += blockDim.x)
+      if (s_counts[i]) atomicAdd(&counts[i], s_counts[i]);
+    if (threadIdx.x <= K && s_hist[threadIdx.x])
+      atomicAdd(&nffn_hist[threadIdx.x], s_hist[threadIdx.x]);
+  }
+}
+
+// Small batches with many split-K slices: one CTA per token sums the S slices of its
+// logits (slice order; eight slices in flight per thread, 16-byte loads when the rows
+// allow) into shared memory and writes them out; warp 0 then routes the token.
+constexpr int kSumThreads = 256;
+
+template <int W>
+__device__ __forceinline__ void sum_slices(const float* __restrict__ row, size_t slice, int S,
+                                           int n, float* __restrict__ out_s,
+                                           float* __restrict__ out_g) {
+  using V = typename std::conditional<W == 4, float4, float>::type;
+  const V* p = reinterpret_cast<const V*>(row);
+  const size_t sl = slice / W;
+  for (int q = threadIdx.x; q < n; q += kSumThreads) {
+    float v[W];
+    {
+      const V a = p[q];
+      const float* f = reinterpret_cast<const float*>(&a);
+#pragma unroll
+      for (int i = 0; i < W; ++i) v[i] = f[i];
+    }
+    int sp = 1;
+    for (; sp + 8 <= S; sp += 8) {
+      V a[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a[u] = p[(size_t)(sp + u) * sl + q];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float* f = reinterpret_cast<const float*>(&a[u]);
+#pragma unroll
+        for (int i = 0; i < W; ++i) v[i] += f[i];
+      }
+    }
+    for (; sp < S; ++sp) {
+      const V a = p[(size_t)sp * sl + q];
+      const float* f = reinterpret_cast<const float*>(&a);
+#pragma unroll
+      for (int i = 0; i < W; ++i) v[i] += f[i];
+    }
+#pragma unroll
+    for (int i = 0; i < W; ++i) out_s[q * W + i] = v[i];
+    V o;
+    float* f = reinterpret_cast<float*>(&o);
+#pragma unroll
+    for (int i = 0; i < W; ++i) f[i] = v[i];
+    reinterpret_cast<V*>(out_g)[q] = o;
+  }
+}
+
+template <int J>
+__global__ void __launch_bounds__(kSumThreads, 1) k_route_topk_sum(
+    const float* __restrict__ src, int S, size_t slice, float* __restrict__ logits_out,
+    const float* __restrict__ bias, int T, int E, int n_ffn, int K,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ counts,
+    int32_t* __restrict__ nffn_hist, float* __restrict__ zgate, int vec4) {
+  __shared__ __align__(16) float s_l[32 * J];
+  __shared__ WarpScratch s_ws;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int t = blockIdx.x;
+  if (vec4)
+    sum_slices<4>(src + (size_t)t * E, slice, S, E / 4, s_l, logits_out + (size_t)t * E);
+  else
+    sum_slices<1>(src + (size_t)t * E, slice, S, E, s_l, logits_out + (size_t)t * E);
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  float bia[J], lv[J];
+  load_bias<J>(bias, E, lane, bia);
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    lv[j] = e < E ? s_l[e] : -INFINITY;
+  }
+  route_token<J>(lv, bia, lane, t, E, n_ffn, K, s_ws, topk_idx, topk_gate, zgate, counts,
+                 nffn_hist);
+}
+
+__global__ void k_zero2(int32_t* __restrict__ a, int na, int32_t* __restrict__ b, int nb) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < na; i += gridDim.x * blockDim.x) a[i] = 0;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nb; i += gridDim.x * blockDim.x) b[i] = 0;
+}
+
+template <int J>
+cudaError_t launch_topk_j(int T, int sm_count, cudaStream_t st, const float* src, int S,
+                          size_t slice, float* logits_out, const float* bias, int E, int n_ffn,
+                          int K, int32_t* idx, float* gate, int32_t* counts, int32_t* hist,
+                          float* zgate) {
+  if (T < 8 * sm_count && S > 4) {
+    // 16-byte rows: E a multiple of 4 and both bases 16-byte aligned
+    const int vec4 = (E % 4 == 0) && ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(logits_out)) & 15) == 0;
+    return launch_kernel(k_route_topk_sum<J>, T, kSumThreads, 0, st, 1, src, S, slice, logits_out,
+                         bias, T, E, n_ffn, K, idx, gate, counts, hist, zgate, vec4);
+  }
+  if (T < 8 * sm_count)
+    return launch_kernel(k_route_topk<J, 1>, T, 32, 0, st, 1, src, S, slice, logits_out, bias, T,
+                         E, n_ffn, K, idx, gate, counts, hist, zgate);
+  int blocks = (T + 7) / 8;
+  if (blocks > 8 * sm_count) blocks = 8 * sm_count;
+  return launch_kernel(k_route_topk<J, 8>, blocks, 256, 0, st, 1, src, S, slice, logits_out, bias,
+                       T, E, n_ffn, K, idx, gate, counts, hist, zgate);
+}
 }  // namespace
+
+bool route_topk_sums_slices(int T, int S, int sm_count) { return S <= 4 || T < 8 * sm_count; }
+
+cudaError_t launch_zero_counts(int32_t* counts, int E, int32_t* nffn_hist, int K, cudaStream_t st) {
+  const cudaError_t e = launch_kernel(k_zero2, (E + 255) / 256, 256, 0, st, 1, counts, E, nffn_hist,
+                                      K + 1);
+  count_launch();
+  return e;
+}
 
 cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const float* bias,
                               int T, int E, int n_ffn, int K, int32_t* topk_idx,
                               float* topk_gate, int32_t* counts, int32_t* nffn_hist,
                               float* zgate, int sm_count, cudaStream_t st) {
-  cudaError_t err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st);
-  if (err != cudaSuccess) return err;
-  err = cudaMemsetAsync(nffn_hist, 0, sizeof(int32_t) * (K + 1), st);
-  if (err != cudaSuccess) return err;
   const size_t slice = (size_t)T * E;
   const int J = (E + 31) / 32;
-#define MOE_TOPK_CASE(JJ)                                                                      \
-  if (J <= JJ) {                                                                               \
-    launch_topk_j<JJ>(T, sm_count, st, src, S, slice, logits_out, bias, E, n_ffn, K, topk_idx, \
-                      topk_gate, counts, nffn_hist, zgate);                                    \
+  cudaError_t err = cudaErrorInvalidValue;
+#define MOE_TOPK_CASE(JJ)                                                                     \
+  if (J <= JJ) {                                                                              \
+    err = launch_topk_j<JJ>(T, sm_count, st, src, S, slice, logits_out, bias, E, n_ffn, K,    \
+                            topk_idx, topk_gate, counts, nffn_hist, zgate);                   \
   } else
   MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4) MOE_TOPK_CASE(6)
   MOE_TOPK_CASE(8) MOE_TOPK_CASE(12) MOE_TOPK_CASE(16) MOE_TOPK_CASE(24) MOE_TOPK_CASE(32) {
@@ -381,7 +581,7 @@ cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const 
   }
 #undef MOE_TOPK_CASE
   count_launch();
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moe

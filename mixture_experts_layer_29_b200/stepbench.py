@@ -41,7 +41,7 @@ def main(argv=None) -> int:
                             ("n_zero", a.zero_experts)) if v is not None}
     cfg = cfg.with_(**kw) if kw else cfg
     dev = torch.device("cuda", 0)
-    need_ffn = a.step in ("ffn", "layer")
+    need_ffn = a.step in ("ffn", "combine", "layer")
     w = wl.draw_weights(cfg, dev, ffn=need_ffn)
     x = wl.draw_tokens(cfg, dev)
     logits_in = wl.draw_skewed_logits(cfg, dev) if cfg.skewed else None

@@ -225,3 +225,41 @@ def test_packed_router_weight_gives_the_same_routing(cuda_device, name, T):
     torch.cuda.synchronize()
     for a, c in zip(ref, (b.logits, b.topk_idx, b.topk_gate, b.counts, b.nffn_hist, b.zgate)):
         assert torch.equal(a, c)
+
+
+@pytest.mark.parametrize("name,T", [("proxy_bf16", 300), ("prefill_bf16", 300),
+                                    ("prefill_bf16", 2000)])
+def test_tied_scores_follow_expert_index(cuda_device, name, T):
+    """Logits on a coarse grid and a zero bias give exactly equal scores on both sides
+    (equal logits, equal softmax values): the picks must then follow the expert index,
+    on every token. Rows with all logits equal have E tied candidates (the fallback of the
+    candidate filter); the other rows have ties at and around the K-th score."""
+    cfg = wl.CONFIGS[name].with_(T=T)
+    g = torch.Generator().manual_seed(11)
+    L = torch.round(torch.randn(T, cfg.E, generator=g) * 2.0) / 2.0
+    L[::7] = 0.25                                     # all experts tied
+    case = gh.Case(cfg, ffn=False, logits=L.to("cuda"))
+    case.w.bias.zero_()
+    b = case.buffers()
+    case.route(b)
+    torch.cuda.synchronize()
+    r = orc.route(L.numpy(), np.zeros(cfg.E, np.float32), cfg.n_ffn, cfg.K)
+    np.testing.assert_array_equal(gh.host(b.topk_idx), r.topk_idx)
+    np.testing.assert_array_equal(gh.host(b.counts), r.counts)
+    np.testing.assert_array_equal(gh.host(b.nffn_hist), r.nffn_hist)
+    np.testing.assert_array_equal(gh.host(b.topk_idx)[::7], np.tile(np.arange(cfg.K), (len(L[::7]), 1)))
+
+
+@pytest.mark.parametrize("T", [128, 1000, 1500, 3000])
+def test_router_split_k_paths(cuda_device, T):
+    """The full-width router at batch sizes that take the different split-K paths (slices
+    summed inside the top-K kernel, by a separate kernel, or no split): logits within the
+    fp32 bound on a sample of rows, routing exact from the GPU's logits."""
+    cfg = wl.CONFIGS["prefill_bf16"].with_(T=T)
+    case = gh.Case(cfg, ffn=False, seed=5)
+    b = case.buffers()
+    case.route(b)
+    torch.cuda.synchronize()
+    rows = np.unique(np.r_[np.arange(0, T, max(1, T // 97)), T - 1])
+    gh.check_logits(case, b, rows)
+    gh.check_routing(case, b)
