@@ -31,12 +31,19 @@ Sources (page title, then the section or claim on that page):
            the fine-grained experts' outputs (ffn_out_scale here; its value is not printed).
   [zero]   "LongCat-Flash" blog, Key Innovations: zero-computation experts bypass
            computation for simple tokens.
+  [lbloss] "LongCat-Flash Technical Report" digest, Key claims, report §2.1.1 / §2.1.2
+           Eqs. 3-5: the zero-computation experts' share is held by a device-level
+           load-balance loss, DeepSeek-V3's balance loss extended so that all
+           zero-computation experts form one virtual group (the equations are not
+           printed).
 
 Readings where the pages are silent (the report's equations are not printed):
   softmax over all E experts; bias added to the float32 probability (not the logit);
   ties broken toward the lower expert index; gates not renormalised over the K picks;
   FFN experts are indices [0, n_ffn); SwiGLU experts W_down (silu(W_gate x) * W_up x);
-  PID in position form with per-expert frequency target target_ratio * K / n_ffn.
+  PID in position form with per-expert frequency target target_ratio * K / n_ffn;
+  load-balance loss as in lb_loss below (DeepSeek's f_i P_i form, device-level grouping
+  with one FFN expert per group and one group of every zero-computation expert).
 
 Parity pins: every function here is pinned in tests/test_oracle.py against closed forms,
 brute force, invariants or independent library routines; none is "parity unpinned".
@@ -51,7 +58,7 @@ import numpy as np
 __all__ = [
     "router_logits", "softmax_probs", "biased_scores", "select_topk", "near_tie_gap",
     "route", "permute", "swiglu_expert", "moe_layer_forward", "PidState", "pid_init",
-    "pid_update", "pid_stats", "RouteResult", "PermuteResult",
+    "pid_update", "pid_stats", "lb_loss", "RouteResult", "PermuteResult",
 ]
 
 
@@ -313,3 +320,36 @@ def pid_stats(counts, nffn_hist, T: int, K: int, n_ffn: int, err=None) -> np.nda
         out[6] = a.mean()
         out[7] = a.max()
     return out
+
+
+# ---------------------------------------------------------------------------------------
+# Device-level load-balance loss (forward value)
+# ---------------------------------------------------------------------------------------
+
+def lb_loss(logits, counts, n_ffn: int, K: int):
+    """Load-balance loss of one batch of T tokens over E = n_ffn + n_zero experts, and
+    the mean router probability of every expert.
+
+    [lbloss] names the loss without printing it; this follows DeepSeek's balance loss:
+      f_i = E * c_i / (K * T)      c_i = tokens that picked expert i (counts)
+      P_i = (1/T) sum_t p[t, i]     p = softmax over all E experts, float64
+    and its device-level form, in which experts are grouped and a group g contributes
+    (mean of f_i over g) * (sum of P_i over g). The groups are one per FFN expert and
+    one virtual group holding every zero-computation expert:
+      L = sum_{i < n_ffn} f_i P_i + mean_{i >= n_ffn}(f_i) * sum_{i >= n_ffn} P_i.
+    A perfectly balanced batch (c_i = K T / E, p = 1/E) gives L = 1. The weight of the
+    loss in the training objective is left to the caller. Returns (L, P) in float64.
+    """
+    L = np.asarray(logits, dtype=np.float64)
+    c = np.asarray(counts, dtype=np.float64)
+    T, E = L.shape
+    m = L.max(axis=1, keepdims=True)
+    ex = np.exp(L - m)
+    p = ex / ex.sum(axis=1, keepdims=True)
+    P = p.sum(axis=0) / T
+    f = E * c / (K * T)
+    loss = float((f[:n_ffn] * P[:n_ffn]).sum())
+    if E > n_ffn:
+        loss += float(f[n_ffn:].mean() * P[n_ffn:].sum())
+    return loss, P
+

@@ -340,6 +340,66 @@ def test_pid_stats_from_histogram_match_per_token_values():
     assert math.isclose(st[5], 1 - per_tok.sum() / (T * K), rel_tol=1e-12)
 
 
+# ----------------------------------------------------------------------------- load-balance loss
+
+@pytest.mark.parametrize("N,Z,K,T", [(4, 2, 3, 4), (16, 8, 4, 6), (8, 0, 2, 4), (6, 6, 4, 3)])
+def test_lb_loss_balanced_batch_is_one(N, Z, K, T):
+    """Uniform probabilities (p = 1/E) and counts K T / E on every expert: f_i = 1, so each
+    FFN expert adds 1/E and the zero group adds Z/E; the loss is exactly 1."""
+    E = N + Z
+    assert (K * T) % E == 0
+    loss, P = orc.lb_loss(np.zeros((T, E)), np.full(E, K * T // E), N, K)
+    assert abs(loss - 1.0) < 1e-12
+    np.testing.assert_allclose(P, 1.0 / E, rtol=1e-12)
+
+
+def test_lb_loss_worked_example_by_hand():
+    """Two tokens, two FFN and two zero experts, K = 2.
+    Token 0 logits (ln 4, ln 2, 0, 0): exp = (4, 2, 1, 1) / 8 -> p = (1/2, 1/4, 1/8, 1/8).
+    Token 1 logits (0, 0, ln 2, ln 4): p = (1/8, 1/8, 1/4, 1/2).
+    P = mean over the tokens = (5/16, 3/16, 3/16, 5/16); f_i = 4 c_i / (2 * 2) = c_i.
+    counts (2, 0, 1, 1): 2 * 5/16 + 0 + mean(1, 1) * (3/16 + 5/16) = 18/16.
+    counts (0, 2, 2, 0): 0 + 2 * 3/16 + mean(2, 0) * 8/16 = 14/16."""
+    L = np.array([[math.log(4), math.log(2), 0, 0], [0, 0, math.log(2), math.log(4)]])
+    loss, P = orc.lb_loss(L, [2, 0, 1, 1], 2, 2)
+    assert abs(loss - 18 / 16) < 1e-12
+    np.testing.assert_allclose(P, [5 / 16, 3 / 16, 3 / 16, 5 / 16], rtol=1e-12)
+    loss2, _ = orc.lb_loss(L, [0, 2, 2, 0], 2, 2)
+    assert abs(loss2 - 14 / 16) < 1e-12
+
+
+def test_lb_loss_zero_experts_form_one_virtual_group():
+    """Moving picks between zero experts leaves the loss unchanged (one group); moving them
+    between FFN experts does not. With a single zero expert every group is a singleton
+    and the loss is DeepSeek's plain balance loss sum_i f_i P_i."""
+    g = rng(5)
+    T, N, Z, K = 50, 6, 4, 3
+    L = g.standard_normal((T, N + Z)) * 2
+    c = np.array([20, 10, 5, 5, 10, 0, 40, 20, 30, 10])
+    base, _ = orc.lb_loss(L, c, N, K)
+    c_zero_moved = c.copy(); c_zero_moved[6:] = [0, 50, 50, 0]
+    assert abs(orc.lb_loss(L, c_zero_moved, N, K)[0] - base) < 1e-12
+    c_ffn_moved = c.copy(); c_ffn_moved[:6] = [0, 0, 0, 0, 0, 50]
+    assert abs(orc.lb_loss(L, c_ffn_moved, N, K)[0] - base) > 1e-3
+    # Z = 1: singletons only
+    L1 = L[:, : N + 1]
+    c1 = c[: N + 1]
+    p = scipy.special.softmax(L1, axis=1)
+    plain = ((N + 1) * c1 / (K * T) * p.mean(axis=0)).sum()
+    assert abs(orc.lb_loss(L1, c1, N, K)[0] - plain) < 1e-12
+
+
+def test_lb_loss_collapsed_routing_reaches_E():
+    """Every token sends its only pick (K = 1) to expert 0 with p_0 -> 1: f_0 = E, P_0 = 1,
+    every other term 0, so the loss is E (its maximum)."""
+    T, N, Z = 16, 5, 3
+    L = np.zeros((T, N + Z)); L[:, 0] = 60.0
+    c = np.zeros(N + Z, int); c[0] = T
+    loss, P = orc.lb_loss(L, c, N, 1)
+    assert abs(loss - (N + Z)) < 1e-9
+    assert abs(P[0] - 1) < 1e-12
+
+
 # ----------------------------------------------------------------------------- pages' numbers
 
 def test_activated_parameter_identity_from_the_pages():
@@ -418,4 +478,32 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(orc, "pid_update", bad_pid)
     with pytest.raises(AssertionError):
         test_pid_constant_error_closed_form()
+    monkeypatch.setattr(orc, "pid_update", orig_pid)
+
+    # 6. load-balance loss: the zero group's f summed instead of averaged -> the
+    #    balanced-batch pin breaks; P averaged over experts instead of tokens -> the
+    #    worked example breaks
+    orig_lb = orc.lb_loss
+
+    def lb_sum(logits, counts, n_ffn, K):
+        loss, P = orig_lb(logits, counts, n_ffn, K)
+        E = np.asarray(logits).shape[1]
+        f = E * np.asarray(counts, float) / (K * np.asarray(logits).shape[0])
+        return loss + (f[n_ffn:].sum() - f[n_ffn:].mean()) * P[n_ffn:].sum(), P
+    monkeypatch.setattr(orc, "lb_loss", lb_sum)
+    with pytest.raises(AssertionError):
+        test_lb_loss_balanced_batch_is_one(4, 2, 3, 4)
+    monkeypatch.setattr(orc, "lb_loss", orig_lb)
+
+    def lb_axis(logits, counts, n_ffn, K):
+        Lg = np.asarray(logits, float)
+        p = np.exp(Lg - Lg.max(1, keepdims=True)); p /= p.sum(1, keepdims=True)
+        P = np.resize(p.mean(axis=1), Lg.shape[1])          # wrong axis
+        E = Lg.shape[1]
+        f = E * np.asarray(counts, float) / (K * Lg.shape[0])
+        return float((f[:n_ffn] * P[:n_ffn]).sum() + f[n_ffn:].mean() * P[n_ffn:].sum()), P
+    monkeypatch.setattr(orc, "lb_loss", lb_axis)
+    with pytest.raises(AssertionError):
+        test_lb_loss_worked_example_by_hand()
+    monkeypatch.setattr(orc, "lb_loss", orig_lb)
     monkeypatch.setattr(orc, "pid_update", orig_pid)
