@@ -45,8 +45,7 @@ UNIT = "tokens/s"
 PID_GAINS = (0.01, 0.001, 0.0, 8 / 12)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-GEMM_SOURCES = [os.path.join(ROOT, "mixture_experts_layer_29_b200", "csrc", f)
-                for f in ("gemm_tc.cu", "common.cuh")]
+CSRC = os.path.join(ROOT, "mixture_experts_layer_29_b200", "csrc")
 
 
 # ------------------------------------------------------------------------------ helpers
@@ -60,25 +59,27 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def gemm_source_hash() -> str:
+def source_hash(files) -> str:
+    """Hash of the named csrc/ files (the traffic figures hold only for the code they were
+    taken on)."""
     h = hashlib.sha256()
-    for p in GEMM_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def traffic_per_launch(workload: str):
-    """DRAM bytes (read + write) per grouped-FFN call from the committed ncu summary, or
-    None when the GEMM source changed since the counters were taken."""
+def traffic_entry(key: str):
+    """The committed ncu DRAM figures for `key` (see profiles/traffic.json), or None when
+    any of the sources they were taken on changed since."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
-    e = d.get(workload)
-    if not e or e.get("gemm_source_sha") != gemm_source_hash():
+    e = d.get(key)
+    if not e or e.get("source_sha") != source_hash(e.get("sources", [])):
         return None
-    return e.get("dram_bytes_per_call")
+    return e
 
 
 class ClockSampler:
@@ -291,7 +292,8 @@ def run_ours(args):
     pk, pk_kind = peaks()
     achieved = flops_ffn / (ffn_ms / 1e3) / 1e12
     peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    traffic = traffic_per_launch(args.workload)
+    te = traffic_entry(f"{args.workload}:grouped_ffn")
+    traffic = te["dram_bytes_per_call"] if te else None
     roofline = {"bound": "tensor", "kernel": "grouped_ffn (gate/up + down tcgen05 GEMMs)",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -313,6 +315,8 @@ def run_ours(args):
         dbytes = (touched * 3.0 * dcfg.H * dcfg.I * 2 + dcfg.E * dcfg.H * 4
                   + 2 * dcfg.T * dcfg.H * 2)
         dstep = dms / dsteps
+        dte = traffic_entry("decode_bf16:step")
+        dtraffic = dte["dram_bytes_per_step"] if dte else None
         dach = dbytes / (dstep / 1e3) / 1e9
         hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         decode = {"workload": "decode_bf16", "value": round(dcfg.T * dsteps * world / (dms / 1e3), 1),
@@ -321,7 +325,7 @@ def run_ours(args):
                   "roofline": {"bound": "hbm", "scope": "whole layer step",
                                "achieved": round(dach, 1), "peak": hbm, "unit": "GB/s",
                                "frac": round(dach / hbm, 4), "frac_of_8TBs": round(dach / 8000, 4),
-                               "traffic": None, "algorithmic_bytes_per_step": dbytes,
+                               "traffic": dtraffic, "algorithmic_bytes_per_step": dbytes,
                                "touched_experts": touched, "peak_kind": pk_kind}}
 
     # ---- end to end through the public API from pinned host memory ----------------------

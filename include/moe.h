@@ -223,6 +223,26 @@ int moe_pid_bias_update(const moe_pid_t* pid, const moe_shape_t* shape, const in
                         const int32_t* nffn_hist, float* bias, float* pid_state,
                         float* stats_out, void* stream);
 
+/* Device-level load-balance loss of one batch, forward value (LongCat-Flash Technical
+ * Report digest, Key claims, report §2.1.1 / §2.1.2 Eqs. 3-5: DeepSeek-V3's balance loss
+ * with every zero-computation expert in one virtual group; the equations are not
+ * printed, so this is the form read from that description):
+ *   f_i = E * counts[i] / (K * T),   P_i = (1/T) * sum_t softmax(logits[t])[i]
+ *   loss = sum_{i < n_ffn} f_i * P_i + mean_{i >= n_ffn}(f_i) * sum_{i >= n_ffn} P_i
+ * A balanced batch gives 1; the loss weight is the caller's. Sums in double, fixed
+ * order (deterministic); T == 0 gives loss 0.
+ *   logits     device [T, E] fp32             the router logits (moe_route's logits_out
+ *                                             or the logits_in it was given)
+ *   counts     device [E] int32               moe_route's counts for the same batch
+ *   prob_mean  device [E] fp32 or NULL        receives P
+ *   loss       device [1] fp32                receives the loss
+ *   ws         device scratch, >= moe_scratch_size bytes
+ * Errors: MOE_ERR_INVALID_ARG for a NULL pointer, MOE_ERR_ALIGNMENT for a device pointer
+ * that is not 16-byte aligned (loss needs none), MOE_ERR_WORKSPACE for a short workspace,
+ * MOE_ERR_CUDA for a failed launch. */
+int moe_lb_loss(const moe_shape_t* shape, const float* logits, const int32_t* counts,
+                float* prob_mean, float* loss, void* ws, size_t ws_bytes, void* stream);
+
 /* The whole layer: moe_route, moe_permute, moe_grouped_ffn and moe_combine on `stream`,
  * with every intermediate in `ws` (>= moe_workspace_size bytes). topk_idx, topk_gate,
  * counts and nffn_hist are returned so the caller can chain moe_pid_bias_update.

@@ -82,6 +82,7 @@ _SIGS = {
     "moe_permute_static_scratch": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 10 + [_P]),
     "moe_router_pack": (ctypes.c_int, [ctypes.POINTER(Shape), _P, _P, _P]),
     "moe_route_packed": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 10 + [_SZ, _P]),
+    "moe_lb_loss": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 5 + [_SZ, _P]),
 }
 
 _lib = None
@@ -236,6 +237,12 @@ def pid_bias_update(pid: Pid, shape, counts, nffn_hist, bias, pid_state, stats_o
     _check(lib().moe_pid_bias_update(ctypes.byref(pid), ctypes.byref(shape), ptr(counts),
                                      ptr(nffn_hist), ptr(bias), ptr(pid_state), ptr(stats_out),
                                      _stream(stream)), "moe_pid_bias_update")
+
+
+def lb_loss(shape, logits, counts, prob_mean, loss, ws, stream=None):
+    """Load-balance loss of the batch (moe_lb_loss): loss [1] fp32, prob_mean [E] or None."""
+    _check(lib().moe_lb_loss(ctypes.byref(shape), ptr(logits), ptr(counts), ptr(prob_mean),
+                             ptr(loss), ptr(ws), _nbytes(ws), _stream(stream)), "moe_lb_loss")
 
 
 def forward(shape, x, w_router, logits_in, bias, w_gate_up, w_down, out, topk_idx, topk_gate,

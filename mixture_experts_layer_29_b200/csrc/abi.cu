@@ -60,7 +60,7 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
   // scratch (all step calls)
-  size_t status, masks, crel, ecount, lpart, scratch_end;
+  size_t status, masks, crel, ecount, lbpart, lpart, scratch_end;
   // intermediates (moe_forward)
   size_t logits, zgate, offsets, perm, rowof, rowgate, xperm, h, yperm, outacc, total;
 };
@@ -93,6 +93,7 @@ Layout layout_of(const moe_shape_t& s) {
   L.masks = o;   o = align_up(o + N * nchunk * 4);
   L.crel = o;    o = align_up(o + N * nchunk * 4);
   L.ecount = o;  o = align_up(o + N * 4);
+  L.lbpart = o;  o = align_up(o + lb_partial_bytes(s.T, (int)E));
   L.lpart = o;   // router scratch: split weight + partials (bf16) or SIMT partials (fp32)
   o = align_up(o + (s.dtype == MOE_BF16 ? router_tc_scratch_bytes(s.T, (int)E, s.H)
                                         : router_partial_bytes(s.T, (int)E, s.H, 0)));
@@ -385,6 +386,22 @@ int moe_pid_bias_update(const moe_pid_t* pid, const moe_shape_t* shape, const in
   return cuda_rc(launch_pid_update(*pid, counts, nffn_hist, bias, pid_state, stats_out, shape->T,
                                    shape->K, shape->n_ffn, shape->n_ffn + shape->n_zero,
                                    as_stream(stream)));
+}
+
+int moe_lb_loss(const moe_shape_t* shape, const float* logits, const int32_t* counts,
+                float* prob_mean, float* loss, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_shape(shape));
+  MOE_TRY(check_ptrs({counts, ws}));
+  MOE_TRY(check_opt({prob_mean}));
+  if (!loss) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0) MOE_TRY(check_ptrs({logits}));
+  const Layout L = layout_of(*shape);
+  if (ws_bytes < L.scratch_end) return MOE_ERR_WORKSPACE;
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  return cuda_rc(launch_lb_loss(logits, counts, shape->T, shape->n_ffn + shape->n_zero,
+                                shape->n_ffn, shape->K, at<double>(ws, L.lbpart), prob_mean, loss,
+                                as_stream(stream)));
 }
 
 int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,

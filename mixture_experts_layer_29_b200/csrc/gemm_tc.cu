@@ -61,6 +61,10 @@ struct alignas(1024) SharedStorage {
   int abort_flag;
   int offs[kMaxExperts + 1];
   int toff[kMaxExperts + 1];
+  // router logits: each epilogue warp turns 32 rows x 16 columns around here so that its
+  // global stores cover whole 64-byte row segments (row stride 20 floats: 16-byte aligned
+  // and conflict-free for the row-wise float4 writes)
+  float epi_stage[kEpiWarps][32][20];
 };
 
 struct GemmArgs {
@@ -122,8 +126,10 @@ __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + _
 // Epilogue of one 128 x 256 accumulator of the expert GEMMs for one thread: its TMEM lane
 // (row) and its half of the columns (gate/up: gate columns [64h, 64h+64) with the matching
 // up columns; down: columns [128h, 128h+128)).
+// stg: the warp's 32 x 80-byte staging rows (deterministic down store: each 32 x 32 chunk
+// goes through them so that a warp store covers 8 rows x 64 bytes).
 __device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t, uint32_t tbase,
-                                                int row, int half) {
+                                                int row, int half, float (*stg)[20], int lane) {
   const bool valid = row < t.row_end;
   if (g.mode == kGateUp) {
     __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(g.out);
@@ -163,10 +169,9 @@ __device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t
     tmem_ld_32x32b_x32(tbase + c, yr);
     tmem_ld_wait();
     const int col = t.nt * BN + c;
-    if (!valid || col >= g.n_valid) continue;
     if (g.mode == kDownStore) {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
-                                            (size_t)row * g.ld_out + col);
+      // this lane's row as 64 bytes of bf16 into the staging row, then 16 bytes per lane
+      // of rows 8i + lane/4 out to global memory
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
         uint32_t w[4];
@@ -175,9 +180,25 @@ __device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t
           const int j = v * 8 + i * 2;
           w[i] = pack_bf16x2(__uint_as_float(yr[j]), __uint_as_float(yr[j + 1]));
         }
-        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(&stg[lane][4 * v]) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-    } else {
+      __syncwarp();
+      if (col < g.n_valid) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 8 * i + (lane >> 2), ch = lane & 3;
+          const int grow = row - lane + r;
+          if (grow < t.row_end)
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                      (size_t)grow * g.ld_out + col + 8 * ch) =
+                *reinterpret_cast<const uint4*>(&stg[r][4 * ch]);
+        }
+      }
+      __syncwarp();
+      continue;
+    }
+    if (!valid || col >= g.n_valid) continue;
+    {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) +
                                               (size_t)tok * g.ld_out + col);
 #pragma unroll
@@ -391,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) sum[c + i] = __fadd_rn(sum[c + i], __uint_as_float(v[i]));
           }
         } else {
-          epilogue_expert(g, t, tbase, row, half);
+          epilogue_expert(g, t, tbase, row, half, s.epi_stage[warp - 2], lane);
         }
         tc_fence_before();
         mbar_arrive(&s.tempty[acc]);
@@ -399,21 +420,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (acc == 0) acc_phase ^= 1u;
       }
       if constexpr (LOGITS) {
-       if (ok && row < t.row_end) {
-        const int col0 = t.nt * BN + 128 * half;
-        float* dst = static_cast<float*>(g.out) + t.split * g.split_stride +
-                     (size_t)row * g.ld_out + col0;
-        if (col0 + 128 <= g.n_valid && (g.ld_out & 3) == 0) {
+        if (ok) {
+          // 32 rows x 16 columns at a time through shared memory: lane l then stores
+          // row 8i + l/4, columns 4(l%4)..+3, so a warp store covers 8 rows x 64 bytes
+          float (*stg)[20] = s.epi_stage[warp - 2];
+          float* outp = static_cast<float*>(g.out) + t.split * g.split_stride;
+          const int col0 = t.nt * BN + 128 * half;
+          const bool vec = (g.ld_out & 3) == 0 && (reinterpret_cast<uintptr_t>(g.out) & 15) == 0;
 #pragma unroll
-          for (int v = 0; v < 32; ++v)
-            reinterpret_cast<float4*>(dst)[v] =
-                make_float4(sum[4 * v], sum[4 * v + 1], sum[4 * v + 2], sum[4 * v + 3]);
-        } else {
+          for (int c = 0; c < 128; c += 16) {
 #pragma unroll
-          for (int v = 0; v < 128; ++v)
-            if (col0 + v < g.n_valid) dst[v] = sum[v];
+            for (int v = 0; v < 4; ++v)
+              *reinterpret_cast<float4*>(&stg[lane][4 * v]) =
+                  make_float4(sum[c + 4 * v], sum[c + 4 * v + 1], sum[c + 4 * v + 2],
+                              sum[c + 4 * v + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = 8 * i + (lane >> 2), cc = 4 * (lane & 3);
+              const float4 val = *reinterpret_cast<const float4*>(&stg[r][cc]);
+              const int grow = t.row0 + q * 32 + r;
+              const int gcol = col0 + c + cc;
+              if (grow < t.row_end) {
+                float* d = outp + (size_t)grow * g.ld_out + gcol;
+                if (vec && gcol + 4 <= g.n_valid) {
+                  *reinterpret_cast<float4*>(d) = val;
+                } else {
+                  const float vv[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+                  for (int j = 0; j < 4; ++j)
+                    if (gcol + j < g.n_valid) d[j] = vv[j];
+                }
+              }
+            }
+            __syncwarp();
+          }
         }
-       }
       }
     }
   }
@@ -458,6 +500,7 @@ struct alignas(1024) PairStorage {
   int abort_flag;
   int offs[kMaxExperts + 1];
   int toff[kMaxExperts + 1];    // prefix of ceil(count / 256)
+  float epi_stage[kEpiWarps][32][20];   // deterministic down store (see epilogue_expert)
 };
 
 __device__ __forceinline__ Tile decode_pair_tile(const PairStorage& s, const GemmArgs& g, int tile) {
@@ -611,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_expert(g, t, tbase, t.row0 + row_in_tile, half);
+      epilogue_expert(g, t, tbase, t.row0 + row_in_tile, half, s.epi_stage[warp - 2], lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
@@ -774,7 +817,15 @@ __global__ void __launch_bounds__(256) k_split_router_weight(const float4* __res
 // Router logits: 128 x 256 tiles, K = 3H (the three weight parts); the tensor cores
 // accumulate kRouterChunk k-blocks at a time and the epilogue sums the chunks in fp32.
 constexpr int kRouterChunk = 6;
-constexpr int kRouterMinSplit = 12;   // k-blocks per split at least (two chunks)
+// k-blocks per split at least (MOE_B200_ROUTER_MINSPLIT overrides it, for measurements)
+int router_min_split() {
+  static const int v = [] {
+    const char* e = getenv("MOE_B200_ROUTER_MINSPLIT");
+    const int n = e ? atoi(e) : 0;
+    return n >= 1 && n <= 1024 ? n : 12;
+  }();
+  return v;
+}
 
 int router_tc_splitk(int T, int E, int H, int sm_count) {
   if (sm_count > 160) sm_count = 160;
@@ -782,7 +833,7 @@ int router_tc_splitk(int T, int E, int H, int sm_count) {
   const int kblocks = 3 * H / BK;
   if (tiles <= 0 || tiles >= sm_count) return 1;   // a full wave already: no partial slices
   long s = (2L * sm_count + tiles - 1) / tiles;
-  long smax = kblocks / kRouterMinSplit;
+  long smax = kblocks / router_min_split();
   if (smax > 64) smax = 64;
   if (s > smax) s = smax;
   if (s < 1) s = 1;

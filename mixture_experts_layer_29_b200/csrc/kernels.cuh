@@ -70,6 +70,11 @@ cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const 
 bool route_topk_sums_slices(int T, int S, int sm_count);
 cudaError_t launch_zero_counts(int32_t* counts, int E, int32_t* nffn_hist, int K, cudaStream_t st);
 
+// ---- load-balance loss -------------------------------------------------------------------
+size_t lb_partial_bytes(int T, int E);
+cudaError_t launch_lb_loss(const float* logits, const int32_t* counts, int T, int E, int n_ffn,
+                           int K, double* part, float* prob_mean, float* loss, cudaStream_t st);
+
 // ---- permutation ------------------------------------------------------------------------
 cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, const float* zgate,
                            const void* x, int x_is_bf16, int T, int H, int n_ffn, int E, int K,

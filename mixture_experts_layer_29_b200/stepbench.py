@@ -28,7 +28,7 @@ def main(argv=None) -> int:
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--workload", default="prefill_bf16", choices=sorted(wl.CONFIGS))
     ap.add_argument("--step", default="route", choices=STEPS)
-    ap.add_argument("--combine", default="fused", choices=["fused", "deterministic"])
+    ap.add_argument("--combine", default="deterministic", choices=["fused", "deterministic"])
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--ffn-experts", type=int, default=None)
     ap.add_argument("--zero-experts", type=int, default=None)

@@ -17,7 +17,7 @@ def L():
 
 def test_library_exports_every_declared_function(L):
     names = abi.header_functions()
-    assert len(names) == 15
+    assert len(names) == 16
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(abi._SIGS)
@@ -66,6 +66,7 @@ def test_workspace_sizes_cover_the_intermediates(L):
             need = rows * cfg.H * esz + rows * cfg.I * esz + cfg.T * cfg.E * 4
             need += rows * cfg.H * esz if comb == "deterministic" else cfg.T * cfg.H * 4
             assert scratch >= 256 + 2 * cfg.n_ffn * ((cfg.T + 31) // 32) * 4
+            assert scratch >= ((cfg.T + 63) // 64) * cfg.E * 8      # load-balance partials
             assert total >= scratch + need, name
     # the full-shape prefill workspace stays a few GB
     s = abi.shape_of(wl.CONFIGS["prefill_bf16"])
@@ -98,6 +99,11 @@ def test_host_checks_run_before_any_device_access(L):
     s0 = _shape(T=0)
     assert L.moe_pid_bias_update(ctypes.byref(pid), ctypes.byref(s0), good, good, good, good,
                                  None, None) == -1
+    # load-balance loss: null counts or loss, unaligned logits, short workspace
+    assert L.moe_lb_loss(ctypes.byref(s), good, None, None, good, good, ws_n, None) == -1
+    assert L.moe_lb_loss(ctypes.byref(s), good, good, None, None, good, ws_n, None) == -1
+    assert L.moe_lb_loss(ctypes.byref(s), bad, good, None, good, good, ws_n, None) == -3
+    assert L.moe_lb_loss(ctypes.byref(s), good, good, None, good, good, ws_n - 1, None) == -5
     assert L.moe_read_device_status(None, 256, None, None) == -1
 
 
