@@ -217,10 +217,16 @@ class Stepper:
 PHASES = ["route", "permute", "grouped_ffn", "combine", "pid"]
 
 
-def timed_loop(st: Stepper, steps: int, warmup: int, dist_on: bool):
+def timed_loop(st: Stepper, steps: int, warmup: int, dist_on: bool, phases: bool = True):
+    """Time `steps` steps (after `warmup`) between CUDA events on the launching stream.
+    phases=True also records an event between the layer's calls for the per-call
+    breakdown; the step time itself is taken without them (phases=False), because an
+    event between two kernels makes the second wait for the first to finish instead of
+    starting as a programmatic dependent launch."""
     for _ in range(warmup):
         st.step()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)] \
+        if phases else None
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist_on:
         torch.distributed.barrier()
@@ -228,7 +234,7 @@ def timed_loop(st: Stepper, steps: int, warmup: int, dist_on: bool):
     n0 = abi.launch_count()
     start.record()
     for k in range(steps):
-        st.step(evs[k])
+        st.step(evs[k] if phases else None)
     end.record()
     torch.cuda.synchronize()
     launches = abi.launch_count() - n0
@@ -236,8 +242,66 @@ def timed_loop(st: Stepper, steps: int, warmup: int, dist_on: bool):
         torch.distributed.barrier()
     total = start.elapsed_time(end)
     per = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps)]
-           for i, p in enumerate(PHASES)}
+           for i, p in enumerate(PHASES)} if phases else None
     return total, per, launches
+
+
+def scmoe_overlap(st: Stepper, device, seed: int, iters: int, warmup: int) -> dict:
+    """The layer's dense SwiGLU FFN (intermediate 12288) beside its MoE step, on one GPU.
+
+    The shortcut-connected MoE (LongCat-Flash Technical Report digest, Key claims, report
+    §2.2) runs a layer's dense FFN while its MoE is under way; across GPUs that hides the
+    dispatch / combine all-to-all, and here the closest analogue is two streams: the MoE
+    step on the launching stream, the dense FFN (the grouped-FFN kernels with one group) on
+    a second one. Times the MoE step alone, the dense FFN alone, both on one stream, and
+    both on two streams, each the mean over `iters` after `warmup`."""
+    cfg = st.cfg
+    wgu, wd = wl.draw_dense_ffn(cfg, device, seed=seed)
+    dense = abi.DenseFFN(cfg.T, wgu, wd)
+    xd = torch.zeros(cfg.T + 128, cfg.H, dtype=torch.bfloat16, device=device)
+    xd[: cfg.T].copy_(st.x)
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream(device=device)
+
+    def timed(fn) -> float:
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(main)
+        for _ in range(iters):
+            fn()
+        e1.record(main)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    def concurrent():
+        fork = torch.cuda.Event()
+        fork.record(main)
+        side.wait_event(fork)
+        with torch.cuda.stream(side):
+            dense.forward(xd)
+        st.step()
+        join = torch.cuda.Event()
+        join.record(side)
+        main.wait_event(join)
+
+    t_moe = timed(st.step)
+    t_dense = timed(lambda: dense.forward(xd))
+    t_serial = timed(lambda: (st.step(), dense.forward(xd)))
+    t_conc = timed(concurrent)
+    flops = 6.0 * cfg.T * cfg.H * wl.DENSE_FFN_INTER
+    saved = t_serial - t_conc
+    out = {"tokens": cfg.T, "dense_inter": wl.DENSE_FFN_INTER,
+           "moe_ms": round(t_moe, 4), "dense_ffn_ms": round(t_dense, 4),
+           "dense_ffn_tflops": round(flops / (t_dense / 1e3) / 1e12, 1),
+           "one_stream_ms": round(t_serial, 4), "two_streams_ms": round(t_conc, 4),
+           "saved_ms": round(saved, 4),
+           "saved_of_shorter": round(saved / min(t_moe, t_dense), 4)}
+    del dense, wgu, wd, xd
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
 
 
 def max_over_ranks(v: float, dist_on: bool) -> float:
@@ -279,7 +343,8 @@ def run_ours(args):
     st = Stepper(cfg, w, x, logits_in, args.combine, device)
 
     with ClockSampler(local) as clk:
-        total_ms, per, launches = timed_loop(st, args.steps, args.warmup, dist_on)
+        total_ms, _, launches = timed_loop(st, args.steps, args.warmup, dist_on, phases=False)
+        _, per, _ = timed_loop(st, min(args.steps, 30), 0, dist_on, phases=True)
     total_ms = max_over_ranks(total_ms, dist_on)
     ms_step = total_ms / args.steps
     tokens = cfg.T * args.steps * world
@@ -308,7 +373,8 @@ def run_ours(args):
         dx = wl.draw_tokens(dcfg, device, seed=seed)
         dst = Stepper(dcfg, w, dx, None, args.combine, device)
         dsteps = max(args.steps, 20)
-        dms, dper, _ = timed_loop(dst, dsteps, max(args.warmup, 3), dist_on)
+        dms, _, _ = timed_loop(dst, dsteps, max(args.warmup, 3), dist_on, phases=False)
+        _, dper, _ = timed_loop(dst, min(dsteps, 30), 0, dist_on, phases=True)
         dms = max_over_ranks(dms, dist_on)
         dc = dst.b.counts.cpu().numpy()
         touched = int((dc[: dcfg.n_ffn] > 0).sum())
@@ -354,6 +420,12 @@ def run_ours(args):
                "note": "moe_forward via MoELayer.forward_host: pinned x in, out back, each step"}
         del layer
 
+    overlap = None
+    if not args.no_overlap and not dist_on and cfg.dtype == wl.BF16:
+        overlap = {"prefill": scmoe_overlap(st, device, seed, 20, 3)}
+        if decode is not None:
+            overlap["decode"] = scmoe_overlap(dst, device, seed, 50, 5)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rng = np.random.default_rng(0)
@@ -381,6 +453,7 @@ def run_ours(args):
         "breakdown_ms": {p: round(float(np.mean(v)), 4) for p, v in per.items()},
         "roofline": roofline,
         "decode": decode,
+        "scmoe_overlap": overlap,
         "e2e": e2e,
         "gpu_launches": int(launches) * world,
         "cpu_baseline": cpu,
@@ -453,6 +526,8 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="skip the dense-FFN-beside-MoE (two streams) measurement")
     args = ap.parse_args(argv)
     if args.impl == "ours":
         args.warmup = max(args.warmup, 3)     # timing rule: at least 3 untimed steps

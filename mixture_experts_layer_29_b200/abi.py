@@ -324,6 +324,34 @@ def run_steps(b: StepBuffers, x, w_router, logits_in, bias, w_gate_up, w_down, s
     return b.out
 
 
+class DenseFFN:
+    """A dense SwiGLU FFN, y = W_d (silu(W_g x) * (W_u x)) for every token, on the grouped-FFN
+    kernels: moe_grouped_ffn with one group that holds all T tokens (deterministic store,
+    so y is written per row). It is the dense FFN a LongCat-Flash layer runs beside its MoE
+    (the shortcut-connected MoE overlaps the two).
+
+    forward(x_padded) reads rows [0, T) of x_padded, a [T + 128, H] buffer whose last 128
+    rows the GEMM tiles may read but never use; it returns a [T, H] view of y."""
+
+    def __init__(self, T: int, w_gate_up, w_down):
+        _, two_i, H = w_gate_up.shape
+        self.T, self.H, self.I = T, H, two_i // 2
+        assert tuple(w_down.shape) == (1, H, self.I)
+        dev = w_gate_up.device
+        self.shape = make_shape(T, H, self.I, 1, 0, 1, "bf16", "deterministic")
+        self.w_gate_up, self.w_down = w_gate_up, w_down
+        self.ws = torch.zeros(max(scratch_size(self.shape), 256), dtype=torch.uint8, device=dev)
+        self.offsets = torch.tensor([0, T], dtype=torch.int32, device=dev)
+        self.h = torch.empty(T + 128, self.I, dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty(T + 128, H, dtype=torch.bfloat16, device=dev)
+
+    def forward(self, x_padded, stream=None):
+        assert x_padded.shape[0] >= self.T + 128 and x_padded.shape[1] == self.H
+        grouped_ffn(self.shape, x_padded, x_padded, self.offsets, self.w_gate_up, self.w_down,
+                    None, None, self.h, self.y, None, self.ws, stream)
+        return self.y[: self.T]
+
+
 class MoELayer:
     """One LongCat-Flash MoE layer on the GPU: weights plus a preallocated workspace.
 

@@ -132,6 +132,26 @@ def draw_weights(cfg: MoEConfig, device="cpu", seed: int | None = None,
     return LayerWeights(w_router, bias, w_gate_up, w_down)
 
 
+# The dense FFN that sits beside the MoE in a LongCat-Flash layer (report §2.4 Model
+# Configurations: dense-FFN intermediate 12288; the shortcut-connected MoE of report §2.2
+# runs it while the MoE's dispatch and combine are under way).
+DENSE_FFN_INTER = 12288
+
+
+def draw_dense_ffn(cfg: MoEConfig, device="cpu", seed: int | None = None,
+                   inter: int = DENSE_FFN_INTER):
+    """A dense SwiGLU FFN of the layer's width: (w_gate_up [1, 2*inter, H], w_down
+    [1, H, inter]) ~ N(0, w_std^2), laid out as one expert of the grouped-FFN weights."""
+    seed = cfg.seed if seed is None else seed
+    g = _gen(device, seed * 7919 + 5)
+    dt = torch_dtype(cfg)
+    w_gate_up = torch.empty(1, 2 * inter, cfg.H, dtype=dt, device=device)
+    w_down = torch.empty(1, cfg.H, inter, dtype=dt, device=device)
+    w_gate_up.normal_(0.0, cfg.w_std, generator=g)
+    w_down.normal_(0.0, cfg.w_std, generator=g)
+    return w_gate_up, w_down
+
+
 def draw_tokens(cfg: MoEConfig, device="cpu", seed: int | None = None) -> torch.Tensor:
     """Draw the token activations x [T, H] ~ N(0, 1) in the layer's dtype."""
     seed = cfg.seed if seed is None else seed
