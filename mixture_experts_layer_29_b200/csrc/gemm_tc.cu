@@ -90,6 +90,7 @@ struct GemmArgs {
   long long split_stride;   // elements between the outputs of consecutive splits
   const int32_t* gather_tok;  // non-null: A row r is row gather_tok[r] of A's tensor
   ZeroSpec zero;              // buffers cleared after the dependency wait
+  int half_tiles;             // pair kernel: tails of at most 128 rows run as M = 128
 };
 
 struct Tile {
@@ -123,92 +124,110 @@ __device__ __forceinline__ int chunk_len(const GemmArgs& g, const Tile& t) {
 
 __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
-// Epilogue of one 128 x 256 accumulator of the expert GEMMs for one thread: its TMEM lane
-// (row) and its half of the columns (gate/up: gate columns [64h, 64h+64) with the matching
-// up columns; down: columns [128h, 128h+128)).
-// stg: the warp's 32 x 80-byte staging rows (deterministic down store: each 32 x 32 chunk
-// goes through them so that a warp store covers 8 rows x 64 bytes).
-__device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t, uint32_t tbase,
-                                                int row, int half, float (*stg)[20], int lane) {
-  const bool valid = row < t.row_end;
-  if (g.mode == kGateUp) {
-    __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(g.out);
-#pragma unroll 1
-    for (int c = 64 * half; c < 64 * half + 64; c += 32) {
-      uint32_t gr[32], ur[32];
-      tmem_ld_32x32b_x32(tbase + c, gr);
-      tmem_ld_32x32b_x32(tbase + BM + c, ur);
-      tmem_ld_wait();
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(hout + (size_t)row * g.ld_out + t.nt * BM + c);
+// ---- epilogue pieces of the expert GEMMs (one thread = one TMEM lane = one row) ---------
+// gate/up: 32 columns of h = silu(G) * U from the gate accumulator columns at tbase + gcol
+// and the up columns at tbase + ucol; h columns [oc, oc + 32) of the tile's 128.
+__device__ __forceinline__ void epi_gateup_chunk(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                                 int row, int gcol, int ucol, int oc) {
+  uint32_t gr[32], ur[32];
+  tmem_ld_32x32b_x32(tbase + gcol, gr);
+  tmem_ld_32x32b_x32(tbase + ucol, ur);
+  tmem_ld_wait();
+  if (row >= t.row_end) return;
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                        (size_t)row * g.ld_out + t.nt * BM + oc);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint32_t w[4];
+  for (int v = 0; v < 4; ++v) {
+    uint32_t w[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int j = v * 8 + i * 2;
-            const float h0 = silu_f(__uint_as_float(gr[j])) * __uint_as_float(ur[j]);
-            const float h1 = silu_f(__uint_as_float(gr[j + 1])) * __uint_as_float(ur[j + 1]);
-            w[i] = pack_bf16x2(h0, h1);
-          }
-          dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+    for (int i = 0; i < 4; ++i) {
+      const int j = v * 8 + i * 2;
+      const float h0 = silu_f(__uint_as_float(gr[j])) * __uint_as_float(ur[j]);
+      const float h1 = silu_f(__uint_as_float(gr[j + 1])) * __uint_as_float(ur[j + 1]);
+      w[i] = pack_bf16x2(h0, h1);
+    }
+    dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// down: 32 columns of y from the accumulator columns at tbase + tcol; output columns
+// [oc, oc + 32) of the tile's 256. Deterministic store: through the warp's staging rows
+// stg (32 x 80 bytes), so that a warp store covers 8 rows x 64 bytes; fused: s * g * y
+// added to the token's fp32 accumulator (tok, sc of this row).
+__device__ __forceinline__ void epi_down_chunk(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                               int row, int tcol, int oc, int tok, float sc,
+                                               float (*stg)[20], int lane) {
+  uint32_t yr[32];
+  tmem_ld_32x32b_x32(tbase + tcol, yr);
+  tmem_ld_wait();
+  const int col = t.nt * BN + oc;
+  if (g.mode == kDownStore) {
+    // this lane's row as 64 bytes of bf16 into the staging row, then 16 bytes per lane of
+    // rows 8i + lane/4 out to global memory
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int j = v * 8 + i * 2;
+        w[i] = pack_bf16x2(__uint_as_float(yr[j]), __uint_as_float(yr[j + 1]));
+      }
+      *reinterpret_cast<uint4*>(&stg[lane][4 * v]) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncwarp();
+    if (col < g.n_valid) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 8 * i + (lane >> 2), ch = lane & 3;
+        const int grow = row - lane + r;
+        if (grow < t.row_end)
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                    (size_t)grow * g.ld_out + col + 8 * ch) =
+              *reinterpret_cast<const uint4*>(&stg[r][4 * ch]);
       }
     }
+    __syncwarp();
     return;
   }
-  int tok = 0;
-  float sc = 0.f;
-  if (g.mode == kDownAtomic && valid) {
+  if (row >= t.row_end || col >= g.n_valid) return;
+  float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)tok * g.ld_out + col);
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    atomicAdd(dst + v, make_float4(sc * __uint_as_float(yr[4 * v + 0]),
+                                   sc * __uint_as_float(yr[4 * v + 1]),
+                                   sc * __uint_as_float(yr[4 * v + 2]),
+                                   sc * __uint_as_float(yr[4 * v + 3])));
+}
+
+__device__ __forceinline__ void row_scale(const GemmArgs& g, const Tile& t, int row, int& tok,
+                                          float& sc) {
+  tok = 0;
+  sc = 0.f;
+  if (g.mode == kDownAtomic && row < t.row_end) {
     tok = g.perm_token[row];
     sc = g.scale * g.row_gate[row];
   }
+}
+
+// Epilogue of one 128 x 256 accumulator of the one-CTA kernel for one thread: its TMEM
+// lane (row) and its half of the columns. The B tile is [128 gate rows | 128 up rows]
+// (gate/up) or 256 rows of W_d (down): gate/up half h makes h columns [64h, 64h + 64)
+// from gate columns [64h, 64h + 64) and up columns 128 + [64h, 64h + 64); down half h
+// stores columns [128h, 128h + 128).
+__device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                                int row, int half, float (*stg)[20], int lane) {
+  if (g.mode == kGateUp) {
 #pragma unroll 1
-  for (int c = 128 * half; c < 128 * half + 128; c += 32) {
-    uint32_t yr[32];
-    tmem_ld_32x32b_x32(tbase + c, yr);
-    tmem_ld_wait();
-    const int col = t.nt * BN + c;
-    if (g.mode == kDownStore) {
-      // this lane's row as 64 bytes of bf16 into the staging row, then 16 bytes per lane
-      // of rows 8i + lane/4 out to global memory
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j = v * 8 + i * 2;
-          w[i] = pack_bf16x2(__uint_as_float(yr[j]), __uint_as_float(yr[j + 1]));
-        }
-        *reinterpret_cast<uint4*>(&stg[lane][4 * v]) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      __syncwarp();
-      if (col < g.n_valid) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = 8 * i + (lane >> 2), ch = lane & 3;
-          const int grow = row - lane + r;
-          if (grow < t.row_end)
-            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
-                                      (size_t)grow * g.ld_out + col + 8 * ch) =
-                *reinterpret_cast<const uint4*>(&stg[r][4 * ch]);
-        }
-      }
-      __syncwarp();
-      continue;
-    }
-    if (!valid || col >= g.n_valid) continue;
-    {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) +
-                                              (size_t)tok * g.ld_out + col);
-#pragma unroll
-      for (int v = 0; v < 8; ++v)
-        atomicAdd(dst + v, make_float4(sc * __uint_as_float(yr[4 * v + 0]),
-                                       sc * __uint_as_float(yr[4 * v + 1]),
-                                       sc * __uint_as_float(yr[4 * v + 2]),
-                                       sc * __uint_as_float(yr[4 * v + 3])));
-    }
+    for (int c = 64 * half; c < 64 * half + 64; c += 32)
+      epi_gateup_chunk(g, t, tbase, row, c, BM + c, c);
+    return;
   }
+  int tok;
+  float sc;
+  row_scale(g, t, row, tok, sc);
+#pragma unroll 1
+  for (int c = 128 * half; c < 128 * half + 128; c += 32)
+    epi_down_chunk(g, t, tbase, row, c, c, tok, sc, stg, lane);
 }
 
 // LOGITS: the router instantiation (mode kLogits, running sums in the epilogue); the
@@ -477,17 +496,67 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- CTA-pair variant of the expert GEMMs (tcgen05 cta_group::2) -------------------------
 // A cluster of two CTAs computes a 256 x 256 tile: CTA r loads rows [128r, 128r+128) of the
-// A tile and B rows [128r, 128r+128) of the N tile (gate/up: CTA 0 the gate rows, CTA 1
-// the up rows), so each CTA moves 32 KB per k-block instead of 48 KB. Both CTAs' TMA loads
-// count on the leader's (rank 0) full barrier; the leader's single thread issues
-// tcgen05.mma.cta_group::2 (M = 256) and commits to the empty / accumulator-full barriers
-// of both CTAs (two commits, one per CTA); both CTAs' epilogues read their own TMEM rows
-// and release the accumulator on the leader's barrier.
+// A tile and 128 rows of the N tile's B (gate/up: gate rows [64r, 64r+64) then the
+// matching up rows, as two 64-row boxes; down: W_d rows [128r, 128r+128)), so each CTA
+// moves 32 KB per k-block instead of 48 KB. Both CTAs' TMA loads count on the leader's
+// (rank 0) full barrier; the leader's single thread issues tcgen05.mma.cta_group::2 and
+// commits to the empty / accumulator-full barriers of both CTAs (two commits, one per
+// CTA); both CTAs' epilogues read their own TMEM rows and release the accumulator on the
+// leader's barrier.
+// An expert's last tile holds count mod 256 rows; when that is at most 128 it runs as an
+// M = 128 MMA (64 rows per CTA: A loaded from row0 + 64r, its first 64 rows used), which
+// halves the padded work of the tail. Its accumulator lands in TMEM as the 2x2 layout:
+// lanes 0-63 hold the CTA's 64 rows for N columns [0, 128), lanes 64-127 the same rows
+// for N columns [128, 256), both in TMEM columns [0, 128) of the accumulator.
 constexpr int BMP = 256;                             // M rows per CTA pair
 constexpr int PSTAGES = 6;                           // 32 KB per stage per CTA
 constexpr int P_B_BYTES = 128 * BK * 2;              // 16 KB: this CTA's half of B
 constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES;   // 32 KB
 constexpr uint32_t kIdescPair = idesc_bf16_f32(BMP, BN);
+constexpr uint32_t kIdescPairHalf = idesc_bf16_f32(128, BN);
+
+__device__ __forceinline__ bool half_tile(const GemmArgs& g, const Tile& t) {
+  return g.half_tiles && t.row_end - t.row0 <= 128;
+}
+
+// Epilogue of one pair tile for one thread (warp quarter q, column half h of the warp pair).
+// Full tile (M = 256): row 128r + 32q + lane; gate/up: h columns [64h, 64h + 64) from gate
+// TMEM columns 128h + [0, 64) and up columns 128h + 64 + [0, 64); down: columns
+// [128h, 128h + 128). Half tile (M = 128): row 64r + 32(q & 1) + lane, N block ib = q >> 1;
+// gate/up: h columns 64 ib + 32h + [0, 32) from gate TMEM columns 32h + [0, 32) and up
+// columns 64 + 32h + [0, 32); down: columns 128 ib + 64h + [0, 64) at TMEM 64h + [0, 64).
+__device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                              uint32_t rank, int q, int h, float (*stg)[20],
+                                              int lane) {
+  if (!half_tile(g, t)) {
+    const int row = t.row0 + 128 * (int)rank + 32 * q + lane;
+    if (g.mode == kGateUp) {
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 32)
+        epi_gateup_chunk(g, t, tbase, row, 128 * h + j, 128 * h + 64 + j, 64 * h + j);
+      return;
+    }
+    int tok;
+    float sc;
+    row_scale(g, t, row, tok, sc);
+#pragma unroll 1
+    for (int c = 128 * h; c < 128 * h + 128; c += 32)
+      epi_down_chunk(g, t, tbase, row, c, c, tok, sc, stg, lane);
+    return;
+  }
+  const int row = t.row0 + 64 * (int)rank + 32 * (q & 1) + lane;
+  const int ib = q >> 1;
+  if (g.mode == kGateUp) {
+    epi_gateup_chunk(g, t, tbase, row, 32 * h, 64 + 32 * h, 64 * ib + 32 * h);
+    return;
+  }
+  int tok;
+  float sc;
+  row_scale(g, t, row, tok, sc);
+#pragma unroll 1
+  for (int j = 0; j < 64; j += 32)
+    epi_down_chunk(g, t, tbase, row, 64 * h + j, 128 * ib + 64 * h + j, tok, sc, stg, lane);
+}
 
 struct alignas(1024) PairStorage {
   uint8_t a[PSTAGES][A_BYTES];
@@ -584,16 +653,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       for (int tile = cluster; tile < total_tiles && !*abort_flag; tile += nclusters) {
         const Tile t = decode_pair_tile(s, g, tile);
-        const int arow = t.row0 + 128 * (int)rank;
-        const int brow = g.mode == kGateUp
-                             ? t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM
-                             : t.e * g.b_rows + t.nt * BN + 128 * (int)rank;
+        const int arow = t.row0 + (half_tile(g, t) ? 64 : 128) * (int)rank;
+        // gate/up: gate rows [64r, 64r+64) of the N tile, then the same up rows (two
+        // 64-row boxes); down: W_d rows [128r, 128r+128) of the N tile
+        const int brow = g.mode == kGateUp ? t.e * g.b_rows + t.nt * BM + 64 * (int)rank
+                                           : t.e * g.b_rows + t.nt * BN + 128 * (int)rank;
         for (int kb = 0; kb < g.kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
           const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * P_STAGE_BYTES);
           tma_load_2d_pair(s.a[stage], &tmA, kb * BK, arow, full_leader);
-          tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
+          if (g.mode == kGateUp) {
+            tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
+            tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB, kb * BK, brow + g.b_second,
+                             full_leader);
+          } else {
+            tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
+          }
           if (++stage == PSTAGES) {
             stage = 0;
             phase ^= 1u;
@@ -610,6 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
+        const uint32_t idesc = half_tile(g, decode_pair_tile(s, g, tile)) ? kIdescPairHalf : kIdescPair;
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -621,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
-                           kIdescPair, (kb > 0 || k > 0) ? 1u : 0u);
+                           idesc, (kb > 0 || k > 0) ? 1u : 0u);
           const uint32_t e_local = smem_u32(&s.empty[stage]);
           umma_commit_pair(mapa_shared(e_local, 0));
           umma_commit_pair(mapa_shared(e_local, 1));
@@ -639,10 +716,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---- epilogue (both CTAs, warps 2..9): this CTA's 128 rows of the 256-row tile ------
+    // ---- epilogue (both CTAs, warps 2..9): this CTA's rows of the tile -------------------
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
-    const int row_in_tile = 128 * (int)rank + q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cluster; tile < total_tiles; tile += nclusters) {
@@ -654,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_expert(g, t, tbase, t.row0 + row_in_tile, half, s.epi_stage[warp - 2], lane);
+      epilogue_pair(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
@@ -772,6 +848,15 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
 
 // The CTA-pair kernel pays off once groups are tall (256-row tiles); small batches keep
 // the one-CTA kernel. MOE_B200_GEMM_PAIR=0 / 1 forces either (for measurements).
+// MOE_B200_PAIR_HALF=0 runs every pair tile as M = 256 (for measurements).
+int pair_half_tiles() {
+  static const int v = [] {
+    const char* e = getenv("MOE_B200_PAIR_HALF");
+    return (e && e[0] == '0') ? 0 : 1;
+  }();
+  return v;
+}
+
 bool use_pair_kernel(int T) {
   static const char* env = getenv("MOE_B200_GEMM_PAIR");
   if (env && env[0] == '0') return false;
@@ -925,7 +1010,10 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   } else {
     if ((rc = make_map(&mx, x, (uint64_t)T, H, 1)) != MOE_OK) return rc;
   }
-  if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H)) != MOE_OK) return rc;
+  // the CTA-pair kernel loads gate/up B as 64-row boxes (gate rows, then the same up rows)
+  const bool pair = use_pair_kernel(T) && x_perm != nullptr;
+  if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H, pair ? 64 : BM)) != MOE_OK)
+    return rc;
   if ((rc = make_map(&mh, h, rows, I)) != MOE_OK) return rc;
   if ((rc = make_map(&mwd, w_down, (uint64_t)n_ffn * H, I)) != MOE_OK) return rc;
 
@@ -944,7 +1032,7 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g1.status = status;
   g1.ksplit = 1;
   g1.kb_per_split = g1.kblocks;
-  const bool pair = use_pair_kernel(T) && !g1.gather_tok;
+  g1.half_tiles = pair_half_tiles();
   if ((rc = pair ? launch_pair(mx, mwgu, g1, sm_count, st) : launch_one(mx, mwgu, g1, sm_count, st)) !=
       MOE_OK)
     return rc;
@@ -966,6 +1054,7 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g2.status = status;
   g2.ksplit = 1;
   g2.kb_per_split = g2.kblocks;
+  g2.half_tiles = pair_half_tiles();
   return pair ? launch_pair(mh, mwd, g2, sm_count, st) : launch_one(mh, mwd, g2, sm_count, st);
 }
 
