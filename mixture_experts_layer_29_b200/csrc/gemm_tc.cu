@@ -914,9 +914,13 @@ int router_min_split() {
 
 int router_tc_splitk(int T, int E, int H, int sm_count) {
   if (sm_count > 160) sm_count = 160;
+  if (sm_count < 1) sm_count = 1;
   const long tiles = (long)((T + BM - 1) / BM) * ((E + BN - 1) / BN);
   const int kblocks = 3 * H / BK;
-  if (tiles <= 0 || tiles >= sm_count) return 1;   // a full wave already: no partial slices
+  if (tiles <= 0) return 1;
+  // a full wave already: no partial slices (splitting K to fill the last wave better
+  // measured slower at T = 8192: 0.322 vs 0.292 ms for the route call)
+  if (tiles >= sm_count) return 1;
   long s = (2L * sm_count + tiles - 1) / tiles;
   long smax = kblocks / router_min_split();
   if (smax > 64) smax = 64;
