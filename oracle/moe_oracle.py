@@ -43,7 +43,9 @@ Readings where the pages are silent (the report's equations are not printed):
   FFN experts are indices [0, n_ffn); SwiGLU experts W_down (silu(W_gate x) * W_up x);
   PID in position form with per-expert frequency target target_ratio * K / n_ffn;
   load-balance loss as in lb_loss below (DeepSeek's f_i P_i form, device-level grouping
-  with one FFN expert per group and one group of every zero-computation expert).
+  with one FFN expert per group and one group of every zero-computation expert);
+  backward with the expert selection held fixed (it is piecewise constant in the inputs)
+  and no gradient to the bias (it only moves the selection and is set by the PID).
 
 Parity pins: every function here is pinned in tests/test_oracle.py against closed forms,
 brute force, invariants or independent library routines; none is "parity unpinned".
@@ -58,7 +60,8 @@ import numpy as np
 __all__ = [
     "router_logits", "softmax_probs", "biased_scores", "select_topk", "near_tie_gap",
     "route", "permute", "swiglu_expert", "moe_layer_forward", "PidState", "pid_init",
-    "pid_update", "pid_stats", "lb_loss", "RouteResult", "PermuteResult",
+    "pid_update", "pid_stats", "lb_loss", "moe_layer_backward", "BackwardResult",
+    "RouteResult", "PermuteResult",
 ]
 
 
@@ -352,4 +355,92 @@ def lb_loss(logits, counts, n_ffn: int, K: int):
     if E > n_ffn:
         loss += float(f[n_ffn:].mean() * P[n_ffn:].sum())
     return loss, P
+
+
+# ---------------------------------------------------------------------------------------
+# Backward of the layer
+# ---------------------------------------------------------------------------------------
+
+@dataclass
+class BackwardResult:
+    dx: np.ndarray          # [T, H]
+    d_router: np.ndarray    # [E, H]
+    d_gate_up: np.ndarray   # [N, 2I, H]
+    d_down: np.ndarray      # [N, H, I]
+    d_logits: np.ndarray    # [T, E]
+    d_gate: np.ndarray      # [T, K]: gradient of each pick's gate
+    topk_idx: np.ndarray    # the selection the gradient was taken at
+
+
+def moe_layer_backward(x, w_router, bias32, w_gate_up, w_down, n_ffn: int, K: int, dout,
+                       ffn_out_scale: float = 1.0, topk_idx=None) -> BackwardResult:
+    """Gradients of the layer output with respect to x, W_r, W_gu and W_d, given the
+    gradient dout of the output, in float64.
+
+    The forward is the one of moe_layer_forward with L = x W_r^T: out[t] = sum over FFN
+    picks of s g_k y_{e_k}(x_t) + sum over zero picks of g_k x_t, g_k = p[t, e_k],
+    p = softmax(L[t]) ([pool], [zero], [scale]). The selection is held fixed (it is
+    piecewise constant in the inputs); the bias only moves the selection ([bias]) and gets
+    no gradient. topk_idx: the selection to differentiate at (default: route() of the
+    float64 logits). Per pick (t, k) of FFN expert e, with G = W_g x, U = W_u x,
+    sig = 1 / (1 + exp(-G)), h = G sig U, y = W_d h:
+      d_gate[t, k] = s <dout_t, y>,      dy = s g_k dout_t
+      d_down[e]   += dy h^T,             dh = W_d^T dy
+      dG = dh U sig (1 + G (1 - sig)),   dU = dh G sig
+      d_gate_up[e] += [dG; dU] x_t^T,   dx_t += W_g^T dG + W_u^T dU
+    per zero pick: d_gate[t, k] = <dout_t, x_t>, dx_t += g_k dout_t; then
+      dp[t, e] = sum of d_gate over the picks of e,   dL = p * (dp - <p, dp>)
+      d_router = dL^T x,   dx += dL W_r.
+    """
+    x64 = np.asarray(x, dtype=np.float64)
+    wr = np.asarray(w_router, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    T, H = x64.shape
+    E = wr.shape[0]
+    L = x64 @ wr.T
+    if topk_idx is None:
+        topk_idx = route(L, bias32, n_ffn, K).topk_idx
+    idx = np.asarray(topk_idx)
+    m = L.max(axis=1, keepdims=True)
+    ex = np.exp(L - m)
+    p = ex / ex.sum(axis=1, keepdims=True)
+    s = float(ffn_out_scale)
+    dx = np.zeros((T, H))
+    d_gate = np.zeros((T, K))
+    N = n_ffn
+    I = np.asarray(w_gate_up[0]).shape[0] // 2
+    d_gu = np.zeros((N, 2 * I, H))
+    d_d = np.zeros((N, H, I))
+    for e in sorted({int(v) for v in idx.ravel() if v < n_ffn}):
+        tk = np.argwhere(idx == e)                       # (t, k) of every pick of e
+        ts, ks = tk[:, 0], tk[:, 1]
+        wgu = np.asarray(w_gate_up[e], dtype=np.float64)
+        wd = np.asarray(w_down[e], dtype=np.float64)
+        X = x64[ts]
+        G = X @ wgu[:I].T
+        U = X @ wgu[I:].T
+        with np.errstate(over="ignore"):
+            sig = 1.0 / (1.0 + np.exp(-G))
+        h = G * sig * U
+        y = h @ wd.T
+        g = p[ts, e]
+        dy = s * g[:, None] * dout[ts]
+        d_gate[ts, ks] = s * (dout[ts] * y).sum(axis=1)
+        d_d[e] = dy.T @ h
+        dh = dy @ wd
+        dG = dh * U * sig * (1.0 + G * (1.0 - sig))
+        dU = dh * G * sig
+        d_gu[e, :I] = dG.T @ X
+        d_gu[e, I:] = dU.T @ X
+        dx[ts] += dG @ wgu[:I] + dU @ wgu[I:]            # a token picks e at most once
+    zt, zk = np.nonzero(idx >= n_ffn)
+    d_gate[zt, zk] = (dout[zt] * x64[zt]).sum(axis=1)
+    for t, k in zip(zt, zk):
+        dx[t] += p[t, idx[t, k]] * dout[t]
+    dp = np.zeros((T, E))
+    np.add.at(dp, (np.repeat(np.arange(T), K), idx.ravel()), d_gate.ravel())
+    dL = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+    d_router = dL.T @ x64
+    dx += dL @ wr
+    return BackwardResult(dx, d_router, d_gu, d_d, dL, d_gate, idx)
 

@@ -400,6 +400,83 @@ def test_lb_loss_collapsed_routing_reaches_E():
     assert abs(P[0] - 1) < 1e-12
 
 
+# ----------------------------------------------------------------------------- backward
+
+def _bwd_case(seed=7, T=6, H=8, I=4, N=3, Z=2, K=3):
+    g = rng(seed)
+    x = g.standard_normal((T, H))
+    wr = g.standard_normal((N + Z, H)) * 0.6
+    bias = (g.uniform(-0.05, 0.05, N + Z)).astype(np.float32)
+    wgu = g.standard_normal((N, 2 * I, H)) * 0.5
+    wd = g.standard_normal((N, H, I)) * 0.5
+    dout = g.standard_normal((T, H))
+    return x, wr, bias, wgu, wd, dout, N, K
+
+
+def _objective(x, wr, bias, wgu, wd, dout, N, K, s, idx):
+    out, *_rest, r = orc.moe_layer_forward(x, x @ wr.T, bias, wgu, wd, N, K, s)
+    assert (np.sort(r.topk_idx, 1) == np.sort(idx, 1)).all()     # selection unchanged
+    return float((dout * out).sum())
+
+
+def test_backward_matches_central_differences():
+    """Directional derivatives of <dout, out> along random directions of each input, by
+    central differences of the (pinned) forward, against the backward's gradients. The
+    step keeps every token's selection (checked); the forward's float32 gates limit the
+    agreement to ~1e-4 relative."""
+    x, wr, bias, wgu, wd, dout, N, K = _bwd_case()
+    s = 1.3
+    b = orc.moe_layer_backward(x, wr, bias, wgu, wd, N, K, dout, s)
+    g = rng(11)
+    eps = 1e-3
+    for name in ("x", "wr", "wgu", "wd"):
+        args = dict(x=x, wr=wr, wgu=wgu, wd=wd)
+        v = g.standard_normal(args[name].shape)
+        grad = {"x": b.dx, "wr": b.d_router, "wgu": b.d_gate_up, "wd": b.d_down}[name]
+        plus = dict(args); plus[name] = args[name] + eps * v
+        minus = dict(args); minus[name] = args[name] - eps * v
+        fd = (_objective(plus["x"], plus["wr"], bias, plus["wgu"], plus["wd"], dout, N, K, s, b.topk_idx)
+              - _objective(minus["x"], minus["wr"], bias, minus["wgu"], minus["wd"], dout, N, K, s,
+                           b.topk_idx)) / (2 * eps)
+        an = float((grad * v).sum())
+        assert abs(fd - an) <= 2e-3 * abs(an) + 1e-6, (name, fd, an)
+
+
+def test_backward_matches_torch_autograd():
+    """The same layer written with torch float64 ops, the selection fixed, differentiated
+    by autograd: every gradient and the logit gradient agree to 1e-10."""
+    x, wr, bias, wgu, wd, dout, N, K = _bwd_case(seed=3, T=9, Z=3, K=3)
+    s = 0.7
+    b = orc.moe_layer_backward(x, wr, bias, wgu, wd, N, K, dout, s)
+    tx = torch.tensor(x, requires_grad=True)
+    twr = torch.tensor(wr, requires_grad=True)
+    twgu = torch.tensor(wgu, requires_grad=True)
+    twd = torch.tensor(wd, requires_grad=True)
+    I = wgu.shape[1] // 2
+    logits = tx @ twr.T
+    logits.retain_grad()
+    p = torch.softmax(logits, dim=1)
+    out = torch.zeros_like(tx)
+    rows = []
+    for t in range(x.shape[0]):
+        acc = torch.zeros(x.shape[1], dtype=torch.float64)
+        for k in range(K):
+            e = int(b.topk_idx[t, k])
+            if e < N:
+                hh = F.silu(F.linear(tx[t], twgu[e, :I])) * F.linear(tx[t], twgu[e, I:])
+                acc = acc + s * p[t, e] * F.linear(hh, twd[e])
+            else:
+                acc = acc + p[t, e] * tx[t]
+        rows.append(acc)
+    out = torch.stack(rows)
+    (out * torch.tensor(dout)).sum().backward()
+    np.testing.assert_allclose(b.dx, tx.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(b.d_router, twr.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(b.d_gate_up, twgu.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(b.d_down, twd.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(b.d_logits, logits.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
 # ----------------------------------------------------------------------------- pages' numbers
 
 def test_activated_parameter_identity_from_the_pages():
@@ -506,4 +583,26 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     with pytest.raises(AssertionError):
         test_lb_loss_worked_example_by_hand()
     monkeypatch.setattr(orc, "lb_loss", orig_lb)
+
+    # 7. backward: a gate/up gradient off by 0.1% -> the autograd pin; the down-projection
+    #    gradient with its columns reversed -> the central-differences pin
+    orig_bwd = orc.moe_layer_backward
+
+    def bwd_scaled(x, wr, bias, wgu, wd, N, K, dout, s=1.0, topk_idx=None):
+        r = orig_bwd(x, wr, bias, wgu, wd, N, K, dout, s, topk_idx)
+        r.d_gate_up = r.d_gate_up * 0.999
+        return r
+    monkeypatch.setattr(orc, "moe_layer_backward", bwd_scaled)
+    with pytest.raises(AssertionError):
+        test_backward_matches_torch_autograd()
+    monkeypatch.setattr(orc, "moe_layer_backward", orig_bwd)
+
+    def bwd_wrong_down(x, wr, bias, wgu, wd, N, K, dout, s=1.0, topk_idx=None):
+        r = orig_bwd(x, wr, bias, wgu, wd, N, K, dout, s, topk_idx)
+        r.d_down = np.ascontiguousarray(np.flip(r.d_down, axis=2))
+        return r
+    monkeypatch.setattr(orc, "moe_layer_backward", bwd_wrong_down)
+    with pytest.raises(AssertionError):
+        test_backward_matches_central_differences()
+    monkeypatch.setattr(orc, "moe_layer_backward", orig_bwd)
     monkeypatch.setattr(orc, "pid_update", orig_pid)
