@@ -223,6 +223,45 @@ int moe_pid_bias_update(const moe_pid_t* pid, const moe_shape_t* shape, const in
                         const int32_t* nffn_hist, float* bias, float* pid_state,
                         float* stats_out, void* stream);
 
+/* ---- backward ---------------------------------------------------------------------------- */
+
+/* Bytes of workspace moe_backward needs: G|U of the FFN rows, dy, dG|dU (bf16,
+ * [T * K + 128, ...] each), dx_perm (fp32 [T * K + 128, H]), the picks' gate gradients
+ * and the logit gradient. */
+int moe_backward_workspace_size(const moe_shape_t* shape, size_t* bytes);
+
+/* Backward of the layer (LongCat-Flash Technical Report digest, Key claims, report §2.1
+ * and §2.4: the combined pool and its SwiGLU experts), differentiated with the expert
+ * selection held fixed (it is piecewise constant) and no gradient to the selection bias
+ * (it only steers selection and is set by the PID, report §2.1.1):
+ *   dy = s g_k dout_t (FFN rows),  d_gate = s <dout_t, y> (FFN) or <dout_t, x_t> (zero),
+ *   dh = dy W_d[e], dG = dh U silu'(G), dU = dh silu(G) (G, U recomputed),
+ *   d_down[e] = sum dy h^T, d_gate_up[e] = sum [dG; dU] x^T, dx_t = sum W_gu[e]^T [dG; dU]
+ *   + zgate_t dout_t + dL_t W_r with dL = p (dp - <p, dp>), d_router = dL^T x.
+ * bf16 layers only (MOE_ERR_UNSUPPORTED otherwise). The inputs are those of a forward in
+ * the deterministic combine mode on the same batch (moe_route, moe_permute with x_perm,
+ * moe_grouped_ffn keeping h and y_perm):
+ *   dout       device [T, H] bf16             gradient of the layer output
+ *   x          device [T, H] bf16
+ *   w_router   device [E, H] fp32;  w_gate_up [n_ffn, 2I, H], w_down [n_ffn, H, I] bf16
+ *   logits     device [T, E] fp32             the logits the batch was routed with
+ *   topk_idx, topk_gate, offsets, row_of      moe_route / moe_permute outputs
+ *   x_perm, h, y_perm   device [T * K + 128, H | I | H] bf16
+ *   dx         device [T, H] fp32             receives d out / d x
+ *   d_router   device [E, H] fp32             receives d / d W_r
+ *   d_gate_up  device [n_ffn, 2I, H] fp32     receives d / d W_gu of every expert with
+ *   d_down     device [n_ffn, H, I] fp32      rows; experts without rows are not written
+ *   ws         device, >= moe_backward_workspace_size bytes, zeroed before first use
+ * The expert GEMMs run on the tensor cores (bf16 in, fp32 accumulate; dy, G, U, dG, dU
+ * rounded to bf16); the router's gradients are fp32 on the CUDA cores. Errors as for the
+ * other calls; device-side timeouts go to the status word at the start of ws. */
+int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
+                 const float* w_router, const void* w_gate_up, const void* w_down,
+                 const float* logits, const int32_t* topk_idx, const float* topk_gate,
+                 const int32_t* offsets, const int32_t* row_of, const void* x_perm,
+                 const void* h, const void* y_perm, float* dx, float* d_router,
+                 float* d_gate_up, float* d_down, void* ws, size_t ws_bytes, void* stream);
+
 /* Device-level load-balance loss of one batch, forward value (LongCat-Flash Technical
  * Report digest, Key claims, report §2.1.1 / §2.1.2 Eqs. 3-5: DeepSeek-V3's balance loss
  * with every zero-computation expert in one virtual group; the equations are not

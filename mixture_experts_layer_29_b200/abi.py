@@ -83,6 +83,8 @@ _SIGS = {
     "moe_router_pack": (ctypes.c_int, [ctypes.POINTER(Shape), _P, _P, _P]),
     "moe_route_packed": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 10 + [_SZ, _P]),
     "moe_lb_loss": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 5 + [_SZ, _P]),
+    "moe_backward_workspace_size": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_SZ)]),
+    "moe_backward": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 18 + [_SZ, _P]),
 }
 
 _lib = None
@@ -237,6 +239,23 @@ def pid_bias_update(pid: Pid, shape, counts, nffn_hist, bias, pid_state, stats_o
     _check(lib().moe_pid_bias_update(ctypes.byref(pid), ctypes.byref(shape), ptr(counts),
                                      ptr(nffn_hist), ptr(bias), ptr(pid_state), ptr(stats_out),
                                      _stream(stream)), "moe_pid_bias_update")
+
+
+def backward_workspace_size(shape) -> int:
+    n = _SZ(0)
+    _check(lib().moe_backward_workspace_size(ctypes.byref(shape), ctypes.byref(n)),
+           "moe_backward_workspace_size")
+    return n.value
+
+
+def backward(shape, dout, x, w_router, w_gate_up, w_down, logits, topk_idx, topk_gate, offsets,
+             row_of, x_perm, h, y_perm, dx, d_router, d_gate_up, d_down, ws, stream=None):
+    """moe_backward: gradients of the layer for dout, from a deterministic-mode forward."""
+    _check(lib().moe_backward(ctypes.byref(shape), ptr(dout), ptr(x), ptr(w_router),
+                              ptr(w_gate_up), ptr(w_down), ptr(logits), ptr(topk_idx),
+                              ptr(topk_gate), ptr(offsets), ptr(row_of), ptr(x_perm), ptr(h),
+                              ptr(y_perm), ptr(dx), ptr(d_router), ptr(d_gate_up), ptr(d_down),
+                              ptr(ws), _nbytes(ws), _stream(stream)), "moe_backward")
 
 
 def lb_loss(shape, logits, counts, prob_mean, loss, ws, stream=None):

@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 SOURCES = ["abi.cu", "router.cu", "permute.cu", "gemm_tc.cu", "ffn_simt.cu", "combine_pid.cu",
-           "permute_static.cu", "lbloss.cu"]
+           "permute_static.cu", "lbloss.cu", "gemm_bwd.cu", "backward.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]

@@ -283,6 +283,74 @@ int moe_workspace_size(const moe_shape_t* shape, size_t* bytes) {
   return MOE_OK;
 }
 
+// Backward workspace: status word, G|U, dy, dG|dU, dx_perm (fp32), the picks' gate
+// gradients and the logit gradient.
+struct BwdLayout {
+  size_t status, gu, dy, dgu, dxp, dgate, dl, total;
+};
+
+static BwdLayout bwd_layout_of(const moe_shape_t& s) {
+  BwdLayout L{};
+  const size_t T = s.T, H = s.H, I = s.I, K = s.K, E = (size_t)s.n_ffn + s.n_zero;
+  const size_t rows = T * K + kRowPad;
+  size_t o = 0;
+  L.status = o; o = align_up(o + 256);
+  L.gu = o;     o = align_up(o + rows * 2 * I * 2);
+  L.dy = o;     o = align_up(o + rows * H * 2);
+  L.dgu = o;    o = align_up(o + rows * 2 * I * 2);
+  L.dxp = o;    o = align_up(o + rows * H * 4);
+  L.dgate = o;  o = align_up(o + T * K * 4);
+  L.dl = o;     o = align_up(o + T * E * 4);
+  L.total = o;
+  return L;
+}
+
+int moe_backward_workspace_size(const moe_shape_t* shape, size_t* bytes) {
+  MOE_TRY(check_shape(shape));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = bwd_layout_of(*shape).total;
+  return MOE_OK;
+}
+
+int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
+                 const float* w_router, const void* w_gate_up, const void* w_down,
+                 const float* logits, const int32_t* topk_idx, const float* topk_gate,
+                 const int32_t* offsets, const int32_t* row_of, const void* x_perm,
+                 const void* h, const void* y_perm, float* dx, float* d_router,
+                 float* d_gate_up, float* d_down, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_shape(shape));
+  if (shape->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(check_ptrs({dout, x, w_router, w_gate_up, w_down, logits, topk_idx, topk_gate, offsets,
+                      row_of, x_perm, h, y_perm, dx, d_router, d_gate_up, d_down, ws}));
+  const BwdLayout L = bwd_layout_of(*shape);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (shape->T == 0) return MOE_OK;
+  DeviceInfo dev;
+  MOE_TRY(current_device_info(&dev));
+  const cudaStream_t st = as_stream(stream);
+  const int T = shape->T, H = shape->H, I = shape->I, K = shape->K, N = shape->n_ffn;
+  const int E = N + shape->n_zero;
+  int* status = at<int>(ws, L.status);
+  void* gu = at<char>(ws, L.gu);
+  void* dy = at<char>(ws, L.dy);
+  void* dgu = at<char>(ws, L.dgu);
+  float* dxp = at<float>(ws, L.dxp);
+  float* dgate = at<float>(ws, L.dgate);
+  float* dl = at<float>(ws, L.dl);
+  // G | U of every FFN row again, then dy and the gates' gradients
+  MOE_TRY(launch_gate_up_raw(x_perm, offsets, w_gate_up, gu, T, H, I, N, K, status, dev.sm_count,
+                             st));
+  MOE_TRY(cuda_rc(launch_bwd_dy_dgate(dout, x, y_perm, topk_idx, topk_gate, row_of, T, H, K, N,
+                                      shape->ffn_out_scale, dy, dgate, st)));
+  // the expert GEMMs: dgu (with the SwiGLU backward), dx_perm, d_down, d_gate_up
+  MOE_TRY(launch_bwd_gemms(dy, gu, h, x_perm, offsets, w_gate_up, w_down, dgu, dxp, d_gate_up,
+                           d_down, T, H, I, N, K, status, dev.sm_count, st));
+  // router: logit gradient, d_router = dL^T x, dx = dL W_r; then the rows and the zero term
+  MOE_TRY(cuda_rc(launch_bwd_router(logits, topk_idx, dgate, T, E, K, dl, st)));
+  MOE_TRY(cuda_rc(launch_router_grads(dl, x, w_router, T, E, H, d_router, dx, st)));
+  return cuda_rc(launch_bwd_dx_combine(dxp, dout, topk_idx, topk_gate, row_of, T, H, K, N, dx, st));
+}
+
 int moe_read_device_status(void* ws, size_t ws_bytes, void* stream, int32_t* status) {
   if (!ws || !status) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < 256) return MOE_ERR_WORKSPACE;

@@ -1,0 +1,332 @@
+// backward.cu - the layer's backward outside the expert GEMMs (those are in gemm_bwd.cu).
+//
+// The forward, differentiated with the expert selection held fixed (it is piecewise
+// constant in the inputs) and no gradient to the selection bias (LongCat-Flash Technical
+// Report digest, Key claims, report §2.1.1: the bias only steers selection and is set by the
+// PID controller):
+//   out[t] = sum over FFN picks of s g_k y_k(x_t) + sum over zero picks of g_k x_t,
+//   g_k = p[t, e_k],  p = softmax(x_t W_r^T)
+// Kernels:
+//   k_bwd_dy_dgate   per token: dy[r] = s g_k dout_t on each FFN row r (bf16), and each
+//                    pick's gate gradient: s <dout_t, y_r> (FFN) or <dout_t, x_t> (zero)
+//   k_bwd_router     per token: p again from the logits (double), dp at the picks,
+//                    dL = p * (dp - <p, dp>) (fp32)
+//   k_simt_gemm      fp32 CUDA-core GEMMs of the router: d_router = dL^T x, dx = dL W_r
+//   k_bwd_dx_combine dx[t] += sum over FFN slots (in order) of dx_perm[row] + zgate_t dout_t
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "launch.cuh"
+
+namespace moe {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&q);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(b[i]);
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+constexpr int kTok = 256;   // threads per token CTA
+
+// One CTA per token; thread i owns columns 8i, 8i + 8 kTok, ... of the row.
+__global__ void __launch_bounds__(kTok) k_bwd_dy_dgate(
+    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ x,
+    const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restrict__ topk_idx,
+    const float* __restrict__ topk_gate, const int32_t* __restrict__ row_of, int H, int K,
+    int n_ffn, float scale, __nv_bfloat16* __restrict__ dy, float* __restrict__ d_gate) {
+  __shared__ int s_row[32];
+  __shared__ float s_g[32];
+  __shared__ float s_red[kTok / 32][33];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int t = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x < K) {
+    const int e = topk_idx[(size_t)t * K + threadIdx.x];
+    s_row[threadIdx.x] = e < n_ffn ? row_of[(size_t)t * K + threadIdx.x] : -1;
+    s_g[threadIdx.x] = topk_gate[(size_t)t * K + threadIdx.x];
+  }
+  __syncthreads();
+  float dot[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) dot[k] = 0.f;
+  for (int c = threadIdx.x * 8; c < H; c += kTok * 8) {
+    float d[8], xv[8];
+    load8(dout + (size_t)t * H + c, d);
+    load8(x + (size_t)t * H + c, xv);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      if (k >= K) break;
+      const int r = s_row[k];
+      if (r >= 0) {
+        float y[8];
+        load8(y_perm + (size_t)r * H + c, y);
+        const float gs = scale * s_g[k];
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(gs * d[2 * i], gs * d[2 * i + 1]);
+        *reinterpret_cast<uint4*>(dy + (size_t)r * H + c) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dot[k] = fmaf(d[i], y[i], dot[k]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dot[k] = fmaf(d[i], xv[i], dot[k]);
+      }
+    }
+  }
+  // block sums of the K dot products (fixed order)
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    if (k >= K) break;
+    float v = dot[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) s_red[warp][k] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < K) {
+    float v = 0.f;
+    for (int w = 0; w < kTok / 32; ++w) v += s_red[w][threadIdx.x];
+    d_gate[(size_t)t * K + threadIdx.x] = s_row[threadIdx.x] >= 0 ? scale * v : v;
+  }
+}
+
+// One warp per token: dL[t, e] = p_e (dp_e - sum_k p_{e_k} dg_k), dp_e = dg_k at e = e_k.
+template <int J>
+__global__ void __launch_bounds__(256) k_bwd_router(const float* __restrict__ logits,
+                                                    const int32_t* __restrict__ topk_idx,
+                                                    const float* __restrict__ d_gate, int T,
+                                                    int E, int K, float* __restrict__ dL) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* Lr = logits + (size_t)t * E;
+  float lv[J];
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    lv[j] = e < E ? Lr[e] : -INFINITY;
+    m = fmaxf(m, lv[j]);
+  }
+  m = warp_max(m);
+  double ex[J], sum = 0.0;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    ex[j] = e < E ? exp((double)lv[j] - (double)m) : 0.0;
+    sum += ex[j];
+  }
+  sum = warp_sum(sum);
+  const double inv = 1.0 / sum;
+  // the picks: lane k < K holds (e_k, dg_k)
+  const int my_e = lane < K ? topk_idx[(size_t)t * K + lane] : -1;
+  const float my_dg = lane < K ? d_gate[(size_t)t * K + lane] : 0.f;
+  double dpe[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) dpe[j] = 0.0;
+  double dot = 0.0;
+  for (int k = 0; k < K; ++k) {
+    const int ek = __shfl_sync(0xffffffffu, my_e, k);
+    const float dgk = __shfl_sync(0xffffffffu, my_dg, k);
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+      if (ek == lane + 32 * j) {
+        dpe[j] = dgk;
+        dot += ex[j] * inv * (double)dgk;
+      }
+  }
+  dot = warp_sum(dot);
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    if (e < E) dL[(size_t)t * E + e] = (float)(ex[j] * inv * (dpe[j] - dot));
+  }
+}
+
+// C[M, N] (fp32, row-major, ld N) = op(A) . B over K, fp32 FMA on the CUDA cores.
+// A_KM: A is stored [K][M] (C = A^T B), else [M][K]; B is [K][N] of TB. 64 x 64 tiles,
+// 16-deep k slices, 256 threads with 4 x 4 outputs each, fixed summation order.
+template <bool A_KM, typename TB>
+__global__ void __launch_bounds__(256) k_simt_gemm(const float* __restrict__ A,
+                                                   const TB* __restrict__ B, int M, int N,
+                                                   int K, float* __restrict__ C) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    // 16 x 64 of A and of B: 1024 values each, four per thread
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tid + 256 * i;
+      int kk, mm;
+      if (A_KM) {
+        kk = idx >> 6;
+        mm = idx & 63;
+      } else {
+        mm = idx >> 4;
+        kk = idx & 15;
+      }
+      const int k = k0 + kk, m = m0 + mm;
+      float a = 0.f;
+      if (k < K && m < M) a = A_KM ? A[(size_t)k * M + m] : A[(size_t)m * K + k];
+      As[kk][mm] = a;
+      const int bk = idx >> 6, bn = idx & 63;
+      float b = 0.f;
+      if (k0 + bk < K && n0 + bn < N) b = to_f32(B[(size_t)(k0 + bk) * N + n0 + bn]);
+      Bs[bk][bn] = b;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < N) C[(size_t)m * N + n] = acc[i][j];
+    }
+  }
+}
+
+// dx[t] += sum over FFN slots k (in order) of dx_perm[row_of[t, k]] + zgate_t * dout_t
+__global__ void __launch_bounds__(kTok) k_bwd_dx_combine(
+    const float* __restrict__ dx_perm, const __nv_bfloat16* __restrict__ dout,
+    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_gate,
+    const int32_t* __restrict__ row_of, int H, int K, int n_ffn, float* __restrict__ dx) {
+  __shared__ int s_row[32];
+  __shared__ float s_z;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int t = blockIdx.x;
+  if (threadIdx.x < 32) {
+    const int k = threadIdx.x;
+    int r = -1;
+    float zg = 0.f;
+    if (k < K) {
+      const int e = topk_idx[(size_t)t * K + k];
+      if (e < n_ffn) r = row_of[(size_t)t * K + k];
+      else zg = topk_gate[(size_t)t * K + k];
+    }
+    s_row[k] = r;
+    // zgate in slot order (lane 0 adds the lanes' terms one by one)
+    float z = 0.f;
+    for (int j = 0; j < K; ++j) z += __shfl_sync(0xffffffffu, zg, j);
+    if (k == 0) s_z = z;
+  }
+  __syncthreads();
+  const float z = s_z;
+  for (int c = threadIdx.x * 8; c < H; c += kTok * 8) {
+    float acc[8], d[8];
+    load8(dx + (size_t)t * H + c, acc);
+    for (int k = 0; k < K; ++k) {
+      const int r = s_row[k];
+      if (r < 0) continue;
+      float v[8];
+      load8(dx_perm + (size_t)r * H + c, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += v[i];
+    }
+    load8(dout + (size_t)t * H + c, d);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = fmaf(z, d[i], acc[i]);
+    *reinterpret_cast<float4*>(dx + (size_t)t * H + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(dx + (size_t)t * H + c + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_dy_dgate(const void* dout, const void* x, const void* y_perm,
+                                const int32_t* topk_idx, const float* topk_gate,
+                                const int32_t* row_of, int T, int H, int K, int n_ffn,
+                                float scale, void* dy, float* d_gate, cudaStream_t st) {
+  const cudaError_t e = launch_kernel(
+      k_bwd_dy_dgate, T, kTok, 0, st, 1, static_cast<const __nv_bfloat16*>(dout),
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm), topk_idx,
+      topk_gate, row_of, H, K, n_ffn, scale, static_cast<__nv_bfloat16*>(dy), d_gate);
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_bwd_router(const float* logits, const int32_t* topk_idx, const float* d_gate,
+                              int T, int E, int K, float* dL, cudaStream_t st) {
+  const int J = (E + 31) / 32;
+  const int blocks = (T + 7) / 8;
+  cudaError_t e = cudaErrorInvalidValue;
+#define MOE_BR_CASE(JJ)                                                                    \
+  if (J <= JJ) {                                                                           \
+    e = launch_kernel(k_bwd_router<JJ>, blocks, 256, 0, st, 1, logits, topk_idx, d_gate, T, \
+                      E, K, dL);                                                           \
+  } else
+  MOE_BR_CASE(4) MOE_BR_CASE(8) MOE_BR_CASE(16) MOE_BR_CASE(24) MOE_BR_CASE(32) {
+    return cudaErrorInvalidValue;
+  }
+#undef MOE_BR_CASE
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_router_grads(const float* dL, const void* x, const float* w_router, int T,
+                                int E, int H, float* d_router, float* dx, cudaStream_t st) {
+  // d_router [E, H] = dL^T x   (K = T)
+  dim3 g1((H + 63) / 64, (E + 63) / 64);
+  cudaError_t e = launch_kernel(k_simt_gemm<true, __nv_bfloat16>, g1, 256, 0, st, 1, dL,
+                                static_cast<const __nv_bfloat16*>(x), E, H, T, d_router);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  // dx [T, H] = dL W_r   (K = E)
+  dim3 g2((H + 63) / 64, (T + 63) / 64);
+  e = launch_kernel(k_simt_gemm<false, float>, g2, 256, 0, st, 1, dL, w_router, T, H, E, dx);
+  count_launch();
+  return e;
+}
+
+cudaError_t launch_bwd_dx_combine(const float* dx_perm, const void* dout, const int32_t* topk_idx,
+                                  const float* topk_gate, const int32_t* row_of, int T, int H,
+                                  int K, int n_ffn, float* dx, cudaStream_t st) {
+  const cudaError_t e =
+      launch_kernel(k_bwd_dx_combine, T, kTok, 0, st, 1, dx_perm,
+                    static_cast<const __nv_bfloat16*>(dout), topk_idx, topk_gate, row_of, H, K,
+                    n_ffn, dx);
+  count_launch();
+  return e;
+}
+
+}  // namespace moe

@@ -299,5 +299,30 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
+// The same with A and / or B MN-major (bit 15: A, bit 16: B).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
+}
+
+// Shared-memory descriptor of an MN-major bf16 operand written by TMA with the 128-byte
+// swizzle as boxes of 64 K-rows x 64 MN-elements (8 KB each, stacked along MN): rows of
+// 128 bytes (64 MN elements), 8-row K groups 1024 bytes apart (stride byte offset), the
+// 64-element MN blocks `mn_block_bytes` apart (leading byte offset), version 1, 128-byte
+// swizzle. One K = 16 step of the MMA is 16 rows = 2048 bytes further.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t mn_block_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((mn_block_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the async proxy (the
+// tensor cores and TMA) before a barrier hands them over.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 }  // namespace moe

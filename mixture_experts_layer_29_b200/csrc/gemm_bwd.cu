@@ -1,0 +1,452 @@
+// gemm_bwd.cu - the expert GEMMs of the layer's backward on the 5th-generation tensor cores.
+//
+// With dy[r] = s * g * dout[token of r] on every FFN row r of expert e (see backward.cu):
+//   kDH  dh = dy . W_d[e]          M = rows of e, K = H, N = I; B = W_d[e] read N-major,
+//        then the SwiGLU backward in the epilogue from the recomputed G, U of the row:
+//        dG = dh * U * sig(G) * (1 + G (1 - sig(G))),  dU = dh * G * sig(G)  -> dgu [dG | dU]
+//   kDX  dx_perm = dgu . W_gu[e]   M = rows of e, K = 2I, N = H; B = W_gu[e] N-major; fp32
+//   kDW  d_down[e]    = dy_e^T  h_e       M = H,  K = rows of e, N = I
+//        d_gate_up[e] = dgu_e^T x_perm_e  M = 2I, K = rows of e, N = H
+//        A and B both MN-major (the row buffers read along their rows); fp32, written for
+//        the experts that have rows only.
+// The forward's SwiGLU expert (LongCat-Flash Technical Report digest, Key claims, report
+// §2.4: per-expert intermediate 2048 at hidden 6144) differentiated with the selection held
+// fixed.
+//
+// Same structure as the forward kernel (one CTA per SM, persistent, warp 0 TMA producer,
+// warp 1 TMEM owner + single-thread tcgen05.mma issuer, warps 2-9 epilogue, 4-stage ring
+// of 48 KB, two 256-column fp32 accumulators, every wait bounded). MN-major operands come
+// in as 64 K-rows x 64 MN-elements TMA boxes with the 128-byte swizzle, stacked along MN
+// 8 KB apart; the shared-memory descriptor then has leading byte offset 8 KB (between MN
+// blocks) and stride byte offset 1 KB (between 8-row K groups), and the instruction
+// descriptor marks the operand MN-major. kDW's K runs over one expert's rows: the last
+// k-block of an expert holds rows of the next one, so its tiles land on a side barrier,
+// the producer warp zeroes the K-rows past the expert in shared memory, fences them to the
+// async proxy and only then releases the stage to the MMA.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "launch.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BOX_BYTES = 64 * BK * 2;               // one 64 x 64 box: 8 KB
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = 64 + kEpiThreads;
+constexpr int kMaxExperts = 1024;
+constexpr uint32_t kTmemCols = 512;
+
+enum BwdMode : int { kDH = 0, kDX = 1, kDW = 2 };
+
+struct BwdArgs {
+  int mode;
+  int n_ffn;
+  int kblocks;            // kDH / kDX: K / 64
+  int m_tiles;            // kDW: M / 128
+  int n_tiles;            // N / 256 (rounded up)
+  int b_krows;            // kDH / kDX: K rows of B per expert in its 2-D view
+  int n_valid;            // output columns N
+  long long ld_out;       // output row length (elements)
+  long long out_expert;   // kDW: elements per expert of the output
+  int I;                  // kDH: G at column c, U at column I + c of gu and dgu
+  const int32_t* offsets;
+  const __nv_bfloat16* gu;
+  void* out;
+  int* status;
+};
+
+struct Tile {
+  int e, row0, row_end, mt, nt;
+};
+
+struct alignas(1024) Smem {
+  uint8_t a[STAGES][A_BYTES];
+  uint8_t b[STAGES][B_BYTES];
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t landed[STAGES];      // kDW last k-block: TMA bytes land here first
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  int offs[kMaxExperts + 1];
+  int toff[kMaxExperts + 1];    // kDH / kDX: prefix of ceil(count / 128); kDW: of (count > 0)
+  float stg[kEpiWarps][32][20];
+};
+
+__device__ __forceinline__ Tile decode(const Smem& s, const BwdArgs& g, int tile) {
+  Tile t;
+  int unit;
+  if (g.mode == kDW) {
+    const int per = g.m_tiles * g.n_tiles;
+    unit = tile / per;
+    const int rem = tile - unit * per;
+    t.mt = rem / g.n_tiles;
+    t.nt = rem - t.mt * g.n_tiles;
+  } else {
+    unit = tile / g.n_tiles;
+    t.nt = tile - unit * g.n_tiles;
+    t.mt = 0;
+  }
+  // largest e with toff[e] <= unit (experts without tiles share the next one's toff)
+  int lo = 0, hi = g.n_ffn - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.toff[mid] <= unit) lo = mid; else hi = mid - 1;
+  }
+  t.e = lo;
+  t.row0 = g.mode == kDW ? s.offs[lo] : s.offs[lo] + (unit - s.toff[lo]) * BM;
+  t.row_end = s.offs[lo + 1];
+  return t;
+}
+
+__device__ __forceinline__ int kblocks_of(const BwdArgs& g, const Tile& t) {
+  return g.mode == kDW ? (t.row_end - t.row0 + BK - 1) / BK : g.kblocks;
+}
+
+// fp32 row stores through the warp's staging block: this thread's row holds 16 values at
+// output columns [col, col + 16); a warp store then covers 8 rows x 64 bytes.
+__device__ __forceinline__ void store_f32_16(float (*stg)[20], int lane, const float* v,
+                                             float* out, long long ld, int row_base,
+                                             int row_end, int col, int n_valid) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<float4*>(&stg[lane][4 * i]) =
+        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = 8 * i + (lane >> 2), c = col + 4 * (lane & 3);
+    const int grow = row_base + r;
+    if (grow < row_end && c < n_valid)
+      *reinterpret_cast<float4*>(out + (size_t)grow * ld + c) =
+          *reinterpret_cast<const float4*>(&stg[r][4 * (lane & 3)]);
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ float sigm(float a) { return 1.0f / (1.0f + __expf(-a)); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const BwdArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                     ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+      mbar_init(&s.landed[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], kEpiThreads);
+    }
+    s.abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  pdl_wait();
+  for (int i = threadIdx.x; i <= g.n_ffn; i += kThreads) s.offs[i] = g.offsets[i];
+  __syncthreads();
+  if (warp == 2) {
+    const int per = (g.n_ffn + 31) / 32;
+    const int b = lane * per;
+    auto units = [&](int e) {
+      const int c = s.offs[e + 1] - s.offs[e];
+      return g.mode == kDW ? (c > 0 ? 1 : 0) : (c + BM - 1) / BM;
+    };
+    int local = 0;
+    for (int i = 0; i < per; ++i)
+      if (b + i < g.n_ffn) local += units(b + i);
+    const int inc = warp_inclusive_scan(local);
+    int run = inc - local;
+    for (int i = 0; i < per; ++i)
+      if (b + i < g.n_ffn) {
+        s.toff[b + i] = run;
+        run += units(b + i);
+      }
+    if (lane == 31) s.toff[g.n_ffn] = inc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s.tmem_base;
+  const int total_tiles =
+      s.toff[g.n_ffn] * (g.mode == kDW ? g.m_tiles * g.n_tiles : g.n_tiles);
+  volatile int* abort_flag = &s.abort_flag;
+  const bool a_mn = g.mode == kDW;
+
+  if (warp == 0) {
+    // ---- TMA producer (whole warp: lane 0 issues, all lanes zero the tail rows) ----------
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t landed_phase = 0;     // bit i: parity of the next completion of landed[i]
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles && !*abort_flag; tile += gridDim.x) {
+      const Tile t = decode(s, g, tile);
+      const int nkb = kblocks_of(g, t);
+      for (int kb = 0; kb < nkb; ++kb) {
+        int w_ok = 1;
+        if (lane == 0) w_ok = mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+          ok = false;
+          break;
+        }
+        const int valid = a_mn ? min(BK, t.row_end - (t.row0 + kb * BK)) : BK;
+        const bool masked = valid < BK;
+        uint64_t* bar = masked ? &s.landed[stage] : &s.full[stage];
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar, STAGE_BYTES);
+          if (a_mn) {
+            const int y = t.row0 + kb * BK;
+            tma_load_2d(s.a[stage], &tmA, t.mt * BM, y, bar);
+            tma_load_2d(s.a[stage] + BOX_BYTES, &tmA, t.mt * BM + 64, y, bar);
+            for (int j = 0; j < 4; ++j)
+              tma_load_2d(s.b[stage] + j * BOX_BYTES, &tmB, t.nt * BN + 64 * j, y, bar);
+          } else {
+            tma_load_2d(s.a[stage], &tmA, kb * BK, t.row0, bar);
+            const int y = t.e * g.b_krows + kb * BK;
+            for (int j = 0; j < 4; ++j)
+              tma_load_2d(s.b[stage] + j * BOX_BYTES, &tmB, t.nt * BN + 64 * j, y, bar);
+          }
+        }
+        if (masked) {
+          // K-rows [valid, 64) of every box belong to the next expert: zero them
+          if (lane == 0)
+            w_ok = mbar_wait(&s.landed[stage], (landed_phase >> stage) & 1u, abort_flag) ? 1 : 0;
+          landed_phase ^= 1u << stage;
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+            ok = false;
+            break;
+          }
+          const int nrow = BK - valid;
+          for (int i = lane; i < 6 * nrow * 8; i += 32) {
+            const int box = i / (nrow * 8), rem = i - box * nrow * 8;
+            const int r = valid + rem / 8, c16 = rem & 7;
+            uint8_t* base = box < 2 ? s.a[stage] + box * BOX_BYTES : s.b[stage] + (box - 2) * BOX_BYTES;
+            *reinterpret_cast<uint4*>(base + r * 128 + c16 * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.full[stage]);
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer -----------------------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32_major(BM, BN, a_mn, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles && !*abort_flag; tile += gridDim.x) {
+        const Tile t = decode(s, g, tile);
+        const int nkb = kblocks_of(g, t);
+        if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(s.a[stage]);
+          const uint32_t b0 = smem_u32(s.b[stage]);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = a_mn ? sw128_mnmajor_desc(a0 + k * 2048, BOX_BYTES)
+                                     : sw128_kmajor_desc(a0 + k * 32);
+            umma_bf16(d_tmem, ad, sw128_mnmajor_desc(b0 + k * 2048, BOX_BYTES), idesc,
+                      (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&s.empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&s.tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ---- epilogue: TMEM lane quarter q = warp % 4, column half h = (warp - 2) / 4 ---------
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
+    float (*stg)[20] = s.stg[warp - 2];
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const Tile t = decode(s, g, tile);
+      int w_ok = 1;
+      if (lane == 0) w_ok = mbar_wait(&s.tfull[acc], acc_phase, abort_flag) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      // kDH / kDX: output row = the tile's row; kDW: the weight row mt * 128 + q * 32 + lane
+      const int row_base = g.mode == kDW ? t.mt * BM + q * 32 : t.row0 + q * 32;
+      const int row_end = g.mode == kDW ? 0x7fffffff : t.row_end;
+      const int row = row_base + lane;
+#pragma unroll 1
+      for (int c = 128 * h; c < 128 * h + 128; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + c, v);
+        tmem_ld_wait();
+        const int col = t.nt * BN + c;
+        if (g.mode == kDH) {
+          if (row < row_end && col < g.n_valid) {
+            const __nv_bfloat16* gr = g.gu + (size_t)row * 2 * g.I + col;
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + (size_t)row * 2 * g.I + col;
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              const uint4 G4 = *reinterpret_cast<const uint4*>(gr + 8 * q8);
+              const uint4 U4 = *reinterpret_cast<const uint4*>(gr + g.I + 8 * q8);
+              const __nv_bfloat16* Gb = reinterpret_cast<const __nv_bfloat16*>(&G4);
+              const __nv_bfloat16* Ub = reinterpret_cast<const __nv_bfloat16*>(&U4);
+              float dG[8], dU[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float G = __bfloat162float(Gb[i]), U = __bfloat162float(Ub[i]);
+                const float dh = __uint_as_float(v[8 * q8 + i]);
+                const float sg = sigm(G);
+                dG[i] = dh * U * sg * (1.0f + G * (1.0f - sg));
+                dU[i] = dh * G * sg;
+              }
+              *reinterpret_cast<uint4*>(dst + 8 * q8) =
+                  make_uint4(pack_bf16x2(dG[0], dG[1]), pack_bf16x2(dG[2], dG[3]),
+                             pack_bf16x2(dG[4], dG[5]), pack_bf16x2(dG[6], dG[7]));
+              *reinterpret_cast<uint4*>(dst + g.I + 8 * q8) =
+                  make_uint4(pack_bf16x2(dU[0], dU[1]), pack_bf16x2(dU[2], dU[3]),
+                             pack_bf16x2(dU[4], dU[5]), pack_bf16x2(dU[6], dU[7]));
+            }
+          }
+        } else {
+          float* out = static_cast<float*>(g.out) +
+                       (g.mode == kDW ? (size_t)t.e * g.out_expert : (size_t)0);
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+          store_f32_16(stg, lane, f, out, g.ld_out, row_base, row_end, col, g.n_valid);
+          store_f32_16(stg, lane, f + 16, out, g.ld_out, row_base, row_end, col + 16, g.n_valid);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s.tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  if (*abort_flag) {
+    set_status(g.status, MOE_ERR_TIMEOUT);
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+int launch(const CUtensorMap& ma, const CUtensorMap& mb, const BwdArgs& g, int sm_count,
+           cudaStream_t st) {
+  constexpr size_t smem = sizeof(Smem) + 1024;
+  static_assert(smem <= 227 * 1024, "shared memory budget");
+  if (cudaFuncSetAttribute(k_bwd_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  const cudaError_t e = launch_kernel(k_bwd_gemm, sm_count, kThreads, smem, st, 1, ma, mb, g);
+  count_launch();
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* x_perm,
+                     const int32_t* offsets, const void* w_gate_up, const void* w_down,
+                     void* dgu, float* dx_perm, float* d_gate_up, float* d_down, int T, int H,
+                     int I, int n_ffn, int K, int* status, int sm_count, cudaStream_t st) {
+  const uint64_t rows = (uint64_t)T * K + BM;          // row buffers' allocation rows
+  CUtensorMap m_dy128, m_dy64, m_dgu128, m_dgu64, m_h64, m_x64, m_wd, m_wgu;
+  int rc;
+  if ((rc = make_tma_map_bf16(&m_dy128, dy, rows, H, 128)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_dy64, dy, rows, H, 64)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_dgu128, dgu, rows, 2ull * I, 128)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_dgu64, dgu, rows, 2ull * I, 64)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_h64, h, rows, I, 64)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_x64, x_perm, rows, H, 64)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_wd, w_down, (uint64_t)n_ffn * H, I, 64)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_wgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H, 64)) != MOE_OK)
+    return rc;
+
+  BwdArgs g{};
+  g.n_ffn = n_ffn;
+  g.offsets = offsets;
+  g.status = status;
+  g.I = I;
+  g.gu = static_cast<const __nv_bfloat16*>(gu);
+  // dh = dy . W_d[e] (+ SwiGLU backward) -> dgu
+  g.mode = kDH;
+  g.kblocks = H / BK;
+  g.n_tiles = (I + BN - 1) / BN;
+  g.b_krows = H;
+  g.n_valid = I;
+  g.out = dgu;
+  if ((rc = launch(m_dy128, m_wd, g, sm_count, st)) != MOE_OK) return rc;
+  // dx_perm = dgu . W_gu[e]
+  g.mode = kDX;
+  g.kblocks = 2 * I / BK;
+  g.n_tiles = (H + BN - 1) / BN;
+  g.b_krows = 2 * I;
+  g.n_valid = H;
+  g.ld_out = H;
+  g.out = dx_perm;
+  if ((rc = launch(m_dgu128, m_wgu, g, sm_count, st)) != MOE_OK) return rc;
+  // d_down[e] = dy^T h
+  g.mode = kDW;
+  g.m_tiles = H / BM;
+  g.n_tiles = (I + BN - 1) / BN;
+  g.n_valid = I;
+  g.ld_out = I;
+  g.out_expert = (long long)H * I;
+  g.out = d_down;
+  if ((rc = launch(m_dy64, m_h64, g, sm_count, st)) != MOE_OK) return rc;
+  // d_gate_up[e] = dgu^T x_perm
+  g.m_tiles = 2 * I / BM;
+  g.n_tiles = (H + BN - 1) / BN;
+  g.n_valid = H;
+  g.ld_out = H;
+  g.out_expert = 2LL * I * H;
+  g.out = d_gate_up;
+  return launch(m_dgu64, m_x64, g, sm_count, st);
+}
+
+}  // namespace moe

@@ -91,6 +91,7 @@ struct GemmArgs {
   const int32_t* gather_tok;  // non-null: A row r is row gather_tok[r] of A's tensor
   ZeroSpec zero;              // buffers cleared after the dependency wait
   int half_tiles;             // pair kernel: tails of at most 128 rows run as M = 128
+  int gu_raw;                 // gate/up: store G and U (bf16, [rows, 2I]) instead of h
 };
 
 struct Tile {
@@ -134,6 +135,24 @@ __device__ __forceinline__ void epi_gateup_chunk(const GemmArgs& g, const Tile& 
   tmem_ld_32x32b_x32(tbase + ucol, ur);
   tmem_ld_wait();
   if (row >= t.row_end) return;
+  if (g.gu_raw) {
+    // G to columns [nt*128 + oc, +32) and U to I + that of the row (ld_out = 2I)
+    __nv_bfloat16* base = static_cast<__nv_bfloat16*>(g.out) + (size_t)row * g.ld_out + t.nt * BM + oc;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t* src = half ? ur : gr;
+      uint4* dst = reinterpret_cast<uint4*>(base + (half ? g.n_valid : 0));
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(src[v * 8 + 2 * i]), __uint_as_float(src[v * 8 + 2 * i + 1]));
+        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    return;
+  }
   uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
                                         (size_t)row * g.ld_out + t.nt * BM + oc);
 #pragma unroll
@@ -1060,6 +1079,42 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g2.kb_per_split = g2.kblocks;
   g2.half_tiles = pair_half_tiles();
   return pair ? launch_pair(mh, mwd, g2, sm_count, st) : launch_one(mh, mwd, g2, sm_count, st);
+}
+
+int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w_gate_up,
+                       void* gu, int T, int H, int I, int n_ffn, int K, int* status, int sm_count,
+                       cudaStream_t st) {
+  if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
+  const uint64_t rows = (uint64_t)T * K + BM;
+  const bool pair = use_pair_kernel(T);
+  CUtensorMap mx, mwgu;
+  int rc;
+  if ((rc = make_map(&mx, x_perm, rows, H)) != MOE_OK) return rc;
+  if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H, pair ? 64 : BM)) != MOE_OK)
+    return rc;
+  GemmArgs g{};
+  g.mode = kGateUp;
+  g.gu_raw = 1;
+  g.n_ffn = n_ffn;
+  g.kblocks = H / BK;
+  g.n_tiles = I / BM;
+  g.b_rows = 2 * I;
+  g.b_second = I;
+  g.n_valid = I;
+  g.ld_out = 2 * I;
+  g.offsets = offsets;
+  g.out = gu;
+  g.status = status;
+  g.ksplit = 1;
+  g.kb_per_split = g.kblocks;
+  g.half_tiles = pair_half_tiles();
+  return pair ? launch_pair(mx, mwgu, g, sm_count, st) : launch_one(mx, mwgu, g, sm_count, st);
+}
+
+int make_tma_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows) {
+  if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
+  return make_map(m, base, rows, cols, box_rows);
 }
 
 }  // namespace moe

@@ -1,6 +1,7 @@
 // kernels.cuh - host-side launchers of the layer's kernels (internal to the library).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -69,6 +70,37 @@ cudaError_t launch_route_topk(const float* src, int S, float* logits_out, const 
 // launch_splitk_sum).
 bool route_topk_sums_slices(int T, int S, int sm_count);
 cudaError_t launch_zero_counts(int32_t* counts, int E, int32_t* nffn_hist, int K, cudaStream_t st);
+
+// rows x cols bf16 row-major tensor map with 128-byte swizzle and a box of 64 columns x
+// box_rows rows (no multicast).
+int make_tma_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows);
+
+// ---- backward ------------------------------------------------------------------------------
+// The gate/up GEMM again, storing G and U (bf16) instead of h: gu [T*K + 128, 2I].
+int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w_gate_up,
+                       void* gu, int T, int H, int I, int n_ffn, int K, int* status, int sm_count,
+                       cudaStream_t st);
+// dh = dy . W_d[e] with the SwiGLU backward in the epilogue -> dgu [rows, 2I] = [dG | dU];
+// dx_perm = dgu . W_gu[e] (fp32); per touched expert d_down[e] = dy^T h and
+// d_gate_up[e] = dgu^T x_perm (fp32, experts without rows untouched).
+int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* x_perm,
+                     const int32_t* offsets, const void* w_gate_up, const void* w_down,
+                     void* dgu, float* dx_perm, float* d_gate_up, float* d_down, int T, int H,
+                     int I, int n_ffn, int K, int* status, int sm_count, cudaStream_t st);
+
+cudaError_t launch_bwd_dy_dgate(const void* dout, const void* x, const void* y_perm,
+                                const int32_t* topk_idx, const float* topk_gate,
+                                const int32_t* row_of, int T, int H, int K, int n_ffn,
+                                float scale, void* dy, float* d_gate, cudaStream_t st);
+cudaError_t launch_bwd_router(const float* logits, const int32_t* topk_idx, const float* d_gate,
+                              int T, int E, int K, float* dL, cudaStream_t st);
+// d_router = dL^T x and dx = dL W_r (fp32, CUDA cores)
+cudaError_t launch_router_grads(const float* dL, const void* x, const float* w_router, int T,
+                                int E, int H, float* d_router, float* dx, cudaStream_t st);
+cudaError_t launch_bwd_dx_combine(const float* dx_perm, const void* dout, const int32_t* topk_idx,
+                                  const float* topk_gate, const int32_t* row_of, int T, int H,
+                                  int K, int n_ffn, float* dx, cudaStream_t st);
 
 // ---- load-balance loss -------------------------------------------------------------------
 size_t lb_partial_bytes(int T, int E);

@@ -17,7 +17,7 @@ def L():
 
 def test_library_exports_every_declared_function(L):
     names = abi.header_functions()
-    assert len(names) == 16
+    assert len(names) == 18
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(abi._SIGS)
@@ -99,6 +99,12 @@ def test_host_checks_run_before_any_device_access(L):
     s0 = _shape(T=0)
     assert L.moe_pid_bias_update(ctypes.byref(pid), ctypes.byref(s0), good, good, good, good,
                                  None, None) == -1
+    # backward: bf16 only, null pointers, short workspace
+    bs = _shape(dtype="bf16", H=256, I=128)
+    bw = abi.backward_workspace_size(bs)
+    assert L.moe_backward(ctypes.byref(s), *([good] * 18), bw, None) == -2      # fp32 layer
+    assert L.moe_backward(ctypes.byref(bs), *([good] * 17), None, bw, None) == -1
+    assert L.moe_backward(ctypes.byref(bs), *([good] * 18), bw - 1, None) == -5
     # load-balance loss: null counts or loss, unaligned logits, short workspace
     assert L.moe_lb_loss(ctypes.byref(s), good, None, None, good, good, ws_n, None) == -1
     assert L.moe_lb_loss(ctypes.byref(s), good, good, None, None, good, ws_n, None) == -1
