@@ -304,6 +304,50 @@ def scmoe_overlap(st: Stepper, device, seed: int, iters: int, warmup: int) -> di
     return out
 
 
+def time_backward(st: Stepper, device, seed: int, iters: int, warmup: int) -> dict:
+    """moe_backward on the batch of the last timed step (deterministic-mode forward), for a
+    random bf16 output gradient; mean CUDA-event time per call. Algorithmic work of the
+    expert GEMMs: the G|U recompute (4 R H I), dh (2 R H I), the rows' dx (4 R H I) and the
+    two weight gradients (2 + 4 R H I), 16 R H I in all; the router's two fp32 GEMMs are
+    4 T E H on the CUDA cores."""
+    cfg, b = st.cfg, st.b
+    g = torch.Generator(device=device).manual_seed(seed + 77)
+    dout = (torch.randn(cfg.T, cfg.H, device=device, generator=g) * 0.5).to(torch.bfloat16)
+    dx = torch.empty(cfg.T, cfg.H, dtype=torch.float32, device=device)
+    d_router = torch.empty(cfg.E, cfg.H, dtype=torch.float32, device=device)
+    d_gu = torch.empty(cfg.n_ffn, 2 * cfg.I, cfg.H, dtype=torch.float32, device=device)
+    d_d = torch.empty(cfg.n_ffn, cfg.H, cfg.I, dtype=torch.float32, device=device)
+    ws = torch.zeros(abi.backward_workspace_size(b.shape), dtype=torch.uint8, device=device)
+    w = st.w
+
+    def call():
+        abi.backward(b.shape, dout, st.x, w.w_router, w.w_gate_up, w.w_down, b.logits,
+                     b.topk_idx, b.topk_gate, b.offsets, b.row_of, b.x_perm, b.h, b.y_perm,
+                     dx, d_router, d_gu, d_d, ws)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / iters
+    assert abi.read_device_status(ws) == 0
+    rows = int(b.counts[: cfg.n_ffn].sum().item())
+    flop = 16.0 * rows * cfg.H * cfg.I
+    out = {"workload": st.cfg.name, "tokens": cfg.T, "ms_per_call": round(ms, 4),
+           "expert_gemm_flop": flop, "ffn_rows": rows,
+           "expert_gemm_tflops_over_call": round(flop / (ms / 1e3) / 1e12, 1),
+           "router_fp32_flop": 4.0 * cfg.T * cfg.E * cfg.H,
+           "note": "whole moe_backward call (router gradients on the CUDA cores included)"}
+    del dout, dx, d_router, d_gu, d_d, ws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 def max_over_ranks(v: float, dist_on: bool) -> float:
     if not dist_on:
         return v
@@ -420,6 +464,11 @@ def run_ours(args):
                "note": "moe_forward via MoELayer.forward_host: pinned x in, out back, each step"}
         del layer
 
+    bwd = None
+    if not args.no_backward and not dist_on and cfg.dtype == wl.BF16 and \
+            args.combine == "deterministic" and not cfg.skewed:
+        bwd = time_backward(st, device, seed, 5, 2)
+
     overlap = None
     if not args.no_overlap and not dist_on and cfg.dtype == wl.BF16:
         overlap = {"prefill": scmoe_overlap(st, device, seed, 20, 3)}
@@ -454,6 +503,7 @@ def run_ours(args):
         "roofline": roofline,
         "decode": decode,
         "scmoe_overlap": overlap,
+        "backward": bwd,
         "e2e": e2e,
         "gpu_launches": int(launches) * world,
         "cpu_baseline": cpu,
@@ -526,6 +576,7 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip timing moe_backward")
     ap.add_argument("--no-overlap", action="store_true",
                     help="skip the dense-FFN-beside-MoE (two streams) measurement")
     args = ap.parse_args(argv)

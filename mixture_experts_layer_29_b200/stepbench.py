@@ -4,7 +4,9 @@
     python -m mixture_experts_layer_29_b200.stepbench --step ffn --ffn-experts 32 --zero-experts 16
 
 Steps: route (moe_route: router logits + top-K), permute (moe_permute), ffn
-(moe_grouped_ffn), combine (moe_combine), pid (moe_pid_bias_update), layer (all of them).
+(moe_grouped_ffn), combine (moe_combine), pid (moe_pid_bias_update), layer (all of them),
+backward (moe_backward after one deterministic-mode forward; fp32 weight gradients of
+every expert are allocated, so keep n_ffn modest at full width).
 Only what the chosen step needs is drawn: the route and permute steps never allocate the
 FFN weights, so they run at the full-shape T and E in well under a GB of device memory.
 Prints one JSON line with the mean CUDA-event time per call.
@@ -20,7 +22,7 @@ import torch
 from . import abi
 from . import workloads as wl
 
-STEPS = ("route", "permute", "ffn", "combine", "pid", "layer")
+STEPS = ("route", "permute", "ffn", "combine", "pid", "layer", "backward")
 
 
 def main(argv=None) -> int:
@@ -41,7 +43,9 @@ def main(argv=None) -> int:
                             ("n_zero", a.zero_experts)) if v is not None}
     cfg = cfg.with_(**kw) if kw else cfg
     dev = torch.device("cuda", 0)
-    need_ffn = a.step in ("ffn", "combine", "layer")
+    need_ffn = a.step in ("ffn", "combine", "layer", "backward")
+    if a.step == "backward":
+        a.combine = "deterministic"
     w = wl.draw_weights(cfg, dev, ffn=need_ffn)
     x = wl.draw_tokens(cfg, dev)
     logits_in = wl.draw_skewed_logits(cfg, dev) if cfg.skewed else None
@@ -71,10 +75,26 @@ def main(argv=None) -> int:
     def pid_step():
         abi.pid_bias_update(pid, shape, b.counts, b.nffn_hist, bias_next, state)
 
+    bwd = {}
+    if a.step == "backward":
+        g = torch.Generator(device=dev).manual_seed(9)
+        bwd["dout"] = (torch.randn(cfg.T, cfg.H, device=dev, generator=g) * 0.5).to(torch.bfloat16)
+        bwd["dx"] = torch.empty(cfg.T, cfg.H, device=dev)
+        bwd["dr"] = torch.empty(cfg.E, cfg.H, device=dev)
+        bwd["dgu"] = torch.empty(cfg.n_ffn, 2 * cfg.I, cfg.H, device=dev)
+        bwd["dd"] = torch.empty(cfg.n_ffn, cfg.H, cfg.I, device=dev)
+        bwd["ws"] = torch.zeros(abi.backward_workspace_size(shape), dtype=torch.uint8, device=dev)
+
+    def backward():
+        abi.backward(shape, bwd["dout"], x, w.w_router, w.w_gate_up, w.w_down, b.logits,
+                     b.topk_idx, b.topk_gate, b.offsets, b.row_of, b.x_perm, b.h, b.y_perm,
+                     bwd["dx"], bwd["dr"], bwd["dgu"], bwd["dd"], bwd["ws"])
+
     steps = {"route": route, "permute": permute, "ffn": ffn, "combine": combine,
-             "pid": pid_step, "layer": lambda: (route(), permute(), ffn(), combine())}
+             "pid": pid_step, "layer": lambda: (route(), permute(), ffn(), combine()),
+             "backward": backward}
     # inputs of the timed step come from the steps before it
-    order = ["route", "permute", "ffn", "combine"]
+    order = ["route", "permute", "ffn", "combine", "backward"]
     if a.step in order[1:]:
         for s in order[: order.index(a.step)]:
             steps[s]()
