@@ -226,8 +226,8 @@ int moe_pid_bias_update(const moe_pid_t* pid, const moe_shape_t* shape, const in
 /* ---- backward ---------------------------------------------------------------------------- */
 
 /* Bytes of workspace moe_backward needs: G|U of the FFN rows, dy, dG|dU (bf16,
- * [T * K + 128, ...] each), dx_perm (fp32 [T * K + 128, H]), the picks' gate gradients
- * and the logit gradient. */
+ * [T * K + 128, ...] each), dx_perm (fp32 [T * K + 128, H]), the picks' gate gradients,
+ * the logit gradient in three bf16 parts and W_r in bf16. */
 int moe_backward_workspace_size(const moe_shape_t* shape, size_t* bytes);
 
 /* Backward of the layer (LongCat-Flash Technical Report digest, Key claims, report §2.1
@@ -252,9 +252,12 @@ int moe_backward_workspace_size(const moe_shape_t* shape, size_t* bytes);
  *   d_gate_up  device [n_ffn, 2I, H] fp32     receives d / d W_gu of every expert with
  *   d_down     device [n_ffn, H, I] fp32      rows; experts without rows are not written
  *   ws         device, >= moe_backward_workspace_size bytes, zeroed before first use
- * The expert GEMMs run on the tensor cores (bf16 in, fp32 accumulate; dy, G, U, dG, dU
- * rounded to bf16); the router's gradients are fp32 on the CUDA cores. Errors as for the
- * other calls; device-side timeouts go to the status word at the start of ws. */
+ * Every GEMM runs on the tensor cores (bf16 in, fp32 accumulate): the expert GEMMs with
+ * dy, G, U, dG, dU rounded to bf16; d_router from the logit gradient split exactly into
+ * three bf16 parts (exact products with the bf16 x); the router's share of dx from
+ * bf16(dL) and bf16(W_r). bf16 layers with E a multiple of 8 (MOE_ERR_UNSUPPORTED
+ * otherwise). Other errors as for the other calls; device-side timeouts go to the status
+ * word at the start of ws. */
 int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
                  const float* w_router, const void* w_gate_up, const void* w_down,
                  const float* logits, const int32_t* topk_idx, const float* topk_gate,

@@ -286,7 +286,7 @@ int moe_workspace_size(const moe_shape_t* shape, size_t* bytes) {
 // Backward workspace: status word, G|U, dy, dG|dU, dx_perm (fp32), the picks' gate
 // gradients and the logit gradient.
 struct BwdLayout {
-  size_t status, gu, dy, dgu, dxp, dgate, dl, total;
+  size_t status, offs, gu, dy, dgu, dxp, dgate, dl3, wr16, total;
 };
 
 static BwdLayout bwd_layout_of(const moe_shape_t& s) {
@@ -294,13 +294,16 @@ static BwdLayout bwd_layout_of(const moe_shape_t& s) {
   const size_t T = s.T, H = s.H, I = s.I, K = s.K, E = (size_t)s.n_ffn + s.n_zero;
   const size_t rows = T * K + kRowPad;
   size_t o = 0;
+  const size_t Tp = (T + 63) / 64 * 64;
   L.status = o; o = align_up(o + 256);
+  L.offs = o;   o = align_up(o + 4 * 4);
   L.gu = o;     o = align_up(o + rows * 2 * I * 2);
   L.dy = o;     o = align_up(o + rows * H * 2);
   L.dgu = o;    o = align_up(o + rows * 2 * I * 2);
   L.dxp = o;    o = align_up(o + rows * H * 4);
   L.dgate = o;  o = align_up(o + T * K * 4);
-  L.dl = o;     o = align_up(o + T * E * 4);
+  L.dl3 = o;    o = align_up(o + 3 * Tp * E * 2);
+  L.wr16 = o;   o = align_up(o + E * (size_t)s.H * 2);
   L.total = o;
   return L;
 }
@@ -320,6 +323,7 @@ int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
                  float* d_gate_up, float* d_down, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(check_shape(shape));
   if (shape->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if ((shape->n_ffn + shape->n_zero) % 8 != 0) return MOE_ERR_UNSUPPORTED;   // dL rows: 16 B
   MOE_TRY(check_ptrs({dout, x, w_router, w_gate_up, w_down, logits, topk_idx, topk_gate, offsets,
                       row_of, x_perm, h, y_perm, dx, d_router, d_gate_up, d_down, ws}));
   const BwdLayout L = bwd_layout_of(*shape);
@@ -336,7 +340,10 @@ int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
   void* dgu = at<char>(ws, L.dgu);
   float* dxp = at<float>(ws, L.dxp);
   float* dgate = at<float>(ws, L.dgate);
-  float* dl = at<float>(ws, L.dl);
+  void* dl3 = at<char>(ws, L.dl3);
+  void* wr16 = at<char>(ws, L.wr16);
+  int32_t* offs = at<int32_t>(ws, L.offs);
+  const int Tp = (T + 63) / 64 * 64;
   // G | U of every FFN row again, then dy and the gates' gradients
   MOE_TRY(launch_gate_up_raw(x_perm, offsets, w_gate_up, gu, T, H, I, N, K, status, dev.sm_count,
                              st));
@@ -345,9 +352,12 @@ int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
   // the expert GEMMs: dgu (with the SwiGLU backward), dx_perm, d_down, d_gate_up
   MOE_TRY(launch_bwd_gemms(dy, gu, h, x_perm, offsets, w_gate_up, w_down, dgu, dxp, d_gate_up,
                            d_down, T, H, I, N, K, status, dev.sm_count, st));
-  // router: logit gradient, d_router = dL^T x, dx = dL W_r; then the rows and the zero term
-  MOE_TRY(cuda_rc(launch_bwd_router(logits, topk_idx, dgate, T, E, K, dl, st)));
-  MOE_TRY(cuda_rc(launch_router_grads(dl, x, w_router, T, E, H, d_router, dx, st)));
+  // router: logit gradient (three bf16 parts), d_router = dL^T x, dx = dL W_r; then the
+  // rows' gradients and the zero-expert term
+  MOE_TRY(cuda_rc(launch_bwd_router(logits, topk_idx, dgate, T, Tp, E, K, dl3, offs, w_router,
+                                    wr16, H, st)));
+  MOE_TRY(launch_bwd_router_gemms(dl3, Tp, x, wr16, offs, offs + 2, T, E, H, d_router, dx,
+                                  status, dev.sm_count, st));
   return cuda_rc(launch_bwd_dx_combine(dxp, dout, topk_idx, topk_gate, row_of, T, H, K, N, dx, st));
 }
 

@@ -10,8 +10,11 @@
 //   k_bwd_dy_dgate   per token: dy[r] = s g_k dout_t on each FFN row r (bf16), and each
 //                    pick's gate gradient: s <dout_t, y_r> (FFN) or <dout_t, x_t> (zero)
 //   k_bwd_router     per token: p again from the logits (double), dp at the picks,
-//                    dL = p * (dp - <p, dp>) (fp32)
-//   k_simt_gemm      fp32 CUDA-core GEMMs of the router: d_router = dL^T x, dx = dL W_r
+//                    dL = p * (dp - <p, dp>), split exactly into three bf16 parts
+//                    (hi = bf16(dL), mid = bf16(dL - hi), lo = dL - hi - mid) for the
+//                    router's tensor-core GEMMs in gemm_bwd.cu: d_router = dL^T x (all
+//                    three parts: exact products, fp32 sums) and dx = dL W_r (hi parts)
+//   k_to_bf16        W_r in bf16 for the latter
 //   k_bwd_dx_combine dx[t] += sum over FFN slots (in order) of dx_perm[row] + zgate_t dout_t
 #include <math.h>
 
@@ -104,16 +107,32 @@ __global__ void __launch_bounds__(kTok) k_bwd_dy_dgate(
 }
 
 // One warp per token: dL[t, e] = p_e (dp_e - sum_k p_{e_k} dg_k), dp_e = dg_k at e = e_k.
+// dl3: [3][Tp][E] bf16, part p of token t at row p Tp + t; rows [T, Tp) of every part are
+// written as zeros. Block 0 also writes the two one-group offset tables of the router
+// GEMMs: offs_k = {0, 3 Tp}, offs_m = {0, T}.
 template <int J>
 __global__ void __launch_bounds__(256) k_bwd_router(const float* __restrict__ logits,
                                                     const int32_t* __restrict__ topk_idx,
                                                     const float* __restrict__ d_gate, int T,
-                                                    int E, int K, float* __restrict__ dL) {
+                                                    int Tp, int E, int K,
+                                                    __nv_bfloat16* __restrict__ dl3,
+                                                    int32_t* __restrict__ offs) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T) return;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    offs[0] = 0;
+    offs[1] = 3 * Tp;
+    offs[2] = 0;
+    offs[3] = T;
+  }
+  if (t >= Tp) return;
+  if (t >= T) {
+    for (int e = lane; e < E; e += 32)
+      for (int p = 0; p < 3; ++p) dl3[((size_t)p * Tp + t) * E + e] = __float2bfloat16_rn(0.f);
+    return;
+  }
   const float* Lr = logits + (size_t)t * E;
   float lv[J];
   float m = -INFINITY;
@@ -154,75 +173,26 @@ __global__ void __launch_bounds__(256) k_bwd_router(const float* __restrict__ lo
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int e = lane + 32 * j;
-    if (e < E) dL[(size_t)t * E + e] = (float)(ex[j] * inv * (dpe[j] - dot));
+    if (e < E) {
+      const float v = (float)(ex[j] * inv * (dpe[j] - dot));
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const float r1 = __fsub_rn(v, __bfloat162float(hi));
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(r1, __bfloat162float(mid)));
+      dl3[(size_t)t * E + e] = hi;
+      dl3[((size_t)Tp + t) * E + e] = mid;
+      dl3[(2 * (size_t)Tp + t) * E + e] = lo;
+    }
   }
 }
 
-// C[M, N] (fp32, row-major, ld N) = op(A) . B over K, fp32 FMA on the CUDA cores.
-// A_KM: A is stored [K][M] (C = A^T B), else [M][K]; B is [K][N] of TB. 64 x 64 tiles,
-// 16-deep k slices, 256 threads with 4 x 4 outputs each, fixed summation order.
-template <bool A_KM, typename TB>
-__global__ void __launch_bounds__(256) k_simt_gemm(const float* __restrict__ A,
-                                                   const TB* __restrict__ B, int M, int N,
-                                                   int K, float* __restrict__ C) {
-  __shared__ float As[16][64 + 4];
-  __shared__ float Bs[16][64 + 4];
+__global__ void __launch_bounds__(256) k_to_bf16(const float* __restrict__ a,
+                                                 __nv_bfloat16* __restrict__ out, size_t n) {
   pdl_launch_dependents();
   pdl_wait();
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    // 16 x 64 of A and of B: 1024 values each, four per thread
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int idx = tid + 256 * i;
-      int kk, mm;
-      if (A_KM) {
-        kk = idx >> 6;
-        mm = idx & 63;
-      } else {
-        mm = idx >> 4;
-        kk = idx & 15;
-      }
-      const int k = k0 + kk, m = m0 + mm;
-      float a = 0.f;
-      if (k < K && m < M) a = A_KM ? A[(size_t)k * M + m] : A[(size_t)m * K + k];
-      As[kk][mm] = a;
-      const int bk = idx >> 6, bn = idx & 63;
-      float b = 0.f;
-      if (k0 + bk < K && n0 + bn < N) b = to_f32(B[(size_t)(k0 + bk) * N + n0 + bn]);
-      Bs[bk][bn] = b;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
-    if (m >= M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
-      if (n < N) C[(size_t)m * N + n] = acc[i][j];
-    }
-  }
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    out[i] = __float2bfloat16_rn(a[i]);
 }
 
 // dx[t] += sum over FFN slots k (in order) of dx_perm[row_of[t, k]] + zgate_t * dout_t
@@ -286,34 +256,26 @@ cudaError_t launch_bwd_dy_dgate(const void* dout, const void* x, const void* y_p
 }
 
 cudaError_t launch_bwd_router(const float* logits, const int32_t* topk_idx, const float* d_gate,
-                              int T, int E, int K, float* dL, cudaStream_t st) {
+                              int T, int Tp, int E, int K, void* dl3, int32_t* offs,
+                              const float* w_router, void* wr16, int H, cudaStream_t st) {
   const int J = (E + 31) / 32;
-  const int blocks = (T + 7) / 8;
+  const int blocks = (Tp + 7) / 8;
   cudaError_t e = cudaErrorInvalidValue;
 #define MOE_BR_CASE(JJ)                                                                    \
   if (J <= JJ) {                                                                           \
     e = launch_kernel(k_bwd_router<JJ>, blocks, 256, 0, st, 1, logits, topk_idx, d_gate, T, \
-                      E, K, dL);                                                           \
+                      Tp, E, K, static_cast<__nv_bfloat16*>(dl3), offs);                  \
   } else
   MOE_BR_CASE(4) MOE_BR_CASE(8) MOE_BR_CASE(16) MOE_BR_CASE(24) MOE_BR_CASE(32) {
     return cudaErrorInvalidValue;
   }
 #undef MOE_BR_CASE
   count_launch();
-  return e;
-}
-
-cudaError_t launch_router_grads(const float* dL, const void* x, const float* w_router, int T,
-                                int E, int H, float* d_router, float* dx, cudaStream_t st) {
-  // d_router [E, H] = dL^T x   (K = T)
-  dim3 g1((H + 63) / 64, (E + 63) / 64);
-  cudaError_t e = launch_kernel(k_simt_gemm<true, __nv_bfloat16>, g1, 256, 0, st, 1, dL,
-                                static_cast<const __nv_bfloat16*>(x), E, H, T, d_router);
-  count_launch();
   if (e != cudaSuccess) return e;
-  // dx [T, H] = dL W_r   (K = E)
-  dim3 g2((H + 63) / 64, (T + 63) / 64);
-  e = launch_kernel(k_simt_gemm<false, float>, g2, 256, 0, st, 1, dL, w_router, T, H, E, dx);
+  const size_t n = (size_t)E * H;
+  int cb = (int)((n + 255) / 256);
+  if (cb > 4096) cb = 4096;
+  e = launch_kernel(k_to_bf16, cb, 256, 0, st, 1, w_router, static_cast<__nv_bfloat16*>(wr16), n);
   count_launch();
   return e;
 }

@@ -39,7 +39,8 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int BOX_BYTES = 64 * BK * 2;               // one 64 x 64 box: 8 KB
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kThreads = 64 + kEpiThreads;
+constexpr int kFixWarp = 2 + kEpiWarps;             // zeroes an expert's tail K-rows
+constexpr int kThreads = 64 + kEpiThreads + 32;
 constexpr int kMaxExperts = 1024;
 constexpr uint32_t kTmemCols = 512;
 
@@ -56,6 +57,8 @@ struct BwdArgs {
   long long ld_out;       // output row length (elements)
   long long out_expert;   // kDW: elements per expert of the output
   int I;                  // kDH: G at column c, U at column I + c of gu and dgu
+  int m_valid;            // kDW: output rows M
+  int b_kwrap;            // kDW: B's row is the K row modulo this (0: no wrap)
   const int32_t* offsets;
   const __nv_bfloat16* gu;
   void* out;
@@ -110,6 +113,14 @@ __device__ __forceinline__ Tile decode(const Smem& s, const BwdArgs& g, int tile
 __device__ __forceinline__ int kblocks_of(const BwdArgs& g, const Tile& t) {
   return g.mode == kDW ? (t.row_end - t.row0 + BK - 1) / BK : g.kblocks;
 }
+
+// kDW: K-rows of k-block kb that belong to the tile's expert (64 for the other modes). The
+// MMA runs ceil(valid / 16) K = 16 steps; the rows in [valid, ceil16(valid)) hold the next
+// expert's data and are zeroed in shared memory first (a "fix" block).
+__device__ __forceinline__ int kvalid(const BwdArgs& g, const Tile& t, int kb) {
+  return g.mode == kDW ? min(BK, t.row_end - (t.row0 + kb * BK)) : BK;
+}
+__device__ __forceinline__ bool fix_block(int valid) { return (valid & 15) != 0; }
 
 // fp32 row stores through the warp's staging block: this thread's row holds 16 values at
 // output columns [col, col + 16); a warp store then covers 8 rows x 64 bytes.
@@ -193,10 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool a_mn = g.mode == kDW;
 
   if (warp == 0) {
-    // ---- TMA producer (whole warp: lane 0 issues, all lanes zero the tail rows) ----------
+    // ---- TMA producer (lane 0) -----------------------------------------------------------
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t landed_phase = 0;     // bit i: parity of the next completion of landed[i]
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles && !*abort_flag; tile += gridDim.x) {
       const Tile t = decode(s, g, tile);
@@ -208,43 +218,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const int valid = a_mn ? min(BK, t.row_end - (t.row0 + kb * BK)) : BK;
-        const bool masked = valid < BK;
-        uint64_t* bar = masked ? &s.landed[stage] : &s.full[stage];
+        // a fix block lands on the side barrier; the fix warp releases it to the MMA
+        uint64_t* bar = fix_block(kvalid(g, t, kb)) ? &s.landed[stage] : &s.full[stage];
         if (lane == 0) {
           mbar_arrive_expect_tx(bar, STAGE_BYTES);
           if (a_mn) {
             const int y = t.row0 + kb * BK;
+            const int yb = g.b_kwrap > 0 ? y % g.b_kwrap : y;
             tma_load_2d(s.a[stage], &tmA, t.mt * BM, y, bar);
             tma_load_2d(s.a[stage] + BOX_BYTES, &tmA, t.mt * BM + 64, y, bar);
             for (int j = 0; j < 4; ++j)
-              tma_load_2d(s.b[stage] + j * BOX_BYTES, &tmB, t.nt * BN + 64 * j, y, bar);
+              tma_load_2d(s.b[stage] + j * BOX_BYTES, &tmB, t.nt * BN + 64 * j, yb, bar);
           } else {
             tma_load_2d(s.a[stage], &tmA, kb * BK, t.row0, bar);
             const int y = t.e * g.b_krows + kb * BK;
             for (int j = 0; j < 4; ++j)
               tma_load_2d(s.b[stage] + j * BOX_BYTES, &tmB, t.nt * BN + 64 * j, y, bar);
           }
-        }
-        if (masked) {
-          // K-rows [valid, 64) of every box belong to the next expert: zero them
-          if (lane == 0)
-            w_ok = mbar_wait(&s.landed[stage], (landed_phase >> stage) & 1u, abort_flag) ? 1 : 0;
-          landed_phase ^= 1u << stage;
-          if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
-            ok = false;
-            break;
-          }
-          const int nrow = BK - valid;
-          for (int i = lane; i < 6 * nrow * 8; i += 32) {
-            const int box = i / (nrow * 8), rem = i - box * nrow * 8;
-            const int r = valid + rem / 8, c16 = rem & 7;
-            uint8_t* base = box < 2 ? s.a[stage] + box * BOX_BYTES : s.b[stage] + (box - 2) * BOX_BYTES;
-            *reinterpret_cast<uint4*>(base + r * 128 + c16 * 16) = make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.full[stage]);
         }
         if (++stage == STAGES) {
           stage = 0;
@@ -275,8 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(s.a[stage]);
           const uint32_t b0 = smem_u32(s.b[stage]);
+          const int nk = (kvalid(g, t, kb) + 15) / 16;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
+            if (k >= nk) break;
             const uint64_t ad = a_mn ? sw128_mnmajor_desc(a0 + k * 2048, BOX_BYTES)
                                      : sw128_kmajor_desc(a0 + k * 32);
             umma_bf16(d_tmem, ad, sw128_mnmajor_desc(b0 + k * 2048, BOX_BYTES), idesc,
@@ -292,6 +284,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&s.tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else if (warp == kFixWarp) {
+    // ---- fix warp: follows the producer's k-blocks; on each fix block it waits for the
+    // TMA bytes, zeroes K-rows [valid, ceil16(valid)) of the six boxes, fences them to the
+    // async proxy and releases the stage to the MMA
+    if (a_mn) {
+      int stage = 0;
+      uint32_t landed_phase = 0;   // bit i: parity of the next completion of landed[i]
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles && !*abort_flag; tile += gridDim.x) {
+        const Tile t = decode(s, g, tile);
+        const int nkb = kblocks_of(g, t);
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int valid = kvalid(g, t, kb);
+          if (fix_block(valid)) {
+            int w_ok = 1;
+            if (lane == 0)
+              w_ok = mbar_wait(&s.landed[stage], (landed_phase >> stage) & 1u, abort_flag) ? 1 : 0;
+            landed_phase ^= 1u << stage;
+            if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+              ok = false;
+              break;
+            }
+            const int nrow = ((valid + 15) & ~15) - valid;
+            for (int i = lane; i < 6 * nrow * 8; i += 32) {
+              const int box = i / (nrow * 8), rem = i - box * nrow * 8;
+              const int r = valid + rem / 8, c16 = rem & 7;
+              uint8_t* base = box < 2 ? s.a[stage] + box * BOX_BYTES : s.b[stage] + (box - 2) * BOX_BYTES;
+              *reinterpret_cast<uint4*>(base + r * 128 + c16 * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.full[stage]);
+          }
+          if (++stage == STAGES) stage = 0;
+        }
       }
     }
   } else {
@@ -311,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              static_cast<uint32_t>(acc * BN);
       // kDH / kDX: output row = the tile's row; kDW: the weight row mt * 128 + q * 32 + lane
       const int row_base = g.mode == kDW ? t.mt * BM + q * 32 : t.row0 + q * 32;
-      const int row_end = g.mode == kDW ? 0x7fffffff : t.row_end;
+      const int row_end = g.mode == kDW ? g.m_valid : t.row_end;
       const int row = row_base + lane;
 #pragma unroll 1
       for (int c = 128 * h; c < 128 * h + 128; c += 32) {
@@ -432,6 +461,7 @@ int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* 
   if ((rc = launch(m_dgu128, m_wgu, g, sm_count, st)) != MOE_OK) return rc;
   // d_down[e] = dy^T h
   g.mode = kDW;
+  g.m_valid = H;
   g.m_tiles = H / BM;
   g.n_tiles = (I + BN - 1) / BN;
   g.n_valid = I;
@@ -440,6 +470,7 @@ int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* 
   g.out = d_down;
   if ((rc = launch(m_dy64, m_h64, g, sm_count, st)) != MOE_OK) return rc;
   // d_gate_up[e] = dgu^T x_perm
+  g.m_valid = 2 * I;
   g.m_tiles = 2 * I / BM;
   g.n_tiles = (H + BN - 1) / BN;
   g.n_valid = H;
@@ -447,6 +478,47 @@ int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* 
   g.out_expert = 2LL * I * H;
   g.out = d_gate_up;
   return launch(m_dgu64, m_x64, g, sm_count, st);
+}
+
+int launch_bwd_router_gemms(const void* dl3, int Tp, const void* x, const void* wr16,
+                            const int32_t* offs_k, const int32_t* offs_m, int T, int E, int H,
+                            float* d_router, float* dx, int* status, int sm_count,
+                            cudaStream_t st) {
+  CUtensorMap m_dl64, m_dl128, m_x64, m_wr64;
+  int rc;
+  if ((rc = make_tma_map_bf16(&m_dl64, dl3, 3ull * Tp, E, 64)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_dl128, dl3, 3ull * Tp, E, 128)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_x64, x, (uint64_t)T, H, 64)) != MOE_OK) return rc;
+  if ((rc = make_tma_map_bf16(&m_wr64, wr16, (uint64_t)E, H, 64)) != MOE_OK) return rc;
+  BwdArgs g{};
+  g.n_ffn = 1;
+  g.status = status;
+  // d_router [E, H] = sum over the three parts p and tokens t of dL_p[t]^T x[t]: one group
+  // of 3 Tp K-rows (part p at rows [p Tp, p Tp + T)), x's row = K row mod Tp
+  g.mode = kDW;
+  g.offsets = offs_k;
+  g.m_valid = E;
+  g.m_tiles = (E + BM - 1) / BM;
+  g.n_tiles = (H + BN - 1) / BN;
+  g.n_valid = H;
+  g.ld_out = H;
+  g.out_expert = 0;
+  g.b_kwrap = Tp;
+  g.out = d_router;
+  if ((rc = launch(m_dl64, m_x64, g, sm_count, st)) != MOE_OK) return rc;
+  // dx [T, H] = dL_hi . W_r (bf16 operands): one group of T rows, K = E
+  g = BwdArgs{};
+  g.n_ffn = 1;
+  g.status = status;
+  g.mode = kDX;
+  g.offsets = offs_m;
+  g.kblocks = (E + BK - 1) / BK;
+  g.n_tiles = (H + BN - 1) / BN;
+  g.b_krows = 0;
+  g.n_valid = H;
+  g.ld_out = H;
+  g.out = dx;
+  return launch(m_dl128, m_wr64, g, sm_count, st);
 }
 
 }  // namespace moe

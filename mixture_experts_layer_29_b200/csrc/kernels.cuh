@@ -93,11 +93,16 @@ cudaError_t launch_bwd_dy_dgate(const void* dout, const void* x, const void* y_p
                                 const int32_t* topk_idx, const float* topk_gate,
                                 const int32_t* row_of, int T, int H, int K, int n_ffn,
                                 float scale, void* dy, float* d_gate, cudaStream_t st);
+// logit gradient of every token as three exact bf16 parts dl3 [3][Tp][E] (Tp = T rounded
+// up to 64, pad rows zero), the offset tables {0, 3Tp, 0, T} and W_r in bf16
 cudaError_t launch_bwd_router(const float* logits, const int32_t* topk_idx, const float* d_gate,
-                              int T, int E, int K, float* dL, cudaStream_t st);
-// d_router = dL^T x and dx = dL W_r (fp32, CUDA cores)
-cudaError_t launch_router_grads(const float* dL, const void* x, const float* w_router, int T,
-                                int E, int H, float* d_router, float* dx, cudaStream_t st);
+                              int T, int Tp, int E, int K, void* dl3, int32_t* offs,
+                              const float* w_router, void* wr16, int H, cudaStream_t st);
+// d_router = dL^T x (three parts) and dx = dL_hi W_r (bf16) on the tensor cores
+int launch_bwd_router_gemms(const void* dl3, int Tp, const void* x, const void* wr16,
+                            const int32_t* offs_k, const int32_t* offs_m, int T, int E, int H,
+                            float* d_router, float* dx, int* status, int sm_count,
+                            cudaStream_t st);
 cudaError_t launch_bwd_dx_combine(const float* dx_perm, const void* dout, const int32_t* topk_idx,
                                   const float* topk_gate, const int32_t* row_of, int T, int H,
                                   int K, int n_ffn, float* dx, cudaStream_t st);
