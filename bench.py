@@ -349,11 +349,24 @@ def time_backward(st: Stepper, device, seed: int, iters: int, warmup: int) -> di
 
 
 def max_over_ranks(v: float, dist_on: bool) -> float:
+    """The largest of the ranks' values (the job's time is the slowest replica's)."""
     if not dist_on:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(cfg, rank: int) -> int:
+    """Each replica routes its own batch: the token seed moves with the rank (the weights
+    are the same on every rank)."""
+    return cfg.seed + rank
+
+
+def job_throughput(tokens_per_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_step * steps * world / (max_ms / 1e3)
 
 
 def workload(args):
@@ -380,7 +393,7 @@ def run_ours(args):
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
     cfg = workload(args)
-    seed = cfg.seed + rank                 # each replica routes its own batch
+    seed = replica_seed(cfg, rank)
     w = wl.draw_weights(cfg, device, seed=cfg.seed)
     x = wl.draw_tokens(cfg, device, seed=seed)
     logits_in = wl.draw_skewed_logits(cfg, device, seed=seed) if cfg.skewed else None
@@ -391,8 +404,7 @@ def run_ours(args):
         _, per, _ = timed_loop(st, min(args.steps, 30), 0, dist_on, phases=True)
     total_ms = max_over_ranks(total_ms, dist_on)
     ms_step = total_ms / args.steps
-    tokens = cfg.T * args.steps * world
-    value = tokens / (total_ms / 1e3)
+    value = job_throughput(cfg.T, args.steps, world, total_ms)
 
     counts = st.b.counts.cpu().numpy()
     rows = int(counts[: cfg.n_ffn].sum())
@@ -560,7 +572,7 @@ def run_reference(args):
     return 0
 
 
-def main(argv=None):
+def parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
@@ -579,7 +591,11 @@ def main(argv=None):
     ap.add_argument("--no-backward", action="store_true", help="skip timing moe_backward")
     ap.add_argument("--no-overlap", action="store_true",
                     help="skip the dense-FFN-beside-MoE (two streams) measurement")
-    args = ap.parse_args(argv)
+    return ap
+
+
+def main(argv=None):
+    args = parser().parse_args(argv)
     if args.impl == "ours":
         args.warmup = max(args.warmup, 3)     # timing rule: at least 3 untimed steps
     return run_reference(args) if args.impl == "reference" else run_ours(args)
