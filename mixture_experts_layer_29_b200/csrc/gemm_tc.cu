@@ -90,7 +90,6 @@ struct GemmArgs {
   long long split_stride;   // elements between the outputs of consecutive splits
   const int32_t* gather_tok;  // non-null: A row r is row gather_tok[r] of A's tensor
   ZeroSpec zero;              // buffers cleared after the dependency wait
-  int half_tiles;             // pair kernel: tails of at most 128 rows run as M = 128
   int gu_raw;                 // gate/up: store G and U (bf16, [rows, 2I]) instead of h
 };
 
@@ -515,67 +514,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- CTA-pair variant of the expert GEMMs (tcgen05 cta_group::2) -------------------------
 // A cluster of two CTAs computes a 256 x 256 tile: CTA r loads rows [128r, 128r+128) of the
-// A tile and 128 rows of the N tile's B (gate/up: gate rows [64r, 64r+64) then the
-// matching up rows, as two 64-row boxes; down: W_d rows [128r, 128r+128)), so each CTA
-// moves 32 KB per k-block instead of 48 KB. Both CTAs' TMA loads count on the leader's
-// (rank 0) full barrier; the leader's single thread issues tcgen05.mma.cta_group::2 and
-// commits to the empty / accumulator-full barriers of both CTAs (two commits, one per
-// CTA); both CTAs' epilogues read their own TMEM rows and release the accumulator on the
+// A tile and B rows [128r, 128r+128) of the N tile (gate/up: CTA 0 the gate rows, CTA 1
+// the up rows), so each CTA moves 32 KB per k-block instead of 48 KB. Both CTAs' TMA loads
+// count on the leader's (rank 0) full barrier; the leader's single thread issues
+// tcgen05.mma.cta_group::2 (M = 256) and commits to the empty / accumulator-full barriers
+// of both CTAs (two commits, one per CTA); both CTAs' epilogues read their own TMEM rows
+// (the same column layout as the one-CTA kernel) and release the accumulator on the
 // leader's barrier.
-// An expert's last tile holds count mod 256 rows; when that is at most 128 it runs as an
-// M = 128 MMA (64 rows per CTA: A loaded from row0 + 64r, its first 64 rows used), which
-// halves the padded work of the tail. Its accumulator lands in TMEM as the 2x2 layout:
-// lanes 0-63 hold the CTA's 64 rows for N columns [0, 128), lanes 64-127 the same rows
-// for N columns [128, 256), both in TMEM columns [0, 128) of the accumulator.
 constexpr int BMP = 256;                             // M rows per CTA pair
 constexpr int PSTAGES = 6;                           // 32 KB per stage per CTA
 constexpr int P_B_BYTES = 128 * BK * 2;              // 16 KB: this CTA's half of B
 constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES;   // 32 KB
 constexpr uint32_t kIdescPair = idesc_bf16_f32(BMP, BN);
-constexpr uint32_t kIdescPairHalf = idesc_bf16_f32(128, BN);
-
-__device__ __forceinline__ bool half_tile(const GemmArgs& g, const Tile& t) {
-  return g.half_tiles && t.row_end - t.row0 <= 128;
-}
-
-// Epilogue of one pair tile for one thread (warp quarter q, column half h of the warp pair).
-// Full tile (M = 256): row 128r + 32q + lane; gate/up: h columns [64h, 64h + 64) from gate
-// TMEM columns 128h + [0, 64) and up columns 128h + 64 + [0, 64); down: columns
-// [128h, 128h + 128). Half tile (M = 128): row 64r + 32(q & 1) + lane, N block ib = q >> 1;
-// gate/up: h columns 64 ib + 32h + [0, 32) from gate TMEM columns 32h + [0, 32) and up
-// columns 64 + 32h + [0, 32); down: columns 128 ib + 64h + [0, 64) at TMEM 64h + [0, 64).
-__device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, uint32_t tbase,
-                                              uint32_t rank, int q, int h, float (*stg)[20],
-                                              int lane) {
-  if (!half_tile(g, t)) {
-    const int row = t.row0 + 128 * (int)rank + 32 * q + lane;
-    if (g.mode == kGateUp) {
-#pragma unroll 1
-      for (int j = 0; j < 64; j += 32)
-        epi_gateup_chunk(g, t, tbase, row, 128 * h + j, 128 * h + 64 + j, 64 * h + j);
-      return;
-    }
-    int tok;
-    float sc;
-    row_scale(g, t, row, tok, sc);
-#pragma unroll 1
-    for (int c = 128 * h; c < 128 * h + 128; c += 32)
-      epi_down_chunk(g, t, tbase, row, c, c, tok, sc, stg, lane);
-    return;
-  }
-  const int row = t.row0 + 64 * (int)rank + 32 * (q & 1) + lane;
-  const int ib = q >> 1;
-  if (g.mode == kGateUp) {
-    epi_gateup_chunk(g, t, tbase, row, 32 * h, 64 + 32 * h, 64 * ib + 32 * h);
-    return;
-  }
-  int tok;
-  float sc;
-  row_scale(g, t, row, tok, sc);
-#pragma unroll 1
-  for (int j = 0; j < 64; j += 32)
-    epi_down_chunk(g, t, tbase, row, 64 * h + j, 128 * ib + 64 * h + j, tok, sc, stg, lane);
-}
 
 struct alignas(1024) PairStorage {
   uint8_t a[PSTAGES][A_BYTES];
@@ -672,23 +622,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       for (int tile = cluster; tile < total_tiles && !*abort_flag; tile += nclusters) {
         const Tile t = decode_pair_tile(s, g, tile);
-        const int arow = t.row0 + (half_tile(g, t) ? 64 : 128) * (int)rank;
-        // gate/up: gate rows [64r, 64r+64) of the N tile, then the same up rows (two
-        // 64-row boxes); down: W_d rows [128r, 128r+128) of the N tile
-        const int brow = g.mode == kGateUp ? t.e * g.b_rows + t.nt * BM + 64 * (int)rank
-                                           : t.e * g.b_rows + t.nt * BN + 128 * (int)rank;
+        const int arow = t.row0 + 128 * (int)rank;
+        const int brow = g.mode == kGateUp
+                             ? t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM
+                             : t.e * g.b_rows + t.nt * BN + 128 * (int)rank;
         for (int kb = 0; kb < g.kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
           const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * P_STAGE_BYTES);
           tma_load_2d_pair(s.a[stage], &tmA, kb * BK, arow, full_leader);
-          if (g.mode == kGateUp) {
-            tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
-            tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB, kb * BK, brow + g.b_second,
-                             full_leader);
-          } else {
-            tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
-          }
+          tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
           if (++stage == PSTAGES) {
             stage = 0;
             phase ^= 1u;
@@ -705,7 +648,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
-        const uint32_t idesc = half_tile(g, decode_pair_tile(s, g, tile)) ? kIdescPairHalf : kIdescPair;
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -717,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
-                           idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                           kIdescPair, (kb > 0 || k > 0) ? 1u : 0u);
           const uint32_t e_local = smem_u32(&s.empty[stage]);
           umma_commit_pair(mapa_shared(e_local, 0));
           umma_commit_pair(mapa_shared(e_local, 1));
@@ -749,7 +691,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_pair(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
+      epilogue_expert(g, t, tbase, t.row0 + 128 * (int)rank + q * 32 + lane, half,
+                      s.epi_stage[warp - 2], lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
@@ -867,15 +810,6 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
 
 // The CTA-pair kernel pays off once groups are tall (256-row tiles); small batches keep
 // the one-CTA kernel. MOE_B200_GEMM_PAIR=0 / 1 forces either (for measurements).
-// MOE_B200_PAIR_HALF=0 runs every pair tile as M = 256 (for measurements).
-int pair_half_tiles() {
-  static const int v = [] {
-    const char* e = getenv("MOE_B200_PAIR_HALF");
-    return (e && e[0] == '0') ? 0 : 1;
-  }();
-  return v;
-}
-
 bool use_pair_kernel(int T) {
   static const char* env = getenv("MOE_B200_GEMM_PAIR");
   if (env && env[0] == '0') return false;
@@ -1033,10 +967,8 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   } else {
     if ((rc = make_map(&mx, x, (uint64_t)T, H, 1)) != MOE_OK) return rc;
   }
-  // the CTA-pair kernel loads gate/up B as 64-row boxes (gate rows, then the same up rows)
   const bool pair = use_pair_kernel(T) && x_perm != nullptr;
-  if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H, pair ? 64 : BM)) != MOE_OK)
-    return rc;
+  if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H)) != MOE_OK) return rc;
   if ((rc = make_map(&mh, h, rows, I)) != MOE_OK) return rc;
   if ((rc = make_map(&mwd, w_down, (uint64_t)n_ffn * H, I)) != MOE_OK) return rc;
 
@@ -1055,7 +987,6 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g1.status = status;
   g1.ksplit = 1;
   g1.kb_per_split = g1.kblocks;
-  g1.half_tiles = pair_half_tiles();
   if ((rc = pair ? launch_pair(mx, mwgu, g1, sm_count, st) : launch_one(mx, mwgu, g1, sm_count, st)) !=
       MOE_OK)
     return rc;
@@ -1077,7 +1008,6 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g2.status = status;
   g2.ksplit = 1;
   g2.kb_per_split = g2.kblocks;
-  g2.half_tiles = pair_half_tiles();
   return pair ? launch_pair(mh, mwd, g2, sm_count, st) : launch_one(mh, mwd, g2, sm_count, st);
 }
 
@@ -1090,8 +1020,7 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
   CUtensorMap mx, mwgu;
   int rc;
   if ((rc = make_map(&mx, x_perm, rows, H)) != MOE_OK) return rc;
-  if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H, pair ? 64 : BM)) != MOE_OK)
-    return rc;
+  if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H)) != MOE_OK) return rc;
   GemmArgs g{};
   g.mode = kGateUp;
   g.gu_raw = 1;
@@ -1107,7 +1036,6 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
   g.status = status;
   g.ksplit = 1;
   g.kb_per_split = g.kblocks;
-  g.half_tiles = pair_half_tiles();
   return pair ? launch_pair(mx, mwgu, g, sm_count, st) : launch_one(mx, mwgu, g, sm_count, st);
 }
 
