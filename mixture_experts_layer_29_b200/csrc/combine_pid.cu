@@ -125,24 +125,30 @@ __global__ void k_pid_init(const float* __restrict__ bias, float* __restrict__ s
   }
 }
 
-// One CTA of 1024 threads; expert i = threadIdx.x (n_ffn <= 1024). The statistics are
-// reduced in one pass: warp butterflies, then thread 0 over the warps (fixed order).
-__global__ void __launch_bounds__(1024) k_pid_update(moe_pid_t pid, const int32_t* __restrict__ counts,
-                                                     const int32_t* __restrict__ hist,
-                                                     float* __restrict__ bias, float* __restrict__ st,
-                                                     float* __restrict__ stats, int T, int K,
-                                                     int n_ffn, int E) {
-  __shared__ double red[32][8];
+// One CTA of kPidThreads; thread i updates experts i, i + kPidThreads, ... (each expert's
+// bias in fp32, in the fixed order of the PID law). The statistics are reduced in one
+// pass: warp butterflies, then warp 0 over the warps (fixed order).
+constexpr int kPidThreads = 256;
+
+__global__ void __launch_bounds__(kPidThreads) k_pid_update(moe_pid_t pid,
+                                                            const int32_t* __restrict__ counts,
+                                                            const int32_t* __restrict__ hist,
+                                                            float* __restrict__ bias,
+                                                            float* __restrict__ st,
+                                                            float* __restrict__ stats, int T,
+                                                            int K, int n_ffn, int E) {
+  constexpr int W = kPidThreads / 32;
+  __shared__ double red[W][8];
   pdl_launch_dependents();
   pdl_wait();
-  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // v: [0] FFN count, [1] max FFN count, [2] FFN experts hit, [3] zero-expert count,
   //    [4] |e|, [5] max |e|, [6] n * hist[n], [7] n^2 * hist[n]
   double v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  if (i < n_ffn) {
+  const float tau = __fdiv_rn(__fmul_rn(pid.target_ratio, (float)K), (float)n_ffn);
+  for (int i = tid; i < n_ffn; i += kPidThreads) {
     const int c = counts[i];
     const float f = __fdiv_rn((float)c, (float)T);
-    const float tau = __fdiv_rn(__fmul_rn(pid.target_ratio, (float)K), (float)n_ffn);
     const float e = __fsub_rn(tau, f);
     const float integ = __fadd_rn(st[n_ffn + i], e);
     const float deriv = __fsub_rn(e, st[2 * n_ffn + i]);
@@ -152,14 +158,16 @@ __global__ void __launch_bounds__(1024) k_pid_update(moe_pid_t pid, const int32_
     bias[i] = b;
     st[n_ffn + i] = integ;
     st[2 * n_ffn + i] = e;
-    v[0] = v[1] = (double)c;
-    v[2] = c > 0 ? 1.0 : 0.0;
-    v[4] = v[5] = fabs((double)e);
+    v[0] += (double)c;
+    v[1] = fmax(v[1], (double)c);
+    v[2] += c > 0 ? 1.0 : 0.0;
+    v[4] += fabs((double)e);
+    v[5] = fmax(v[5], fabs((double)e));
   }
-  for (int j = n_ffn + i; j < E; j += blockDim.x) v[3] += (double)counts[j];
-  if (i <= K) {
-    v[6] = (double)hist[i] * i;
-    v[7] = (double)hist[i] * i * i;
+  for (int j = n_ffn + tid; j < E; j += kPidThreads) v[3] += (double)counts[j];
+  for (int n = tid; n <= K; n += kPidThreads) {
+    v[6] += (double)hist[n] * n;
+    v[7] += (double)hist[n] * n * n;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -173,22 +181,29 @@ __global__ void __launch_bounds__(1024) k_pid_update(moe_pid_t pid, const int32_
 #pragma unroll
     for (int k = 0; k < 8; ++k) red[warp][k] = v[k];
   __syncthreads();
-  if (stats && i == 0) {
-    double r[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w)
+  if (stats && warp == 0) {
+    // lane k < 8 combines statistic k over the warps in order
+    double r = 0.0;
+    if (lane < 8) {
+      const bool mx = lane == 1 || lane == 5;
+      for (int w = 0; w < W; ++w) r = mx ? fmax(r, red[w][lane]) : r + red[w][lane];
+    }
+    double rr[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) r[k] = (k == 1 || k == 5) ? fmax(r[k], red[w][k]) : r[k] + red[w][k];
-    const double mean = r[6] / T;
-    const double var = fmax(0.0, r[7] / T - mean * mean);
-    const double mean_load = r[0] / n_ffn;
-    stats[0] = (float)(mean / K);
-    stats[1] = (float)mean;
-    stats[2] = (float)sqrt(var);
-    stats[3] = (float)(mean_load > 0.0 ? r[1] / mean_load : 0.0);
-    stats[4] = (float)r[2];
-    stats[5] = (float)(r[3] / ((double)T * K));
-    stats[6] = (float)(r[4] / n_ffn);
-    stats[7] = (float)r[5];
+    for (int k = 0; k < 8; ++k) rr[k] = __shfl_sync(0xffffffffu, r, k);
+    if (lane == 0) {
+      const double mean = rr[6] / T;
+      const double var = fmax(0.0, rr[7] / T - mean * mean);
+      const double mean_load = rr[0] / n_ffn;
+      stats[0] = (float)(mean / K);
+      stats[1] = (float)mean;
+      stats[2] = (float)sqrt(var);
+      stats[3] = (float)(mean_load > 0.0 ? rr[1] / mean_load : 0.0);
+      stats[4] = (float)rr[2];
+      stats[5] = (float)(rr[3] / ((double)T * K));
+      stats[6] = (float)(rr[4] / n_ffn);
+      stats[7] = (float)rr[5];
+    }
   }
 }
 
@@ -243,7 +258,7 @@ cudaError_t launch_pid_init(const float* bias, float* pid_state, int n_ffn, cuda
 cudaError_t launch_pid_update(const moe_pid_t& pid, const int32_t* counts,
                               const int32_t* nffn_hist, float* bias, float* pid_state,
                               float* stats, int T, int K, int n_ffn, int E, cudaStream_t st) {
-  const cudaError_t e = launch_kernel(k_pid_update, 1, 1024, 0, st, 1, pid, counts, nffn_hist,
+  const cudaError_t e = launch_kernel(k_pid_update, 1, kPidThreads, 0, st, 1, pid, counts, nffn_hist,
                                       bias, pid_state, stats, T, K, n_ffn, E);
   count_launch();
   return e;

@@ -183,7 +183,6 @@ __global__ void __launch_bounds__(256) k_perm_scatter(
 
 // ---- small batches (T <= 512): all index work in one CTA, then a wide copy kernel -------
 constexpr int kSmallT = 512;
-constexpr int kSmallChunks = kSmallT / 32;
 
 // One CTA of 512 threads: bitmasks [n_ffn][16] and their per-expert prefixes in shared
 // memory, the expert counts, the offsets (block scan), then every pick's row. The same
@@ -193,16 +192,17 @@ __global__ void __launch_bounds__(512) k_perm_index_small(
     int E, int K, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
     int32_t* __restrict__ row_of, float* __restrict__ row_gate, int* status) {
   extern __shared__ uint32_t sm[];
-  uint32_t* masks = sm;                                          // [n_ffn][16]
-  int32_t* crel = reinterpret_cast<int32_t*>(sm + n_ffn * kSmallChunks);   // [n_ffn][16]
-  int32_t* offs = crel + n_ffn * kSmallChunks;                   // [n_ffn + 1]
+  const int nch = (T + 31) / 32;                                 // 32-token chunks (<= 16)
+  uint32_t* masks = sm;                                          // [n_ffn][nch]
+  int32_t* crel = reinterpret_cast<int32_t*>(sm + n_ffn * nch);  // [n_ffn][nch]
+  int32_t* offs = crel + n_ffn * nch;                            // [n_ffn + 1]
   __shared__ int32_t s_wsum[16];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_launch_dependents();
-  for (int i = tid; i < n_ffn * kSmallChunks; i += blockDim.x) masks[i] = 0u;
+  for (int i = tid; i < n_ffn * nch; i += blockDim.x) masks[i] = 0u;
   pdl_wait();
   __syncthreads();
-  const int t = tid;
+  const int t = tid;          // warp w holds the tokens of chunk w, lane = token bit
   // keep[k]: slot k is in range and the first slot of its expert (a repeated expert shows
   // as its bit already set: a token's own slots run in order, other tokens use other bits)
   uint32_t keep = 0u;
@@ -220,8 +220,8 @@ __global__ void __launch_bounds__(512) k_perm_index_small(
         continue;
       }
       if (e < n_ffn) {
-        const uint32_t bit = 1u << (t & 31);
-        if (atomicOr(&masks[e * kSmallChunks + (t >> 5)], bit) & bit) {
+        const uint32_t bit = 1u << lane;
+        if (atomicOr(&masks[e * nch + warp], bit) & bit) {
           set_status(status, MOE_ERR_DEVICE_CHECK);
           continue;
         }
@@ -244,9 +244,9 @@ __global__ void __launch_bounds__(512) k_perm_index_small(
   int local = 0;
   for (int e = tid; e < n_ffn; e += blockDim.x) {
     int run = 0;
-    for (int c = 0; c < kSmallChunks; ++c) {
-      crel[e * kSmallChunks + c] = run;
-      run += __popc(masks[e * kSmallChunks + c]);
+    for (int c = 0; c < nch; ++c) {
+      crel[e * nch + c] = run;
+      run += __popc(masks[e * nch + c]);
     }
     offs[e] = run;          // count for now
   }
@@ -285,8 +285,8 @@ __global__ void __launch_bounds__(512) k_perm_index_small(
       const int e = ek[k];
       if (((keep >> k) & 1u) && e < n_ffn) {
         const int c = t >> 5;
-        r = offs[e] + crel[e * kSmallChunks + c] +
-            __popc(masks[e * kSmallChunks + c] & ((1u << (t & 31)) - 1u));
+        r = offs[e] + crel[e * nch + c] +
+            __popc(masks[e * nch + c] & ((1u << (t & 31)) - 1u));
         perm_token[r] = t;
         row_gate[r] = topk_gate[(size_t)t * K + k];
       }
@@ -347,7 +347,7 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, cons
                            float* out_acc, int* status, cudaStream_t st) {
   if (T <= kSmallT && n_ffn <= 1024) {
     // one CTA for the indices, then a wide copy (short chain for small batches)
-    const size_t smem = sizeof(uint32_t) * (size_t)n_ffn * kSmallChunks * 2 + sizeof(int32_t) * (n_ffn + 1);
+    const size_t smem = sizeof(uint32_t) * (size_t)n_ffn * ((T + 31) / 32) * 2 + sizeof(int32_t) * (n_ffn + 1);
     if (smem > 48 * 1024) {
       const cudaError_t e = cudaFuncSetAttribute(k_perm_index_small,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
