@@ -48,6 +48,7 @@ constexpr int kMaxExperts = 1024;
 constexpr uint32_t kTmemCols = 512;                  // two 256-column fp32 accumulators
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
 
+
 enum Mode : int { kGateUp = 0, kDownStore = 1, kDownAtomic = 2, kLogits = 3 };
 
 struct alignas(1024) SharedStorage {
@@ -91,6 +92,7 @@ struct GemmArgs {
   const int32_t* gather_tok;  // non-null: A row r is row gather_tok[r] of A's tensor
   ZeroSpec zero;              // buffers cleared after the dependency wait
   int gu_raw;                 // gate/up: store G and U (bf16, [rows, 2I]) instead of h
+  int logit_n;                // router: N tile (128 or 256 logits)
 };
 
 struct Tile {
@@ -248,9 +250,9 @@ __device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t
     epi_down_chunk(g, t, tbase, row, c, c, tok, sc, stg, lane);
 }
 
-// LOGITS: the router instantiation (mode kLogits, running sums in the epilogue); the
-// expert GEMMs use the other one.
-template <bool LOGITS>
+// LOGITS: the router instantiations (mode kLogits, running sums in the epilogue), with N
+// tiles of NL logits; the expert GEMMs use <false, BN>.
+template <bool LOGITS, int NL>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
@@ -357,15 +359,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
         const Tile t = decode_tile(s, g, tile);
-        const int brow0 = t.e * g.b_rows + t.nt * (g.mode == kGateUp ? BM : BN);
+        const int brow0 = t.e * g.b_rows + t.nt * (LOGITS ? NL : g.mode == kGateUp ? BM : BN);
         const int brow1 = brow0 + g.b_second;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
-          mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
+          mbar_arrive_expect_tx(&s.full[stage], LOGITS ? A_BYTES + NL * BK * 2 : STAGE_BYTES);
           const int ka = g.a_kwrap > 0 ? kb % g.a_kwrap : kb;
           tma_load_2d(s.a[stage], &tmA, ka * BK, t.row0, &s.full[stage]);
           tma_load_2d(s.b[stage], &tmB, kb * BK, brow0, &s.full[stage]);
-          tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
+          if (!LOGITS || NL == 256)
+            tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -397,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
               umma_bf16(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
-                        kIdesc, (kb > c0 || k > 0) ? 1u : 0u);
+                        LOGITS ? idesc_bf16_f32(BM, NL) : kIdesc, (kb > c0 || k > 0) ? 1u : 0u);
             umma_commit(&s.empty[stage]);
             if (++stage == STAGES) {
               stage = 0;
@@ -424,10 +427,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = t.row0 + row_in_tile;
       const int cl = chunk_len(g, t);
       constexpr bool logits = LOGITS;
-      float sum[LOGITS ? 128 : 1];   // router logits: running fp32 sum of this half-row
+      constexpr int NH = NL / 2;     // router: columns per thread (half of the tile)
+      float sum[LOGITS ? NH : 1];    // router logits: running fp32 sum of this half-row
       if constexpr (LOGITS) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) sum[i] = 0.f;
+        for (int i = 0; i < NH; ++i) sum[i] = 0.f;
       }
       for (int c0 = t.kb0; c0 < t.kb1; c0 += cl) {
         // one lane waits, the warp follows it: tcgen05.ld below needs all 32 lanes
@@ -441,9 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (LOGITS) {
           // add this chunk to the running sum (fp32, round to nearest)
 #pragma unroll
-          for (int c = 0; c < 128; c += 32) {
+          for (int c = 0; c < NH; c += 32) {
             uint32_t v[32];
-            tmem_ld_32x32b_x32(tbase + 128 * half + c, v);
+            tmem_ld_32x32b_x32(tbase + NH * half + c, v);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) sum[c + i] = __fadd_rn(sum[c + i], __uint_as_float(v[i]));
@@ -462,10 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // row 8i + l/4, columns 4(l%4)..+3, so a warp store covers 8 rows x 64 bytes
           float (*stg)[20] = s.epi_stage[warp - 2];
           float* outp = static_cast<float*>(g.out) + t.split * g.split_stride;
-          const int col0 = t.nt * BN + 128 * half;
+          const int col0 = t.nt * NL + NH * half;
           const bool vec = (g.ld_out & 3) == 0 && (reinterpret_cast<uintptr_t>(g.out) & 15) == 0;
 #pragma unroll
-          for (int c = 0; c < 128; c += 16) {
+          for (int c = 0; c < NH; c += 16) {
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               *reinterpret_cast<float4*>(&stg[lane][4 * v]) =
@@ -751,7 +755,8 @@ int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, 
                cudaStream_t st) {
   constexpr size_t smem = sizeof(SharedStorage) + 1024;
   static_assert(smem <= 227 * 1024, "shared memory budget");
-  auto kern = g.mode == kLogits ? k_grouped_gemm_tc<true> : k_grouped_gemm_tc<false>;
+  auto kern = g.mode != kLogits ? k_grouped_gemm_tc<false, BN>
+               : g.logit_n == 128 ? k_grouped_gemm_tc<true, 128> : k_grouped_gemm_tc<true, 256>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
@@ -852,7 +857,7 @@ __global__ void __launch_bounds__(256) k_split_router_weight(const float4* __res
 
 }  // namespace
 
-// Router logits: 128 x 256 tiles, K = 3H (the three weight parts); the tensor cores
+// Router logits: 128 x 128 tiles, K = 3H (the three weight parts); the tensor cores
 // accumulate kRouterChunk k-blocks at a time and the epilogue sums the chunks in fp32.
 constexpr int kRouterChunk = 6;
 // k-blocks per split at least (MOE_B200_ROUTER_MINSPLIT overrides it, for measurements)
@@ -865,10 +870,19 @@ int router_min_split() {
   return v;
 }
 
+// The router GEMM's N tile: 256 logits when the 256-wide tiles fill a wave of SMs (the
+// A tile is then read once per 256 logits), else 128 (twice the tiles for a small batch:
+// decode's 128 tokens x 768 logits fill 144 CTAs with the K split instead of 72).
+int router_tile_n(int T, int E, int sm_count) {
+  const long tiles256 = (long)((T + BM - 1) / BM) * ((E + 255) / 256);
+  return tiles256 >= sm_count ? 256 : 128;
+}
+
 int router_tc_splitk(int T, int E, int H, int sm_count) {
   if (sm_count > 160) sm_count = 160;
   if (sm_count < 1) sm_count = 1;
-  const long tiles = (long)((T + BM - 1) / BM) * ((E + BN - 1) / BN);
+  const int nl = router_tile_n(T, E, sm_count);
+  const long tiles = (long)((T + BM - 1) / BM) * ((E + nl - 1) / nl);
   const int kblocks = 3 * H / BK;
   if (tiles <= 0) return 1;
   // a full wave already: no partial slices (splitting K to fill the last wave better
@@ -884,7 +898,11 @@ int router_tc_splitk(int T, int E, int H, int sm_count) {
 }
 
 size_t router_tc_scratch_bytes(int T, int E, int H) {
-  const int S = router_tc_splitk(T, E, H, 160);
+  int S = 1;                                          // the most slices any SM count takes
+  for (int sm = 1; sm <= 160; ++sm) {
+    const int s_sm = router_tc_splitk(T, E, H, sm);
+    if (s_sm > S) S = s_sm;
+  }
   size_t b = (size_t)E * 3 * H * 2;                  // split weight
   b = (b + 1023) / 1024 * 1024;
   if (S > 1) b += (size_t)S * T * E * sizeof(float); // per-split partial logits
@@ -936,7 +954,8 @@ int launch_router_logits_tc(const void* x, const float* w_router, const void* w_
   g.ksplit = S;
   g.kb_per_split = (g.kblocks + S - 1) / S;
   g.kchunk = kRouterChunk;
-  g.n_tiles = (E + BN - 1) / BN;
+  g.logit_n = router_tile_n(T, E, sm_count > 160 ? 160 : sm_count);
+  g.n_tiles = (E + g.logit_n - 1) / g.logit_n;
   g.b_rows = 0;
   g.b_second = BM;
   g.n_valid = E;
