@@ -144,22 +144,25 @@ def oracle_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(cfg, w, x_dev, tokens):
+def oracle_sample(cfg, w, x_dev, tokens, logits_dev=None):
     """Time the oracle on `tokens` of the workload: logits (float64), routing, and the
     SwiGLU experts of those tokens. Weights of the experts they hit are copied to the
-    host first (outside the timed region). Returns (seconds, tokens)."""
+    host first (outside the timed region). Where the workload's logits are an input
+    (`logits_dev`, the skewed workload), the oracle takes those rows instead of computing
+    them. Returns (seconds, tokens)."""
     import oracle.moe_oracle as orc
     x = x_dev[tokens].float().cpu().numpy()
     wr = w.w_router.cpu().numpy()
     bias = w.bias.cpu().numpy()
+    given = None if logits_dev is None else logits_dev[tokens].cpu().numpy()
     # routing decides which experts' weights to stage; staging is not timed
-    L_probe = orc.router_logits(x, wr).astype(np.float32)
+    L_probe = given if given is not None else orc.router_logits(x, wr).astype(np.float32)
     r = orc.route(L_probe, bias, cfg.n_ffn, cfg.K)
     experts = sorted({int(e) for e in r.topk_idx.ravel() if e < cfg.n_ffn})
     wgu = {e: w.w_gate_up[e].float().cpu().numpy() for e in experts}
     wd = {e: w.w_down[e].float().cpu().numpy() for e in experts}
     t0 = time.perf_counter()
-    L = orc.router_logits(x, wr).astype(np.float32)
+    L = given if given is not None else orc.router_logits(x, wr).astype(np.float32)
     orc.moe_layer_forward(x, L, bias, wgu, wd, cfg.n_ffn, cfg.K, cfg.ffn_out_scale)
     return time.perf_counter() - t0, len(tokens)
 
@@ -381,6 +384,14 @@ def workload(args):
     return cfg.with_(**kw) if kw else cfg
 
 
+def workload_config(args, cfg) -> dict:
+    """The `config` keys both arms report: the workload and the layer's sizes."""
+    name = args.workload if cfg == wl.CONFIGS[args.workload] else \
+        f"{args.workload} (overridden: T={cfg.T}, n_ffn={cfg.n_ffn}, n_zero={cfg.n_zero})"
+    return {"workload": name, "tokens": cfg.T, "hidden": cfg.H, "expert_intermediate": cfg.I,
+            "ffn_experts": cfg.n_ffn, "zero_experts": cfg.n_zero, "top_k": cfg.K}
+
+
 def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -491,7 +502,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rng = np.random.default_rng(0)
         toks = sorted(rng.choice(cfg.T, size=min(args.cpu_tokens, cfg.T), replace=False).tolist())
-        secs, n = oracle_sample(cfg, w, x, toks)
+        secs, n = oracle_sample(cfg, w, x, toks, logits_in)
         cpu = {"value": round(n / secs, 3), "unit": UNIT, "cores": oracle_threads(),
                "kind": "oracle",
                "sample": f"{n} of the {cfg.T} tokens (logits, routing and SwiGLU experts in "
@@ -502,11 +513,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded normal inputs and random-init weights of the layer's shape)",
-        "config": {"workload": args.workload if cfg == wl.CONFIGS[args.workload] else
-                   f"{args.workload} (overridden: T={cfg.T}, n_ffn={cfg.n_ffn}, n_zero={cfg.n_zero})",
-                   "tokens": cfg.T, "hidden": cfg.H,
-                   "expert_intermediate": cfg.I, "ffn_experts": cfg.n_ffn,
-                   "zero_experts": cfg.n_zero, "top_k": cfg.K, "combine": args.combine,
+        "config": {**workload_config(args, cfg), "combine": args.combine,
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "no flush: each step streams the touched experts' weights "
                          f"({roofline['ffn_rows']} FFN rows) and writes x_perm, both far above "
@@ -546,11 +553,12 @@ def run_reference(args):
         return 0
     w = wl.draw_weights(cfg, device)
     x = wl.draw_tokens(cfg, device)
+    logits_in = wl.draw_skewed_logits(cfg, device) if cfg.skewed else None
     rng = np.random.default_rng(1)
     times, n_tok = [], 0
     for k in range(args.warmup + args.steps):
         toks = sorted(rng.choice(cfg.T, size=args.ref_tokens, replace=False).tolist())
-        secs, n = oracle_sample(cfg, w, x, toks)
+        secs, n = oracle_sample(cfg, w, x, toks, logits_in)
         if k >= args.warmup:
             times.append(secs)
             n_tok += n
@@ -563,7 +571,7 @@ def run_reference(args):
             "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload, "tokens": cfg.T},
+            "data": "synthetic", "config": workload_config(args, cfg),
             "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
