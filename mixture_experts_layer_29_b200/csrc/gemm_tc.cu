@@ -93,6 +93,7 @@ struct GemmArgs {
   ZeroSpec zero;              // buffers cleared after the dependency wait
   int gu_raw;                 // gate/up: store G and U (bf16, [rows, 2I]) instead of h
   int logit_n;                // router: N tile (128 or 256 logits)
+  int half_tiles;             // pair kernel: an expert's last tile of <= 128 rows runs as M = 128
 };
 
 struct Tile {
@@ -525,11 +526,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // of both CTAs (two commits, one per CTA); both CTAs' epilogues read their own TMEM rows
 // (the same column layout as the one-CTA kernel) and release the accumulator on the
 // leader's barrier.
+// Half tiles: an expert's last tile holds count mod 256 rows; when that is at most 128 it
+// runs as an M = 128 MMA over both CTAs (64 rows each: A loaded from row0 + 64r, its first
+// 64 rows used), which halves the tail's padded work. The accumulator then lands in TMEM
+// columns [0, 128) as the 2 x 2 layout: lanes 0-63 hold the CTA's 64 rows for N columns
+// [0, 128) (the leader's B rows), lanes 64-127 the same rows for N columns [128, 256) (the
+// peer's B rows). So that each lane quarter holds gate and up columns of the same h
+// columns, the gate/up half tile loads CTA r's B as gate rows [64r, 64r + 64) of the N tile
+// followed by the same up rows (two 64-row boxes, the same shared-memory layout as one
+// 128-row box); full tiles keep the 128-row gate / up boxes.
 constexpr int BMP = 256;                             // M rows per CTA pair
 constexpr int PSTAGES = 6;                           // 32 KB per stage per CTA
 constexpr int P_B_BYTES = 128 * BK * 2;              // 16 KB: this CTA's half of B
 constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES;   // 32 KB
 constexpr uint32_t kIdescPair = idesc_bf16_f32(BMP, BN);
+constexpr uint32_t kIdescPairHalf = idesc_bf16_f32(128, BN);
 
 struct alignas(1024) PairStorage {
   uint8_t a[PSTAGES][A_BYTES];
@@ -563,9 +574,41 @@ __device__ __forceinline__ Tile decode_pair_tile(const PairStorage& s, const Gem
   return t;
 }
 
+__device__ __forceinline__ bool half_tile(const GemmArgs& g, const Tile& t) {
+  return g.half_tiles && t.row_end - t.row0 <= 128;
+}
+
+// Epilogue of one pair tile for one thread of warp quarter q and column half h. Full tile
+// (M = 256): row 128r + 32q + lane, as in the one-CTA kernel. Half tile (M = 128): row
+// 64r + 32(q & 1) + lane and N block ib = q >> 1; gate/up: h columns 64 ib + 32h + [0, 32)
+// from the gate TMEM columns 32h + [0, 32) and the up columns 64 + 32h + [0, 32); down:
+// output columns 128 ib + 64h + [0, 64) from TMEM columns 64h + [0, 64).
+__device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                              uint32_t rank, int q, int h, float (*stg)[20],
+                                              int lane) {
+  if (!half_tile(g, t)) {
+    epilogue_expert(g, t, tbase, t.row0 + 128 * (int)rank + q * 32 + lane, h, stg, lane);
+    return;
+  }
+  const int row = t.row0 + 64 * (int)rank + 32 * (q & 1) + lane;
+  const int ib = q >> 1;
+  if (g.mode == kGateUp) {
+    epi_gateup_chunk(g, t, tbase, row, 32 * h, 64 + 32 * h, 64 * ib + 32 * h);
+    return;
+  }
+  int tok;
+  float sc;
+  row_scale(g, t, row, tok, sc);
+#pragma unroll 1
+  for (int j = 0; j < 64; j += 32)
+    epi_down_chunk(g, t, tbase, row, 64 * h + j, 128 * ib + 64 * h + j, tok, sc, stg, lane);
+}
+
+// tmB64: the gate/up B tensor with 64-row boxes (half tiles); unused by the down GEMM.
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB64, const GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
   PairStorage& s = *reinterpret_cast<PairStorage*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -588,6 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    if (g.half_tiles && g.mode == kGateUp) prefetch_tensormap(&tmB64);
   }
   pdl_wait();
   for (int i = threadIdx.x; i <= g.n_ffn; i += kThreads) s.offs[i] = g.offsets[i];
@@ -626,16 +670,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       for (int tile = cluster; tile < total_tiles && !*abort_flag; tile += nclusters) {
         const Tile t = decode_pair_tile(s, g, tile);
-        const int arow = t.row0 + 128 * (int)rank;
-        const int brow = g.mode == kGateUp
-                             ? t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM
-                             : t.e * g.b_rows + t.nt * BN + 128 * (int)rank;
+        const bool half = half_tile(g, t);
+        const bool split_b = half && g.mode == kGateUp;   // 64 gate + 64 up rows
+        const int arow = t.row0 + (half ? 64 : 128) * (int)rank;
+        const int brow = g.mode != kGateUp ? t.e * g.b_rows + t.nt * BN + 128 * (int)rank
+                         : split_b ? t.e * g.b_rows + t.nt * BM + 64 * (int)rank
+                                   : t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM;
         for (int kb = 0; kb < g.kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
           const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * P_STAGE_BYTES);
           tma_load_2d_pair(s.a[stage], &tmA, kb * BK, arow, full_leader);
-          tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
+          if (split_b) {
+            tma_load_2d_pair(s.b[stage], &tmB64, kb * BK, brow, full_leader);
+            tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB64, kb * BK, brow + g.b_second,
+                             full_leader);
+          } else {
+            tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
+          }
           if (++stage == PSTAGES) {
             stage = 0;
             phase ^= 1u;
@@ -652,6 +704,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
+        const uint32_t idesc =
+            half_tile(g, decode_pair_tile(s, g, tile)) ? kIdescPairHalf : kIdescPair;
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -663,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
-                           kIdescPair, (kb > 0 || k > 0) ? 1u : 0u);
+                           idesc, (kb > 0 || k > 0) ? 1u : 0u);
           const uint32_t e_local = smem_u32(&s.empty[stage]);
           umma_commit_pair(mapa_shared(e_local, 0));
           umma_commit_pair(mapa_shared(e_local, 1));
@@ -695,8 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_expert(g, t, tbase, t.row0 + 128 * (int)rank + q * 32 + lane, half,
-                      s.epi_stage[warp - 2], lane);
+      epilogue_pair(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
@@ -767,8 +820,8 @@ int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, 
 
 // Cluster-of-two launch of the CTA-pair kernel: as many clusters as fit at once (cached
 // per device), so the persistent tile loop never waits for a cluster slot.
-int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int sm_count,
-                cudaStream_t st) {
+int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb64,
+                const GemmArgs& g, int sm_count, cudaStream_t st) {
   constexpr size_t smem = sizeof(PairStorage) + 1024;
   static_assert(smem <= 227 * 1024, "shared memory budget");
   static std::mutex mu;
@@ -804,7 +857,7 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
     nclusters = clusters_of[dev];
   }
   if (nclusters > sm_count / 2) nclusters = sm_count / 2;
-  if (launch_kernel(k_grouped_gemm_pair, 2 * nclusters, kThreads, smem, st, 2, ma, mb, g) !=
+  if (launch_kernel(k_grouped_gemm_pair, 2 * nclusters, kThreads, smem, st, 2, ma, mb, mb64, g) !=
       cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -815,6 +868,15 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
 
 // The CTA-pair kernel pays off once groups are tall (256-row tiles); small batches keep
 // the one-CTA kernel. MOE_B200_GEMM_PAIR=0 / 1 forces either (for measurements).
+// MOE_B200_PAIR_HALF=0 runs every pair tile as M = 256 (for measurements).
+int pair_half_tiles() {
+  static const int v = [] {
+    const char* e = getenv("MOE_B200_PAIR_HALF");
+    return (e && e[0] == '0') ? 0 : 1;
+  }();
+  return v;
+}
+
 bool use_pair_kernel(int T) {
   static const char* env = getenv("MOE_B200_GEMM_PAIR");
   if (env && env[0] == '0') return false;
@@ -978,7 +1040,7 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
                           cudaStream_t st) {
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   const uint64_t rows = (uint64_t)T * K + BM;   // x_perm / h / y_perm allocation rows
-  CUtensorMap mx, mwgu, mh, mwd;
+  CUtensorMap mx, mwgu, mwgu64, mh, mwd;
   int rc;
   // A of the gate/up GEMM: the permuted rows, or the token rows gathered through perm_token
   if (x_perm) {
@@ -988,6 +1050,8 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   }
   const bool pair = use_pair_kernel(T) && x_perm != nullptr;
   if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H)) != MOE_OK) return rc;
+  if (pair && (rc = make_map(&mwgu64, w_gate_up, (uint64_t)n_ffn * 2 * I, H, 64)) != MOE_OK)
+    return rc;
   if ((rc = make_map(&mh, h, rows, I)) != MOE_OK) return rc;
   if ((rc = make_map(&mwd, w_down, (uint64_t)n_ffn * H, I)) != MOE_OK) return rc;
 
@@ -1006,8 +1070,9 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g1.status = status;
   g1.ksplit = 1;
   g1.kb_per_split = g1.kblocks;
-  if ((rc = pair ? launch_pair(mx, mwgu, g1, sm_count, st) : launch_one(mx, mwgu, g1, sm_count, st)) !=
-      MOE_OK)
+  g1.half_tiles = pair ? pair_half_tiles() : 0;
+  if ((rc = pair ? launch_pair(mx, mwgu, mwgu64, g1, sm_count, st)
+                 : launch_one(mx, mwgu, g1, sm_count, st)) != MOE_OK)
     return rc;
 
   GemmArgs g2{};
@@ -1027,7 +1092,9 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g2.status = status;
   g2.ksplit = 1;
   g2.kb_per_split = g2.kblocks;
-  return pair ? launch_pair(mh, mwd, g2, sm_count, st) : launch_one(mh, mwd, g2, sm_count, st);
+  g2.half_tiles = pair ? pair_half_tiles() : 0;
+  return pair ? launch_pair(mh, mwd, mwd, g2, sm_count, st)
+              : launch_one(mh, mwd, g2, sm_count, st);
 }
 
 int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w_gate_up,
@@ -1036,10 +1103,12 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   const uint64_t rows = (uint64_t)T * K + BM;
   const bool pair = use_pair_kernel(T);
-  CUtensorMap mx, mwgu;
+  CUtensorMap mx, mwgu, mwgu64;
   int rc;
   if ((rc = make_map(&mx, x_perm, rows, H)) != MOE_OK) return rc;
   if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H)) != MOE_OK) return rc;
+  if (pair && (rc = make_map(&mwgu64, w_gate_up, (uint64_t)n_ffn * 2 * I, H, 64)) != MOE_OK)
+    return rc;
   GemmArgs g{};
   g.mode = kGateUp;
   g.gu_raw = 1;
@@ -1055,7 +1124,9 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
   g.status = status;
   g.ksplit = 1;
   g.kb_per_split = g.kblocks;
-  return pair ? launch_pair(mx, mwgu, g, sm_count, st) : launch_one(mx, mwgu, g, sm_count, st);
+  g.half_tiles = pair ? pair_half_tiles() : 0;
+  return pair ? launch_pair(mx, mwgu, mwgu64, g, sm_count, st)
+              : launch_one(mx, mwgu, g, sm_count, st);
 }
 
 int make_tma_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
