@@ -15,7 +15,8 @@
  *    [n_ffn, n_ffn + n_zero). E = n_ffn + n_zero.
  *  - Pointers marked "device" are CUDA device pointers on the current device; the caller
  *    owns every buffer. The library never allocates, frees or synchronises, except
- *    moe_read_device_status, which synchronises the given stream.
+ *    moe_read_device_status, which synchronises the given stream, and the host pipeline
+ *    (its own streams and events).
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
  *    legacy default stream).
  *  - Layouts are row-major and contiguous. Device pointers must be 16-byte aligned.
@@ -293,6 +294,55 @@ int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,
                 const float* logits_in, const float* bias, const void* w_gate_up,
                 const void* w_down, void* out, int32_t* topk_idx, float* topk_gate,
                 int32_t* counts, int32_t* nffn_hist, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- end-to-end runs from host memory ------------------------------------------------------
+ * The pages have no counterpart to these calls: they serve a caller whose batches live in
+ * host memory (a serving loop), and overlap each batch's PCIe copies with the previous and
+ * next batches' layer kernels. A pipeline owns two copy streams and a few events (created
+ * by moe_host_pipeline_create, the one place besides moe_read_device_status where the
+ * library touches device state outside a stream) and uses the caller's device staging
+ * buffers: two slots of x [T, H] dtype, out [T, H] dtype and, optionally, logits [T, E]
+ * fp32. Slots alternate per batch, so a buffer is never overwritten while a copy or a
+ * kernel still reads it.
+ *
+ * moe_host_pipeline_create(shape, x_dev, logits_dev, out_dev, stream, &pipe)
+ *   x_dev, out_dev  two device pointers each (16-byte aligned), as above
+ *   logits_dev      two device pointers, or NULL when no batch passes logits
+ *   stream          the stream the layer's kernels run on (the caller's compute stream)
+ *   Errors: MOE_ERR_INVALID_ARG (NULL pipe / buffers), MOE_ERR_ALIGNMENT, the shape's
+ *   errors, MOE_ERR_NO_DEVICE, MOE_ERR_CUDA (stream or event creation; nothing is kept).
+ *
+ * moe_host_pipeline_submit(pipe, x_host, logits_in_host, out_host, weights..., ws, ws_bytes)
+ *   x_host          host [T, H] dtype, the batch's tokens
+ *   logits_in_host  host [T, E] fp32 or NULL: given router logits, as logits_in of moe_route
+ *   out_host        host [T, H] dtype, receives the layer's output
+ *   w_router ... ws_bytes: as in moe_forward; topk_idx, topk_gate, counts and nffn_hist
+ *   are overwritten by every batch (read them on `stream` before the next batch's kernels).
+ *   Queues: the copy of x (and logits) into slot n mod 2 on the input copy stream; the
+ *   layer (moe_forward) on `stream` after that copy; the copy of out back on the output
+ *   copy stream after the layer. The first submit after create or join orders the copy
+ *   streams after the work already on `stream`. Host buffers must be page-locked (for
+ *   example cudaHostAlloc) for the copies to run asynchronously and overlap; a host
+ *   buffer must stay untouched until the batch's output copy has completed (join, then
+ *   synchronise `stream`). Every check happens before anything is queued.
+ *
+ * moe_host_pipeline_join(pipe): makes `stream` wait for every copy queued so far, so that
+ *   work or an event recorded on `stream` afterwards follows the last output copy.
+ *   Asynchronous.
+ * moe_host_pipeline_destroy(pipe): waits for the pipeline's copy streams, releases its
+ *   streams and events and frees it. NULL is a no-op. */
+typedef struct moe_host_pipeline moe_host_pipeline;
+
+int moe_host_pipeline_create(const moe_shape_t* shape, void* const x_dev[2],
+                             float* const logits_dev[2], void* const out_dev[2], void* stream,
+                             moe_host_pipeline** pipe);
+int moe_host_pipeline_submit(moe_host_pipeline* pipe, const void* x_host,
+                             const float* logits_in_host, void* out_host, const float* w_router,
+                             const float* bias, const void* w_gate_up, const void* w_down,
+                             int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                             int32_t* nffn_hist, void* ws, size_t ws_bytes);
+int moe_host_pipeline_join(moe_host_pipeline* pipe);
+int moe_host_pipeline_destroy(moe_host_pipeline* pipe);
 
 /* ---- allocation-free variant ------------------------------------------------------------
  * The pages have no counterpart to this call: it is moe_permute for callers that cannot

@@ -85,6 +85,12 @@ _SIGS = {
     "moe_lb_loss": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 5 + [_SZ, _P]),
     "moe_backward_workspace_size": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_SZ)]),
     "moe_backward": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 18 + [_SZ, _P]),
+    "moe_host_pipeline_create": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_P),
+                                                 ctypes.POINTER(_P), ctypes.POINTER(_P), _P,
+                                                 ctypes.POINTER(_P)]),
+    "moe_host_pipeline_submit": (ctypes.c_int, [_P] * 13 + [_SZ]),
+    "moe_host_pipeline_join": (ctypes.c_int, [_P]),
+    "moe_host_pipeline_destroy": (ctypes.c_int, [_P]),
 }
 
 _lib = None
@@ -421,3 +427,51 @@ class MoELayer:
             self.forward(self._x_dev, logits_in, st)
             out_host.copy_(self.out[: x_host.shape[0]], non_blocking=True)
         return out_host
+
+
+class HostPipeline:
+    """moe_host_pipeline_*: a layer over batches held in page-locked host memory, each
+    batch's copies overlapped with the neighbouring batches' kernels (see include/moe.h).
+
+    Holds the two slots of device staging buffers the C pipeline uses. submit(x_host,
+    out_host[, logits_in_host]) queues one batch; join() makes the compute stream wait for
+    every queued copy; close() waits for the copies and releases the pipeline."""
+
+    def __init__(self, layer: "MoELayer", with_logits: bool = False, stream=None):
+        self.layer = layer
+        sh = layer.shape
+        dev = layer.out.device
+        dt = layer.out.dtype
+        self.x = [torch.empty(sh.T, sh.H, dtype=dt, device=dev) for _ in range(2)]
+        self.out = [torch.empty(max(sh.T, 1), sh.H, dtype=dt, device=dev) for _ in range(2)]
+        self.logits = ([torch.empty(sh.T, sh.E, dtype=torch.float32, device=dev)
+                        for _ in range(2)] if with_logits else None)
+        arr = _P * 2
+        lg = arr(*[ptr(t) for t in self.logits]) if self.logits is not None else None
+        self._handle = _P()
+        _check(lib().moe_host_pipeline_create(ctypes.byref(sh), arr(*[ptr(t) for t in self.x]),
+                                              lg, arr(*[ptr(t) for t in self.out]),
+                                              _stream(stream), ctypes.byref(self._handle)),
+               "moe_host_pipeline_create")
+
+    def submit(self, x_host, out_host, logits_in_host=None):
+        L = self.layer
+        _check(lib().moe_host_pipeline_submit(
+            self._handle, ptr(x_host), ptr(logits_in_host), ptr(out_host), ptr(L.w_router),
+            ptr(L.bias), ptr(L.w_gate_up), ptr(L.w_down), ptr(L.topk_idx), ptr(L.topk_gate),
+            ptr(L.counts), ptr(L.nffn_hist), ptr(L.ws), _nbytes(L.ws)),
+            "moe_host_pipeline_submit")
+
+    def join(self):
+        _check(lib().moe_host_pipeline_join(self._handle), "moe_host_pipeline_join")
+
+    def close(self):
+        if getattr(self, "_handle", None) is not None and self._handle.value:
+            _check(lib().moe_host_pipeline_destroy(self._handle), "moe_host_pipeline_destroy")
+        self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass

@@ -1,6 +1,7 @@
 // abi.cu - the extern "C" entry points of include/moe.h: host-side argument checks, the
 // workspace layout and the launch order of the layer's kernels. No call here allocates
-// memory or waits for the device, except moe_read_device_status.
+// device memory or waits for the device, except moe_read_device_status and the host
+// pipeline's create (streams and events) and destroy (waits for its copies).
 #include <atomic>
 #include <initializer_list>
 #include <mutex>
@@ -511,6 +512,158 @@ int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,
   MOE_TRY(grouped_ffn_impl(shape, x, xperm, offsets, w_gate_up, w_down, perm, rowgate, h, yperm,
                            outacc, ws, ws_bytes, stream));
   return combine_impl(shape, x, yperm, outacc, topk_gate, rowof, zgate, out, stream);
+}
+
+}  // extern "C"
+
+// ---- end-to-end runs from host memory, overlapped across batches --------------------------
+// Batch i's layer kernels run on the caller's stream while batch i+1's input crosses to the
+// device on one copy stream and batch i-1's output crosses back on another. Two slots of
+// device staging buffers (the caller's) alternate; per slot, "staged" orders the kernels
+// after the input copy, "consumed" the next input copy into the slot after the kernels that
+// read it, and "drained" the next kernels writing the slot's output after its copy out.
+struct moe_host_pipeline {
+  moe_shape_t shape;
+  int device;
+  cudaStream_t compute, h2d, d2h;
+  void* x_dev[2];
+  float* logits_dev[2];
+  void* out_dev[2];
+  cudaEvent_t staged[2], consumed[2], drained[2], fork, tail;
+  bool used[2];
+  bool forked;
+  uint64_t n;
+};
+
+namespace moe {
+namespace {
+
+size_t elt_bytes(const moe_shape_t& s) { return s.dtype == MOE_BF16 ? 2 : 4; }
+
+void destroy_pipeline_parts(moe_host_pipeline* p) {
+  for (int b = 0; b < 2; ++b) {
+    if (p->staged[b]) cudaEventDestroy(p->staged[b]);
+    if (p->consumed[b]) cudaEventDestroy(p->consumed[b]);
+    if (p->drained[b]) cudaEventDestroy(p->drained[b]);
+  }
+  if (p->fork) cudaEventDestroy(p->fork);
+  if (p->tail) cudaEventDestroy(p->tail);
+  if (p->h2d) cudaStreamDestroy(p->h2d);
+  if (p->d2h) cudaStreamDestroy(p->d2h);
+  cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int moe_host_pipeline_create(const moe_shape_t* shape, void* const x_dev[2],
+                             float* const logits_dev[2], void* const out_dev[2], void* stream,
+                             moe_host_pipeline** pipe) {
+  using namespace moe;
+  if (!pipe || !x_dev || !out_dev) return MOE_ERR_INVALID_ARG;
+  *pipe = nullptr;
+  MOE_TRY(check_shape(shape));
+  MOE_TRY(check_ptrs({x_dev[0], x_dev[1], out_dev[0], out_dev[1]}));
+  if (logits_dev) MOE_TRY(check_ptrs({logits_dev[0], logits_dev[1]}));
+  DeviceInfo info;
+  MOE_TRY(current_device_info(&info));
+  moe_host_pipeline* p = static_cast<moe_host_pipeline*>(calloc(1, sizeof(moe_host_pipeline)));
+  if (!p) return MOE_ERR_INVALID_ARG;
+  p->shape = *shape;
+  p->device = info.device;
+  p->compute = as_stream(stream);
+  for (int b = 0; b < 2; ++b) {
+    p->x_dev[b] = x_dev[b];
+    p->logits_dev[b] = logits_dev ? logits_dev[b] : nullptr;
+    p->out_dev[b] = out_dev[b];
+  }
+  bool ok = cudaStreamCreateWithFlags(&p->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p->d2h, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p->fork, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p->tail, cudaEventDisableTiming) == cudaSuccess;
+  for (int b = 0; ok && b < 2; ++b)
+    ok = cudaEventCreateWithFlags(&p->staged[b], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p->consumed[b], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p->drained[b], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    destroy_pipeline_parts(p);
+    free(p);
+    return MOE_ERR_CUDA;
+  }
+  *pipe = p;
+  return MOE_OK;
+}
+
+int moe_host_pipeline_submit(moe_host_pipeline* p, const void* x_host,
+                             const float* logits_in_host, void* out_host, const float* w_router,
+                             const float* bias, const void* w_gate_up, const void* w_down,
+                             int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                             int32_t* nffn_hist, void* ws, size_t ws_bytes) {
+  using namespace moe;
+  if (!p || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if (logits_in_host && !p->logits_dev[0]) return MOE_ERR_INVALID_ARG;
+  const moe_shape_t& s = p->shape;
+  // every check moe_forward makes, before anything is queued
+  MOE_TRY(check_ptrs({bias, w_gate_up, w_down, topk_idx, topk_gate, counts, nffn_hist, ws}));
+  if (!logits_in_host) MOE_TRY(check_ptrs({w_router}));
+  if (ws_bytes < layout_of(s).total) return MOE_ERR_WORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) {
+    cudaGetLastError();
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (s.T == 0) return MOE_OK;
+  const int b = static_cast<int>(p->n & 1);
+  const size_t xb = (size_t)s.T * s.H * elt_bytes(s);
+  const size_t lb = (size_t)s.T * (s.n_ffn + s.n_zero) * sizeof(float);
+  if (!p->forked) {
+    // a new sequence starts after the work already on the caller's stream
+    MOE_TRY(cuda_rc(cudaEventRecord(p->fork, p->compute)));
+    MOE_TRY(cuda_rc(cudaStreamWaitEvent(p->h2d, p->fork, 0)));
+    MOE_TRY(cuda_rc(cudaStreamWaitEvent(p->d2h, p->fork, 0)));
+    p->forked = true;
+  }
+  if (p->used[b]) MOE_TRY(cuda_rc(cudaStreamWaitEvent(p->h2d, p->consumed[b], 0)));
+  MOE_TRY(cuda_rc(cudaMemcpyAsync(p->x_dev[b], x_host, xb, cudaMemcpyHostToDevice, p->h2d)));
+  if (logits_in_host)
+    MOE_TRY(cuda_rc(cudaMemcpyAsync(p->logits_dev[b], logits_in_host, lb,
+                                    cudaMemcpyHostToDevice, p->h2d)));
+  MOE_TRY(cuda_rc(cudaEventRecord(p->staged[b], p->h2d)));
+  MOE_TRY(cuda_rc(cudaStreamWaitEvent(p->compute, p->staged[b], 0)));
+  if (p->used[b]) MOE_TRY(cuda_rc(cudaStreamWaitEvent(p->compute, p->drained[b], 0)));
+  MOE_TRY(moe_forward(&s, p->x_dev[b], w_router, logits_in_host ? p->logits_dev[b] : nullptr,
+                      bias, w_gate_up, w_down, p->out_dev[b], topk_idx, topk_gate, counts,
+                      nffn_hist, ws, ws_bytes, p->compute));
+  MOE_TRY(cuda_rc(cudaEventRecord(p->consumed[b], p->compute)));
+  MOE_TRY(cuda_rc(cudaStreamWaitEvent(p->d2h, p->consumed[b], 0)));
+  MOE_TRY(cuda_rc(cudaMemcpyAsync(out_host, p->out_dev[b], xb, cudaMemcpyDeviceToHost, p->d2h)));
+  MOE_TRY(cuda_rc(cudaEventRecord(p->drained[b], p->d2h)));
+  p->used[b] = true;
+  ++p->n;
+  return MOE_OK;
+}
+
+int moe_host_pipeline_join(moe_host_pipeline* p) {
+  using namespace moe;
+  if (!p) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(cuda_rc(cudaEventRecord(p->tail, p->h2d)));
+  MOE_TRY(cuda_rc(cudaStreamWaitEvent(p->compute, p->tail, 0)));
+  MOE_TRY(cuda_rc(cudaEventRecord(p->tail, p->d2h)));
+  MOE_TRY(cuda_rc(cudaStreamWaitEvent(p->compute, p->tail, 0)));
+  p->forked = false;
+  return MOE_OK;
+}
+
+int moe_host_pipeline_destroy(moe_host_pipeline* p) {
+  using namespace moe;
+  if (!p) return MOE_OK;
+  const bool ok = cudaStreamSynchronize(p->h2d) == cudaSuccess &&
+                  cudaStreamSynchronize(p->d2h) == cudaSuccess;
+  destroy_pipeline_parts(p);
+  free(p);
+  return ok ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -17,7 +17,7 @@ def L():
 
 def test_library_exports_every_declared_function(L):
     names = abi.header_functions()
-    assert len(names) == 18
+    assert len(names) == 22
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(abi._SIGS)
@@ -111,6 +111,31 @@ def test_host_checks_run_before_any_device_access(L):
     assert L.moe_lb_loss(ctypes.byref(s), bad, good, None, good, good, ws_n, None) == -3
     assert L.moe_lb_loss(ctypes.byref(s), good, good, None, good, good, ws_n - 1, None) == -5
     assert L.moe_read_device_status(None, 256, None, None) == -1
+
+
+def test_host_pipeline_host_checks(L):
+    """moe_host_pipeline_*: argument checks on the host; without a GPU, a valid create
+    stops at the device query and keeps nothing."""
+    s = _shape(dtype="bf16", H=256, I=128)
+    good, bad = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 4)
+    arr = ctypes.c_void_p * 2
+    two = arr(good, good)
+    h = ctypes.c_void_p()
+    assert L.moe_host_pipeline_create(ctypes.byref(s), two, None, two, None, None) == -1
+    assert L.moe_host_pipeline_create(ctypes.byref(s), None, None, two, None, ctypes.byref(h)) == -1
+    assert L.moe_host_pipeline_create(ctypes.byref(s), arr(good, bad), None, two, None,
+                                      ctypes.byref(h)) == -3
+    assert L.moe_host_pipeline_create(ctypes.byref(s), two, arr(good, None), two, None,
+                                      ctypes.byref(h)) == -1
+    sk = _shape(dtype="bf16", H=256, I=128, K=25)
+    assert L.moe_host_pipeline_create(ctypes.byref(sk), two, None, two, None, ctypes.byref(h)) == -1
+    if not torch.cuda.is_available():
+        assert L.moe_host_pipeline_create(ctypes.byref(s), two, None, two, None,
+                                          ctypes.byref(h)) == -8
+        assert not h.value
+    assert L.moe_host_pipeline_submit(None, *([good] * 12), 1 << 30) == -1
+    assert L.moe_host_pipeline_join(None) == -1
+    assert L.moe_host_pipeline_destroy(None) == 0
 
 
 def test_empty_batch_is_a_no_op(L):
