@@ -309,10 +309,13 @@ def scmoe_overlap(st: Stepper, device, seed: int, iters: int, warmup: int) -> di
 
 def time_backward(st: Stepper, device, seed: int, iters: int, warmup: int) -> dict:
     """moe_backward on the batch of the last timed step (deterministic-mode forward), for a
-    random bf16 output gradient; mean CUDA-event time per call. Algorithmic work of the
-    expert GEMMs: the G|U recompute (4 R H I), dh (2 R H I), the rows' dx (4 R H I) and the
-    two weight gradients (2 + 4 R H I), 16 R H I in all; the router's two fp32 GEMMs are
-    4 T E H on the CUDA cores."""
+    random bf16 output gradient; mean CUDA-event time per call.
+
+    Training mode: the forward's moe_grouped_ffn keeps G | U (gu_out) and the backward
+    takes them. Also timed: the backward that recomputes G | U itself, and the forward's
+    grouped FFN with and without keeping G | U. Algorithmic work of the backward's expert
+    GEMMs: dh (2 R H I), the rows' dx (4 R H I) and the two weight gradients (2 + 4 R H I),
+    12 R H I in all (16 R H I with the recompute); the router's GEMMs are 4 T E H."""
     cfg, b = st.cfg, st.b
     g = torch.Generator(device=device).manual_seed(seed + 77)
     dout = (torch.randn(cfg.T, cfg.H, device=device, generator=g) * 0.5).to(torch.bfloat16)
@@ -321,31 +324,47 @@ def time_backward(st: Stepper, device, seed: int, iters: int, warmup: int) -> di
     d_gu = torch.empty(cfg.n_ffn, 2 * cfg.I, cfg.H, dtype=torch.float32, device=device)
     d_d = torch.empty(cfg.n_ffn, cfg.H, cfg.I, dtype=torch.float32, device=device)
     ws = torch.zeros(abi.backward_workspace_size(b.shape), dtype=torch.uint8, device=device)
+    gu = torch.empty(cfg.T * cfg.K + 128, 2 * cfg.I, dtype=torch.bfloat16, device=device)
     w = st.w
 
-    def call():
+    def ffn(keep):
+        abi.grouped_ffn(b.shape, st.x, b.x_perm, b.offsets, w.w_gate_up, w.w_down, b.perm_token,
+                        b.row_gate, b.h, b.y_perm, b.out_acc, b.ws, gu_out=gu if keep else None)
+
+    def bwd(saved):
         abi.backward(b.shape, dout, st.x, w.w_router, w.w_gate_up, w.w_down, b.logits,
                      b.topk_idx, b.topk_gate, b.offsets, b.row_of, b.x_perm, b.h, b.y_perm,
-                     dx, d_router, d_gu, d_d, ws)
-    for _ in range(warmup):
-        call()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(iters):
-        call()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / iters
+                     dx, d_router, d_gu, d_d, ws, gu=gu if saved else None)
+
+    def timed(fn, n):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    ffn_plain = timed(lambda: ffn(False), iters)
+    ffn_keep = timed(lambda: ffn(True), iters)      # leaves G | U of this batch in gu
+    ms = timed(lambda: bwd(True), iters)
+    ms_re = timed(lambda: bwd(False), iters)
     assert abi.read_device_status(ws) == 0
     rows = int(b.counts[: cfg.n_ffn].sum().item())
-    flop = 16.0 * rows * cfg.H * cfg.I
+    flop = 12.0 * rows * cfg.H * cfg.I
     out = {"workload": st.cfg.name, "tokens": cfg.T, "ms_per_call": round(ms, 4),
            "expert_gemm_flop": flop, "ffn_rows": rows,
            "expert_gemm_tflops_over_call": round(flop / (ms / 1e3) / 1e12, 1),
-           "router_fp32_flop": 4.0 * cfg.T * cfg.E * cfg.H,
-           "note": "whole moe_backward call (router gradients on the CUDA cores included)"}
-    del dout, dx, d_router, d_gu, d_d, ws
+           "ms_per_call_recompute_gu": round(ms_re, 4),
+           "forward_grouped_ffn_ms": round(ffn_plain, 4),
+           "forward_grouped_ffn_keep_gu_ms": round(ffn_keep, 4),
+           "router_flop": 4.0 * cfg.T * cfg.E * cfg.H,
+           "note": "whole moe_backward call given the forward's G | U (gu_out); "
+                   "the recompute variant runs the gate/up GEMM again"}
+    del dout, dx, d_router, d_gu, d_d, ws, gu
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return out

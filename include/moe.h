@@ -186,12 +186,16 @@ int moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* 
  *   y_perm     device [T * K + 128, H] dtype  deterministic combine: receives y = h W_d^T
  *   out_acc    device [T, H] fp32             fused combine: out_acc[perm_token[r]] +=
  *                                             s * row_gate[r] * y[r] (atomic fp32 adds)
+ *   gu_out     device [T * K + 128, 2I] bf16  or NULL (bf16 layers only): also receives
+ *              or NULL                        G = x W_g^T (columns [0, I)) and U = x W_u^T
+ *                                             (columns [I, 2I)) of every row, rounded to
+ *                                             bf16, for moe_backward (a training forward)
  * bf16 runs on the tensor cores (tcgen05, fp32 accumulate, h rounded to bf16); fp32 runs
  * a plain fp32 kernel. The call reads the row counts on the device: it never waits. */
 int moe_grouped_ffn(const moe_shape_t* shape, const void* x, const void* x_perm,
                     const int32_t* offsets, const void* w_gate_up, const void* w_down,
                     const int32_t* perm_token, const float* row_gate, void* h, void* y_perm,
-                    float* out_acc, void* ws, size_t ws_bytes, void* stream);
+                    float* out_acc, void* gu_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Combine (report §2.1: zero-computation experts contribute g * x).
  * Fused: out = out_acc rounded to dtype. Deterministic: out[t] = sum over the FFN slots k
@@ -236,7 +240,7 @@ int moe_backward_workspace_size(const moe_shape_t* shape, size_t* bytes);
  * selection held fixed (it is piecewise constant) and no gradient to the selection bias
  * (it only steers selection and is set by the PID, report §2.1.1):
  *   dy = s g_k dout_t (FFN rows),  d_gate = s <dout_t, y> (FFN) or <dout_t, x_t> (zero),
- *   dh = dy W_d[e], dG = dh U silu'(G), dU = dh silu(G) (G, U recomputed),
+ *   dh = dy W_d[e], dG = dh U silu'(G), dU = dh silu(G),
  *   d_down[e] = sum dy h^T, d_gate_up[e] = sum [dG; dU] x^T, dx_t = sum W_gu[e]^T [dG; dU]
  *   + zgate_t dout_t + dL_t W_r with dL = p (dp - <p, dp>), d_router = dL^T x.
  * bf16 layers only (MOE_ERR_UNSUPPORTED otherwise). The inputs are those of a forward in
@@ -248,6 +252,10 @@ int moe_backward_workspace_size(const moe_shape_t* shape, size_t* bytes);
  *   logits     device [T, E] fp32             the logits the batch was routed with
  *   topk_idx, topk_gate, offsets, row_of      moe_route / moe_permute outputs
  *   x_perm, h, y_perm   device [T * K + 128, H | I | H] bf16
+ *   gu         device [T * K + 128, 2I] bf16  G | U saved by moe_grouped_ffn's gu_out, or
+ *              or NULL                        NULL: the call recomputes them (x_perm W_gu^T,
+ *                                             the same kernels and rounding, so the results
+ *                                             are the same bits either way)
  *   dx         device [T, H] fp32             receives d out / d x
  *   d_router   device [E, H] fp32             receives d / d W_r
  *   d_gate_up  device [n_ffn, 2I, H] fp32     receives d / d W_gu of every expert with
@@ -263,7 +271,7 @@ int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
                  const float* w_router, const void* w_gate_up, const void* w_down,
                  const float* logits, const int32_t* topk_idx, const float* topk_gate,
                  const int32_t* offsets, const int32_t* row_of, const void* x_perm,
-                 const void* h, const void* y_perm, float* dx, float* d_router,
+                 const void* h, const void* y_perm, const void* gu, float* dx, float* d_router,
                  float* d_gate_up, float* d_down, void* ws, size_t ws_bytes, void* stream);
 
 /* Device-level load-balance loss of one batch, forward value (LongCat-Flash Technical

@@ -73,7 +73,7 @@ _SIGS = {
     "moe_launch_count": (ctypes.c_uint64, []),
     "moe_route": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 11 + [_SZ, _P]),
     "moe_permute": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 11 + [_SZ, _P]),
-    "moe_grouped_ffn": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 11 + [_SZ, _P]),
+    "moe_grouped_ffn": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 12 + [_SZ, _P]),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 7 + [_P]),
     "moe_pid_init": (ctypes.c_int, [ctypes.POINTER(Shape), _P, _P, _P]),
     "moe_pid_bias_update": (ctypes.c_int, [ctypes.POINTER(Pid), ctypes.POINTER(Shape)]
@@ -84,7 +84,7 @@ _SIGS = {
     "moe_route_packed": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 10 + [_SZ, _P]),
     "moe_lb_loss": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 5 + [_SZ, _P]),
     "moe_backward_workspace_size": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_SZ)]),
-    "moe_backward": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 18 + [_SZ, _P]),
+    "moe_backward": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 19 + [_SZ, _P]),
     "moe_host_pipeline_create": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_P),
                                                  ctypes.POINTER(_P), ctypes.POINTER(_P), _P,
                                                  ctypes.POINTER(_P)]),
@@ -221,12 +221,13 @@ def permute_static_scratch(shape, topk_idx, topk_gate, zgate, x, offsets, perm_t
 
 
 def grouped_ffn(shape, x, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h, y_perm,
-                out_acc, ws, stream=None):
-    """x_perm None (bf16): the gate/up GEMM gathers the token rows of x via perm_token."""
+                out_acc, ws, stream=None, gu_out=None):
+    """x_perm None (bf16): the gate/up GEMM gathers the token rows of x via perm_token.
+    gu_out [T*K+128, 2I] bf16: also keep G | U for moe_backward (training forward)."""
     _check(lib().moe_grouped_ffn(ctypes.byref(shape), ptr(x), ptr(x_perm), ptr(offsets),
                                  ptr(w_gate_up), ptr(w_down), ptr(perm_token), ptr(row_gate),
-                                 ptr(h), ptr(y_perm), ptr(out_acc), ptr(ws), _nbytes(ws),
-                                 _stream(stream)), "moe_grouped_ffn")
+                                 ptr(h), ptr(y_perm), ptr(out_acc), ptr(gu_out), ptr(ws),
+                                 _nbytes(ws), _stream(stream)), "moe_grouped_ffn")
 
 
 def combine(shape, x, y_perm, out_acc, topk_gate, row_of, zgate, out, stream=None):
@@ -255,13 +256,15 @@ def backward_workspace_size(shape) -> int:
 
 
 def backward(shape, dout, x, w_router, w_gate_up, w_down, logits, topk_idx, topk_gate, offsets,
-             row_of, x_perm, h, y_perm, dx, d_router, d_gate_up, d_down, ws, stream=None):
-    """moe_backward: gradients of the layer for dout, from a deterministic-mode forward."""
+             row_of, x_perm, h, y_perm, dx, d_router, d_gate_up, d_down, ws, stream=None,
+             gu=None):
+    """moe_backward: gradients of the layer for dout, from a deterministic-mode forward;
+    gu: G | U saved by grouped_ffn(gu_out=...), or None to recompute them."""
     _check(lib().moe_backward(ctypes.byref(shape), ptr(dout), ptr(x), ptr(w_router),
                               ptr(w_gate_up), ptr(w_down), ptr(logits), ptr(topk_idx),
                               ptr(topk_gate), ptr(offsets), ptr(row_of), ptr(x_perm), ptr(h),
-                              ptr(y_perm), ptr(dx), ptr(d_router), ptr(d_gate_up), ptr(d_down),
-                              ptr(ws), _nbytes(ws), _stream(stream)), "moe_backward")
+                              ptr(y_perm), ptr(gu), ptr(dx), ptr(d_router), ptr(d_gate_up),
+                              ptr(d_down), ptr(ws), _nbytes(ws), _stream(stream)), "moe_backward")
 
 
 def lb_loss(shape, logits, counts, prob_mean, loss, ws, stream=None):
@@ -330,11 +333,11 @@ class StepBuffers:
 
 
 def run_steps(b: StepBuffers, x, w_router, logits_in, bias, w_gate_up, w_down, stream=None,
-              gather=None):
+              gather=None, gu_out=None):
     """The layer as its four ABI steps on one stream (moe_route, moe_permute,
     moe_grouped_ffn, moe_combine); returns b.out. gather=True (bf16 only) skips the
     permuted copy of x and lets the gate/up GEMM gather the token rows (less memory,
-    slower GEMM)."""
+    slower GEMM). gu_out: keep G | U for moe_backward (a training forward)."""
     s = b.shape
     if gather is None:
         gather = False
@@ -344,7 +347,7 @@ def run_steps(b: StepBuffers, x, w_router, logits_in, bias, w_gate_up, w_down, s
     permute(s, b.topk_idx, b.topk_gate, b.zgate, x, b.offsets, b.perm_token, b.row_of,
             b.row_gate, xp, b.out_acc, b.ws, stream)
     grouped_ffn(s, x, xp, b.offsets, w_gate_up, w_down, b.perm_token, b.row_gate, b.h,
-                b.y_perm, b.out_acc, b.ws, stream)
+                b.y_perm, b.out_acc, b.ws, stream, gu_out=gu_out)
     combine(s, x, b.y_perm, b.out_acc, b.topk_gate, b.row_of, b.zgate, b.out, stream)
     return b.out
 

@@ -219,9 +219,11 @@ int permute_impl(const moe_shape_t* s, const int32_t* topk_idx, const float* top
 int grouped_ffn_impl(const moe_shape_t* s, const void* x, const void* x_perm,
                      const int32_t* offsets, const void* w_gate_up, const void* w_down,
                      const int32_t* perm_token, const float* row_gate, void* h, void* y_perm,
-                     float* out_acc, void* ws, size_t ws_bytes, void* stream) {
+                     float* out_acc, void* gu_out, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(check_shape(s));
   MOE_TRY(check_ptrs({offsets, w_gate_up, w_down, h, ws}));
+  MOE_TRY(check_opt({gu_out}));
+  if (gu_out && s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (x_perm) MOE_TRY(check_ptrs({x_perm}));
   else if (s->dtype == MOE_BF16) MOE_TRY(check_ptrs({x, perm_token}));   // gathered rows
   else return MOE_ERR_INVALID_ARG;                                      // fp32 needs x_perm
@@ -236,7 +238,7 @@ int grouped_ffn_impl(const moe_shape_t* s, const void* x, const void* x_perm,
   const cudaStream_t st = as_stream(stream);
   if (s->dtype == MOE_BF16)
     return launch_grouped_ffn_tc(x, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h, y_perm,
-                                 out_acc, s->T, s->H, s->I, s->n_ffn, s->K, s->ffn_out_scale, fused,
+                                 out_acc, gu_out, s->T, s->H, s->I, s->n_ffn, s->K, s->ffn_out_scale, fused,
                                  at<int>(ws, L.status), dev.sm_count, st);
   return cuda_rc(launch_grouped_ffn_simt(
       static_cast<const float*>(x_perm), offsets, static_cast<const float*>(w_gate_up),
@@ -320,13 +322,15 @@ int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
                  const float* w_router, const void* w_gate_up, const void* w_down,
                  const float* logits, const int32_t* topk_idx, const float* topk_gate,
                  const int32_t* offsets, const int32_t* row_of, const void* x_perm,
-                 const void* h, const void* y_perm, float* dx, float* d_router,
-                 float* d_gate_up, float* d_down, void* ws, size_t ws_bytes, void* stream) {
+                 const void* h, const void* y_perm, const void* gu_saved, float* dx,
+                 float* d_router, float* d_gate_up, float* d_down, void* ws, size_t ws_bytes,
+                 void* stream) {
   MOE_TRY(check_shape(shape));
   if (shape->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if ((shape->n_ffn + shape->n_zero) % 8 != 0) return MOE_ERR_UNSUPPORTED;   // dL rows: 16 B
   MOE_TRY(check_ptrs({dout, x, w_router, w_gate_up, w_down, logits, topk_idx, topk_gate, offsets,
                       row_of, x_perm, h, y_perm, dx, d_router, d_gate_up, d_down, ws}));
+  MOE_TRY(check_opt({gu_saved}));
   const BwdLayout L = bwd_layout_of(*shape);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   if (shape->T == 0) return MOE_OK;
@@ -336,7 +340,7 @@ int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
   const int T = shape->T, H = shape->H, I = shape->I, K = shape->K, N = shape->n_ffn;
   const int E = N + shape->n_zero;
   int* status = at<int>(ws, L.status);
-  void* gu = at<char>(ws, L.gu);
+  const void* gu = gu_saved ? gu_saved : at<char>(ws, L.gu);
   void* dy = at<char>(ws, L.dy);
   void* dgu = at<char>(ws, L.dgu);
   float* dxp = at<float>(ws, L.dxp);
@@ -345,9 +349,11 @@ int moe_backward(const moe_shape_t* shape, const void* dout, const void* x,
   void* wr16 = at<char>(ws, L.wr16);
   int32_t* offs = at<int32_t>(ws, L.offs);
   const int Tp = (T + 63) / 64 * 64;
-  // G | U of every FFN row again, then dy and the gates' gradients
-  MOE_TRY(launch_gate_up_raw(x_perm, offsets, w_gate_up, gu, T, H, I, N, K, status, dev.sm_count,
-                             st));
+  // G | U of every FFN row again (unless the forward saved them), then dy and the gates'
+  // gradients
+  if (!gu_saved)
+    MOE_TRY(launch_gate_up_raw(x_perm, offsets, w_gate_up, at<char>(ws, L.gu), T, H, I, N, K,
+                               status, dev.sm_count, st));
   MOE_TRY(cuda_rc(launch_bwd_dy_dgate(dout, x, y_perm, topk_idx, topk_gate, row_of, T, H, K, N,
                                       shape->ffn_out_scale, dy, dgate, st)));
   // the expert GEMMs: dgu (with the SwiGLU backward), dx_perm, d_down, d_gate_up
@@ -433,9 +439,9 @@ int moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* 
 int moe_grouped_ffn(const moe_shape_t* shape, const void* x, const void* x_perm,
                     const int32_t* offsets, const void* w_gate_up, const void* w_down,
                     const int32_t* perm_token, const float* row_gate, void* h, void* y_perm,
-                    float* out_acc, void* ws, size_t ws_bytes, void* stream) {
+                    float* out_acc, void* gu_out, void* ws, size_t ws_bytes, void* stream) {
   return grouped_ffn_impl(shape, x, x_perm, offsets, w_gate_up, w_down, perm_token, row_gate, h,
-                          y_perm, out_acc, ws, ws_bytes, stream);
+                          y_perm, out_acc, gu_out, ws, ws_bytes, stream);
 }
 
 int moe_combine(const moe_shape_t* shape, const void* x, const void* y_perm, const float* out_acc,
@@ -510,7 +516,7 @@ int moe_forward(const moe_shape_t* shape, const void* x, const float* w_router,
   MOE_TRY(permute_impl(shape, topk_idx, topk_gate, zgate, x, offsets, perm, rowof, rowgate, xperm,
                        outacc, ws, ws_bytes, stream));
   MOE_TRY(grouped_ffn_impl(shape, x, xperm, offsets, w_gate_up, w_down, perm, rowgate, h, yperm,
-                           outacc, ws, ws_bytes, stream));
+                           outacc, nullptr, ws, ws_bytes, stream));
   return combine_impl(shape, x, yperm, outacc, topk_gate, rowof, zgate, out, stream);
 }
 

@@ -94,6 +94,7 @@ struct GemmArgs {
   int gu_raw;                 // gate/up: store G and U (bf16, [rows, 2I]) instead of h
   int logit_n;                // router: N tile (128 or 256 logits)
   int half_tiles;             // pair kernel: an expert's last tile of <= 128 rows runs as M = 128
+  void* gu_out;               // gate/up: also store G and U (bf16, [rows, 2I]) beside h, or null
 };
 
 struct Tile {
@@ -168,6 +169,25 @@ __device__ __forceinline__ void epi_gateup_chunk(const GemmArgs& g, const Tile& 
       w[i] = pack_bf16x2(h0, h1);
     }
     dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (g.gu_out) {
+    // the same G and U, rounded to bf16 as the raw store rounds them, for the backward
+    __nv_bfloat16* base = static_cast<__nv_bfloat16*>(g.gu_out) + (size_t)row * 2 * g.n_valid +
+                          t.nt * BM + oc;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t* src = part ? ur : gr;
+      uint4* gdst = reinterpret_cast<uint4*>(base + (part ? g.n_valid : 0));
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(src[v * 8 + 2 * i]),
+                             __uint_as_float(src[v * 8 + 2 * i + 1]));
+        gdst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
   }
 }
 
@@ -1035,9 +1055,9 @@ int launch_router_logits_tc(const void* x, const float* w_router, const void* w_
 int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offsets,
                           const void* w_gate_up,
                           const void* w_down, const int32_t* perm_token, const float* row_gate,
-                          void* h, void* y_perm, float* out_acc, int T, int H, int I, int n_ffn,
-                          int K, float scale, int fused, int* status, int sm_count,
-                          cudaStream_t st) {
+                          void* h, void* y_perm, float* out_acc, void* gu_out, int T, int H,
+                          int I, int n_ffn, int K, float scale, int fused, int* status,
+                          int sm_count, cudaStream_t st) {
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   const uint64_t rows = (uint64_t)T * K + BM;   // x_perm / h / y_perm allocation rows
   CUtensorMap mx, mwgu, mwgu64, mh, mwd;
@@ -1067,6 +1087,7 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g1.offsets = offsets;
   g1.gather_tok = x_perm ? nullptr : perm_token;
   g1.out = h;
+  g1.gu_out = gu_out;
   g1.status = status;
   g1.ksplit = 1;
   g1.kb_per_split = g1.kblocks;

@@ -125,9 +125,9 @@ cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, cons
 int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offsets,
                           const void* w_gate_up,
                           const void* w_down, const int32_t* perm_token, const float* row_gate,
-                          void* h, void* y_perm, float* out_acc, int T, int H, int I, int n_ffn,
-                          int K, float scale, int fused, int* status, int sm_count,
-                          cudaStream_t st);
+                          void* h, void* y_perm, float* out_acc, void* gu_out, int T, int H,
+                          int I, int n_ffn, int K, float scale, int fused, int* status,
+                          int sm_count, cudaStream_t st);
 // fp32 on the CUDA cores.
 cudaError_t launch_grouped_ffn_simt(const float* x_perm, const int32_t* offsets,
                                     const float* w_gate_up, const float* w_down,

@@ -89,7 +89,9 @@ def test_host_checks_run_before_any_device_access(L):
     assert L.moe_route(ctypes.byref(s), *args, ws_n - 1, None) == -5
     # permute / grouped_ffn / forward with a workspace that is too small
     assert L.moe_permute(ctypes.byref(s), *([good] * 11), 16, None) == -5
-    assert L.moe_grouped_ffn(ctypes.byref(s), *([good] * 11), 16, None) == -5
+    assert L.moe_grouped_ffn(ctypes.byref(s), *([good] * 10), None, good, 16, None) == -5
+    # gu_out (the training forward's G | U) is for bf16 layers only
+    assert L.moe_grouped_ffn(ctypes.byref(s), *([good] * 12), ws_n, None) == -2
     assert L.moe_forward(ctypes.byref(s), *([good] * 12), abi.workspace_size(s) - 1, None) == -5
     # combine: fused mode needs out_acc
     assert L.moe_combine(ctypes.byref(s), good, None, None, None, None, None, good, None) == -1
@@ -102,9 +104,11 @@ def test_host_checks_run_before_any_device_access(L):
     # backward: bf16 only, null pointers, short workspace
     bs = _shape(dtype="bf16", H=256, I=128)
     bw = abi.backward_workspace_size(bs)
-    assert L.moe_backward(ctypes.byref(s), *([good] * 18), bw, None) == -2      # fp32 layer
-    assert L.moe_backward(ctypes.byref(bs), *([good] * 17), None, bw, None) == -1
-    assert L.moe_backward(ctypes.byref(bs), *([good] * 18), bw - 1, None) == -5
+    assert L.moe_backward(ctypes.byref(s), *([good] * 19), bw, None) == -2      # fp32 layer
+    assert L.moe_backward(ctypes.byref(bs), *([good] * 18), None, bw, None) == -1
+    assert L.moe_backward(ctypes.byref(bs), *([good] * 19), bw - 1, None) == -5
+    # the saved G | U is optional but must be aligned
+    assert L.moe_backward(ctypes.byref(bs), *([good] * 13), bad, *([good] * 5), bw, None) == -3
     # load-balance loss: null counts or loss, unaligned logits, short workspace
     assert L.moe_lb_loss(ctypes.byref(s), good, None, None, good, good, ws_n, None) == -1
     assert L.moe_lb_loss(ctypes.byref(s), good, good, None, None, good, ws_n, None) == -1
@@ -144,7 +148,7 @@ def test_empty_batch_is_a_no_op(L):
     ws_n = abi.scratch_size(s)
     assert L.moe_route(ctypes.byref(s), *([p] * 11), ws_n, None) == 0
     assert L.moe_permute(ctypes.byref(s), *([p] * 11), ws_n, None) == 0
-    assert L.moe_grouped_ffn(ctypes.byref(s), *([p] * 11), ws_n, None) == 0
+    assert L.moe_grouped_ffn(ctypes.byref(s), *([p] * 10), None, p, ws_n, None) == 0
     assert L.moe_combine(ctypes.byref(s), *([p] * 7), None) == 0
     assert L.moe_forward(ctypes.byref(s), *([p] * 12), abi.workspace_size(s), None) == 0
 

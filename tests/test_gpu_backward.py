@@ -95,3 +95,32 @@ def test_backward_is_bit_reproducible(cuda_device):
     r2 = _run(cfg, seed=4)
     for a, c in zip(r1[3:], r2[3:]):
         assert torch.equal(a, c)
+
+
+@pytest.mark.parametrize("T", [300, 2048])
+def test_backward_from_saved_gate_up(cuda_device, T):
+    """A training forward (moe_grouped_ffn with gu_out) keeps G | U; moe_backward given them
+    skips the recompute and returns the same bits as the recomputing call, and the
+    forward's own outputs do not change. T = 300 runs the one-CTA kernels, T = 2048 the
+    CTA pairs (with half tiles)."""
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=T)
+    case, b, dout, dx, d_router, d_gu, d_d = _run(cfg, seed=6)
+    out_plain = b.out.clone()
+    h_plain = b.h[: int(b.offsets[cfg.n_ffn].item())].clone()
+    gu = torch.full((cfg.T * cfg.K + 128, 2 * cfg.I), 3.0, dtype=torch.bfloat16, device="cuda")
+    abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up,
+                  case.w.w_down, gu_out=gu)
+    torch.cuda.synchronize()
+    assert torch.equal(b.out, out_plain)
+    assert torch.equal(b.h[: h_plain.shape[0]], h_plain)
+    dx2, dr2 = torch.empty_like(dx), torch.empty_like(d_router)
+    gu2 = torch.full_like(d_gu, SENTINEL)
+    dd2 = torch.full_like(d_d, SENTINEL)
+    ws = torch.zeros(abi.backward_workspace_size(b.shape), dtype=torch.uint8, device="cuda")
+    abi.backward(b.shape, dout, case.x, case.w.w_router, case.w.w_gate_up, case.w.w_down,
+                 b.logits, b.topk_idx, b.topk_gate, b.offsets, b.row_of, b.x_perm, b.h,
+                 b.y_perm, dx2, dr2, gu2, dd2, ws, gu=gu)
+    torch.cuda.synchronize()
+    assert abi.read_device_status(ws) == 0
+    for a, c in ((dx, dx2), (d_router, dr2), (d_gu, gu2), (d_d, dd2)):
+        assert torch.equal(a, c)
