@@ -220,6 +220,31 @@ class Stepper:
 PHASES = ["route", "permute", "grouped_ffn", "combine", "pid"]
 
 
+def graph_step_ms(st: Stepper, n: int) -> float:
+    """One step captured into a CUDA graph (the calls neither allocate nor synchronise),
+    then `n` replays between CUDA events: the step without the host's launch work."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        st.step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st.step()
+    for _ in range(3):
+        g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(n):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / n
+
+
 def timed_loop(st: Stepper, steps: int, warmup: int, dist_on: bool, phases: bool = True):
     """Time `steps` steps (after `warmup`) between CUDA events on the launching stream.
     phases=True also records an event between the layer's calls for the per-call
@@ -471,8 +496,10 @@ def run_ours(args):
         dtraffic = dte["dram_bytes_per_step"] if dte else None
         dach = dbytes / (dstep / 1e3) / 1e9
         hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        dgraph = graph_step_ms(dst, dsteps) if not dist_on else None
         decode = {"workload": "decode_bf16", "value": round(dcfg.T * dsteps * world / (dms / 1e3), 1),
                   "unit": UNIT, "ms_per_step": round(dstep, 4),
+                  "graph_ms_per_step": round(dgraph, 4) if dgraph else None,
                   "breakdown_ms": {p: round(float(np.mean(v)), 4) for p, v in dper.items()},
                   "roofline": {"bound": "hbm", "scope": "whole layer step",
                                "achieved": round(dach, 1), "peak": hbm, "unit": "GB/s",
