@@ -395,6 +395,36 @@ def time_backward(st: Stepper, device, seed: int, iters: int, warmup: int) -> di
     return out
 
 
+def pid_trajectory(cfg, w, device, seed: int) -> dict:
+    """The skewed workload's closed loop, untimed: for each of cfg.pid_steps steps, route
+    that step's drawn logits with the current bias (moe_route) and update the FFN experts'
+    biases from the histogram (moe_pid_bias_update), starting from the workload's bias.
+    Reports, after every step, the FFN activation ratio (mean FFN picks per token / K),
+    the spread of FFN picks per token and the FFN experts' max / mean load."""
+    shape = abi.shape_of(cfg)
+    b = abi.StepBuffers.allocate(abi.shape_of(cfg.with_(H=128, I=128)), device)
+    ws = torch.zeros(abi.scratch_size(shape), dtype=torch.uint8, device=device)
+    bias = w.bias.clone()
+    state = torch.empty(3 * cfg.n_ffn, dtype=torch.float32, device=device)
+    stats = torch.zeros(8, dtype=torch.float32, device=device)
+    abi.pid_init(shape, bias, state)
+    pid = abi.Pid(*PID_GAINS)
+    ratio, spread, imbalance = [], [], []
+    for k in range(cfg.pid_steps):
+        logits = wl.draw_skewed_logits(cfg, device, seed=seed, step=k)
+        abi.route(shape, None, None, logits, bias, None, b.topk_idx, b.topk_gate, b.counts,
+                  b.nffn_hist, b.zgate, ws)
+        abi.pid_bias_update(pid, shape, b.counts, b.nffn_hist, bias, state, stats)
+        st = stats.cpu()
+        ratio.append(round(float(st[0]), 4))
+        spread.append(round(float(st[2]), 3))
+        imbalance.append(round(float(st[3]), 2))
+    assert abi.read_device_status(ws) == 0
+    return {"steps": cfg.pid_steps, "target_ratio": round(PID_GAINS[3], 4),
+            "gains": {"kp": PID_GAINS[0], "ki": PID_GAINS[1], "kd": PID_GAINS[2]},
+            "ffn_ratio": ratio, "ffn_picks_std": spread, "ffn_max_over_mean_load": imbalance}
+
+
 def max_over_ranks(v: float, dist_on: bool) -> float:
     """The largest of the ranks' values (the job's time is the slowest replica's)."""
     if not dist_on:
@@ -564,6 +594,10 @@ def run_ours(args):
         if decode is not None:
             overlap["decode"] = scmoe_overlap(dst, device, seed, 50, 5)
 
+    pid_traj = None
+    if cfg.pid_steps > 0 and rank == 0:
+        pid_traj = pid_trajectory(cfg, w, device, seed)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rng = np.random.default_rng(0)
@@ -589,6 +623,7 @@ def run_ours(args):
         "decode": decode,
         "scmoe_overlap": overlap,
         "backward": bwd,
+        "pid_trajectory": pid_traj,
         "e2e": e2e,
         "gpu_launches": int(launches) * world,
         "cpu_baseline": cpu,
