@@ -92,7 +92,7 @@ struct GemmArgs {
   const int32_t* gather_tok;  // non-null: A row r is row gather_tok[r] of A's tensor
   ZeroSpec zero;              // buffers cleared after the dependency wait
   int gu_raw;                 // gate/up: store G and U (bf16, [rows, 2I]) instead of h
-  int logit_n;                // router: N tile (128 or 256 logits)
+  int logit_n;                // router: N tile (128, 192 or 256 logits)
   int half_tiles;             // pair kernel: an expert's last tile of <= 128 rows runs as M = 128
   void* gu_out;               // gate/up: also store G and U (bf16, [rows, 2I]) beside h, or null
 };
@@ -829,7 +829,9 @@ int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, 
   constexpr size_t smem = sizeof(SharedStorage) + 1024;
   static_assert(smem <= 227 * 1024, "shared memory budget");
   auto kern = g.mode != kLogits ? k_grouped_gemm_tc<false, BN>
-               : g.logit_n == 128 ? k_grouped_gemm_tc<true, 128> : k_grouped_gemm_tc<true, 256>;
+               : g.logit_n == 128 ? k_grouped_gemm_tc<true, 128>
+               : g.logit_n == 192 ? k_grouped_gemm_tc<true, 192>
+                                  : k_grouped_gemm_tc<true, 256>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
@@ -955,9 +957,29 @@ int router_min_split() {
 // The router GEMM's N tile: 256 logits when the 256-wide tiles fill a wave of SMs (the
 // A tile is then read once per 256 logits), else 128 (twice the tiles for a small batch:
 // decode's 128 tokens x 768 logits fill 144 CTAs with the K split instead of 72).
+// MOE_B200_ROUTER_N=192 / 256 forces that width where 256-logit tiles fill a wave (for
+// measurements).
+int router_n_override() {
+  static const int v = [] {
+    const char* e = getenv("MOE_B200_ROUTER_N");
+    const int n = e ? atoi(e) : 0;
+    return (n == 192 || n == 256) ? n : 0;
+  }();
+  return v;
+}
+
 int router_tile_n(int T, int E, int sm_count) {
-  const long tiles256 = (long)((T + BM - 1) / BM) * ((E + 255) / 256);
-  return tiles256 >= sm_count ? 256 : 128;
+  const long mt = (T + BM - 1) / BM;
+  const long tiles256 = mt * ((E + 255) / 256);
+  if (tiles256 < sm_count) return 128;
+  if (router_n_override()) return router_n_override();
+  // whole waves times the tile width (a tile's time grows with its width): 192-logit
+  // tiles when they need less of it, e.g. 8192 tokens x 768 experts on 148 SMs: 256 tiles
+  // in two waves of 192 against 192 tiles in two waves of 256
+  const long tiles192 = mt * ((E + 191) / 192);
+  const long c256 = (tiles256 + sm_count - 1) / sm_count * 256;
+  const long c192 = (tiles192 + sm_count - 1) / sm_count * 192;
+  return c192 < c256 ? 192 : 256;
 }
 
 int router_tc_splitk(int T, int E, int H, int sm_count) {
@@ -1024,8 +1046,11 @@ int launch_router_logits_tc(const void* x, const float* w_router, const void* w_
   }
   CUtensorMap mx, mw;
   int rc;
+  const int nl = router_tile_n(T, E, sm_count > 160 ? 160 : sm_count);
   if ((rc = make_map(&mx, x, (uint64_t)T, H)) != MOE_OK) return rc;
-  if ((rc = make_map(&mw, wsplit, (uint64_t)E, 3ull * H)) != MOE_OK) return rc;
+  // B boxes: 128 rows (two per 256-logit tile) or one 192-row box
+  if ((rc = make_map(&mw, wsplit, (uint64_t)E, 3ull * H, nl == 192 ? 192 : BM)) != MOE_OK)
+    return rc;
   const int S = router_tc_splitk(T, E, H, sm_count);
   GemmArgs g{};
   g.mode = kLogits;
@@ -1036,7 +1061,7 @@ int launch_router_logits_tc(const void* x, const float* w_router, const void* w_
   g.ksplit = S;
   g.kb_per_split = (g.kblocks + S - 1) / S;
   g.kchunk = kRouterChunk;
-  g.logit_n = router_tile_n(T, E, sm_count > 160 ? 160 : sm_count);
+  g.logit_n = nl;
   g.n_tiles = (E + g.logit_n - 1) / g.logit_n;
   g.b_rows = 0;
   g.b_second = BM;
