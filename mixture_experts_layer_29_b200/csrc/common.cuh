@@ -319,6 +319,15 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint3
   return d;
 }
 
+// Backward of h = silu(G) * U for the upstream gradient dh, with s = sigmoid(G):
+// dG = dh U s (1 + G (1 - s)), dU = dh G s.
+__device__ __forceinline__ void swiglu_backward(float G, float U, float dh, float& dG,
+                                                float& dU) {
+  const float s = 1.0f / (1.0f + __expf(-G));
+  dG = dh * U * s * (1.0f + G * (1.0f - s));
+  dU = dh * G * s;
+}
+
 // Makes this thread's generic-proxy shared-memory writes visible to the async proxy (the
 // tensor cores and TMA) before a barrier hands them over.
 __device__ __forceinline__ void fence_proxy_async_smem() {

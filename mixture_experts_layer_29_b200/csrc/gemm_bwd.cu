@@ -143,8 +143,6 @@ __device__ __forceinline__ void store_f32_16(float (*stg)[20], int lane, const f
   __syncwarp();
 }
 
-__device__ __forceinline__ float sigm(float a) { return 1.0f / (1.0f + __expf(-a)); }
-
 __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const BwdArgs g) {
@@ -361,11 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               float dG[8], dU[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const float G = __bfloat162float(Gb[i]), U = __bfloat162float(Ub[i]);
-                const float dh = __uint_as_float(v[8 * q8 + i]);
-                const float sg = sigm(G);
-                dG[i] = dh * U * sg * (1.0f + G * (1.0f - sg));
-                dU[i] = dh * G * sg;
+                swiglu_backward(__bfloat162float(Gb[i]), __bfloat162float(Ub[i]),
+                                __uint_as_float(v[8 * q8 + i]), dG[i], dU[i]);
               }
               *reinterpret_cast<uint4*>(dst + 8 * q8) =
                   make_uint4(pack_bf16x2(dG[0], dG[1]), pack_bf16x2(dG[2], dG[3]),
@@ -442,15 +437,24 @@ int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* 
   g.status = status;
   g.I = I;
   g.gu = static_cast<const __nv_bfloat16*>(gu);
-  // dh = dy . W_d[e] (+ SwiGLU backward) -> dgu
+  // dh = dy . W_d[e] (+ SwiGLU backward) -> dgu, then dx_perm = dgu . W_gu[e]: on the
+  // CTA-pair kernel where the forward uses it
+  const bool pair = dgrad_use_pair(T);
+  if (pair) {
+    if ((rc = launch_dgrad_pair(0, dy, H, w_down, H, I, gu, dgu, offsets, T, K, n_ffn, status,
+                                sm_count, st)) != MOE_OK)
+      return rc;
+    if ((rc = launch_dgrad_pair(1, dgu, 2 * I, w_gate_up, 2 * I, H, nullptr, dx_perm, offsets, T,
+                                K, n_ffn, status, sm_count, st)) != MOE_OK)
+      return rc;
+  }
   g.mode = kDH;
   g.kblocks = H / BK;
   g.n_tiles = (I + BN - 1) / BN;
   g.b_krows = H;
   g.n_valid = I;
   g.out = dgu;
-  if ((rc = launch(m_dy128, m_wd, g, sm_count, st)) != MOE_OK) return rc;
-  // dx_perm = dgu . W_gu[e]
+  if (!pair && (rc = launch(m_dy128, m_wd, g, sm_count, st)) != MOE_OK) return rc;
   g.mode = kDX;
   g.kblocks = 2 * I / BK;
   g.n_tiles = (H + BN - 1) / BN;
@@ -458,7 +462,7 @@ int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* 
   g.n_valid = H;
   g.ld_out = H;
   g.out = dx_perm;
-  if ((rc = launch(m_dgu128, m_wgu, g, sm_count, st)) != MOE_OK) return rc;
+  if (!pair && (rc = launch(m_dgu128, m_wgu, g, sm_count, st)) != MOE_OK) return rc;
   // d_down[e] = dy^T h
   g.mode = kDW;
   g.m_valid = H;

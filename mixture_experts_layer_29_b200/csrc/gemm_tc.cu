@@ -49,7 +49,11 @@ constexpr uint32_t kTmemCols = 512;                  // two 256-column fp32 accu
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
 
 
-enum Mode : int { kGateUp = 0, kDownStore = 1, kDownAtomic = 2, kLogits = 3 };
+// kDgradDH / kDgradDX: the backward's dgrad GEMMs on the CTA-pair kernel, B read MN-major
+// (dh = dy . W_d[e] with the SwiGLU backward in the epilogue; dx rows = [dG | dU] . W_gu[e])
+enum Mode : int {
+  kGateUp = 0, kDownStore = 1, kDownAtomic = 2, kLogits = 3, kDgradDH = 4, kDgradDX = 5
+};
 
 struct alignas(1024) SharedStorage {
   uint8_t a[STAGES][A_BYTES];
@@ -95,6 +99,7 @@ struct GemmArgs {
   int logit_n;                // router: N tile (128, 192 or 256 logits)
   int half_tiles;             // pair kernel: an expert's last tile of <= 128 rows runs as M = 128
   void* gu_out;               // gate/up: also store G and U (bf16, [rows, 2I]) beside h, or null
+  const __nv_bfloat16* gu_in; // kDgradDH: G | U of the rows ([rows, 2I], I = n_valid)
 };
 
 struct Tile {
@@ -247,6 +252,69 @@ __device__ __forceinline__ void row_scale(const GemmArgs& g, const Tile& t, int 
   if (g.mode == kDownAtomic && row < t.row_end) {
     tok = g.perm_token[row];
     sc = g.scale * g.row_gate[row];
+  }
+}
+
+// dgrad dh: 32 columns of dh at TMEM column tcol for this thread's row, output columns
+// [oc, oc + 32) of the tile: dG, dU from the row's G and U (bf16), stored to [dG | dU].
+__device__ __forceinline__ void epi_dh_chunk(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                             int row, int tcol, int oc) {
+  uint32_t v[32];
+  tmem_ld_32x32b_x32(tbase + tcol, v);
+  tmem_ld_wait();
+  const int col = t.nt * BN + oc;
+  if (row >= t.row_end || col >= g.n_valid) return;
+  const int I = g.n_valid;
+  const __nv_bfloat16* gr = g.gu_in + (size_t)row * 2 * I + col;
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + (size_t)row * 2 * I + col;
+#pragma unroll
+  for (int q8 = 0; q8 < 4; ++q8) {
+    const uint4 G4 = *reinterpret_cast<const uint4*>(gr + 8 * q8);
+    const uint4 U4 = *reinterpret_cast<const uint4*>(gr + I + 8 * q8);
+    const __nv_bfloat16* Gb = reinterpret_cast<const __nv_bfloat16*>(&G4);
+    const __nv_bfloat16* Ub = reinterpret_cast<const __nv_bfloat16*>(&U4);
+    float dG[8], dU[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      swiglu_backward(__bfloat162float(Gb[i]), __bfloat162float(Ub[i]),
+                      __uint_as_float(v[8 * q8 + i]), dG[i], dU[i]);
+    *reinterpret_cast<uint4*>(dst + 8 * q8) =
+        make_uint4(pack_bf16x2(dG[0], dG[1]), pack_bf16x2(dG[2], dG[3]),
+                   pack_bf16x2(dG[4], dG[5]), pack_bf16x2(dG[6], dG[7]));
+    *reinterpret_cast<uint4*>(dst + I + 8 * q8) =
+        make_uint4(pack_bf16x2(dU[0], dU[1]), pack_bf16x2(dU[2], dU[3]),
+                   pack_bf16x2(dU[4], dU[5]), pack_bf16x2(dU[6], dU[7]));
+  }
+}
+
+// dgrad dx rows: 32 fp32 columns at TMEM column tcol, output columns [oc, oc + 32) of the
+// tile, through the warp's staging rows (16 columns at a time) so that a warp store covers
+// 8 rows x 64 bytes; rows past the expert's group are not stored.
+__device__ __forceinline__ void epi_dx_chunk(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                             int row, int tcol, int oc, float (*stg)[20],
+                                             int lane) {
+  uint32_t v[32];
+  tmem_ld_32x32b_x32(tbase + tcol, v);
+  tmem_ld_wait();
+  float* out = static_cast<float*>(g.out);
+  const int row_base = row - lane;
+#pragma unroll
+  for (int h16 = 0; h16 < 2; ++h16) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(&stg[lane][4 * i]) = make_float4(
+          __uint_as_float(v[16 * h16 + 4 * i]), __uint_as_float(v[16 * h16 + 4 * i + 1]),
+          __uint_as_float(v[16 * h16 + 4 * i + 2]), __uint_as_float(v[16 * h16 + 4 * i + 3]));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 8 * i + (lane >> 2);
+      const int c = t.nt * BN + oc + 16 * h16 + 4 * (lane & 3);
+      if (row_base + r < t.row_end && c < g.n_valid)
+        *reinterpret_cast<float4*>(out + (size_t)(row_base + r) * g.ld_out + c) =
+            *reinterpret_cast<const float4*>(&stg[r][4 * (lane & 3)]);
+    }
+    __syncwarp();
   }
 }
 
@@ -559,8 +627,6 @@ constexpr int BMP = 256;                             // M rows per CTA pair
 constexpr int PSTAGES = 6;                           // 32 KB per stage per CTA
 constexpr int P_B_BYTES = 128 * BK * 2;              // 16 KB: this CTA's half of B
 constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES;   // 32 KB
-constexpr uint32_t kIdescPair = idesc_bf16_f32(BMP, BN);
-constexpr uint32_t kIdescPairHalf = idesc_bf16_f32(128, BN);
 
 struct alignas(1024) PairStorage {
   uint8_t a[PSTAGES][A_BYTES];
@@ -606,6 +672,21 @@ __device__ __forceinline__ bool half_tile(const GemmArgs& g, const Tile& t) {
 __device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, uint32_t tbase,
                                               uint32_t rank, int q, int h, float (*stg)[20],
                                               int lane) {
+  if (g.mode == kDgradDH || g.mode == kDgradDX) {
+    // full tile: row 128r + 32q + lane, columns [128h, 128h + 128); half tile: as the down
+    // store below
+    const bool half = half_tile(g, t);
+    const int row = half ? t.row0 + 64 * (int)rank + 32 * (q & 1) + lane
+                         : t.row0 + 128 * (int)rank + q * 32 + lane;
+#pragma unroll 1
+    for (int j = 0; j < (half ? 64 : 128); j += 32) {
+      const int tcol = half ? 64 * h + j : 128 * h + j;
+      const int oc = half ? 128 * (q >> 1) + 64 * h + j : 128 * h + j;
+      if (g.mode == kDgradDH) epi_dh_chunk(g, t, tbase, row, tcol, oc);
+      else epi_dx_chunk(g, t, tbase, row, tcol, oc, stg, lane);
+    }
+    return;
+  }
   if (!half_tile(g, t)) {
     epilogue_expert(g, t, tbase, t.row0 + 128 * (int)rank + q * 32 + lane, h, stg, lane);
     return;
@@ -692,16 +773,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = decode_pair_tile(s, g, tile);
         const bool half = half_tile(g, t);
         const bool split_b = half && g.mode == kGateUp;   // 64 gate + 64 up rows
+        const bool b_mn = g.mode == kDgradDH || g.mode == kDgradDX;
         const int arow = t.row0 + (half ? 64 : 128) * (int)rank;
         const int brow = g.mode != kGateUp ? t.e * g.b_rows + t.nt * BN + 128 * (int)rank
                          : split_b ? t.e * g.b_rows + t.nt * BM + 64 * (int)rank
                                    : t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM;
+        // MN-major B (dgrad): this CTA's 128 N columns as two 64 x 64 boxes of K rows
+        const int bcol = t.nt * BN + 128 * (int)rank;
         for (int kb = 0; kb < g.kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
           const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * P_STAGE_BYTES);
           tma_load_2d_pair(s.a[stage], &tmA, kb * BK, arow, full_leader);
-          if (split_b) {
+          if (b_mn) {
+            const int y = t.e * g.b_rows + kb * BK;
+            tma_load_2d_pair(s.b[stage], &tmB, bcol, y, full_leader);
+            tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB, bcol + 64, y, full_leader);
+          } else if (split_b) {
             tma_load_2d_pair(s.b[stage], &tmB64, kb * BK, brow, full_leader);
             tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB64, kb * BK, brow + g.b_second,
                              full_leader);
@@ -724,8 +812,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
-        const uint32_t idesc =
-            half_tile(g, decode_pair_tile(s, g, tile)) ? kIdescPairHalf : kIdescPair;
+        const bool b_mn = g.mode == kDgradDH || g.mode == kDgradDX;
+        const uint32_t idesc = idesc_bf16_f32_major(
+            half_tile(g, decode_pair_tile(s, g, tile)) ? 128 : BMP, BN, false, b_mn);
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -736,7 +825,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b0 = smem_u32(s.b[stage]);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
+            umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + k * 32),
+                           b_mn ? sw128_mnmajor_desc(b0 + k * 2048, P_B_BYTES / 2)
+                                : sw128_kmajor_desc(b0 + k * 32),
                            idesc, (kb > 0 || k > 0) ? 1u : 0u);
           const uint32_t e_local = smem_u32(&s.empty[stage]);
           umma_commit_pair(mapa_shared(e_local, 0));
@@ -1173,6 +1264,41 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
   g.half_tiles = pair ? pair_half_tiles() : 0;
   return pair ? launch_pair(mx, mwgu, mwgu64, g, sm_count, st)
               : launch_one(mx, mwgu, g, sm_count, st);
+}
+
+// MOE_B200_BWD_PAIR=0 keeps the dgrad GEMMs on the one-CTA backward kernel (for
+// measurements).
+bool dgrad_use_pair(int T) {
+  static const char* env = getenv("MOE_B200_BWD_PAIR");
+  if (env && env[0] == '0') return false;
+  return use_pair_kernel(T);
+}
+
+int launch_dgrad_pair(int mode_dx, const void* a_rows, int a_cols, const void* w, int b_rows,
+                      int n, const void* gu, void* out, const int32_t* offsets, int T, int K,
+                      int n_ffn, int* status, int sm_count, cudaStream_t st) {
+  if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
+  const uint64_t rows = (uint64_t)T * K + BM;   // row buffers' allocation rows
+  CUtensorMap ma, mb;
+  int rc;
+  if ((rc = make_map(&ma, a_rows, rows, (uint64_t)a_cols)) != MOE_OK) return rc;
+  if ((rc = make_map(&mb, w, (uint64_t)n_ffn * b_rows, (uint64_t)n, 64)) != MOE_OK) return rc;
+  GemmArgs g{};
+  g.mode = mode_dx ? kDgradDX : kDgradDH;
+  g.n_ffn = n_ffn;
+  g.kblocks = a_cols / BK;
+  g.n_tiles = (n + BN - 1) / BN;
+  g.b_rows = b_rows;
+  g.n_valid = n;
+  g.ld_out = mode_dx ? n : 2 * n;
+  g.offsets = offsets;
+  g.out = out;
+  g.gu_in = static_cast<const __nv_bfloat16*>(gu);
+  g.status = status;
+  g.ksplit = 1;
+  g.kb_per_split = g.kblocks;
+  g.half_tiles = pair_half_tiles();
+  return launch_pair(ma, mb, mb, g, sm_count, st);
 }
 
 int make_tma_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,

@@ -76,6 +76,16 @@ cudaError_t launch_zero_counts(int32_t* counts, int E, int32_t* nffn_hist, int K
 int make_tma_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                       uint32_t box_rows);
 
+// The backward's dgrad GEMMs on the CTA-pair kernel (B read MN-major), for batches where
+// the forward uses it (dgrad_use_pair): mode_dx 0: dh = a_rows . W (W = w_down, b_rows = H,
+// n = I) with the SwiGLU backward from gu into out = [dG | dU] (bf16 [rows, 2I]);
+// mode_dx 1: dx rows = a_rows . W (a_rows = [dG | dU], W = w_gate_up, b_rows = 2I, n = H)
+// into out (fp32 [rows, H]).
+bool dgrad_use_pair(int T);
+int launch_dgrad_pair(int mode_dx, const void* a_rows, int a_cols, const void* w, int b_rows,
+                      int n, const void* gu, void* out, const int32_t* offsets, int T, int K,
+                      int n_ffn, int* status, int sm_count, cudaStream_t st);
+
 // ---- backward ------------------------------------------------------------------------------
 // The gate/up GEMM again, storing G and U (bf16) instead of h: gu [T*K + 128, 2I].
 int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w_gate_up,

@@ -89,8 +89,10 @@ def test_backward_full_width(cuda_device):
     _check(wl.CONFIGS["prefill_bf16"].with_(T=64, n_ffn=16, n_zero=8))
 
 
-def test_backward_is_bit_reproducible(cuda_device):
-    cfg = wl.CONFIGS["proxy_bf16"].with_(T=700)
+@pytest.mark.parametrize("T", [700, 2048])
+def test_backward_is_bit_reproducible(cuda_device, T):
+    """T = 700: the one-CTA backward GEMMs; T = 2048: the dgrad GEMMs on CTA pairs."""
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=T)
     r1 = _run(cfg, seed=4)
     r2 = _run(cfg, seed=4)
     for a, c in zip(r1[3:], r2[3:]):
