@@ -669,10 +669,11 @@ __device__ __forceinline__ bool half_tile(const GemmArgs& g, const Tile& t) {
 // 64r + 32(q & 1) + lane and N block ib = q >> 1; gate/up: h columns 64 ib + 32h + [0, 32)
 // from the gate TMEM columns 32h + [0, 32) and the up columns 64 + 32h + [0, 32); down:
 // output columns 128 ib + 64h + [0, 64) from TMEM columns 64h + [0, 64).
+template <bool DGRAD>
 __device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, uint32_t tbase,
                                               uint32_t rank, int q, int h, float (*stg)[20],
                                               int lane) {
-  if (g.mode == kDgradDH || g.mode == kDgradDX) {
+  if constexpr (DGRAD) {
     // full tile: row 128r + 32q + lane, columns [128h, 128h + 128); half tile: as the down
     // store below
     const bool half = half_tile(g, t);
@@ -685,27 +686,30 @@ __device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, 
       if (g.mode == kDgradDH) epi_dh_chunk(g, t, tbase, row, tcol, oc);
       else epi_dx_chunk(g, t, tbase, row, tcol, oc, stg, lane);
     }
-    return;
-  }
-  if (!half_tile(g, t)) {
-    epilogue_expert(g, t, tbase, t.row0 + 128 * (int)rank + q * 32 + lane, h, stg, lane);
-    return;
-  }
-  const int row = t.row0 + 64 * (int)rank + 32 * (q & 1) + lane;
-  const int ib = q >> 1;
-  if (g.mode == kGateUp) {
-    epi_gateup_chunk(g, t, tbase, row, 32 * h, 64 + 32 * h, 64 * ib + 32 * h);
-    return;
-  }
-  int tok;
-  float sc;
-  row_scale(g, t, row, tok, sc);
+  } else {
+    if (!half_tile(g, t)) {
+      epilogue_expert(g, t, tbase, t.row0 + 128 * (int)rank + q * 32 + lane, h, stg, lane);
+      return;
+    }
+    const int row = t.row0 + 64 * (int)rank + 32 * (q & 1) + lane;
+    const int ib = q >> 1;
+    if (g.mode == kGateUp) {
+      epi_gateup_chunk(g, t, tbase, row, 32 * h, 64 + 32 * h, 64 * ib + 32 * h);
+      return;
+    }
+    int tok;
+    float sc;
+    row_scale(g, t, row, tok, sc);
 #pragma unroll 1
-  for (int j = 0; j < 64; j += 32)
-    epi_down_chunk(g, t, tbase, row, 64 * h + j, 128 * ib + 64 * h + j, tok, sc, stg, lane);
+    for (int j = 0; j < 64; j += 32)
+      epi_down_chunk(g, t, tbase, row, 64 * h + j, 128 * ib + 64 * h + j, tok, sc, stg, lane);
+  }
 }
 
 // tmB64: the gate/up B tensor with 64-row boxes (half tiles); unused by the down GEMM.
+// DGRAD: the backward's dgrad modes (B read MN-major), a separate instantiation so that
+// the forward carries none of their code.
+template <bool DGRAD>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -773,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = decode_pair_tile(s, g, tile);
         const bool half = half_tile(g, t);
         const bool split_b = half && g.mode == kGateUp;   // 64 gate + 64 up rows
-        const bool b_mn = g.mode == kDgradDH || g.mode == kDgradDX;
+        constexpr bool b_mn = DGRAD;
         const int arow = t.row0 + (half ? 64 : 128) * (int)rank;
         const int brow = g.mode != kGateUp ? t.e * g.b_rows + t.nt * BN + 128 * (int)rank
                          : split_b ? t.e * g.b_rows + t.nt * BM + 64 * (int)rank
@@ -812,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
-        const bool b_mn = g.mode == kDgradDH || g.mode == kDgradDX;
+        constexpr bool b_mn = DGRAD;
         const uint32_t idesc = idesc_bf16_f32_major(
             half_tile(g, decode_pair_tile(s, g, tile)) ? 128 : BMP, BN, false, b_mn);
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
@@ -860,7 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_pair(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
+      epilogue_pair<DGRAD>(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
@@ -941,8 +945,10 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap&
   static int clusters_of[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return MOE_ERR_CUDA;
-  if (cudaFuncSetAttribute(k_grouped_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  auto kern = (g.mode == kDgradDH || g.mode == kDgradDX) ? k_grouped_gemm_pair<true>
+                                                          : k_grouped_gemm_pair<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -961,7 +967,7 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap&
     if (clusters_of[dev] == 0) {
       cfg.gridDim = dim3(sm_count & ~1);
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, k_grouped_gemm_pair, &cfg) != cudaSuccess || n < 1) {
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
       }
@@ -970,8 +976,7 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap&
     nclusters = clusters_of[dev];
   }
   if (nclusters > sm_count / 2) nclusters = sm_count / 2;
-  if (launch_kernel(k_grouped_gemm_pair, 2 * nclusters, kThreads, smem, st, 2, ma, mb, mb64, g) !=
-      cudaSuccess) {
+  if (launch_kernel(kern, 2 * nclusters, kThreads, smem, st, 2, ma, mb, mb64, g) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
