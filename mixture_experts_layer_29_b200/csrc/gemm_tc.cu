@@ -136,6 +136,9 @@ __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + _
 // ---- epilogue pieces of the expert GEMMs (one thread = one TMEM lane = one row) ---------
 // gate/up: 32 columns of h = silu(G) * U from the gate accumulator columns at tbase + gcol
 // and the up columns at tbase + ucol; h columns [oc, oc + 32) of the tile's 128.
+// KEEP: whether G and U are also stored for the backward: 0 never, 1 always, 2 when
+// g.gu_out is set (checked at run time).
+template <int KEEP>
 __device__ __forceinline__ void epi_gateup_chunk(const GemmArgs& g, const Tile& t, uint32_t tbase,
                                                  int row, int gcol, int ucol, int oc) {
   uint32_t gr[32], ur[32];
@@ -175,7 +178,7 @@ __device__ __forceinline__ void epi_gateup_chunk(const GemmArgs& g, const Tile& 
     }
     dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  if (g.gu_out) {
+  if (KEEP == 1 || (KEEP == 2 && g.gu_out)) {
     // the same G and U, rounded to bf16 as the raw store rounds them, for the backward
     __nv_bfloat16* base = static_cast<__nv_bfloat16*>(g.gu_out) + (size_t)row * 2 * g.n_valid +
                           t.nt * BM + oc;
@@ -323,12 +326,13 @@ __device__ __forceinline__ void epi_dx_chunk(const GemmArgs& g, const Tile& t, u
 // (gate/up) or 256 rows of W_d (down): gate/up half h makes h columns [64h, 64h + 64)
 // from gate columns [64h, 64h + 64) and up columns 128 + [64h, 64h + 64); down half h
 // stores columns [128h, 128h + 128).
+template <int KEEP>
 __device__ __forceinline__ void epilogue_expert(const GemmArgs& g, const Tile& t, uint32_t tbase,
                                                 int row, int half, float (*stg)[20], int lane) {
   if (g.mode == kGateUp) {
 #pragma unroll 1
     for (int c = 64 * half; c < 64 * half + 64; c += 32)
-      epi_gateup_chunk(g, t, tbase, row, c, BM + c, c);
+      epi_gateup_chunk<KEEP>(g, t, tbase, row, c, BM + c, c);
     return;
   }
   int tok;
@@ -542,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) sum[c + i] = __fadd_rn(sum[c + i], __uint_as_float(v[i]));
           }
         } else {
-          epilogue_expert(g, t, tbase, row, half, s.epi_stage[warp - 2], lane);
+          epilogue_expert<2>(g, t, tbase, row, half, s.epi_stage[warp - 2], lane);
         }
         tc_fence_before();
         mbar_arrive(&s.tempty[acc]);
@@ -669,11 +673,15 @@ __device__ __forceinline__ bool half_tile(const GemmArgs& g, const Tile& t) {
 // 64r + 32(q & 1) + lane and N block ib = q >> 1; gate/up: h columns 64 ib + 32h + [0, 32)
 // from the gate TMEM columns 32h + [0, 32) and the up columns 64 + 32h + [0, 32); down:
 // output columns 128 ib + 64h + [0, 64) from TMEM columns 64h + [0, 64).
-template <bool DGRAD>
+// Kinds of the CTA-pair kernel: the forward, the forward that also keeps G | U, and the
+// backward's dgrad modes (B read MN-major); each its own instantiation.
+constexpr int kPairFwd = 0, kPairFwdKeep = 1, kPairDgrad = 2;
+
+template <int KIND>
 __device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, uint32_t tbase,
                                               uint32_t rank, int q, int h, float (*stg)[20],
                                               int lane) {
-  if constexpr (DGRAD) {
+  if constexpr (KIND == kPairDgrad) {
     // full tile: row 128r + 32q + lane, columns [128h, 128h + 128); half tile: as the down
     // store below
     const bool half = half_tile(g, t);
@@ -688,13 +696,16 @@ __device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, 
     }
   } else {
     if (!half_tile(g, t)) {
-      epilogue_expert(g, t, tbase, t.row0 + 128 * (int)rank + q * 32 + lane, h, stg, lane);
+      epilogue_expert<KIND == kPairFwdKeep ? 1 : 0>(g, t, tbase,
+                                                     t.row0 + 128 * (int)rank + q * 32 + lane,
+                                                     h, stg, lane);
       return;
     }
     const int row = t.row0 + 64 * (int)rank + 32 * (q & 1) + lane;
     const int ib = q >> 1;
     if (g.mode == kGateUp) {
-      epi_gateup_chunk(g, t, tbase, row, 32 * h, 64 + 32 * h, 64 * ib + 32 * h);
+      epi_gateup_chunk<KIND == kPairFwdKeep ? 1 : 0>(g, t, tbase, row, 32 * h, 64 + 32 * h,
+                                                      64 * ib + 32 * h);
       return;
     }
     int tok;
@@ -707,9 +718,9 @@ __device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, 
 }
 
 // tmB64: the gate/up B tensor with 64-row boxes (half tiles); unused by the down GEMM.
-// DGRAD: the backward's dgrad modes (B read MN-major), a separate instantiation so that
-// the forward carries none of their code.
-template <bool DGRAD>
+// KIND: kPairFwd, kPairFwdKeep or kPairDgrad (see epilogue_pair), so that the plain
+// forward carries none of the other kinds' code.
+template <int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -777,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = decode_pair_tile(s, g, tile);
         const bool half = half_tile(g, t);
         const bool split_b = half && g.mode == kGateUp;   // 64 gate + 64 up rows
-        constexpr bool b_mn = DGRAD;
+        constexpr bool b_mn = KIND == kPairDgrad;
         const int arow = t.row0 + (half ? 64 : 128) * (int)rank;
         const int brow = g.mode != kGateUp ? t.e * g.b_rows + t.nt * BN + 128 * (int)rank
                          : split_b ? t.e * g.b_rows + t.nt * BM + 64 * (int)rank
@@ -816,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
-        constexpr bool b_mn = DGRAD;
+        constexpr bool b_mn = KIND == kPairDgrad;
         const uint32_t idesc = idesc_bf16_f32_major(
             half_tile(g, decode_pair_tile(s, g, tile)) ? 128 : BMP, BN, false, b_mn);
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
@@ -864,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_pair<DGRAD>(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
+      epilogue_pair<KIND>(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
@@ -945,8 +956,9 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap&
   static int clusters_of[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return MOE_ERR_CUDA;
-  auto kern = (g.mode == kDgradDH || g.mode == kDgradDX) ? k_grouped_gemm_pair<true>
-                                                          : k_grouped_gemm_pair<false>;
+  auto kern = (g.mode == kDgradDH || g.mode == kDgradDX) ? k_grouped_gemm_pair<kPairDgrad>
+               : g.gu_out                                  ? k_grouped_gemm_pair<kPairFwdKeep>
+                                                           : k_grouped_gemm_pair<kPairFwd>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
