@@ -34,6 +34,8 @@ def main(argv=None) -> int:
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--ffn-experts", type=int, default=None)
     ap.add_argument("--zero-experts", type=int, default=None)
+    ap.add_argument("--gather", action="store_true",
+                    help="no permuted copy of x: the gate/up GEMM gathers the token rows")
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     a = ap.parse_args(argv)
@@ -61,12 +63,14 @@ def main(argv=None) -> int:
                   None if logits_in is not None else b.logits, b.topk_idx, b.topk_gate,
                   b.counts, b.nffn_hist, b.zgate, b.ws)
 
+    xp = None if a.gather else b.x_perm
+
     def permute():
         abi.permute(shape, b.topk_idx, b.topk_gate, b.zgate, x, b.offsets, b.perm_token,
-                    b.row_of, b.row_gate, b.x_perm, b.out_acc, b.ws)
+                    b.row_of, b.row_gate, xp, b.out_acc, b.ws)
 
     def ffn():
-        abi.grouped_ffn(shape, x, b.x_perm, b.offsets, w.w_gate_up, w.w_down, b.perm_token,
+        abi.grouped_ffn(shape, x, xp, b.offsets, w.w_gate_up, w.w_down, b.perm_token,
                         b.row_gate, b.h, b.y_perm, b.out_acc, b.ws)
 
     def combine():

@@ -83,6 +83,27 @@ def test_layer_output_small(cuda_device, name, combine):
     _ffn_checks(case, combine)
 
 
+@pytest.mark.parametrize("T", [300, 700])
+def test_gathered_rows_match_copied_rows_bit_for_bit(cuda_device, T):
+    """x_perm NULL: the one-CTA gate/up GEMM reads the token rows of x itself with TMA
+    four-row gathers. Its MMAs see the same A values as with the permuted copy (the same
+    kernel below 1024 tokens), so the outputs are the same bits."""
+    case = gh.Case(wl.CONFIGS["proxy_bf16"].with_(T=T), seed=8)
+    b = case.buffers("deterministic")
+    copied = abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up,
+                           case.w.w_down).clone()
+    h_copied = b.h.clone()
+    b.out.zero_()
+    b.h.zero_()
+    gathered = abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up,
+                             case.w.w_down, gather=True)
+    torch.cuda.synchronize()
+    rows = int(b.offsets[case.cfg.n_ffn].item())
+    assert torch.equal(b.h[:rows], h_copied[:rows])
+    assert torch.equal(gathered, copied)
+    assert abi.read_device_status(b.ws) == 0
+
+
 @pytest.mark.parametrize("combine", ["fused", "deterministic"])
 def test_layer_output_gathered_rows_path(cuda_device, combine):
     """bf16 with token rows gathered by the GEMM instead of the permuted copy."""
