@@ -17,6 +17,7 @@
 //   k_to_bf16        W_r in bf16 for the latter
 //   k_bwd_dx_combine dx[t] += sum over FFN slots (in order) of dx_perm[row] + zgate_t dout_t
 #include <math.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -44,7 +45,9 @@ __device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
 
 constexpr int kTok = 256;   // threads per token CTA
 
-// One CTA per token; thread i owns columns 8i, 8i + 8 kTok, ... of the row.
+// One CTA per token; thread i owns columns 8i, 8i + 8 kTok, ... of the row. G slots' rows
+// are loaded before they are used (more loads in flight per thread).
+template <int G>
 __global__ void __launch_bounds__(kTok) k_bwd_dy_dgate(
     const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ x,
     const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restrict__ topk_idx,
@@ -56,10 +59,11 @@ __global__ void __launch_bounds__(kTok) k_bwd_dy_dgate(
   pdl_launch_dependents();
   pdl_wait();
   const int t = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x < K) {
-    const int e = topk_idx[(size_t)t * K + threadIdx.x];
-    s_row[threadIdx.x] = e < n_ffn ? row_of[(size_t)t * K + threadIdx.x] : -1;
-    s_g[threadIdx.x] = topk_gate[(size_t)t * K + threadIdx.x];
+  if (threadIdx.x < 32) {
+    const bool in = threadIdx.x < K;
+    const int e = in ? topk_idx[(size_t)t * K + threadIdx.x] : 0;
+    s_row[threadIdx.x] = in && e < n_ffn ? row_of[(size_t)t * K + threadIdx.x] : -1;
+    s_g[threadIdx.x] = in ? topk_gate[(size_t)t * K + threadIdx.x] : 0.f;
   }
   __syncthreads();
   float dot[32];
@@ -70,22 +74,31 @@ __global__ void __launch_bounds__(kTok) k_bwd_dy_dgate(
     load8(dout + (size_t)t * H + c, d);
     load8(x + (size_t)t * H + c, xv);
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      if (k >= K) break;
-      const int r = s_row[k];
-      if (r >= 0) {
-        float y[8];
-        load8(y_perm + (size_t)r * H + c, y);
-        const float gs = scale * s_g[k];
-        uint32_t w[4];
+    for (int k0 = 0; k0 < 32; k0 += G) {
+      if (k0 >= K) break;
+      float y[G][8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(gs * d[2 * i], gs * d[2 * i + 1]);
-        *reinterpret_cast<uint4*>(dy + (size_t)r * H + c) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int u = 0; u < G; ++u) {
+        const int r = s_row[k0 + u];
+        if (k0 + u < K && r >= 0) load8(y_perm + (size_t)r * H + c, y[u]);
+      }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dot[k] = fmaf(d[i], y[i], dot[k]);
-      } else {
+      for (int u = 0; u < G; ++u) {
+        const int k = k0 + u;
+        if (k >= K) break;
+        const int r = s_row[k];
+        if (r >= 0) {
+          const float gs = scale * s_g[k];
+          uint32_t w[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dot[k] = fmaf(d[i], xv[i], dot[k]);
+          for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(gs * d[2 * i], gs * d[2 * i + 1]);
+          *reinterpret_cast<uint4*>(dy + (size_t)r * H + c) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dot[k] = fmaf(d[i], y[u][i], dot[k]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dot[k] = fmaf(d[i], xv[i], dot[k]);
+        }
       }
     }
   }
@@ -247,8 +260,13 @@ cudaError_t launch_bwd_dy_dgate(const void* dout, const void* x, const void* y_p
                                 const int32_t* topk_idx, const float* topk_gate,
                                 const int32_t* row_of, int T, int H, int K, int n_ffn,
                                 float scale, void* dy, float* d_gate, cudaStream_t st) {
+  static const int g_env = [] {
+    const char* v = getenv("MOE_B200_DY_G");
+    return v ? atoi(v) : 4;
+  }();
   const cudaError_t e = launch_kernel(
-      k_bwd_dy_dgate, T, kTok, 0, st, 1, static_cast<const __nv_bfloat16*>(dout),
+      g_env == 1 ? k_bwd_dy_dgate<1> : k_bwd_dy_dgate<4>, T, kTok, 0, st, 1,
+      static_cast<const __nv_bfloat16*>(dout),
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm), topk_idx,
       topk_gate, row_of, H, K, n_ffn, scale, static_cast<__nv_bfloat16*>(dy), d_gate);
   count_launch();
