@@ -167,6 +167,20 @@ def oracle_sample(cfg, w, x_dev, tokens, logits_dev=None):
     return time.perf_counter() - t0, len(tokens)
 
 
+def cpu_baseline_sample(cfg, w, x, logits_in, first: int, target_s: float):
+    """The oracle on a bounded token sample sized for about `target_s` seconds of oracle
+    time: `first` tokens, then as many more (up to the batch) as that rate allows. The
+    tokens are a fixed-seed random permutation of the batch. Returns (seconds, tokens)."""
+    order = np.random.default_rng(0).permutation(cfg.T).tolist()
+    n1 = min(first, cfg.T)
+    secs, n = oracle_sample(cfg, w, x, sorted(order[:n1]), logits_in)
+    more = min(cfg.T - n1, int(n * max(0.0, target_s - secs) / max(secs, 1e-9)))
+    if more > 0:
+        s2, n2 = oracle_sample(cfg, w, x, sorted(order[n1:n1 + more]), logits_in)
+        secs, n = secs + s2, n + n2
+    return secs, n
+
+
 # ------------------------------------------------------------------------------ our arm
 
 class Stepper:
@@ -600,13 +614,11 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rng = np.random.default_rng(0)
-        toks = sorted(rng.choice(cfg.T, size=min(args.cpu_tokens, cfg.T), replace=False).tolist())
-        secs, n = oracle_sample(cfg, w, x, toks, logits_in)
+        secs, n = cpu_baseline_sample(cfg, w, x, logits_in, args.cpu_tokens, args.cpu_seconds)
         cpu = {"value": round(n / secs, 3), "unit": UNIT, "cores": oracle_threads(),
                "kind": "oracle",
-               "sample": f"{n} of the {cfg.T} tokens (logits, routing and SwiGLU experts in "
-                         f"float64 numpy), {secs:.1f} s"}
+               "sample": f"{n} of the {cfg.T} tokens, drawn with a fixed seed (logits, routing "
+                         f"and SwiGLU experts in float64 numpy), {secs:.1f} s of oracle time"}
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -689,7 +701,10 @@ def parser() -> argparse.ArgumentParser:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_bf16", choices=sorted(wl.CONFIGS))
     ap.add_argument("--combine", default="deterministic", choices=["fused", "deterministic"])
-    ap.add_argument("--cpu-tokens", type=int, default=400)
+    ap.add_argument("--cpu-tokens", type=int, default=400,
+                    help="first slice of the oracle's token sample")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="oracle time the CPU baseline's sample is sized for")
     ap.add_argument("--ref-tokens", type=int, default=8)
     ap.add_argument("--tokens", type=int, default=None, help="override the workload's T")
     ap.add_argument("--ffn-experts", type=int, default=None, help="override n_ffn (profiling)")
