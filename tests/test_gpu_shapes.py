@@ -1,0 +1,97 @@
+"""The layer on shapes the named workloads do not reach, against the oracle.
+
+The named workloads have hidden sizes that are multiples of 256, E a multiple of 8 and
+K >= 4. These bf16 layers put the other edges under test:
+  * H % 256 == 128 (a half-valid last N tile of the down GEMM and of the router);
+  * I an odd multiple of 128 (gate/up N tiles of 128 gate + 128 up rows);
+  * H = 128 (two k-blocks);
+  * E not a multiple of 8 or 32, K = 1, no zero experts;
+  * T on both sides of the CTA-pair threshold (1024), ragged against every tile.
+Each runs the four step calls in both combine modes and checks routing bit for bit (away
+from near ties), every permuted row's y (deterministic mode) and the whole output within
+the bf16 bar, on every token. One shape also runs the backward."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_harness as gh
+import oracle.moe_oracle as orc
+from mixture_experts_layer_29_b200 import abi
+from mixture_experts_layer_29_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = {
+    #            T,    H,   I,  N,  Z, K
+    "h384":    (777, 384, 128, 8, 4, 3),
+    "h640_pair": (1100, 640, 384, 12, 0, 2),
+    "e27":     (513, 896, 256, 20, 7, 5),
+    "k1_i640": (2048, 384, 640, 6, 2, 1),
+    "h128":    (64, 128, 128, 3, 1, 2),
+}
+
+
+def _cfg(name):
+    T, H, I, N, Z, K = SHAPES[name]
+    return wl.CONFIGS["proxy_bf16"].with_(name=f"shape_{name}", T=T, H=H, I=I, n_ffn=N,
+                                          n_zero=Z, K=K)
+
+
+@pytest.mark.parametrize("name", sorted(SHAPES))
+@pytest.mark.parametrize("combine", ["deterministic", "fused"])
+def test_odd_shape_layer_matches_oracle(cuda_device, name, combine):
+    cfg = _cfg(name)
+    case = gh.Case(cfg, seed=21)
+    b = case.buffers(combine)
+    out = abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up,
+                        case.w.w_down)
+    torch.cuda.synchronize()
+    assert abi.read_device_status(b.ws) == 0
+    gh.check_routing(case, b)
+    gh.check_permutation(case, b, zero_init=False)
+    L = case.gpu_logits(b)
+    toks = list(range(cfg.T))
+    o_out, _, _, y_rows, _, _ = gh.oracle_layer(case, L, toks)
+    # tokens whose selection is a near tie may route differently on the two sides
+    r = orc.route(L, gh.host(case.w.bias), cfg.n_ffn, cfg.K)
+    same = np.all(np.sort(gh.host(b.topk_idx), 1) == np.sort(r.topk_idx, 1), axis=1)
+    err = gh.row_rel_err(gh.host(out)[: cfg.T][same], o_out[same])
+    assert err <= gh.TOL["bf16"], err
+    if combine == "deterministic":
+        row_of = gh.host(b.row_of).reshape(cfg.T, cfg.K)
+        yp = gh.host(b.y_perm)
+        keys = [key for key in sorted(y_rows) if same[key[0]]]
+        if keys:
+            got = np.stack([yp[row_of[t, k]] for (t, k) in keys])
+            want = np.stack([y_rows[key] for key in keys])
+            assert gh.row_rel_err(got, want) <= gh.TOL["bf16"]
+
+
+def test_odd_shape_backward_matches_oracle(cuda_device):
+    """H = 384 (half-valid last N tiles in every backward GEMM), I = 384, E = 16."""
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=600, H=384, I=384, n_ffn=12, n_zero=4, K=3)
+    case = gh.Case(cfg, seed=22)
+    b = case.buffers("deterministic")
+    abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up, case.w.w_down)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    dout = (torch.randn(cfg.T, cfg.H, device="cuda", generator=g) * 0.5).to(torch.bfloat16)
+    dx = torch.empty(cfg.T, cfg.H, dtype=torch.float32, device="cuda")
+    d_router = torch.empty(cfg.E, cfg.H, dtype=torch.float32, device="cuda")
+    d_gu = torch.zeros(cfg.n_ffn, 2 * cfg.I, cfg.H, dtype=torch.float32, device="cuda")
+    d_d = torch.zeros(cfg.n_ffn, cfg.H, cfg.I, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(abi.backward_workspace_size(b.shape), dtype=torch.uint8, device="cuda")
+    abi.backward(b.shape, dout, case.x, case.w.w_router, case.w.w_gate_up, case.w.w_down,
+                 b.logits, b.topk_idx, b.topk_gate, b.offsets, b.row_of, b.x_perm, b.h,
+                 b.y_perm, dx, d_router, d_gu, d_d, ws)
+    torch.cuda.synchronize()
+    assert abi.read_device_status(ws) == 0
+    ref = orc.moe_layer_backward(gh.host(case.x), gh.host(case.w.w_router), gh.host(case.w.bias),
+                                 gh.host(case.w.w_gate_up), gh.host(case.w.w_down), cfg.n_ffn,
+                                 cfg.K, gh.host(dout), cfg.ffn_out_scale,
+                                 topk_idx=gh.host(b.topk_idx))
+    assert gh.row_rel_err(gh.host(dx), ref.dx) <= gh.TOL["bf16"]
+    assert gh.row_rel_err(gh.host(d_router), ref.d_router) <= gh.TOL["bf16"]
+    counts = gh.host(b.counts)[: cfg.n_ffn]
+    for e in np.nonzero(counts > 0)[0]:
+        for got, want in ((gh.host(d_gu[e]), ref.d_gate_up[e]), (gh.host(d_d[e]), ref.d_down[e])):
+            assert np.abs(got - want).max() / max(np.abs(want).max(), 1e-30) <= gh.TOL["bf16"]
