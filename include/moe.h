@@ -29,7 +29,8 @@
  *    read back with moe_read_device_status; kernels never trap.
  *  - T = 0 is valid: the call checks its arguments and launches nothing.
  *  - Limits: 1 <= E <= 1024, 1 <= K <= min(32, E), n_ffn >= 1, n_zero >= 0, T < 2^24,
- *    T * K < 2^31. bf16: H % 128 == 0 and I % 128 == 0. fp32: H, I >= 1.
+ *    T * K < 2^31, H % 16 == 0 (rows move 16 bytes at a time), I >= 1. bf16 also needs
+ *    H % 128 == 0 and I % 128 == 0. Other shapes give MOE_ERR_UNSUPPORTED.
  */
 #ifndef MOE_B200_H_
 #define MOE_B200_H_

@@ -95,3 +95,35 @@ def test_odd_shape_backward_matches_oracle(cuda_device):
     for e in np.nonzero(counts > 0)[0]:
         for got, want in ((gh.host(d_gu[e]), ref.d_gate_up[e]), (gh.host(d_d[e]), ref.d_down[e])):
             assert np.abs(got - want).max() / max(np.abs(want).max(), 1e-30) <= gh.TOL["bf16"]
+
+
+FP32_SHAPES = {
+    #            T,   H,   I,  N, Z, K
+    "f_odd":   (50, 112, 36, 5, 3, 2),
+    "f_prime": (301, 272, 129, 9, 0, 4),
+    "f_k1":    (97, 64, 1, 2, 5, 1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FP32_SHAPES))
+@pytest.mark.parametrize("combine", ["deterministic", "fused"])
+def test_odd_fp32_shape_layer_matches_oracle(cuda_device, name, combine):
+    """fp32 layers (the CUDA-core FFN) take any I >= 1 and H % 16 == 0: I = 1, 36, 129 and
+    H = 112, 272 (not multiples of 32), against the oracle within 1e-5."""
+    T, H, I, N, Z, K = FP32_SHAPES[name]
+    cfg = wl.CONFIGS["tiny_fp32"].with_(name=f"shape_{name}", T=T, H=H, I=I, n_ffn=N,
+                                        n_zero=Z, K=K)
+    case = gh.Case(cfg, seed=23)
+    b = case.buffers(combine)
+    out = abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up,
+                        case.w.w_down)
+    torch.cuda.synchronize()
+    assert abi.read_device_status(b.ws) == 0
+    gh.check_routing(case, b)
+    gh.check_permutation(case, b, zero_init=False)
+    L = case.gpu_logits(b)
+    o_out, _, _, _, _, _ = gh.oracle_layer(case, L, list(range(cfg.T)))
+    r = orc.route(L, gh.host(case.w.bias), cfg.n_ffn, cfg.K)
+    same = np.all(np.sort(gh.host(b.topk_idx), 1) == np.sort(r.topk_idx, 1), axis=1)
+    err = gh.row_rel_err(gh.host(out)[: cfg.T][same], o_out[same])
+    assert err <= gh.TOL["fp32"], err
