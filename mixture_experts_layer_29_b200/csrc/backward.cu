@@ -50,9 +50,9 @@ constexpr int kTok = 256;   // threads per token CTA
 template <int G>
 __global__ void __launch_bounds__(kTok) k_bwd_dy_dgate(
     const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ x,
-    const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restrict__ topk_idx,
-    const float* __restrict__ topk_gate, const int32_t* __restrict__ row_of, int H, int K,
-    int n_ffn, float scale, __nv_bfloat16* __restrict__ dy, float* __restrict__ d_gate) {
+    const __nv_bfloat16* y_perm, const int32_t* topk_idx,
+    const float* topk_gate, const int32_t* row_of, int H, int K,
+    int n_ffn, float scale, __nv_bfloat16* dy, float* d_gate) {
   __shared__ int s_row[32];
   __shared__ float s_g[32];
   __shared__ float s_red[kTok / 32][33];
@@ -124,12 +124,12 @@ __global__ void __launch_bounds__(kTok) k_bwd_dy_dgate(
 // written as zeros. Block 0 also writes the two one-group offset tables of the router
 // GEMMs: offs_k = {0, 3 Tp}, offs_m = {0, T}.
 template <int J>
-__global__ void __launch_bounds__(256) k_bwd_router(const float* __restrict__ logits,
-                                                    const int32_t* __restrict__ topk_idx,
-                                                    const float* __restrict__ d_gate, int T,
+__global__ void __launch_bounds__(256) k_bwd_router(const float* logits,
+                                                    const int32_t* topk_idx,
+                                                    const float* d_gate, int T,
                                                     int Tp, int E, int K,
-                                                    __nv_bfloat16* __restrict__ dl3,
-                                                    int32_t* __restrict__ offs) {
+                                                    __nv_bfloat16* dl3,
+                                                    int32_t* offs) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -199,8 +199,8 @@ __global__ void __launch_bounds__(256) k_bwd_router(const float* __restrict__ lo
   }
 }
 
-__global__ void __launch_bounds__(256) k_to_bf16(const float* __restrict__ a,
-                                                 __nv_bfloat16* __restrict__ out, size_t n) {
+__global__ void __launch_bounds__(256) k_to_bf16(const float* a,
+                                                 __nv_bfloat16* out, size_t n) {
   pdl_launch_dependents();
   pdl_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
@@ -210,9 +210,9 @@ __global__ void __launch_bounds__(256) k_to_bf16(const float* __restrict__ a,
 
 // dx[t] += sum over FFN slots k (in order) of dx_perm[row_of[t, k]] + zgate_t * dout_t
 __global__ void __launch_bounds__(kTok) k_bwd_dx_combine(
-    const float* __restrict__ dx_perm, const __nv_bfloat16* __restrict__ dout,
-    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_gate,
-    const int32_t* __restrict__ row_of, int H, int K, int n_ffn, float* __restrict__ dx) {
+    const float* dx_perm, const __nv_bfloat16* __restrict__ dout,
+    const int32_t* topk_idx, const float* topk_gate,
+    const int32_t* row_of, int H, int K, int n_ffn, float* dx) {
   __shared__ int s_row[32];
   __shared__ float s_z;
   pdl_launch_dependents();

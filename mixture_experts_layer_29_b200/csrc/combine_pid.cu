@@ -45,7 +45,7 @@ struct Vec<float> {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(256) k_finalize(const float* __restrict__ acc, T* __restrict__ out,
+__global__ void __launch_bounds__(256) k_finalize(const float* acc, T* out,
                                                   size_t n) {
   pdl_launch_dependents();
   pdl_wait();
@@ -66,11 +66,11 @@ __global__ void __launch_bounds__(256) k_finalize(const float* __restrict__ acc,
 // G rows are loaded before they are summed: G = 4 for small batches (more loads in
 // flight per thread), 1 for large ones (fewer registers, more CTAs per SM).
 template <typename T, int G>
-__global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, const T* __restrict__ y_perm,
-                                                     const float* __restrict__ topk_gate,
-                                                     const int32_t* __restrict__ row_of,
-                                                     const float* __restrict__ zgate,
-                                                     T* __restrict__ out, int H, int K, float scale) {
+__global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, const T* y_perm,
+                                                     const float* topk_gate,
+                                                     const int32_t* row_of,
+                                                     const float* zgate,
+                                                     T* out, int H, int K, float scale) {
   constexpr int V = Vec<T>::N;
   __shared__ int s_row[32 + G];
   __shared__ float s_g[32 + G];
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, co
   }
 }
 
-__global__ void k_pid_init(const float* __restrict__ bias, float* __restrict__ st, int n_ffn) {
+__global__ void k_pid_init(const float* bias, float* st, int n_ffn) {
   pdl_launch_dependents();
   pdl_wait();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_ffn; i += gridDim.x * blockDim.x) {
@@ -131,11 +131,11 @@ __global__ void k_pid_init(const float* __restrict__ bias, float* __restrict__ s
 constexpr int kPidThreads = 256;
 
 __global__ void __launch_bounds__(kPidThreads) k_pid_update(moe_pid_t pid,
-                                                            const int32_t* __restrict__ counts,
-                                                            const int32_t* __restrict__ hist,
-                                                            float* __restrict__ bias,
-                                                            float* __restrict__ st,
-                                                            float* __restrict__ stats, int T,
+                                                            const int32_t* counts,
+                                                            const int32_t* hist,
+                                                            float* bias,
+                                                            float* st,
+                                                            float* stats, int T,
                                                             int K, int n_ffn, int E) {
   constexpr int W = kPidThreads / 32;
   __shared__ double red[W][8];

@@ -22,9 +22,9 @@ __device__ __forceinline__ int expert_of_row(const int32_t* offsets, int n_ffn, 
   return lo;
 }
 
-__global__ void __launch_bounds__(128) k_ffn_up_simt(const float* __restrict__ x_perm,
-                                                     const int32_t* __restrict__ offsets,
-                                                     const float* __restrict__ wgu, float* __restrict__ h,
+__global__ void __launch_bounds__(128) k_ffn_up_simt(const float* x_perm,
+                                                     const int32_t* offsets,
+                                                     const float* __restrict__ wgu, float* h,
                                                      int H, int I, int n_ffn) {
   pdl_launch_dependents();
   pdl_wait();
@@ -46,13 +46,13 @@ __global__ void __launch_bounds__(128) k_ffn_up_simt(const float* __restrict__ x
   }
 }
 
-__global__ void __launch_bounds__(128) k_ffn_down_simt(const float* __restrict__ h,
-                                                       const int32_t* __restrict__ offsets,
+__global__ void __launch_bounds__(128) k_ffn_down_simt(const float* h,
+                                                       const int32_t* offsets,
                                                        const float* __restrict__ wd,
-                                                       const int32_t* __restrict__ perm_token,
-                                                       const float* __restrict__ row_gate,
-                                                       float* __restrict__ y_perm,
-                                                       float* __restrict__ out_acc, int H, int I,
+                                                       const int32_t* perm_token,
+                                                       const float* row_gate,
+                                                       float* y_perm,
+                                                       float* out_acc, int H, int I,
                                                        int n_ffn, float scale, int fused) {
   pdl_launch_dependents();
   pdl_wait();

@@ -28,9 +28,9 @@ constexpr int kLbTokens = 64;                        // tokens per CTA
 constexpr int kLbPerWarp = kLbTokens / kLbWarps;
 
 template <int J>
-__global__ void __launch_bounds__(kLbWarps * 32) k_lb_partial(const float* __restrict__ logits,
+__global__ void __launch_bounds__(kLbWarps * 32) k_lb_partial(const float* logits,
                                                              int T, int E,
-                                                             double* __restrict__ part) {
+                                                             double* part) {
   __shared__ double s_acc[kLbWarps][32 * J];
   pdl_launch_dependents();
   pdl_wait();
@@ -94,11 +94,11 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
   return red[32];
 }
 
-__global__ void __launch_bounds__(1024) k_lb_finish(const double* __restrict__ part, int nchunk,
-                                                    const int32_t* __restrict__ counts, int T,
+__global__ void __launch_bounds__(1024) k_lb_finish(const double* part, int nchunk,
+                                                    const int32_t* counts, int T,
                                                     int E, int n_ffn, int K,
-                                                    float* __restrict__ prob_mean,
-                                                    float* __restrict__ loss) {
+                                                    float* prob_mean,
+                                                    float* loss) {
   __shared__ double red[33];
   pdl_launch_dependents();
   pdl_wait();

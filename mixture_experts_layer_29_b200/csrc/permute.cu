@@ -38,9 +38,9 @@ __device__ __forceinline__ bool valid_pick(const int32_t* idx_row, int k, int E,
   return true;
 }
 
-__global__ void __launch_bounds__(256) k_perm_masks(const int32_t* __restrict__ topk_idx, int T,
+__global__ void __launch_bounds__(256) k_perm_masks(const int32_t* topk_idx, int T,
                                                     int n_ffn, int E, int K, int nchunk,
-                                                    uint32_t* __restrict__ masks, int* status) {
+                                                    uint32_t* masks, int* status) {
   extern __shared__ uint32_t sm_masks[];   // [8][n_ffn]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   pdl_launch_dependents();
@@ -66,9 +66,9 @@ __global__ void __launch_bounds__(256) k_perm_masks(const int32_t* __restrict__ 
 }
 
 // one warp per FFN expert
-__global__ void __launch_bounds__(256) k_perm_scan(const uint32_t* __restrict__ masks, int n_ffn,
-                                                   int nchunk, int32_t* __restrict__ crel,
-                                                   int32_t* __restrict__ ecount) {
+__global__ void __launch_bounds__(256) k_perm_scan(const uint32_t* masks, int n_ffn,
+                                                   int nchunk, int32_t* crel,
+                                                   int32_t* ecount) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -90,12 +90,12 @@ __global__ void __launch_bounds__(256) k_perm_scan(const uint32_t* __restrict__ 
 // 8 tokens per CTA (one warp each). VEC = 16-byte vectors per row of x.
 template <bool XBF16>
 __global__ void __launch_bounds__(256) k_perm_scatter(
-    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_gate,
-    const float* __restrict__ zgate, const void* __restrict__ x, int T, int H, int n_ffn, int E,
-    int K, int nchunk, const uint32_t* __restrict__ masks, const int32_t* __restrict__ crel,
-    const int32_t* __restrict__ ecount, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ perm_token, int32_t* __restrict__ row_of, float* __restrict__ row_gate,
-    void* __restrict__ x_perm, float* __restrict__ out_acc, int* status) {
+    const int32_t* topk_idx, const float* topk_gate,
+    const float* zgate, const void* __restrict__ x, int T, int H, int n_ffn, int E,
+    int K, int nchunk, const uint32_t* masks, const int32_t* crel,
+    const int32_t* ecount, int32_t* offsets,
+    int32_t* perm_token, int32_t* row_of, float* row_gate,
+    void* x_perm, float* out_acc, int* status) {
   __shared__ int32_t s_off[1025];
   __shared__ int32_t s_wsum[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -188,9 +188,9 @@ constexpr int kSmallT = 512;
 // memory, the expert counts, the offsets (block scan), then every pick's row. The same
 // ranking as the three-kernel path, so the same rows.
 __global__ void __launch_bounds__(512) k_perm_index_small(
-    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_gate, int T, int n_ffn,
-    int E, int K, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
-    int32_t* __restrict__ row_of, float* __restrict__ row_gate, int* status) {
+    const int32_t* topk_idx, const float* topk_gate, int T, int n_ffn,
+    int E, int K, int32_t* offsets, int32_t* perm_token,
+    int32_t* row_of, float* row_gate, int* status) {
   extern __shared__ uint32_t sm[];
   const int nch = (T + 31) / 32;                                 // 32-token chunks (<= 16)
   uint32_t* masks = sm;                                          // [n_ffn][nch]
@@ -298,11 +298,11 @@ __global__ void __launch_bounds__(512) k_perm_index_small(
 // Copy x[t] into the rows of its FFN picks (and out_acc = zgate * x): block (t, seg) takes
 // one contiguous slice of the row, 16 bytes per thread per step.
 template <bool XBF16>
-__global__ void __launch_bounds__(128) k_perm_copy(const int32_t* __restrict__ row_of,
-                                                   const float* __restrict__ zgate,
+__global__ void __launch_bounds__(128) k_perm_copy(const int32_t* row_of,
+                                                   const float* zgate,
                                                    const void* __restrict__ x, int H, int K,
-                                                   void* __restrict__ x_perm,
-                                                   float* __restrict__ out_acc) {
+                                                   void* x_perm,
+                                                   float* out_acc) {
   __shared__ int32_t s_rows[32];
   pdl_launch_dependents();
   pdl_wait();
@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(128) k_perm_copy(const int32_t* __restrict__ r
 }  // namespace
 
 cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, const float* zgate,
-                           const void* x, int x_is_bf16, int T, int H, int n_ffn, int E, int K,
+                           const void* __restrict__ x, int x_is_bf16, int T, int H, int n_ffn, int E, int K,
                            uint32_t* masks, int32_t* crel, int32_t* ecount, int32_t* offsets,
                            int32_t* perm_token, int32_t* row_of, float* row_gate, void* x_perm,
                            float* out_acc, int* status, cudaStream_t st) {

@@ -25,7 +25,7 @@ constexpr int RB = 128, RK = 16, RPAD = 4;
 constexpr int kSmMax = 160;   // sizing bound for the split-K partial buffer
 
 template <bool XBF16>
-__device__ __forceinline__ void load_x_slice(const void* x, int T, int H, int row0, int k0,
+__device__ __forceinline__ void load_x_slice(const void* __restrict__ x, int T, int H, int row0, int k0,
                                              float (&v)[8], int& r, int& kk) {
   const int tid = threadIdx.x;
   if (XBF16) {
@@ -56,7 +56,7 @@ __device__ __forceinline__ void load_x_slice(const void* x, int T, int H, int ro
   }
 }
 
-__device__ __forceinline__ void load_w_slice(const float* w, int E, int H, int col0, int k0,
+__device__ __forceinline__ void load_w_slice(const float* __restrict__ w, int E, int H, int col0, int k0,
                                              float (&v)[8]) {
   const int tid = threadIdx.x;
   const int r = tid >> 2, kk = (tid & 3) * 4;
@@ -72,7 +72,7 @@ __device__ __forceinline__ void load_w_slice(const float* w, int E, int H, int c
 template <bool XBF16>
 __global__ void __launch_bounds__(256, 2) k_router_logits(const void* __restrict__ x,
                                                        const float* __restrict__ w, int T, int E,
-                                                       int H, int kchunk, float* __restrict__ out,
+                                                       int H, int kchunk, float* out,
                                                        size_t split_stride, ZeroSpec zero) {
   __shared__ __align__(16) float As[2][RK][RB + RPAD];
   __shared__ __align__(16) float Bs[2][RK][RB + RPAD];
@@ -155,8 +155,8 @@ __global__ void __launch_bounds__(256, 2) k_router_logits(const void* __restrict
 }
 
 // logits = sum over splits s = 0, 1, ... of partial[s] (fixed order)
-__global__ void k_router_splitk_sum(const float* __restrict__ partial, int S, size_t n,
-                                    float* __restrict__ logits) {
+__global__ void k_router_splitk_sum(const float* partial, int S, size_t n,
+                                    float* logits) {
   pdl_launch_dependents();
   pdl_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
@@ -195,7 +195,7 @@ size_t router_partial_bytes(int T, int E, int H, int sm_count_max) {
   return s > 1 ? (size_t)s * T * E * sizeof(float) : 0;
 }
 
-cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_router, int T,
+cudaError_t launch_router_logits(const void* __restrict__ x, int x_is_bf16, const float* w_router, int T,
                                  int E, int H, float* logits, float* partial, int splitk,
                                  ZeroSpec zero, cudaStream_t st) {
   int kchunk = (H + splitk - 1) / splitk;
@@ -252,9 +252,9 @@ struct WarpScratch {        // per warp, in shared memory
 template <int J>
 __device__ __forceinline__ void route_token(float (&lv)[J], const float (&bia)[J], int lane, int t,
                                             int E, int n_ffn, int K, WarpScratch& ws,
-                                            int32_t* __restrict__ topk_idx,
-                                            float* __restrict__ topk_gate,
-                                            float* __restrict__ zgate, int* cnt, int* hist) {
+                                            int32_t* topk_idx,
+                                            float* topk_gate,
+                                            float* zgate, int* cnt, int* hist) {
   constexpr unsigned kFull = 0xffffffffu;
   float m = -INFINITY;
 #pragma unroll
@@ -389,7 +389,7 @@ __device__ __forceinline__ void route_token(float (&lv)[J], const float (&bia)[J
 }
 
 template <int J>
-__device__ __forceinline__ void load_bias(const float* __restrict__ bias, int E, int lane,
+__device__ __forceinline__ void load_bias(const float* bias, int E, int lane,
                                           float (&bia)[J]) {
 #pragma unroll
   for (int j = 0; j < J; ++j) {
@@ -403,10 +403,10 @@ __device__ __forceinline__ void load_bias(const float* __restrict__ bias, int E,
 // in slice order (S = 1: the logits themselves; S > 1: the sum is also written out).
 template <int J, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1) k_route_topk(
-    const float* __restrict__ src, int S, size_t slice, float* __restrict__ logits_out,
-    const float* __restrict__ bias, int T, int E, int n_ffn, int K,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ counts,
-    int32_t* __restrict__ nffn_hist, float* __restrict__ zgate) {
+    const float* src, int S, size_t slice, float* logits_out,
+    const float* bias, int T, int E, int n_ffn, int K,
+    int32_t* topk_idx, float* topk_gate, int32_t* counts,
+    int32_t* nffn_hist, float* zgate) {
   __shared__ int s_counts[WARPS > 1 ? 1024 : 1];
   __shared__ int s_hist[33];
   __shared__ WarpScratch s_ws[WARPS];
@@ -455,9 +455,9 @@ __global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1) k_route_topk(
 constexpr int kSumThreads = 256;
 
 template <int W>
-__device__ __forceinline__ void sum_slices(const float* __restrict__ row, size_t slice, int S,
-                                           int n, float* __restrict__ out_s,
-                                           float* __restrict__ out_g) {
+__device__ __forceinline__ void sum_slices(const float* row, size_t slice, int S,
+                                           int n, float* out_s,
+                                           float* out_g) {
   using V = typename std::conditional<W == 4, float4, float>::type;
   const V* p = reinterpret_cast<const V*>(row);
   const size_t sl = slice / W;
@@ -499,10 +499,10 @@ __device__ __forceinline__ void sum_slices(const float* __restrict__ row, size_t
 
 template <int J>
 __global__ void __launch_bounds__(kSumThreads, 1) k_route_topk_sum(
-    const float* __restrict__ src, int S, size_t slice, float* __restrict__ logits_out,
-    const float* __restrict__ bias, int T, int E, int n_ffn, int K,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ counts,
-    int32_t* __restrict__ nffn_hist, float* __restrict__ zgate, int vec4) {
+    const float* src, int S, size_t slice, float* logits_out,
+    const float* bias, int T, int E, int n_ffn, int K,
+    int32_t* topk_idx, float* topk_gate, int32_t* counts,
+    int32_t* nffn_hist, float* zgate, int vec4) {
   __shared__ __align__(16) float s_l[32 * J];
   __shared__ WarpScratch s_ws;
   pdl_launch_dependents();
@@ -526,7 +526,7 @@ __global__ void __launch_bounds__(kSumThreads, 1) k_route_topk_sum(
                  nffn_hist);
 }
 
-__global__ void k_zero2(int32_t* __restrict__ a, int na, int32_t* __restrict__ b, int nb) {
+__global__ void k_zero2(int32_t* a, int na, int32_t* b, int nb) {
   pdl_launch_dependents();
   pdl_wait();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < na; i += gridDim.x * blockDim.x) a[i] = 0;

@@ -28,11 +28,11 @@ def _capture(fn, mode):
 
 
 @pytest.mark.parametrize("mode", ["global", "thread_local"])
-@pytest.mark.parametrize("name,T", [("decode_like", 128), ("proxy_bf16", 2048)])
+@pytest.mark.parametrize("name,T", [("proxy_bf16", 128), ("proxy_bf16", 2048), ("tiny_fp32", 64)])
 def test_step_calls_replay_bit_identical(cuda_device, name, T, mode):
     """T = 128: the small-batch kernels (split-K router sum, one-CTA permutation index);
-    T = 2048: the CTA-pair GEMMs."""
-    cfg = wl.CONFIGS["proxy_bf16"].with_(T=T)
+    T = 2048: the CTA-pair GEMMs; the fp32 layer: the CUDA-core router and FFN."""
+    cfg = wl.CONFIGS[name].with_(T=T)
     case = gh.Case(cfg, seed=12)
     b = case.buffers("deterministic")
     x = case.x.clone()

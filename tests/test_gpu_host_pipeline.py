@@ -42,11 +42,11 @@ def test_forward_host_matches_device_forward(cuda_device):
     assert torch.equal(oh, want.cpu())
 
 
-@pytest.mark.parametrize("T", [300, 2048])
-def test_pipeline_batches_match_device_forward(cuda_device, T):
+@pytest.mark.parametrize("name,T", [("proxy_bf16", 300), ("proxy_bf16", 2048), ("tiny_fp32", 64)])
+def test_pipeline_batches_match_device_forward(cuda_device, name, T):
     """Five batches through two slots: every slot is reused, and each batch's input copy
-    overlaps the previous batch's kernels."""
-    cfg = wl.CONFIGS["proxy_bf16"].with_(T=T)
+    overlaps the previous batch's kernels (bf16 on both GEMM kernels, and an fp32 layer)."""
+    cfg = wl.CONFIGS[name].with_(T=T)
     layer, _ = _layer(cfg)
     xs = [wl.draw_tokens(cfg, "cuda", seed=20 + i) for i in range(5)]
     want = [_device_out(layer, x) for x in xs]

@@ -1,0 +1,44 @@
+"""Source rules the kernels keep, checked on the text of csrc/ (no GPU).
+
+Every kernel is launched as a programmatic dependent of the one before it and triggers
+its dependents first. A kernel can therefore be resident while its predecessors still
+write its inputs. Loads through `const __restrict__` pointers or `__ldg` compile to the
+non-coherent form, which is only valid for memory that no one writes while the kernel
+lives. So those qualifiers may mark only weights and the caller's inputs, which no kernel
+of the chain writes."""
+import pathlib
+import re
+
+CSRC = pathlib.Path(__file__).resolve().parents[1] / "mixture_experts_layer_29_b200" / "csrc"
+
+# caller inputs and weights: never written by a kernel of the launch chain
+READ_ONLY_NAMES = {"x", "w", "wgu", "wd", "dout"}
+# k_split_router_weight writes a bf16 copy of the router weight through `out`
+WRITE_ONLY = {("gemm_tc.cu", "out")}
+
+
+def _sources():
+    files = sorted(CSRC.glob("*.cu")) + sorted(CSRC.glob("*.cuh"))
+    assert files
+    return [(f.name, f.read_text()) for f in files]
+
+
+def test_restrict_marks_only_inputs_and_weights():
+    bad = []
+    for name, text in _sources():
+        for m in re.finditer(r"__restrict__\s+(\w+)", text):
+            p = m.group(1)
+            if p not in READ_ONLY_NAMES and (name, p) not in WRITE_ONLY:
+                line = text.count("\n", 0, m.start()) + 1
+                bad.append(f"{name}:{line} {p}")
+    assert not bad, bad
+
+
+def test_ldg_reads_only_the_token_rows():
+    """The two __ldg users read rows of the caller's x (`src` points into x)."""
+    for name, text in _sources():
+        for m in re.finditer(r"__ldg\(\s*(\w+)", text):
+            assert m.group(1) == "src", (name, m.group(0))
+            before = text[: m.start()]
+            decl = before[before.rfind("const uint4* src"):]
+            assert "static_cast<const char*>(x)" in decl.split(";")[0], name
