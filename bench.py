@@ -167,17 +167,24 @@ def oracle_sample(cfg, w, x_dev, tokens, logits_dev=None):
     return time.perf_counter() - t0, len(tokens)
 
 
-def cpu_baseline_sample(cfg, w, x, logits_in, first: int, target_s: float):
+def cpu_baseline_sample(cfg, w, x, logits_in, first: int, target_s: float, max_slices: int = 5):
     """The oracle on a bounded token sample sized for about `target_s` seconds of oracle
-    time: `first` tokens, then as many more (up to the batch) as that rate allows. The
-    tokens are a fixed-seed random permutation of the batch. Returns (seconds, tokens)."""
+    time. The tokens are a fixed-seed random permutation of the batch, taken in slices:
+    `first` tokens, then each further slice sized from the previous slice's rate to fill
+    the time left. A slice's cost per token falls as the slice grows (the experts it hits
+    are converted to float64 once per slice), so one linear extrapolation undershoots.
+    Stops at 90% of the target, at the end of the batch or after `max_slices` slices.
+    Returns (seconds, tokens)."""
     order = np.random.default_rng(0).permutation(cfg.T).tolist()
-    n1 = min(first, cfg.T)
-    secs, n = oracle_sample(cfg, w, x, sorted(order[:n1]), logits_in)
-    more = min(cfg.T - n1, int(n * max(0.0, target_s - secs) / max(secs, 1e-9)))
-    if more > 0:
-        s2, n2 = oracle_sample(cfg, w, x, sorted(order[n1:n1 + more]), logits_in)
-        secs, n = secs + s2, n + n2
+    secs, n = 0.0, 0
+    size = min(first, cfg.T)
+    for _ in range(max_slices):
+        s1, n1 = oracle_sample(cfg, w, x, sorted(order[n:n + size]), logits_in)
+        secs, n = secs + s1, n + n1
+        left = target_s - secs
+        if n >= cfg.T or left <= 0.1 * target_s:
+            break
+        size = min(cfg.T - n, max(1, int(n1 * left / max(s1, 1e-9))))
     return secs, n
 
 

@@ -519,7 +519,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile t = decode_tile(s, g, tile);
       const int row = t.row0 + row_in_tile;
       const int cl = chunk_len(g, t);
-      constexpr bool logits = LOGITS;
       constexpr int NH = NL / 2;     // router: columns per thread (half of the tile)
       float sum[LOGITS ? NH : 1];    // router logits: running fp32 sum of this half-row
       if constexpr (LOGITS) {
