@@ -5,7 +5,11 @@ launched with the programmatic stream-serialisation attribute (the default) and 
 MOE_B200_PDL=0 (plain stream order); in the deterministic combine mode every output is a
 fixed function of the inputs, so the two runs must agree bit for bit. Each child runs
 several steps back to back, with a PID bias update between them, so every kernel of the
-chain has a predecessor still in flight when it is launched."""
+chain has a predecessor still in flight when it is launched. The step calls leave host
+gaps between the calls, so each child also runs moe_forward (the whole chain from one C
+call, no gaps) on several fresh batches in a row, fp32 and bf16: a kernel that read a
+predecessor's output through a non-coherent load before the data was final would differ
+there."""
 import os
 import subprocess
 import sys
@@ -40,6 +44,17 @@ for name, T in (("proxy_bf16", 4096), ("proxy_bf16", 200), ("decode_bf16", 128),
                  ("counts", b.counts), ("hist", b.nffn_hist), ("logits", b.logits),
                  ("bias", w.bias)):
         out[f"{name}_{T}_{k}"] = t.detach().cpu().clone()
+for name, T in (("tiny_fp32", 64), ("proxy_bf16", 512)):
+    cfg = wl.CONFIGS[name].with_(T=T)
+    w = wl.draw_weights(cfg, "cuda", seed=4)
+    xs = [wl.draw_tokens(cfg, "cuda", seed=30 + i) for i in range(6)]
+    layer = abi.MoELayer(abi.shape_of(cfg, "deterministic"), w.w_router, w.bias, w.w_gate_up,
+                         w.w_down)
+    torch.cuda.synchronize()
+    got = [layer.forward(x)[0].clone() for x in xs]
+    torch.cuda.synchronize()
+    for i, o in enumerate(got):
+        out[f"forward_{name}_{T}_{i}"] = o[:T].cpu()
 torch.save(out, sys.argv[2])
 """
 
