@@ -49,7 +49,7 @@ constexpr int kTok = 256;   // threads per token CTA
 // are loaded before they are used (more loads in flight per thread).
 template <int G>
 __global__ void __launch_bounds__(kTok) k_bwd_dy_dgate(
-    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ x,
+    const __nv_bfloat16* dout, const __nv_bfloat16* x,
     const __nv_bfloat16* y_perm, const int32_t* topk_idx,
     const float* topk_gate, const int32_t* row_of, int H, int K,
     int n_ffn, float scale, __nv_bfloat16* dy, float* d_gate) {
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(256) k_to_bf16(const float* a,
 
 // dx[t] += sum over FFN slots k (in order) of dx_perm[row_of[t, k]] + zgate_t * dout_t
 __global__ void __launch_bounds__(kTok) k_bwd_dx_combine(
-    const float* dx_perm, const __nv_bfloat16* __restrict__ dout,
+    const float* dx_perm, const __nv_bfloat16* dout,
     const int32_t* topk_idx, const float* topk_gate,
     const int32_t* row_of, int H, int K, int n_ffn, float* dx) {
   __shared__ int s_row[32];

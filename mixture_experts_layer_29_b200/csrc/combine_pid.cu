@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(256) k_finalize(const float* acc, T* out,
 // G rows are loaded before they are summed: G = 4 for small batches (more loads in
 // flight per thread), 1 for large ones (fewer registers, more CTAs per SM).
 template <typename T, int G>
-__global__ void __launch_bounds__(256) k_combine_det(const T* __restrict__ x, const T* y_perm,
+__global__ void __launch_bounds__(256) k_combine_det(const T* x, const T* y_perm,
                                                      const float* topk_gate,
                                                      const int32_t* row_of,
                                                      const float* zgate,

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256) k_perm_scan(const uint32_t* masks, int n_
 template <bool XBF16>
 __global__ void __launch_bounds__(256) k_perm_scatter(
     const int32_t* topk_idx, const float* topk_gate,
-    const float* zgate, const void* __restrict__ x, int T, int H, int n_ffn, int E,
+    const float* zgate, const void* x, int T, int H, int n_ffn, int E,
     int K, int nchunk, const uint32_t* masks, const int32_t* crel,
     const int32_t* ecount, int32_t* offsets,
     int32_t* perm_token, int32_t* row_of, float* row_gate,
@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(256) k_perm_scatter(
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + (size_t)t * H * esz);
   if (!x_perm && !out_acc) return;
   for (int v = lane; v < nvec; v += 32) {
-    const uint4 q = __ldg(src + v);
+    const uint4 q = src[v];
     if (x_perm) {
       for (int k = 0; k < K; ++k) {
         const int r = s_rows[warp][k];
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(512) k_perm_index_small(
 template <bool XBF16>
 __global__ void __launch_bounds__(128) k_perm_copy(const int32_t* row_of,
                                                    const float* zgate,
-                                                   const void* __restrict__ x, int H, int K,
+                                                   const void* x, int H, int K,
                                                    void* x_perm,
                                                    float* out_acc) {
   __shared__ int32_t s_rows[32];
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(128) k_perm_copy(const int32_t* row_of,
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + (size_t)t * H * esz);
   const float zg = out_acc ? zgate[t] : 0.f;
   for (int v = blockIdx.y * per + threadIdx.x; v < v_end; v += blockDim.x) {
-    const uint4 q = __ldg(src + v);
+    const uint4 q = src[v];
     if (x_perm)
       for (int k = 0; k < K; ++k) {
         const int r = s_rows[k];
@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(128) k_perm_copy(const int32_t* row_of,
 }  // namespace
 
 cudaError_t launch_permute(const int32_t* topk_idx, const float* topk_gate, const float* zgate,
-                           const void* __restrict__ x, int x_is_bf16, int T, int H, int n_ffn, int E, int K,
+                           const void* x, int x_is_bf16, int T, int H, int n_ffn, int E, int K,
                            uint32_t* masks, int32_t* crel, int32_t* ecount, int32_t* offsets,
                            int32_t* perm_token, int32_t* row_of, float* row_gate, void* x_perm,
                            float* out_acc, int* status, cudaStream_t st) {

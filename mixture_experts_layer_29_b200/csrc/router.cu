@@ -25,7 +25,7 @@ constexpr int RB = 128, RK = 16, RPAD = 4;
 constexpr int kSmMax = 160;   // sizing bound for the split-K partial buffer
 
 template <bool XBF16>
-__device__ __forceinline__ void load_x_slice(const void* __restrict__ x, int T, int H, int row0, int k0,
+__device__ __forceinline__ void load_x_slice(const void* x, int T, int H, int row0, int k0,
                                              float (&v)[8], int& r, int& kk) {
   const int tid = threadIdx.x;
   if (XBF16) {
@@ -70,7 +70,7 @@ __device__ __forceinline__ void load_w_slice(const float* __restrict__ w, int E,
 }
 
 template <bool XBF16>
-__global__ void __launch_bounds__(256, 2) k_router_logits(const void* __restrict__ x,
+__global__ void __launch_bounds__(256, 2) k_router_logits(const void* x,
                                                        const float* __restrict__ w, int T, int E,
                                                        int H, int kchunk, float* out,
                                                        size_t split_stride, ZeroSpec zero) {
@@ -195,7 +195,7 @@ size_t router_partial_bytes(int T, int E, int H, int sm_count_max) {
   return s > 1 ? (size_t)s * T * E * sizeof(float) : 0;
 }
 
-cudaError_t launch_router_logits(const void* __restrict__ x, int x_is_bf16, const float* w_router, int T,
+cudaError_t launch_router_logits(const void* x, int x_is_bf16, const float* w_router, int T,
                                  int E, int H, float* logits, float* partial, int splitk,
                                  ZeroSpec zero, cudaStream_t st) {
   int kchunk = (H + splitk - 1) / splitk;

@@ -7,9 +7,9 @@ fixed function of the inputs, so the two runs must agree bit for bit. Each child
 several steps back to back, with a PID bias update between them, so every kernel of the
 chain has a predecessor still in flight when it is launched. The step calls leave host
 gaps between the calls, so each child also runs moe_forward (the whole chain from one C
-call, no gaps) on several fresh batches in a row, fp32 and bf16: a kernel that read a
-predecessor's output through a non-coherent load before the data was final would differ
-there."""
+call, no gaps) on several fresh batches in a row, fp32 and bf16, and two layers stacked
+with the first layer's output as the second layer's x: a kernel that read a predecessor's
+output through a non-coherent load before the data was final would differ there."""
 import os
 import subprocess
 import sys
@@ -55,6 +55,19 @@ for name, T in (("tiny_fp32", 64), ("proxy_bf16", 512)):
     torch.cuda.synchronize()
     for i, o in enumerate(got):
         out[f"forward_{name}_{T}_{i}"] = o[:T].cpu()
+    # two layers stacked: layer 2 reads layer 1's output buffer as its x, so the first
+    # kernels of the second call depend on the last kernel of the first
+    w2 = wl.draw_weights(cfg, "cuda", seed=5)
+    layer2 = abi.MoELayer(abi.shape_of(cfg, "deterministic"), w2.w_router, w2.bias,
+                          w2.w_gate_up, w2.w_down)
+    torch.cuda.synchronize()
+    stacked = []
+    for x in xs:
+        o1 = layer.forward(x)[0]
+        stacked.append(layer2.forward(o1[:T])[0].clone())
+    torch.cuda.synchronize()
+    for i, o in enumerate(stacked):
+        out[f"stacked_{name}_{T}_{i}"] = o[:T].cpu()
 torch.save(out, sys.argv[2])
 """
 

@@ -4,15 +4,16 @@ Every kernel is launched as a programmatic dependent of the one before it and tr
 its dependents first. A kernel can therefore be resident while its predecessors still
 write its inputs. Loads through `const __restrict__` pointers or `__ldg` compile to the
 non-coherent form, which is only valid for memory that no one writes while the kernel
-lives. So those qualifiers may mark only weights and the caller's inputs, which no kernel
-of the chain writes."""
+lives. So those qualifiers may mark only weights. The caller's x may itself be the output
+of this library's previous call on the stream (two layers stacked back to back), so it is
+read with plain loads like every other activation."""
 import pathlib
 import re
 
 CSRC = pathlib.Path(__file__).resolve().parents[1] / "mixture_experts_layer_29_b200" / "csrc"
 
-# caller inputs and weights: never written by a kernel of the launch chain
-READ_ONLY_NAMES = {"x", "w", "wgu", "wd", "dout"}
+# weights: no kernel of this library writes them
+READ_ONLY_NAMES = {"w", "wgu", "wd"}
 # k_split_router_weight writes a bf16 copy of the router weight through `out`
 WRITE_ONLY = {("gemm_tc.cu", "out")}
 
@@ -34,11 +35,6 @@ def test_restrict_marks_only_inputs_and_weights():
     assert not bad, bad
 
 
-def test_ldg_reads_only_the_token_rows():
-    """The two __ldg users read rows of the caller's x (`src` points into x)."""
+def test_no_ldg():
     for name, text in _sources():
-        for m in re.finditer(r"__ldg\(\s*(\w+)", text):
-            assert m.group(1) == "src", (name, m.group(0))
-            before = text[: m.start()]
-            decl = before[before.rfind("const uint4* src"):]
-            assert "static_cast<const char*>(x)" in decl.split(";")[0], name
+        assert "__ldg(" not in text, name
