@@ -1,4 +1,12 @@
 // kernels.cuh - host-side launchers of the layer's kernels (internal to the library).
+//
+// Every kernel behind these launchers keeps the launch contract of launch.cuh, and one
+// more rule: only weights are read through `const __restrict__` pointers, and nothing
+// through __ldg. Both compile to non-coherent loads. Those assume the memory stays
+// unchanged for the kernel's whole life, and the compiler may schedule them ahead of
+// pdl_wait(). A kernel launched as a programmatic dependent is resident while its
+// predecessors still write its inputs, and the caller's x may be this library's own
+// output from the previous call. So activations are read with plain loads after the wait.
 #pragma once
 
 #include <cuda.h>
