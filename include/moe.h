@@ -18,7 +18,11 @@
  *    moe_read_device_status, which synchronises the given stream, and the host pipeline
  *    (its own streams and events).
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
- *    legacy default stream).
+ *    legacy default stream). Stream order is the only requirement on inputs: any input
+ *    may be written by earlier work on the same stream, including this library's own
+ *    previous call (one layer's `out` passed as the next layer's `x`). The kernels start
+ *    early as programmatic dependents of their predecessors, but they read nothing a
+ *    predecessor may write until it has completed.
  *  - Layouts are row-major and contiguous. Device pointers must be 16-byte aligned.
  *  - x, x_perm, h, y_perm and out hold `dtype` elements (bf16 or fp32); logits, gates,
  *    biases and out_acc are fp32; indices and counts are int32.
