@@ -107,6 +107,51 @@ const char* moe_status_string(int code);
  * threads). A benchmark reads it before and after a timed region. */
 uint64_t moe_launch_count(void);
 
+/* ---- tuning switches (measurements and tests) -------------------------------------------
+ * The pages have no counterpart: these switches select between kernel variants that give
+ * the same results, so that a measurement can compare them, plus one testing hook. Every
+ * switch starts at its default. The library reads no environment variable. A switch is
+ * process-wide: it applies to every device, and to every call made after it is set.
+ * Changing one while another host thread is queuing calls gives that thread either
+ * setting.
+ *   MOE_TUNE_PDL              1 (default): kernels launch as programmatic dependents of
+ *                             their predecessors on the stream; 0: plain stream order.
+ *   MOE_TUNE_GEMM_PAIR        -1 (default): the bf16 expert GEMMs use CTA pairs
+ *                             (tcgen05 cta_group::2, 256-row tiles) for T >= 1024, one CTA
+ *                             per tile otherwise; 0: always one CTA; 1: always pairs.
+ *   MOE_TUNE_PAIR_HALF        1 (default): in the CTA-pair GEMMs, an expert's last tile of
+ *                             at most 128 rows runs as an M = 128 tile; 0: as M = 256.
+ *   MOE_TUNE_ROUTER_N         0 (default): the bf16 router GEMM's tile width (128, 192 or
+ *                             256 logits) follows from the shape; 192 or 256: that width
+ *                             wherever 256-wide tiles fill a wave of SMs.
+ *   MOE_TUNE_ROUTER_MIN_SPLIT 12 (default): fewest k-blocks of 64 in one split-K slice of
+ *                             the bf16 router GEMM; 1 to 1024.
+ *   MOE_TUNE_BWD_PAIR         1 (default): moe_backward's dgrad GEMMs run on CTA pairs
+ *                             wherever the forward does; 0: one CTA per tile.
+ *   MOE_TUNE_BWD_DY_ROWS      4 (default): y rows each thread of the backward's dy kernel
+ *                             loads before using them; 1: one at a time.
+ *   MOE_TUNE_TEST_STALL       testing hook, 0 (default). Set to 1, the next gate/up GEMM
+ *                             of moe_grouped_ffn (or moe_forward) leaves the first
+ *                             k-block of its first tile unloaded. The waits on that stage
+ *                             run out after their limit (2 s) and write MOE_ERR_TIMEOUT to
+ *                             the status word; that call's outputs are undefined. The
+ *                             switch returns to 0 when that launch is queued.
+ * moe_set_tuning returns MOE_ERR_INVALID_ARG for an unknown switch or a value outside its
+ * range. moe_get_tuning writes the current value. */
+typedef enum {
+  MOE_TUNE_PDL = 0,
+  MOE_TUNE_GEMM_PAIR = 1,
+  MOE_TUNE_PAIR_HALF = 2,
+  MOE_TUNE_ROUTER_N = 3,
+  MOE_TUNE_ROUTER_MIN_SPLIT = 4,
+  MOE_TUNE_BWD_PAIR = 5,
+  MOE_TUNE_BWD_DY_ROWS = 6,
+  MOE_TUNE_TEST_STALL = 7
+} moe_tune_t;
+
+int moe_set_tuning(int knob, int64_t value);
+int moe_get_tuning(int knob, int64_t* value);
+
 /* ---- the steps of the layer ------------------------------------------------------------ */
 
 /* Router: logits, softmax over all E experts, bias-adjusted top-K, gates and histograms
@@ -365,14 +410,17 @@ int moe_host_pipeline_destroy(moe_host_pipeline* pipe);
  * in and out, and latency-bound paths that cannot afford a cudaMalloc, which may
  * synchronise the whole device.
  *
- * Arguments and results are exactly those of moe_permute without ws and ws_bytes. The
- * scratch is a fixed 4 MiB array in the library's own device memory; each GPU that loads
- * the library keeps it until the process exits. A call needs
+ * Arguments and results are exactly those of moe_permute without ws and ws_bytes;
+ * x_perm may be NULL as there (the indices and gates only, for the gathered-rows FFN).
+ * The scratch is a fixed 4 MiB array in the library's own device memory; each GPU that
+ * loads the library keeps it until the process exits. A call needs
  * 1024 + 2 * round_up_1024(n_ffn * ceil(T / 32) * 4) + 4 * n_ffn bytes of it and returns
  * MOE_ERR_WORKSPACE, launching nothing, when the shape needs more (with n_ffn = 512:
  * T <= 32736). The call never calls cudaMalloc, cudaFree or any allocating routine.
- * The first call on a device looks up the array's device address and caches it: make
- * that first call before any stream capture on that device.
+ * The first call in a device's context looks up the array's device address there and
+ * caches it with that context's unique id: make that first call before any stream
+ * capture on that device. A new context on the device (after cudaDeviceReset, say)
+ * gets its own lookup on its first call.
  * Every call uses the same array, which keeps what the last call left there. Calls whose
  * GPU work can overlap (unordered streams, several host threads) race on it and give
  * wrong results: order them on one stream. Each call clears the array's status word;

@@ -71,6 +71,8 @@ _SIGS = {
     "moe_read_device_status": (ctypes.c_int, [_P, _SZ, _P, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_launch_count": (ctypes.c_uint64, []),
+    "moe_set_tuning": (ctypes.c_int, [ctypes.c_int, ctypes.c_int64]),
+    "moe_get_tuning": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]),
     "moe_route": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 11 + [_SZ, _P]),
     "moe_permute": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 11 + [_SZ, _P]),
     "moe_grouped_ffn": (ctypes.c_int, [ctypes.POINTER(Shape)] + [_P] * 12 + [_SZ, _P]),
@@ -165,6 +167,22 @@ def workspace_size(shape: Shape) -> int:
 
 def launch_count() -> int:
     return int(lib().moe_launch_count())
+
+
+# moe_set_tuning switches (include/moe.h): kernel variants with the same results, for
+# measurements and tests, and one testing hook
+TUNE_PDL, TUNE_GEMM_PAIR, TUNE_PAIR_HALF, TUNE_ROUTER_N = 0, 1, 2, 3
+TUNE_ROUTER_MIN_SPLIT, TUNE_BWD_PAIR, TUNE_BWD_DY_ROWS, TUNE_TEST_STALL = 4, 5, 6, 7
+
+
+def set_tuning(knob: int, value: int):
+    _check(lib().moe_set_tuning(int(knob), int(value)), "moe_set_tuning")
+
+
+def get_tuning(knob: int) -> int:
+    v = ctypes.c_int64(0)
+    _check(lib().moe_get_tuning(int(knob), ctypes.byref(v)), "moe_get_tuning")
+    return int(v.value)
 
 
 def read_device_status(ws, stream=None) -> int:

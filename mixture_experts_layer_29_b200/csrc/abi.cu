@@ -5,7 +5,6 @@
 #include <atomic>
 #include <initializer_list>
 #include <mutex>
-#include <stdlib.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -17,13 +16,31 @@ namespace moe {
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
-bool pdl_enabled() {
-  static const bool on = [] {
-    const char* v = getenv("MOE_B200_PDL");
-    return !(v && v[0] == '0');
-  }();
-  return on;
+// Process-wide tuning switches (moe_set_tuning), each at its default until changed.
+namespace {
+constexpr int kTuneCount = MOE_TUNE_TEST_STALL + 1;
+std::atomic<int64_t> g_tune[kTuneCount] = {{1}, {-1}, {1}, {0}, {12}, {1}, {4}, {0}};
+
+bool tune_value_ok(int knob, int64_t v) {
+  switch (knob) {
+    case MOE_TUNE_PDL:
+    case MOE_TUNE_PAIR_HALF:
+    case MOE_TUNE_BWD_PAIR:
+    case MOE_TUNE_TEST_STALL: return v == 0 || v == 1;
+    case MOE_TUNE_GEMM_PAIR: return v >= -1 && v <= 1;
+    case MOE_TUNE_ROUTER_N: return v == 0 || v == 192 || v == 256;
+    case MOE_TUNE_ROUTER_MIN_SPLIT: return v >= 1 && v <= 1024;
+    case MOE_TUNE_BWD_DY_ROWS: return v == 1 || v == 4;
+    default: return false;
+  }
 }
+}  // namespace
+
+int64_t tuning(int knob) { return g_tune[knob].load(std::memory_order_relaxed); }
+
+bool take_test_stall() { return g_tune[MOE_TUNE_TEST_STALL].exchange(0) != 0; }
+
+bool pdl_enabled() { return tuning(MOE_TUNE_PDL) != 0; }
 
 int current_device_info(DeviceInfo* info) {
   static std::mutex mu;
@@ -399,6 +416,18 @@ const char* moe_status_string(int code) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_set_tuning(int knob, int64_t value) {
+  if (knob < 0 || knob >= kTuneCount || !tune_value_ok(knob, value)) return MOE_ERR_INVALID_ARG;
+  g_tune[knob].store(value, std::memory_order_relaxed);
+  return MOE_OK;
+}
+
+int moe_get_tuning(int knob, int64_t* value) {
+  if (knob < 0 || knob >= kTuneCount || !value) return MOE_ERR_INVALID_ARG;
+  *value = tuning(knob);
+  return MOE_OK;
+}
 
 int moe_route(const moe_shape_t* shape, const void* x, const float* w_router,
               const float* logits_in, const float* bias, float* logits_out, int32_t* topk_idx,

@@ -17,7 +17,6 @@
 //   k_to_bf16        W_r in bf16 for the latter
 //   k_bwd_dx_combine dx[t] += sum over FFN slots (in order) of dx_perm[row] + zgate_t dout_t
 #include <math.h>
-#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -260,12 +259,8 @@ cudaError_t launch_bwd_dy_dgate(const void* dout, const void* x, const void* y_p
                                 const int32_t* topk_idx, const float* topk_gate,
                                 const int32_t* row_of, int T, int H, int K, int n_ffn,
                                 float scale, void* dy, float* d_gate, cudaStream_t st) {
-  static const int g_env = [] {
-    const char* v = getenv("MOE_B200_DY_G");
-    return v ? atoi(v) : 4;
-  }();
   const cudaError_t e = launch_kernel(
-      g_env == 1 ? k_bwd_dy_dgate<1> : k_bwd_dy_dgate<4>, T, kTok, 0, st, 1,
+      tuning(MOE_TUNE_BWD_DY_ROWS) == 1 ? k_bwd_dy_dgate<1> : k_bwd_dy_dgate<4>, T, kTok, 0, st, 1,
       static_cast<const __nv_bfloat16*>(dout),
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm), topk_idx,
       topk_gate, row_of, H, K, n_ffn, scale, static_cast<__nv_bfloat16*>(dy), d_gate);

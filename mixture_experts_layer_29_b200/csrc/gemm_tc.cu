@@ -28,7 +28,6 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
-#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -100,7 +99,14 @@ struct GemmArgs {
   int half_tiles;             // pair kernel: an expert's last tile of <= 128 rows runs as M = 128
   void* gu_out;               // gate/up: also store G and U (bf16, [rows, 2I]) beside h, or null
   const __nv_bfloat16* gu_in; // kDgradDH: G | U of the rows ([rows, 2I], I = n_valid)
+  int test_stall;             // testing (MOE_TUNE_TEST_STALL): tile 0 leaves its first
+                              // k-block unloaded, so the waits on that stage run out
 };
+
+// The testing hook of GemmArgs::test_stall: this (tile, k-block) is not loaded.
+__device__ __forceinline__ bool stalled_stage(const GemmArgs& g, int tile, int kb, int kb0) {
+  return g.test_stall != 0 && tile == 0 && kb == kb0;
+}
 
 struct Tile {
   int e, row0, row_end, nt, kb0, kb1, split;
@@ -422,10 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int brow0 = t.e * g.b_rows + t.nt * (g.mode == kGateUp ? BM : BN);
       const int brow1 = brow0 + g.b_second;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        const bool stall = stalled_stage(g, tile, kb, t.kb0);
         int w_ok = 1;
         if (lane == 0) {
           w_ok = mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag) ? 1 : 0;
-          if (w_ok) mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
+          if (w_ok && !stall) mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
         }
         w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
         if (!w_ok) {
@@ -433,11 +440,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const int ka = g.a_kwrap > 0 ? kb % g.a_kwrap : kb;
-        tma_gather4(s.a[stage] + lane * 4 * (BK * 2), &tmA, ka * BK, r[0], r[1], r[2], r[3],
-                    &s.full[stage]);
-        if (lane == 0) {
-          tma_load_2d(s.b[stage], &tmB, kb * BK, brow0, &s.full[stage]);
-          tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
+        if (!stall) {
+          tma_gather4(s.a[stage] + lane * 4 * (BK * 2), &tmA, ka * BK, r[0], r[1], r[2], r[3],
+                      &s.full[stage]);
+          if (lane == 0) {
+            tma_load_2d(s.b[stage], &tmB, kb * BK, brow0, &s.full[stage]);
+            tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
+          }
         }
         if (++stage == STAGES) {
           stage = 0;
@@ -456,12 +465,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int brow1 = brow0 + g.b_second;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
-          mbar_arrive_expect_tx(&s.full[stage], LOGITS ? A_BYTES + NL * BK * 2 : STAGE_BYTES);
-          const int ka = g.a_kwrap > 0 ? kb % g.a_kwrap : kb;
-          tma_load_2d(s.a[stage], &tmA, ka * BK, t.row0, &s.full[stage]);
-          tma_load_2d(s.b[stage], &tmB, kb * BK, brow0, &s.full[stage]);
-          if (!LOGITS || NL == 256)
-            tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
+          if (!stalled_stage(g, tile, kb, t.kb0)) {
+            mbar_arrive_expect_tx(&s.full[stage], LOGITS ? A_BYTES + NL * BK * 2 : STAGE_BYTES);
+            const int ka = g.a_kwrap > 0 ? kb % g.a_kwrap : kb;
+            tma_load_2d(s.a[stage], &tmA, ka * BK, t.row0, &s.full[stage]);
+            tma_load_2d(s.b[stage], &tmB, kb * BK, brow0, &s.full[stage]);
+            if (!LOGITS || NL == 256)
+              tma_load_2d(s.b[stage] + B_BYTES / 2, &tmB, kb * BK, brow1, &s.full[stage]);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -796,6 +807,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bcol = t.nt * BN + 128 * (int)rank;
         for (int kb = 0; kb < g.kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
+          if (stalled_stage(g, tile, kb, 0)) {   // neither CTA loads; nothing is expected
+            if (++stage == PSTAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * P_STAGE_BYTES);
           tma_load_2d_pair(s.a[stage], &tmA, kb * BK, arow, full_leader);
@@ -996,20 +1014,14 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap&
 }
 
 // The CTA-pair kernel pays off once groups are tall (256-row tiles); small batches keep
-// the one-CTA kernel. MOE_B200_GEMM_PAIR=0 / 1 forces either (for measurements).
-// MOE_B200_PAIR_HALF=0 runs every pair tile as M = 256 (for measurements).
-int pair_half_tiles() {
-  static const int v = [] {
-    const char* e = getenv("MOE_B200_PAIR_HALF");
-    return (e && e[0] == '0') ? 0 : 1;
-  }();
-  return v;
-}
+// the one-CTA kernel. MOE_TUNE_GEMM_PAIR forces either, MOE_TUNE_PAIR_HALF = 0 runs every
+// pair tile as M = 256 (for measurements).
+int pair_half_tiles() { return tuning(MOE_TUNE_PAIR_HALF) != 0 ? 1 : 0; }
 
 bool use_pair_kernel(int T) {
-  static const char* env = getenv("MOE_B200_GEMM_PAIR");
-  if (env && env[0] == '0') return false;
-  if (env && env[0] == '1') return true;
+  const int64_t v = tuning(MOE_TUNE_GEMM_PAIR);
+  if (v == 0) return false;
+  if (v == 1) return true;
   return T >= 1024;
 }
 
@@ -1051,29 +1063,15 @@ __global__ void __launch_bounds__(256) k_split_router_weight(const float4* __res
 // Router logits: 128 x 128 tiles, K = 3H (the three weight parts); the tensor cores
 // accumulate kRouterChunk k-blocks at a time and the epilogue sums the chunks in fp32.
 constexpr int kRouterChunk = 6;
-// k-blocks per split at least (MOE_B200_ROUTER_MINSPLIT overrides it, for measurements)
-int router_min_split() {
-  static const int v = [] {
-    const char* e = getenv("MOE_B200_ROUTER_MINSPLIT");
-    const int n = e ? atoi(e) : 0;
-    return n >= 1 && n <= 1024 ? n : 12;
-  }();
-  return v;
-}
+// k-blocks per split at least (MOE_TUNE_ROUTER_MIN_SPLIT, 12 by default)
+int router_min_split() { return (int)tuning(MOE_TUNE_ROUTER_MIN_SPLIT); }
 
 // The router GEMM's N tile: 256 logits when the 256-wide tiles fill a wave of SMs (the
 // A tile is then read once per 256 logits), else 128 (twice the tiles for a small batch:
 // decode's 128 tokens x 768 logits fill 144 CTAs with the K split instead of 72).
-// MOE_B200_ROUTER_N=192 / 256 forces that width where 256-logit tiles fill a wave (for
+// MOE_TUNE_ROUTER_N = 192 / 256 forces that width where 256-logit tiles fill a wave (for
 // measurements).
-int router_n_override() {
-  static const int v = [] {
-    const char* e = getenv("MOE_B200_ROUTER_N");
-    const int n = e ? atoi(e) : 0;
-    return (n == 192 || n == 256) ? n : 0;
-  }();
-  return v;
-}
+int router_n_override() { return (int)tuning(MOE_TUNE_ROUTER_N); }
 
 int router_tile_n(int T, int E, int sm_count) {
   const long mt = (T + BM - 1) / BM;
@@ -1224,6 +1222,7 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g1.ksplit = 1;
   g1.kb_per_split = g1.kblocks;
   g1.half_tiles = pair ? pair_half_tiles() : 0;
+  g1.test_stall = take_test_stall() ? 1 : 0;
   if ((rc = pair ? launch_pair(mx, mwgu, mwgu64, g1, sm_count, st)
                  : launch_one(mx, mwgu, g1, sm_count, st)) != MOE_OK)
     return rc;
@@ -1282,11 +1281,10 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
               : launch_one(mx, mwgu, g, sm_count, st);
 }
 
-// MOE_B200_BWD_PAIR=0 keeps the dgrad GEMMs on the one-CTA backward kernel (for
+// MOE_TUNE_BWD_PAIR = 0 keeps the dgrad GEMMs on the one-CTA backward kernel (for
 // measurements).
 bool dgrad_use_pair(int T) {
-  static const char* env = getenv("MOE_B200_BWD_PAIR");
-  if (env && env[0] == '0') return false;
+  if (tuning(MOE_TUNE_BWD_PAIR) == 0) return false;
   return use_pair_kernel(T);
 }
 

@@ -21,6 +21,11 @@ namespace moe {
 // One launch of one of this library's kernels (counted for moe_launch_count).
 void count_launch(int n = 1);
 
+// Current value of a moe_set_tuning switch (MOE_TUNE_*).
+int64_t tuning(int knob);
+// Reads and clears MOE_TUNE_TEST_STALL: true once per arming.
+bool take_test_stall();
+
 struct DeviceInfo {
   int device = -1;
   int sm_count = 0;

@@ -11,7 +11,7 @@
 //     every CTA executes it before exiting (so a kernel never completes ahead of the one
 //     it depends on, and completion stays transitive down the stream).
 // pdl_wait() returns once all prerequisite grids have completed and their memory is
-// visible; without the attribute (or with MOE_B200_PDL=0) it returns at once.
+// visible; without the attribute (MOE_TUNE_PDL set to 0) it returns at once.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -25,7 +25,7 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// False when the environment sets MOE_B200_PDL=0 (read once per process).
+// False when moe_set_tuning(MOE_TUNE_PDL, 0) is in effect.
 bool pdl_enabled();
 
 // kern<<<grid, block, smem, st>>>(args...) with the PDL attribute (and, for cluster > 1,

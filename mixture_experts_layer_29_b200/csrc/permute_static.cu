@@ -5,8 +5,13 @@
 // sums and the expert counts) lives in one file-scope __device__ array of a fixed size,
 // so the call allocates nothing. Host code may not use the array's name as an address
 // (on the host it names a stand-in object, not device memory): the device address is
-// looked up once per device with cudaGetSymbolAddress, with that device current, and
-// cached. Every call shares the array and it keeps the last call's contents.
+// looked up with cudaGetSymbolAddress, with the device current, and cached per device
+// together with the unique id of the context it was looked up in. A context created
+// later on the same device (after cudaDeviceReset, say) has another id, so the address
+// is looked up again there. Every call shares the array and it keeps the last call's
+// contents.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -22,6 +27,37 @@ __device__ __align__(256) unsigned char g_permute_scratch[kStaticScratchBytes];
 
 std::mutex g_addr_mu;
 void* g_addr[kMaxDevices] = {};
+unsigned long long g_addr_ctx[kMaxDevices] = {};
+
+// The driver's current-context queries, reached through the runtime (no link to libcuda).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+// Unique id of the calling thread's current context (0 if there is none or the driver
+// cannot say).
+unsigned long long current_context_id() {
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_ctx_id = reinterpret_cast<CtxGetIdFn>(fn);
+    cudaGetLastError();
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!g_ctx_current || !g_ctx_id || g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      g_ctx_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 inline size_t up1k(size_t v) { return (v + 1023) / 1024 * 1024; }
 
@@ -39,17 +75,21 @@ StaticLayout static_layout(int T, int n_ffn) {
   return L;
 }
 
-// Device address of the array on the current device (looked up on the first call there).
+// Device address of the array on the current device, looked up the first time a context
+// of that device calls here.
 int scratch_address(int dev, void** out) {
   std::lock_guard<std::mutex> lock(g_addr_mu);
-  if (!g_addr[dev]) {
+  unsigned long long ctx = current_context_id();
+  if (!g_addr[dev] || ctx == 0 || g_addr_ctx[dev] != ctx) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
     if (e != cudaSuccess || !p) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
+    ctx = current_context_id();   // the lookup makes the device's context current
     g_addr[dev] = p;
+    g_addr_ctx[dev] = ctx;
   }
   *out = g_addr[dev];
   return MOE_OK;
@@ -70,11 +110,12 @@ extern "C" int moe_permute_static_scratch(const moe_shape_t* shape, const int32_
   size_t unused = 0;
   const int rc = moe_scratch_size(shape, &unused);   // the same shape checks as moe_permute
   if (rc != MOE_OK) return rc;
-  const void* need[] = {topk_idx, topk_gate, x, offsets, perm_token, row_of, row_gate, x_perm};
+  const void* need[] = {topk_idx, topk_gate, x, offsets, perm_token, row_of, row_gate};
   for (const void* p : need) {
     if (!p) return MOE_ERR_INVALID_ARG;
     if (!ok_ptr(p)) return MOE_ERR_ALIGNMENT;
   }
+  if (x_perm && !ok_ptr(x_perm)) return MOE_ERR_ALIGNMENT;   // NULL: indices only, no copy
   if (out_acc) {                          // the zero-expert term needs zgate
     if (!zgate) return MOE_ERR_INVALID_ARG;
     if (!ok_ptr(out_acc) || !ok_ptr(zgate)) return MOE_ERR_ALIGNMENT;

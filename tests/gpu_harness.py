@@ -151,22 +151,25 @@ def check_permutation(case: Case, b: abi.StepBuffers, zero_init: bool, copied: b
     return pm
 
 
+class LazyExperts:
+    """A device weight tensor [n_ffn, ...] that hands the oracle one expert at a time on
+    the host, so that only the experts it touches are copied."""
+
+    def __init__(self, w):
+        self.w = w
+
+    def __getitem__(self, e):
+        return host(self.w[e])
+
+
 def oracle_layer(case: Case, L: np.ndarray, tokens):
     """Oracle output for the given tokens (float64) from the GPU's logits; weights of the
     experts those tokens hit are brought to the host one expert at a time."""
     cfg = case.cfg
     r = orc.route(L, host(case.w.bias), cfg.n_ffn, cfg.K)
     experts = sorted({int(e) for t in tokens for e in r.topk_idx[t] if e < cfg.n_ffn})
-
-    class _Lazy:
-        def __init__(self, w):
-            self.w = w
-
-        def __getitem__(self, e):
-            return host(self.w[e])
-
     x = host(case.x)
     out, ffn, zg, y_rows, rr = orc.moe_layer_forward(
-        x, L, host(case.w.bias), _Lazy(case.w.w_gate_up), _Lazy(case.w.w_down), cfg.n_ffn, cfg.K,
-        cfg.ffn_out_scale, tokens=tokens)
+        x, L, host(case.w.bias), LazyExperts(case.w.w_gate_up), LazyExperts(case.w.w_down),
+        cfg.n_ffn, cfg.K, cfg.ffn_out_scale, tokens=tokens)
     return out, ffn, zg, y_rows, rr, experts

@@ -2,7 +2,7 @@
 
 The same seeded layer steps run in two child processes, one with the library's kernels
 launched with the programmatic stream-serialisation attribute (the default) and one with
-MOE_B200_PDL=0 (plain stream order); in the deterministic combine mode every output is a
+moe_set_tuning(MOE_TUNE_PDL, 0) (plain stream order); in the deterministic combine mode every output is a
 fixed function of the inputs, so the two runs must agree bit for bit. Each child runs
 several steps back to back, with a PID bias update between them, so every kernel of the
 chain has a predecessor still in flight when it is launched. The step calls leave host
@@ -25,6 +25,8 @@ CHILD = r"""
 import sys, torch
 sys.path.insert(0, sys.argv[1])
 from mixture_experts_layer_29_b200 import abi, workloads as wl
+abi.set_tuning(abi.TUNE_PDL, int(sys.argv[3]))
+assert abi.get_tuning(abi.TUNE_PDL) == int(sys.argv[3])
 out = {}
 for name, T in (("proxy_bf16", 4096), ("proxy_bf16", 200), ("decode_bf16", 128), ("tiny_fp32", 64)):
     cfg = wl.CONFIGS[name].with_(T=T)
@@ -74,8 +76,7 @@ torch.save(out, sys.argv[2])
 
 def _run(tmp_path, pdl: str):
     path = os.path.join(tmp_path, f"pdl{pdl}.pt")
-    env = dict(os.environ, MOE_B200_PDL=pdl)
-    r = subprocess.run([sys.executable, "-c", CHILD, ROOT, path], env=env, capture_output=True,
+    r = subprocess.run([sys.executable, "-c", CHILD, ROOT, path, pdl], capture_output=True,
                        text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
     return torch.load(path)

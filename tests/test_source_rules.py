@@ -38,3 +38,10 @@ def test_restrict_marks_only_inputs_and_weights():
 def test_no_ldg():
     for name, text in _sources():
         assert "__ldg(" not in text, name
+
+
+def test_no_environment_reads():
+    """Kernel choices come from the call's arguments and moe_set_tuning, never from the
+    process environment."""
+    for name, text in _sources():
+        assert "getenv" not in text, name
