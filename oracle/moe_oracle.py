@@ -373,7 +373,8 @@ class BackwardResult:
 
 
 def moe_layer_backward(x, w_router, bias32, w_gate_up, w_down, n_ffn: int, K: int, dout,
-                       ffn_out_scale: float = 1.0, topk_idx=None) -> BackwardResult:
+                       ffn_out_scale: float = 1.0, topk_idx=None, tokens=None,
+                       experts=None) -> BackwardResult:
     """Gradients of the layer output with respect to x, W_r, W_gu and W_d, given the
     gradient dout of the output, in float64.
 
@@ -391,6 +392,13 @@ def moe_layer_backward(x, w_router, bias32, w_gate_up, w_down, n_ffn: int, K: in
     per zero pick: d_gate[t, k] = <dout_t, x_t>, dx_t += g_k dout_t; then
       dp[t, e] = sum of d_gate over the picks of e,   dL = p * (dp - <p, dp>)
       d_router = dL^T x,   dx += dL W_r.
+
+    tokens / experts (full-size checks, where every gradient at once does not fit in host
+    memory): the same quantities for a part only. With tokens given, dx, d_gate and
+    d_logits hold those tokens' rows (every other row is zero) and d_router is None: a
+    token's dx, gate and logit gradients need only its own picks' rows. With experts given,
+    d_gate_up and d_down are dicts holding those experts' gradients only: an expert's
+    weight gradients need all of its rows, whatever `tokens` says.
     """
     x64 = np.asarray(x, dtype=np.float64)
     wr = np.asarray(w_router, dtype=np.float64)
@@ -405,14 +413,26 @@ def moe_layer_backward(x, w_router, bias32, w_gate_up, w_down, n_ffn: int, K: in
     ex = np.exp(L - m)
     p = ex / ex.sum(axis=1, keepdims=True)
     s = float(ffn_out_scale)
+    want = np.ones(T, dtype=bool)
+    if tokens is not None:
+        want = np.zeros(T, dtype=bool)
+        want[np.asarray(tokens, dtype=np.int64)] = True
     dx = np.zeros((T, H))
     d_gate = np.zeros((T, K))
     N = n_ffn
     I = np.asarray(w_gate_up[0]).shape[0] // 2
-    d_gu = np.zeros((N, 2 * I, H))
-    d_d = np.zeros((N, H, I))
-    for e in sorted({int(v) for v in idx.ravel() if v < n_ffn}):
+    if experts is None:
+        full = set(range(N))
+        d_gu = np.zeros((N, 2 * I, H))
+        d_d = np.zeros((N, H, I))
+    else:
+        full = {int(e) for e in experts}
+        d_gu, d_d = {}, {}
+    hit = {int(v) for v in idx[want].ravel() if v < n_ffn}
+    for e in sorted(hit | {e for e in full if (idx == e).any()}):
         tk = np.argwhere(idx == e)                       # (t, k) of every pick of e
+        if e not in full:
+            tk = tk[want[tk[:, 0]]]                      # only the wanted tokens' rows
         ts, ks = tk[:, 0], tk[:, 1]
         wgu = np.asarray(w_gate_up[e], dtype=np.float64)
         wd = np.asarray(w_down[e], dtype=np.float64)
@@ -426,21 +446,26 @@ def moe_layer_backward(x, w_router, bias32, w_gate_up, w_down, n_ffn: int, K: in
         g = p[ts, e]
         dy = s * g[:, None] * dout[ts]
         d_gate[ts, ks] = s * (dout[ts] * y).sum(axis=1)
-        d_d[e] = dy.T @ h
         dh = dy @ wd
         dG = dh * U * sig * (1.0 + G * (1.0 - sig))
         dU = dh * G * sig
-        d_gu[e, :I] = dG.T @ X
-        d_gu[e, I:] = dU.T @ X
+        if e in full:
+            d_d[e] = dy.T @ h
+            gu_e = np.empty((2 * I, H))
+            gu_e[:I] = dG.T @ X
+            gu_e[I:] = dU.T @ X
+            d_gu[e] = gu_e
         dx[ts] += dG @ wgu[:I] + dU @ wgu[I:]            # a token picks e at most once
-    zt, zk = np.nonzero(idx >= n_ffn)
+    zt, zk = np.nonzero((idx >= n_ffn) & want[:, None])
     d_gate[zt, zk] = (dout[zt] * x64[zt]).sum(axis=1)
     for t, k in zip(zt, zk):
         dx[t] += p[t, idx[t, k]] * dout[t]
+    d_gate[~want] = 0.0
     dp = np.zeros((T, E))
     np.add.at(dp, (np.repeat(np.arange(T), K), idx.ravel()), d_gate.ravel())
     dL = p * (dp - (p * dp).sum(axis=1, keepdims=True))
-    d_router = dL.T @ x64
+    dL[~want] = 0.0
+    d_router = dL.T @ x64 if tokens is None else None
     dx += dL @ wr
+    dx[~want] = 0.0
     return BackwardResult(dx, d_router, d_gu, d_d, dL, d_gate, idx)
-

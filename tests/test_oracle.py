@@ -477,6 +477,34 @@ def test_backward_matches_torch_autograd():
     np.testing.assert_allclose(b.d_logits, logits.grad.numpy(), rtol=1e-10, atol=1e-12)
 
 
+def test_backward_restricted_to_tokens_and_experts_equals_the_full_one():
+    """The backward restricted to some tokens (dx, gate and logit gradients) and some
+    experts (weight gradients), as the full-size GPU check uses it, gives the same values
+    as the full (pinned above) backward on those rows and experts, zero rows elsewhere
+    and no router gradient."""
+    x, wr, bias, wgu, wd, dout, N, K = _bwd_case(seed=5, T=12, N=4, Z=2, K=3)
+    s = 0.9
+    full = orc.moe_layer_backward(x, wr, bias, wgu, wd, N, K, dout, s)
+    toks = [1, 4, 5, 11]
+    hit = sorted({int(e) for e in full.topk_idx.ravel() if e < N})
+    experts = hit[:2] + [e for e in range(N) if e not in hit][:1]
+    part = orc.moe_layer_backward(x, wr, bias, wgu, wd, N, K, dout, s,
+                                  topk_idx=full.topk_idx, tokens=toks, experts=experts)
+    rest = np.setdiff1d(np.arange(x.shape[0]), toks)
+    for a, b in ((part.dx, full.dx), (part.d_gate, full.d_gate), (part.d_logits, full.d_logits)):
+        np.testing.assert_allclose(a[toks], b[toks], rtol=1e-12, atol=1e-14)
+        assert (a[rest] == 0).all()
+    assert part.d_router is None
+    for e in experts:
+        if e in hit:
+            np.testing.assert_allclose(part.d_gate_up[e], full.d_gate_up[e], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(part.d_down[e], full.d_down[e], rtol=1e-12, atol=1e-14)
+        else:
+            assert e not in part.d_gate_up and e not in part.d_down
+            assert (full.d_gate_up[e] == 0).all()
+    assert set(part.d_gate_up) == set(experts) & set(hit)
+
+
 # ----------------------------------------------------------------------------- pages' numbers
 
 def test_activated_parameter_identity_from_the_pages():
