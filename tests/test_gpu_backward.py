@@ -126,3 +126,56 @@ def test_backward_from_saved_gate_up(cuda_device, T):
     assert abi.read_device_status(ws) == 0
     for a, c in ((dx, dx2), (d_router, dr2), (d_gu, gu2), (d_d, dd2)):
         assert torch.equal(a, c)
+
+
+def test_backward_full_shape_prefill(cuda_device, parity_report):
+    """The prefill workload the benchmark times (T = 8192, hidden 6144, 512 + 256 experts,
+    intermediate 2048), from a training forward that keeps G | U, as the benchmark runs
+    it. Against the oracle's backward restricted to what fits on the host: dx of 256
+    sampled tokens (with every expert they picked), and d_gate_up / d_down of the expert
+    with the most rows (thousands of rows: the K-grouped weight-gradient GEMMs run over
+    many k-blocks and a ragged last one), a mid-size expert and the expert with the fewest
+    rows. Every expert without rows keeps its sentinel."""
+    cfg = wl.CONFIGS["prefill_bf16"]
+    torch.cuda.empty_cache()
+    case = gh.Case(cfg)
+    b = case.buffers("deterministic")
+    gu = torch.empty(cfg.T * cfg.K + 128, 2 * cfg.I, dtype=torch.bfloat16, device="cuda")
+    abi.run_steps(b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up,
+                  case.w.w_down, gu_out=gu)
+    g = torch.Generator(device="cuda").manual_seed(177)
+    dout = (torch.randn(cfg.T, cfg.H, device="cuda", generator=g) * 0.5).to(torch.bfloat16)
+    dx = torch.empty(cfg.T, cfg.H, dtype=torch.float32, device="cuda")
+    d_router = torch.empty(cfg.E, cfg.H, dtype=torch.float32, device="cuda")
+    d_gu = torch.full((cfg.n_ffn, 2 * cfg.I, cfg.H), SENTINEL, dtype=torch.float32, device="cuda")
+    d_d = torch.full((cfg.n_ffn, cfg.H, cfg.I), SENTINEL, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(abi.backward_workspace_size(b.shape), dtype=torch.uint8, device="cuda")
+    abi.backward(b.shape, dout, case.x, case.w.w_router, case.w.w_gate_up, case.w.w_down,
+                 b.logits, b.topk_idx, b.topk_gate, b.offsets, b.row_of, b.x_perm, b.h,
+                 b.y_perm, dx, d_router, d_gu, d_d, ws, gu=gu)
+    torch.cuda.synchronize()
+    assert abi.read_device_status(ws) == 0
+    assert abi.read_device_status(b.ws) == 0
+    counts = gh.host(b.counts)[: cfg.n_ffn]
+    hit = np.nonzero(counts > 0)[0]
+    by_rows = hit[np.argsort(counts[hit], kind="stable")]
+    experts = sorted({int(by_rows[-1]), int(by_rows[len(by_rows) // 2]), int(by_rows[0])})
+    assert counts[by_rows[-1]] > 4000
+    toks = sorted(np.random.default_rng(5).choice(cfg.T, size=256, replace=False).tolist())
+    ref = orc.moe_layer_backward(gh.host(case.x), gh.host(case.w.w_router), gh.host(case.w.bias),
+                                 gh.LazyExperts(case.w.w_gate_up), gh.LazyExperts(case.w.w_down),
+                                 cfg.n_ffn, cfg.K, gh.host(dout), cfg.ffn_out_scale,
+                                 topk_idx=gh.host(b.topk_idx), tokens=toks, experts=experts)
+    errs = {"dx": gh.row_rel_err(gh.host(dx)[toks], ref.dx[toks])}
+    for e in experts:
+        errs[f"d_gate_up[{e}] ({counts[e]} rows)"] = _mat_rel_err(gh.host(d_gu[e]), ref.d_gate_up[e])
+        errs[f"d_down[{e}] ({counts[e]} rows)"] = _mat_rel_err(gh.host(d_d[e]), ref.d_down[e])
+    parity_report("backward prefill_bf16 T=8192: max rel err "
+                  + ", ".join(f"{k} {v:.2e}" for k, v in errs.items()) + f" (bar {TOL:g})")
+    for k, v in errs.items():
+        assert v <= TOL, (k, v, errs)
+    for e in np.nonzero(counts == 0)[0]:
+        assert bool((d_gu[e] == SENTINEL).all()) and bool((d_d[e] == SENTINEL).all()), e
+    del d_gu, d_d, gu, ws, b, case
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
