@@ -6,13 +6,17 @@
 
 One step = one pass of the whole hot path over one batch: router logits + softmax/top-K
 + histogram (moe_route_packed, with the router weight packed once at set-up), permutation
-(moe_permute), grouped SwiGLU FFN on the tensor
-cores with the fused combine epilogue (moe_grouped_ffn), finalize (moe_combine) and the
-PID bias update (moe_pid_bias_update, written to a second bias buffer so every step
-routes the same batch). Workload: the full-shape prefill layer (hidden 6144, 512 SwiGLU
-FFN experts of intermediate 2048 + 256 zero-computation experts, K = 12, 8192 tokens,
-bf16, synthetic seeded inputs). A second timed loop runs the same layer in the decode
-regime (128 tokens) and reports it against the HBM roofline.
+(moe_permute), grouped SwiGLU FFN on the tensor cores (moe_grouped_ffn; the deterministic
+combine by default: the down GEMM stores y per permuted row), the combine (moe_combine:
+each token's slots summed in slot order plus the zero-expert term) and the PID bias update
+(moe_pid_bias_update, written to a second bias buffer so every step routes the same
+batch). --combine fused times the fused epilogue (fp32 atomics into the token's
+accumulator) and the finalize instead. Workload: the full-shape prefill layer (hidden
+6144, 512 SwiGLU FFN experts of intermediate 2048 + 256 zero-computation experts, K = 12,
+8192 tokens, bf16, synthetic seeded inputs). The default run also times the same layer in
+the decode regime (128 tokens, against the HBM roofline), the skewed-routing workload
+(16384 tokens, drawn Zipf-skewed logits, with its 50-step PID trajectory) and the
+768-wide proxy layer (4096 tokens).
 
 Multi-GPU: every rank runs its own replica of the layer on its own batch (no exchange in
 the forward pass: weak scaling); the time is the max over ranks.
@@ -23,6 +27,7 @@ workload on the host cores; under torchrun only rank 0 runs it.
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import os
@@ -43,6 +48,9 @@ from mixture_experts_layer_29_b200 import workloads as wl  # noqa: E402
 METRIC = "MoE-layer tokens/s on 1 B200; % of bf16 TC peak (prefill) / HBM BW (decode)"
 UNIT = "tokens/s"
 PID_GAINS = (0.01, 0.001, 0.0, 8 / 12)
+# faster integral action for the skewed workload's closed loop (reported beside the
+# default gains; the pages do not print theirs)
+PID_GAINS_FAST = (0.01, 0.05, 0.0, 8 / 12)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 CSRC = os.path.join(ROOT, "mixture_experts_layer_29_b200", "csrc")
@@ -147,7 +155,7 @@ def oracle_threads() -> int:
 def oracle_sample(cfg, w, x_dev, tokens, logits_dev=None):
     """Time the oracle on `tokens` of the workload: logits (float64), routing, and the
     SwiGLU experts of those tokens. Weights of the experts they hit are copied to the
-    host first (outside the timed region). Where the workload's logits are an input
+    host and converted to float64 first (outside the timed region). Where the workload's logits are an input
     (`logits_dev`, the skewed workload), the oracle takes those rows instead of computing
     them. Returns (seconds, tokens)."""
     import oracle.moe_oracle as orc
@@ -161,6 +169,10 @@ def oracle_sample(cfg, w, x_dev, tokens, logits_dev=None):
     experts = sorted({int(e) for e in r.topk_idx.ravel() if e < cfg.n_ffn})
     wgu = {e: w.w_gate_up[e].float().cpu().numpy() for e in experts}
     wd = {e: w.w_down[e].float().cpu().numpy() for e in experts}
+    # the oracle computes in float64: hand it float64 weights, so that the timed region
+    # holds its arithmetic, not the conversion of every touched expert's 75 MB of weights
+    wgu = {e: v.astype(np.float64) for e, v in wgu.items()}
+    wd = {e: v.astype(np.float64) for e, v in wd.items()}
     t0 = time.perf_counter()
     L = given if given is not None else orc.router_logits(x, wr).astype(np.float32)
     orc.moe_layer_forward(x, L, bias, wgu, wd, cfg.n_ffn, cfg.K, cfg.ffn_out_scale)
@@ -416,7 +428,7 @@ def time_backward(st: Stepper, device, seed: int, iters: int, warmup: int) -> di
     return out
 
 
-def pid_trajectory(cfg, w, device, seed: int) -> dict:
+def pid_trajectory(cfg, w, device, seed: int, gains=PID_GAINS) -> dict:
     """The skewed workload's closed loop, untimed: for each of cfg.pid_steps steps, route
     that step's drawn logits with the current bias (moe_route) and update the FFN experts'
     biases from the histogram (moe_pid_bias_update), starting from the workload's bias.
@@ -429,7 +441,7 @@ def pid_trajectory(cfg, w, device, seed: int) -> dict:
     state = torch.empty(3 * cfg.n_ffn, dtype=torch.float32, device=device)
     stats = torch.zeros(8, dtype=torch.float32, device=device)
     abi.pid_init(shape, bias, state)
-    pid = abi.Pid(*PID_GAINS)
+    pid = abi.Pid(*gains)
     ratio, spread, imbalance = [], [], []
     for k in range(cfg.pid_steps):
         logits = wl.draw_skewed_logits(cfg, device, seed=seed, step=k)
@@ -441,9 +453,30 @@ def pid_trajectory(cfg, w, device, seed: int) -> dict:
         spread.append(round(float(st[2]), 3))
         imbalance.append(round(float(st[3]), 2))
     assert abi.read_device_status(ws) == 0
-    return {"steps": cfg.pid_steps, "target_ratio": round(PID_GAINS[3], 4),
-            "gains": {"kp": PID_GAINS[0], "ki": PID_GAINS[1], "kd": PID_GAINS[2]},
+    return {"steps": cfg.pid_steps, "target_ratio": round(gains[3], 4),
+            "gains": {"kp": gains[0], "ki": gains[1], "kd": gains[2]},
             "ffn_ratio": ratio, "ffn_picks_std": spread, "ffn_max_over_mean_load": imbalance}
+
+
+def ffn_roofline(workload: str, rows: int, cfg, ffn_ms: float, timed_ms: float) -> dict:
+    """The grouped FFN (gate/up + down tcgen05 GEMMs) against the bf16 tensor-core peak.
+    Algorithmic work: 6 H I FLOP per FFN row (gate, up and down projections). The timed
+    region lasts well under a second, so the burst peak applies; the sustained one (a
+    seconds-long loop under the power cap) is printed beside it."""
+    pk, pk_kind = peaks()
+    flop = rows * 6.0 * cfg.H * cfg.I
+    achieved = flop / (ffn_ms / 1e3) / 1e12
+    burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    sustained = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    te = traffic_entry(f"{workload}:grouped_ffn")
+    return {"bound": "tensor", "kernel": "grouped_ffn (gate/up + down tcgen05 GEMMs)",
+            "achieved": round(achieved, 1), "peak": burst, "unit": "TFLOP/s",
+            "frac": round(achieved / burst, 4),
+            "traffic": te["dram_bytes_per_call"] if te else None,
+            "peak_kind": f"bf16 burst, {pk_kind} (timed region {timed_ms / 1e3:.2f} s)",
+            "frac_of_sustained": round(achieved / sustained, 4), "sustained_peak": sustained,
+            "algorithmic_flop_per_call": flop, "ffn_rows": rows,
+            "kernel_ms": round(ffn_ms, 4)}
 
 
 def max_over_ranks(v: float, dist_on: bool) -> float:
@@ -477,6 +510,45 @@ def workload(args):
     if args.zero_experts is not None:
         kw["n_zero"] = args.zero_experts
     return cfg.with_(**kw) if kw else cfg
+
+
+def time_workload(name: str, args, device, rank: int, dist_on: bool, world: int) -> dict:
+    """Another workload of the layer, timed like the main one in the same run: its own
+    weights, batch (and drawn logits), the same step, the per-call breakdown and the
+    grouped FFN's roofline; for the skewed workload also its closed PID loop, with the
+    default gains and with PID_GAINS_FAST."""
+    cfg = wl.CONFIGS[name]
+    seed = replica_seed(cfg, rank)
+    w = wl.draw_weights(cfg, device, seed=cfg.seed)
+    x = wl.draw_tokens(cfg, device, seed=seed)
+    logits_in = wl.draw_skewed_logits(cfg, device, seed=seed) if cfg.skewed else None
+    st = Stepper(cfg, w, x, logits_in, args.combine, device)
+    # short steps get more of them, so that the timed region is not a few microseconds
+    steps = max(args.steps, 200) if cfg.T * cfg.H < 8192 * 6144 // 4 else args.steps
+    ms, _, launches = timed_loop(st, steps, max(args.warmup, 3), dist_on, phases=False)
+    _, per, _ = timed_loop(st, min(steps, 30), 0, dist_on, phases=True)
+    ms = max_over_ranks(ms, dist_on)
+    counts = st.b.counts.cpu().numpy()
+    rows = int(counts[: cfg.n_ffn].sum())
+    out = {"workload": name, "tokens": cfg.T, "hidden": cfg.H, "expert_intermediate": cfg.I,
+           "ffn_experts": cfg.n_ffn, "zero_experts": cfg.n_zero, "top_k": cfg.K,
+           "value": round(job_throughput(cfg.T, steps, world, ms), 1), "unit": UNIT,
+           "ms_per_step": round(ms / steps, 4), "steps": steps,
+           "gpu_launches": int(launches) * world,
+           "breakdown_ms": {p: round(float(np.mean(v)), 4) for p, v in per.items()},
+           "roofline": ffn_roofline(name, rows, cfg, float(np.mean(per["grouped_ffn"])), ms),
+           "routing": {"ffn_rows": rows, "ffn_experts_hit": int((counts[: cfg.n_ffn] > 0).sum()),
+                       "max_rows_per_expert": int(counts[: cfg.n_ffn].max())}}
+    if cfg.H * cfg.I * cfg.n_ffn * 6 < 126e6:
+        out["l2"] = "the experts' weights fit in the 126 MB L2; no flush between steps"
+    if cfg.pid_steps > 0 and rank == 0:
+        out["pid_trajectory"] = pid_trajectory(cfg, w, device, seed)
+        out["pid_trajectory_fast"] = pid_trajectory(cfg, w, device, seed, PID_GAINS_FAST)
+    del st, w, x, logits_in
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
 
 
 def workload_config(args, cfg) -> dict:
@@ -514,22 +586,12 @@ def run_ours(args):
 
     counts = st.b.counts.cpu().numpy()
     rows = int(counts[: cfg.n_ffn].sum())
-    flops_ffn = rows * 6.0 * cfg.H * cfg.I
     ffn_ms = float(np.mean(per["grouped_ffn"]))
-    pk, pk_kind = peaks()
-    achieved = flops_ffn / (ffn_ms / 1e3) / 1e12
-    peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    te = traffic_entry(f"{args.workload}:grouped_ffn")
-    traffic = te["dram_bytes_per_call"] if te else None
-    roofline = {"bound": "tensor", "kernel": "grouped_ffn (gate/up + down tcgen05 GEMMs)",
-                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_kind": f"bf16 sustained, {pk_kind}",
-                "frac_of_burst": round(achieved / pk.get("bf16_tflops", peak), 4),
-                "algorithmic_flop_per_call": flops_ffn, "ffn_rows": rows}
+    roofline = ffn_roofline(args.workload, rows, cfg, ffn_ms, total_ms)
 
     # ---- decode regime: same layer (same weights), 128 tokens ---------------------------
     decode = None
+    dst = None
     if args.workload == "prefill_bf16" and not args.no_decode:
         dcfg = cfg.with_(T=wl.CONFIGS["decode_bf16"].T)
         dx = wl.draw_tokens(dcfg, device, seed=seed)
@@ -546,6 +608,7 @@ def run_ours(args):
         dte = traffic_entry("decode_bf16:step")
         dtraffic = dte["dram_bytes_per_step"] if dte else None
         dach = dbytes / (dstep / 1e3) / 1e9
+        pk, pk_kind = peaks()
         hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         dgraph = graph_step_ms(dst, dsteps) if not dist_on else None
         decode = {"workload": "decode_bf16", "value": round(dcfg.T * dsteps * world / (dms / 1e3), 1),
@@ -627,6 +690,16 @@ def run_ours(args):
                "sample": f"{n} of the {cfg.T} tokens, drawn with a fixed seed (logits, routing "
                          f"and SwiGLU experts in float64 numpy), {secs:.1f} s of oracle time"}
 
+    # ---- the other workloads of the layer, after the main one's weights are freed ---------
+    others = None
+    if args.workload == "prefill_bf16" and not args.no_others:
+        del st, dst, w, x, logits_in
+        gc.collect()
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        others = {"skew_pid": time_workload("skew_pid_bf16", args, device, rank, dist_on, world),
+                  "proxy": time_workload("proxy_bf16", args, device, rank, dist_on, world)}
+
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -643,6 +716,7 @@ def run_ours(args):
         "scmoe_overlap": overlap,
         "backward": bwd,
         "pid_trajectory": pid_traj,
+        "workloads": others,
         "e2e": e2e,
         "gpu_launches": int(launches) * world,
         "cpu_baseline": cpu,
@@ -722,6 +796,8 @@ def parser() -> argparse.ArgumentParser:
     ap.add_argument("--no-backward", action="store_true", help="skip timing moe_backward")
     ap.add_argument("--no-overlap", action="store_true",
                     help="skip the dense-FFN-beside-MoE (two streams) measurement")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the skewed-routing + PID and proxy workloads of the default run")
     return ap
 
 
