@@ -136,6 +136,21 @@ uint64_t moe_launch_count(void);
  *                             run out after their limit (2 s) and write MOE_ERR_TIMEOUT to
  *                             the status word; that call's outputs are undefined. The
  *                             switch returns to 0 when that launch is queued.
+ *   MOE_TUNE_GATE_UP_BAND     0 (default): the library's choice; 1 to 64: the CTA-pair
+ *   MOE_TUNE_DOWN_BAND        gate/up (down) GEMM visits an expert's 256-row M tiles in
+ *                             bands of this many, each band N tile by N tile with its M
+ *                             tiles fastest (1: M tile by M tile, N tiles fastest).
+ *   MOE_TUNE_PAIR_INTERLEAVE  0 (default): plain expert order; 1: the CTA-pair GEMMs
+ *                             spread the tiles of experts with at most 256 rows (one M
+ *                             tile) evenly among the other experts' tiles.
+ *   MOE_TUNE_PAIR_A_TRIM      1 (default): in the CTA-pair GEMMs each CTA loads only the A
+ *                             rows of the expert's group that its MMA rows cover (boxes of
+ *                             16, 64 or 128 rows, or none); 0: always 128-row boxes.
+ *   MOE_TUNE_PAIR_SWAP_AB     1 (default): in the forward's CTA-pair GEMMs a tile of at
+ *                             most 128 rows (a small expert, an expert's tail) runs with
+ *                             the operands swapped: the expert's weights as the M = 256
+ *                             side, the tile's rows (rounded up to 16, 32, 64 or 128) as
+ *                             N; 0: such tiles run as M = 128 tiles.
  * moe_set_tuning returns MOE_ERR_INVALID_ARG for an unknown switch or a value outside its
  * range. moe_get_tuning writes the current value. */
 typedef enum {
@@ -146,7 +161,12 @@ typedef enum {
   MOE_TUNE_ROUTER_MIN_SPLIT = 4,
   MOE_TUNE_BWD_PAIR = 5,
   MOE_TUNE_BWD_DY_ROWS = 6,
-  MOE_TUNE_TEST_STALL = 7
+  MOE_TUNE_TEST_STALL = 7,
+  MOE_TUNE_GATE_UP_BAND = 8,
+  MOE_TUNE_DOWN_BAND = 9,
+  MOE_TUNE_PAIR_INTERLEAVE = 10,
+  MOE_TUNE_PAIR_A_TRIM = 11,
+  MOE_TUNE_PAIR_SWAP_AB = 12
 } moe_tune_t;
 
 int moe_set_tuning(int knob, int64_t value);

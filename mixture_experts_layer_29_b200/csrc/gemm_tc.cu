@@ -27,6 +27,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstddef>
 #include <mutex>
 
 #include "common.cuh"
@@ -68,8 +69,11 @@ struct alignas(1024) SharedStorage {
   // router logits: each epilogue warp turns 32 rows x 16 columns around here so that its
   // global stores cover whole 64-byte row segments (row stride 20 floats: 16-byte aligned
   // and conflict-free for the row-wise float4 writes)
-  float epi_stage[kEpiWarps][32][20];
+  alignas(16) float epi_stage[kEpiWarps][32][20];
 };
+static_assert(offsetof(SharedStorage, epi_stage) % 16 == 0, "16-byte staging rows");
+static_assert(offsetof(SharedStorage, a) % 1024 == 0 && offsetof(SharedStorage, b) % 1024 == 0,
+              "128-byte-swizzled TMA boxes need 1024-byte alignment");
 
 struct GemmArgs {
   int mode;
@@ -101,6 +105,10 @@ struct GemmArgs {
   const __nv_bfloat16* gu_in; // kDgradDH: G | U of the rows ([rows, 2I], I = n_valid)
   int test_stall;             // testing (MOE_TUNE_TEST_STALL): tile 0 leaves its first
                               // k-block unloaded, so the waits on that stage run out
+  int band;                   // pair kernel: M tiles per band of the tile order (1: M-major)
+  int interleave;             // pair kernel: spread single-tile experts' tiles (see below)
+  int a_trim;                 // pair kernel: load only the A rows of the group (a_box_rows)
+  int swap_ab;                // pair kernel, forward: tiles of <= 128 rows run swapped (swap_npad)
 };
 
 // The testing hook of GemmArgs::test_stall: this (tile, k-block) is not loaded.
@@ -640,7 +648,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int BMP = 256;                             // M rows per CTA pair
 constexpr int PSTAGES = 6;                           // 32 KB per stage per CTA
 constexpr int P_B_BYTES = 128 * BK * 2;              // 16 KB: this CTA's half of B
-constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES;   // 32 KB
 
 struct alignas(1024) PairStorage {
   uint8_t a[PSTAGES][A_BYTES];
@@ -652,30 +659,207 @@ struct alignas(1024) PairStorage {
   uint32_t tmem_base;
   int abort_flag;
   int offs[kMaxExperts + 1];
-  int toff[kMaxExperts + 1];    // prefix of ceil(count / 256)
-  float epi_stage[kEpiWarps][32][20];   // deterministic down store (see epilogue_expert)
+  int toff[kMaxExperts + 1];    // prefix of ceil(count / 256) over the multi-tile experts
+  int n_single;                 // experts of one M tile spread through the order (see below)
+  int16_t single[kMaxExperts];  // those experts, in index order
+  // deterministic down store (see epilogue_expert); read and written as 16-byte vectors
+  alignas(16) float epi_stage[kEpiWarps][32][20];
 };
+static_assert(offsetof(PairStorage, epi_stage) % 16 == 0, "16-byte staging rows");
+static_assert(offsetof(PairStorage, a) % 1024 == 0 && offsetof(PairStorage, b) % 1024 == 0,
+              "128-byte-swizzled TMA boxes need 1024-byte alignment");
 
+// Tile order of the CTA-pair kernel. Tiles are handed out round-robin in this order, so
+// the order is also roughly the time at which a tile runs.
+//  * Experts of a single M tile (at most 256 rows; g.interleave) stream their whole weight
+//    matrix for one tile each: their tiles are DRAM-bound, while the multi-tile experts'
+//    tiles reuse each B tile over several M tiles and are bound by the tensor pipe. So the
+//    single-tile experts' tiles ("S") are spread evenly through the others ("L"):
+//    position i is an S tile when floor((i+1) TS / Ttot) > floor(i TS / Ttot), with TS S
+//    tiles out of Ttot. Their weight streams then overlap the L tiles' MMAs instead of
+//    filling whole waves with DRAM-bound tiles. S tiles go expert by expert, N fastest.
+//  * L tiles: expert e owns L tiles [toff[e], toff[e+1]) * n_tiles. Inside an expert the
+//    M tiles go in bands of g.band: a band's tiles run N tile by N tile, its M tiles
+//    fastest. g.band = 1 is plain M-major order (N fastest).
 __device__ __forceinline__ Tile decode_pair_tile(const PairStorage& s, const GemmArgs& g, int tile) {
   Tile t;
   t.split = 0;
   t.kb0 = 0;
   t.kb1 = g.kblocks;
-  const int mt = tile / g.n_tiles;
-  t.nt = tile - mt * g.n_tiles;
+  if (s.n_single > 0) {
+    const long long ts = (long long)s.n_single * g.n_tiles;
+    const long long tot = ts + (long long)s.toff[g.n_ffn] * g.n_tiles;
+    const int ns0 = (int)((long long)tile * ts / tot);
+    const int ns1 = (int)((long long)(tile + 1) * ts / tot);
+    if (ns1 > ns0) {                                    // the ns0-th S tile
+      const int k = ns0 / g.n_tiles;
+      const int e = s.single[k];
+      t.nt = ns0 - k * g.n_tiles;
+      t.e = e;
+      t.row0 = s.offs[e];
+      t.row_end = s.offs[e + 1];
+      return t;
+    }
+    tile -= ns0;                                        // the tile-th L tile
+  }
+  const int mt_any = tile / g.n_tiles;
   int lo = 0, hi = g.n_ffn - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (s.toff[mid] <= mt) lo = mid; else hi = mid - 1;
+    if (s.toff[mid] <= mt_any) lo = mid; else hi = mid - 1;
+  }
+  int mt;
+  if (g.band > 1) {
+    const int l = tile - s.toff[lo] * g.n_tiles;       // tile within the expert
+    const int per_band = g.band * g.n_tiles;
+    const int j = l / per_band;
+    const int o = l - j * per_band;
+    const int h = min(g.band, s.toff[lo + 1] - s.toff[lo] - j * g.band);   // band height
+    t.nt = o / h;
+    mt = j * g.band + (o - t.nt * h);
+  } else {
+    mt = mt_any - s.toff[lo];
+    t.nt = tile - mt_any * g.n_tiles;
   }
   t.e = lo;
-  t.row0 = s.offs[lo] + (mt - s.toff[lo]) * BMP;
+  t.row0 = s.offs[lo] + mt * BMP;
   t.row_end = s.offs[lo + 1];
   return t;
 }
 
 __device__ __forceinline__ bool half_tile(const GemmArgs& g, const Tile& t) {
   return g.half_tiles && t.row_end - t.row0 <= 128;
+}
+
+// Rows of CTA r's A box in a pair tile. The CTA's MMA rows are [row0 + per r, + per) with
+// per = 64 (half tile) or 128; only those inside the expert's group are ever stored, so
+// with g.a_trim only they are loaded: a box of 16, 64 or 128 rows, or nothing. The MMA
+// reads whatever the rest of the A stage holds, and the rows it makes there are dropped.
+// A single-row expert then moves 2 KB of A per k-block instead of 16 KB, which matters
+// because such tiles are bound by how fast the SM fills its shared memory.
+__device__ __forceinline__ int a_box_rows(const GemmArgs& g, const Tile& t, bool half, int r) {
+  const int per = half ? 64 : 128;
+  if (!g.a_trim) return 128;
+  const int need = min(t.row_end - (t.row0 + per * r), per);
+  return need <= 0 ? 0 : need <= 16 ? 16 : need <= 64 ? 64 : 128;
+}
+
+// Swap tiles (g.swap_ab, forward GEMMs). An M = 128 tile over the CTA pair (64 rows per
+// CTA) costs the tensor pipe as many cycles as an M = 256 one, so a tile of few rows
+// (small experts, an expert's tail) costs a full tile of MMA time. With the operands
+// swapped the expert's weights are the M = 256 side and the tile's rows the N side,
+// N = npad (16, 32, 64 or 128: the rows rounded up), and the MMA time shrinks with the
+// rows: such a tile is bound by streaming its weights. CTA r then holds weight rows
+// [128r, 128r + 128) of the N tile (gate/up: 64 gate rows and the same 64 up rows, as the
+// half tiles load them) and rows [row0 + r npad/2, + npad/2) of the tile's rows.
+// The accumulator is transposed: TMEM lane = output feature, column = row of the tile.
+__device__ __forceinline__ int swap_npad(const GemmArgs& g, const Tile& t) {
+  if (!g.swap_ab) return 0;
+  const int rows = t.row_end - t.row0;
+  if (rows > 128) return 0;
+  return rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
+}
+
+// The pair kernel's 8 epilogue warps (256 threads) meet here; named barrier 1.
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Epilogue of a swap tile, for every epilogue thread of CTA `rank` (warp quarter q, column
+// half h); all 8 epilogue warps take part (named barrier 1). Per 32 columns (rows of the
+// tile): each warp moves 16 columns of its 32 lanes
+// from TMEM into S[row][feature] (fp32, row stride 132 floats), then the 256 threads write
+// whole output rows from S. TMEM lane l is output feature l of the CTA's 128: gate/up:
+// h column nt * 128 + 64 rank + (l mod 64), from gate (l < 64) and up (l >= 64); down:
+// output column nt * 256 + 128 rank + l. KEEP: as epi_gateup_chunk.
+template <int KEEP>
+__device__ __forceinline__ void epilogue_swap(const GemmArgs& g, const Tile& t, uint32_t tbase,
+                                              uint32_t rank, int q, int h, float* S, int npad) {
+  constexpr int SS = 132;
+  const int lane = threadIdx.x & 31;
+  const int u = threadIdx.x - 64;                     // 0..255 over the epilogue warps
+  // S spans every warp's staging rows: wait until all warps are done with the last tile
+  epi_bar();
+#pragma unroll 1
+  for (int c0 = 0; c0 < npad; c0 += 32) {
+    const int ncol = min(32, npad - c0);
+    if (16 * h < ncol) {
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(tbase + (uint32_t)(c0 + 16 * h), v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) S[(16 * h + j) * SS + 32 * q + lane] = __uint_as_float(v[j]);
+    }
+    epi_bar();
+    if (g.mode == kGateUp) {
+      // 32 rows x 8 groups of 8 h columns: one 16-byte store of h (or of G and U)
+      const int j = u >> 3, f8 = u & 7;
+      const int row = t.row0 + c0 + j;
+      if (j < ncol && row < t.row_end) {
+        const float4* sg = reinterpret_cast<const float4*>(S + j * SS + 8 * f8);
+        const float4* su = reinterpret_cast<const float4*>(S + j * SS + 64 + 8 * f8);
+        const float4 g0 = sg[0], g1 = sg[1], u0 = su[0], u1 = su[1];
+        const float G[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const float U[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        const int col = t.nt * BM + 64 * (int)rank + 8 * f8;
+        if (g.gu_raw) {
+          __nv_bfloat16* base = static_cast<__nv_bfloat16*>(g.out) + (size_t)row * g.ld_out + col;
+          *reinterpret_cast<uint4*>(base) =
+              make_uint4(pack_bf16x2(G[0], G[1]), pack_bf16x2(G[2], G[3]),
+                         pack_bf16x2(G[4], G[5]), pack_bf16x2(G[6], G[7]));
+          *reinterpret_cast<uint4*>(base + g.n_valid) =
+              make_uint4(pack_bf16x2(U[0], U[1]), pack_bf16x2(U[2], U[3]),
+                         pack_bf16x2(U[4], U[5]), pack_bf16x2(U[6], U[7]));
+        } else {
+          float hv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) hv[i] = silu_f(G[i]) * U[i];
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (size_t)row * g.ld_out + col) =
+              make_uint4(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]),
+                         pack_bf16x2(hv[4], hv[5]), pack_bf16x2(hv[6], hv[7]));
+          if (KEEP == 1 || (KEEP == 2 && g.gu_out)) {
+            __nv_bfloat16* base = static_cast<__nv_bfloat16*>(g.gu_out) +
+                                  (size_t)row * 2 * g.n_valid + col;
+            *reinterpret_cast<uint4*>(base) =
+                make_uint4(pack_bf16x2(G[0], G[1]), pack_bf16x2(G[2], G[3]),
+                           pack_bf16x2(G[4], G[5]), pack_bf16x2(G[6], G[7]));
+            *reinterpret_cast<uint4*>(base + g.n_valid) =
+                make_uint4(pack_bf16x2(U[0], U[1]), pack_bf16x2(U[2], U[3]),
+                           pack_bf16x2(U[4], U[5]), pack_bf16x2(U[6], U[7]));
+          }
+        }
+      }
+    } else if (g.mode == kDownStore) {
+      // 32 rows x 16 groups of 8 output columns
+#pragma unroll 1
+      for (int it = u; it < 32 * 16; it += 256) {
+        const int j = it >> 4, f8 = it & 15;
+        const int row = t.row0 + c0 + j;
+        const int col = t.nt * BN + 128 * (int)rank + 8 * f8;
+        if (j < ncol && row < t.row_end && col < g.n_valid) {
+          const float4* sy = reinterpret_cast<const float4*>(S + j * SS + 8 * f8);
+          const float4 a = sy[0], b = sy[1];
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (size_t)row * g.ld_out + col) =
+              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                         pack_bf16x2(b.z, b.w));
+        }
+      }
+    } else {
+      // fused: s * g * y added into the token's fp32 accumulator, 4 columns at a time
+#pragma unroll 1
+      for (int it = u; it < 32 * 32; it += 256) {
+        const int j = it >> 5, f4 = it & 31;
+        const int row = t.row0 + c0 + j;
+        const int col = t.nt * BN + 128 * (int)rank + 4 * f4;
+        if (j < ncol && row < t.row_end && col < g.n_valid) {
+          const int tok = g.perm_token[row];
+          const float sc = g.scale * g.row_gate[row];
+          const float4 y = *reinterpret_cast<const float4*>(S + j * SS + 4 * f4);
+          atomicAdd(reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)tok * g.ld_out + col),
+                    make_float4(sc * y.x, sc * y.y, sc * y.z, sc * y.w));
+        }
+      }
+    }
+    epi_bar();
+  }
 }
 
 // Epilogue of one pair tile for one thread of warp quarter q and column half h. Full tile
@@ -733,6 +917,10 @@ __device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, 
 template <int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmA64,
+                        const __grid_constant__ CUtensorMap tmA32,
+                        const __grid_constant__ CUtensorMap tmA16,
+                        const __grid_constant__ CUtensorMap tmA8,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmB64, const GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
@@ -758,6 +946,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     if (g.half_tiles && g.mode == kGateUp) prefetch_tensormap(&tmB64);
+    if (g.a_trim || g.swap_ab) {
+      prefetch_tensormap(&tmA64);
+      prefetch_tensormap(&tmA16);
+    }
+    if (g.swap_ab) {
+      prefetch_tensormap(&tmA32);
+      prefetch_tensormap(&tmA8);
+    }
   }
   pdl_wait();
   for (int i = threadIdx.x; i <= g.n_ffn; i += kThreads) s.offs[i] = g.offsets[i];
@@ -768,25 +964,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish_pair();
   }
   if (warp == 2) {
+    // L tiles per expert (multi-tile experts, or all with g.interleave off) and the list
+    // of single-tile experts; lane l takes a contiguous run of experts
     const int per = (g.n_ffn + 31) / 32;
     const int b = lane * per;
-    int local = 0;
+    int local = 0, nsingle = 0;
     for (int i = 0; i < per; ++i)
-      if (b + i < g.n_ffn) local += (s.offs[b + i + 1] - s.offs[b + i] + BMP - 1) / BMP;
+      if (b + i < g.n_ffn) {
+        const int m = (s.offs[b + i + 1] - s.offs[b + i] + BMP - 1) / BMP;
+        if (g.interleave && m == 1) ++nsingle;
+        else local += m;
+      }
     const int inc = warp_inclusive_scan(local);
-    int run = inc - local;
+    const int sinc = warp_inclusive_scan(nsingle);
+    int run = inc - local, srun = sinc - nsingle;
     for (int i = 0; i < per; ++i)
       if (b + i < g.n_ffn) {
         s.toff[b + i] = run;
-        run += (s.offs[b + i + 1] - s.offs[b + i] + BMP - 1) / BMP;
+        const int m = (s.offs[b + i + 1] - s.offs[b + i] + BMP - 1) / BMP;
+        if (g.interleave && m == 1) s.single[srun++] = (int16_t)(b + i);
+        else run += m;
       }
-    if (lane == 31) s.toff[g.n_ffn] = inc;
+    if (lane == 31) {
+      s.toff[g.n_ffn] = inc;
+      s.n_single = sinc;
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = s.tmem_base;
-  const int total_tiles = s.toff[g.n_ffn] * g.n_tiles;
+  const int total_tiles = (s.toff[g.n_ffn] + s.n_single) * g.n_tiles;
   volatile int* abort_flag = &s.abort_flag;
 
   if (warp == 0) {
@@ -796,15 +1004,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       for (int tile = cluster; tile < total_tiles && !*abort_flag; tile += nclusters) {
         const Tile t = decode_pair_tile(s, g, tile);
-        const bool half = half_tile(g, t);
-        const bool split_b = half && g.mode == kGateUp;   // 64 gate + 64 up rows
+        const int npad = swap_npad(g, t);                  // swap tile: npad / 2 rows per CTA
+        const bool half = !npad && half_tile(g, t);
+        const bool split_b = (half || npad) && g.mode == kGateUp;   // 64 gate + 64 up rows
         constexpr bool b_mn = KIND == kPairDgrad;
-        const int arow = t.row0 + (half ? 64 : 128) * (int)rank;
+        const int arow = npad ? t.row0 + (npad / 2) * (int)rank
+                              : t.row0 + (half ? 64 : 128) * (int)rank;
         const int brow = g.mode != kGateUp ? t.e * g.b_rows + t.nt * BN + 128 * (int)rank
                          : split_b ? t.e * g.b_rows + t.nt * BM + 64 * (int)rank
                                    : t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM;
         // MN-major B (dgrad): this CTA's 128 N columns as two 64 x 64 boxes of K rows
         const int bcol = t.nt * BN + 128 * (int)rank;
+        const int a_rows = npad ? npad / 2 : a_box_rows(g, t, half, (int)rank);
+        const CUtensorMap* a_map = a_rows == 128 ? &tmA : a_rows == 64 ? &tmA64
+                                 : a_rows == 32 ? &tmA32 : a_rows == 16 ? &tmA16 : &tmA8;
+        // the leader expects both CTAs' bytes: B halves of 16 KB and the two A boxes
+        const uint32_t tx = 2 * P_B_BYTES +
+            (npad ? (uint32_t)npad * BK * 2
+                  : (uint32_t)(a_box_rows(g, t, half, 0) + a_box_rows(g, t, half, 1)) * BK * 2);
         for (int kb = 0; kb < g.kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
           if (stalled_stage(g, tile, kb, 0)) {   // neither CTA loads; nothing is expected
@@ -815,8 +1032,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
-          if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * P_STAGE_BYTES);
-          tma_load_2d_pair(s.a[stage], &tmA, kb * BK, arow, full_leader);
+          if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], tx);
+          if (a_rows > 0) tma_load_2d_pair(s.a[stage], a_map, kb * BK, arow, full_leader);
           if (b_mn) {
             const int y = t.e * g.b_rows + kb * BK;
             tma_load_2d_pair(s.b[stage], &tmB, bcol, y, full_leader);
@@ -845,8 +1062,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
         constexpr bool b_mn = KIND == kPairDgrad;
-        const uint32_t idesc = idesc_bf16_f32_major(
-            half_tile(g, decode_pair_tile(s, g, tile)) ? 128 : BMP, BN, false, b_mn);
+        const Tile mt = decode_pair_tile(s, g, tile);
+        const int npad = swap_npad(g, mt);
+        // swap tile: A = the weights (s.b), B = the tile's rows (s.a), N = npad
+        const uint32_t idesc = npad ? idesc_bf16_f32(BMP, npad)
+                                    : idesc_bf16_f32_major(half_tile(g, mt) ? 128 : BMP, BN,
+                                                           false, b_mn);
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -855,12 +1076,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(s.a[stage]);
           const uint32_t b0 = smem_u32(s.b[stage]);
+          if (npad) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + k * 32),
-                           b_mn ? sw128_mnmajor_desc(b0 + k * 2048, P_B_BYTES / 2)
-                                : sw128_kmajor_desc(b0 + k * 32),
-                           idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16_pair(d_tmem, sw128_kmajor_desc(b0 + k * 32), sw128_kmajor_desc(a0 + k * 32),
+                             idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + k * 32),
+                             b_mn ? sw128_mnmajor_desc(b0 + k * 2048, P_B_BYTES / 2)
+                                  : sw128_kmajor_desc(b0 + k * 32),
+                             idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
           const uint32_t e_local = smem_u32(&s.empty[stage]);
           umma_commit_pair(mapa_shared(e_local, 0));
           umma_commit_pair(mapa_shared(e_local, 1));
@@ -892,7 +1120,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_pair<KIND>(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
+      int npad = 0;
+      if constexpr (KIND != kPairDgrad) npad = swap_npad(g, t);
+      if (npad) {
+        if constexpr (KIND != kPairDgrad)
+          epilogue_swap<KIND == kPairFwdKeep ? 1 : 0>(g, t, tbase, rank, q, half,
+                                                      &s.epi_stage[0][0][0], npad);
+      } else {
+        epilogue_pair<KIND>(g, t, tbase, rank, q, half, s.epi_stage[warp - 2], lane);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
@@ -965,8 +1201,23 @@ int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, 
 
 // Cluster-of-two launch of the CTA-pair kernel: as many clusters as fit at once (cached
 // per device), so the persistent tile loop never waits for a cluster slot.
-int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb64,
-                const GemmArgs& g, int sm_count, cudaStream_t st) {
+// A's tensor with boxes of 128, 64, 32, 16 and 8 rows (see a_box_rows and swap_npad).
+struct AMaps {
+  CUtensorMap m128, m64, m32, m16, m8;
+};
+int make_amaps(AMaps* m, const void* base, uint64_t rows, uint64_t cols) {
+  int rc;
+  if ((rc = make_map(&m->m128, base, rows, cols, 128)) != MOE_OK ||
+      (rc = make_map(&m->m64, base, rows, cols, 64)) != MOE_OK ||
+      (rc = make_map(&m->m32, base, rows, cols, 32)) != MOE_OK ||
+      (rc = make_map(&m->m16, base, rows, cols, 16)) != MOE_OK ||
+      (rc = make_map(&m->m8, base, rows, cols, 8)) != MOE_OK)
+    return rc;
+  return MOE_OK;
+}
+
+int launch_pair(const AMaps& ma, const CUtensorMap& mb, const CUtensorMap& mb64, const GemmArgs& g,
+                int sm_count, cudaStream_t st) {
   constexpr size_t smem = sizeof(PairStorage) + 1024;
   static_assert(smem <= 227 * 1024, "shared memory budget");
   static std::mutex mu;
@@ -1005,7 +1256,13 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap&
     nclusters = clusters_of[dev];
   }
   if (nclusters > sm_count / 2) nclusters = sm_count / 2;
-  if (launch_kernel(kern, 2 * nclusters, kThreads, smem, st, 2, ma, mb, mb64, g) != cudaSuccess) {
+  GemmArgs ga = g;
+  ga.interleave = tuning(MOE_TUNE_PAIR_INTERLEAVE) != 0 ? 1 : 0;
+  ga.a_trim = tuning(MOE_TUNE_PAIR_A_TRIM) != 0 ? 1 : 0;
+  ga.swap_ab = (g.mode != kDgradDH && g.mode != kDgradDX && tuning(MOE_TUNE_PAIR_SWAP_AB) != 0)
+                   ? 1 : 0;
+  if (launch_kernel(kern, 2 * nclusters, kThreads, smem, st, 2, ma.m128, ma.m64, ma.m32, ma.m16,
+                    ma.m8, mb, mb64, ga) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
@@ -1017,6 +1274,12 @@ int launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap&
 // the one-CTA kernel. MOE_TUNE_GEMM_PAIR forces either, MOE_TUNE_PAIR_HALF = 0 runs every
 // pair tile as M = 256 (for measurements).
 int pair_half_tiles() { return tuning(MOE_TUNE_PAIR_HALF) != 0 ? 1 : 0; }
+
+// M tiles per band of the CTA-pair tile order (see decode_pair_tile); 0 picks the default.
+int band_of(int knob) {
+  const int v = (int)tuning(knob);
+  return v > 0 ? v : 1;
+}
 
 bool use_pair_kernel(int T) {
   const int64_t v = tuning(MOE_TUNE_GEMM_PAIR);
@@ -1191,6 +1454,7 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   const uint64_t rows = (uint64_t)T * K + BM;   // x_perm / h / y_perm allocation rows
   CUtensorMap mx, mwgu, mwgu64, mh, mwd;
+  AMaps ax, ah;
   int rc;
   // A of the gate/up GEMM: the permuted rows, or the token rows gathered through perm_token
   if (x_perm) {
@@ -1203,6 +1467,9 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   if (pair && (rc = make_map(&mwgu64, w_gate_up, (uint64_t)n_ffn * 2 * I, H, 64)) != MOE_OK)
     return rc;
   if ((rc = make_map(&mh, h, rows, I)) != MOE_OK) return rc;
+  if (pair && ((rc = make_amaps(&ax, x_perm, rows, H)) != MOE_OK ||
+               (rc = make_amaps(&ah, h, rows, I)) != MOE_OK))
+    return rc;
   if ((rc = make_map(&mwd, w_down, (uint64_t)n_ffn * H, I)) != MOE_OK) return rc;
 
   GemmArgs g1{};
@@ -1222,8 +1489,9 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g1.ksplit = 1;
   g1.kb_per_split = g1.kblocks;
   g1.half_tiles = pair ? pair_half_tiles() : 0;
+  g1.band = band_of(MOE_TUNE_GATE_UP_BAND);
   g1.test_stall = take_test_stall() ? 1 : 0;
-  if ((rc = pair ? launch_pair(mx, mwgu, mwgu64, g1, sm_count, st)
+  if ((rc = pair ? launch_pair(ax, mwgu, mwgu64, g1, sm_count, st)
                  : launch_one(mx, mwgu, g1, sm_count, st)) != MOE_OK)
     return rc;
 
@@ -1245,7 +1513,8 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g2.ksplit = 1;
   g2.kb_per_split = g2.kblocks;
   g2.half_tiles = pair ? pair_half_tiles() : 0;
-  return pair ? launch_pair(mh, mwd, mwd, g2, sm_count, st)
+  g2.band = band_of(MOE_TUNE_DOWN_BAND);
+  return pair ? launch_pair(ah, mwd, mwd, g2, sm_count, st)
               : launch_one(mh, mwd, g2, sm_count, st);
 }
 
@@ -1256,10 +1525,12 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
   const uint64_t rows = (uint64_t)T * K + BM;
   const bool pair = use_pair_kernel(T);
   CUtensorMap mx, mwgu, mwgu64;
+  AMaps ax;
   int rc;
   if ((rc = make_map(&mx, x_perm, rows, H)) != MOE_OK) return rc;
   if ((rc = make_map(&mwgu, w_gate_up, (uint64_t)n_ffn * 2 * I, H)) != MOE_OK) return rc;
-  if (pair && (rc = make_map(&mwgu64, w_gate_up, (uint64_t)n_ffn * 2 * I, H, 64)) != MOE_OK)
+  if (pair && ((rc = make_map(&mwgu64, w_gate_up, (uint64_t)n_ffn * 2 * I, H, 64)) != MOE_OK ||
+               (rc = make_amaps(&ax, x_perm, rows, H)) != MOE_OK))
     return rc;
   GemmArgs g{};
   g.mode = kGateUp;
@@ -1277,7 +1548,7 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
   g.ksplit = 1;
   g.kb_per_split = g.kblocks;
   g.half_tiles = pair ? pair_half_tiles() : 0;
-  return pair ? launch_pair(mx, mwgu, mwgu64, g, sm_count, st)
+  return pair ? launch_pair(ax, mwgu, mwgu64, g, sm_count, st)
               : launch_one(mx, mwgu, g, sm_count, st);
 }
 
@@ -1293,9 +1564,10 @@ int launch_dgrad_pair(int mode_dx, const void* a_rows, int a_cols, const void* w
                       int n_ffn, int* status, int sm_count, cudaStream_t st) {
   if (get_encoder() != MOE_OK) return MOE_ERR_CUDA;
   const uint64_t rows = (uint64_t)T * K + BM;   // row buffers' allocation rows
-  CUtensorMap ma, mb;
+  AMaps ma;
+  CUtensorMap mb;
   int rc;
-  if ((rc = make_map(&ma, a_rows, rows, (uint64_t)a_cols)) != MOE_OK) return rc;
+  if ((rc = make_amaps(&ma, a_rows, rows, (uint64_t)a_cols)) != MOE_OK) return rc;
   if ((rc = make_map(&mb, w, (uint64_t)n_ffn * b_rows, (uint64_t)n, 64)) != MOE_OK) return rc;
   GemmArgs g{};
   g.mode = mode_dx ? kDgradDX : kDgradDH;

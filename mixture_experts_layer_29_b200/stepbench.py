@@ -36,10 +36,16 @@ def main(argv=None) -> int:
     ap.add_argument("--zero-experts", type=int, default=None)
     ap.add_argument("--gather", action="store_true",
                     help="no permuted copy of x: the gate/up GEMM gathers the token rows")
+    ap.add_argument("--tune", action="append", default=[], metavar="KNOB=VALUE",
+                    help="moe_set_tuning switch by its abi.TUNE_* name without the prefix, "
+                         "e.g. --tune GATE_UP_BAND=8 (repeatable)")
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     a = ap.parse_args(argv)
 
+    for kv in a.tune:
+        k, v = kv.split("=")
+        abi.set_tuning(getattr(abi, "TUNE_" + k.upper()), int(v))
     cfg = wl.CONFIGS[a.workload]
     kw = {k: v for k, v in (("T", a.tokens), ("n_ffn", a.ffn_experts),
                             ("n_zero", a.zero_experts)) if v is not None}

@@ -127,3 +127,54 @@ def test_odd_fp32_shape_layer_matches_oracle(cuda_device, name, combine):
     same = np.all(np.sort(gh.host(b.topk_idx), 1) == np.sort(r.topk_idx, 1), axis=1)
     err = gh.row_rel_err(gh.host(out)[: cfg.T][same], o_out[same])
     assert err <= gh.TOL["fp32"], err
+
+
+@pytest.mark.parametrize("bands", [(3, 5, 1, 1, 1), (8, 1, 0, 0, 1), (64, 64, 1, 0, 1),
+                                   (1, 8, 0, 1, 1), (1, 1, 0, 0, 1), (1, 1, 0, 1, 0)])
+def test_tile_order_changes_no_bits(cuda_device, bands):
+    """The CTA-pair GEMMs visit an expert's M tiles in bands (MOE_TUNE_GATE_UP_BAND /
+    MOE_TUNE_DOWN_BAND) and spread the tiles of single-tile experts among the others
+    (MOE_TUNE_PAIR_INTERLEAVE), and load only the A rows of the group (MOE_TUNE_PAIR_A_TRIM;
+    the MMA rows past the group see stale shared memory and are dropped). Every output
+    tile is still one cluster's, summed over K in the same order from the same rows, so
+    any setting gives the same bits as the default one; with the largest expert holding
+    thousands of rows (a dozen M tiles) and several experts of one tile, the settings here
+    cut it into full and partial bands, with and without the spread and the trim. Swapped
+    tiles of at most 128 rows (MOE_TUNE_PAIR_SWAP_AB) against M = 128 tiles are other MMA
+    shapes, so other fp32 summation orders: those two agree within rounding."""
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=3001)
+    case = gh.Case(cfg, seed=21)
+    b = case.buffers("deterministic")
+    args = (b, case.x, case.w.w_router, None, case.w.bias, case.w.w_gate_up, case.w.w_down)
+    abi.run_steps(*args)
+    torch.cuda.synchronize()
+    R = int(b.offsets[-1].item())
+    counts = b.counts[: cfg.n_ffn]
+    assert int(counts.max().item()) > 6 * 256
+    assert int(((counts > 0) & (counts <= 256)).sum().item()) >= 3     # single-tile experts
+    want = [b.h[:R].clone(), b.y_perm[:R].clone(), b.out.clone()]
+    try:
+        abi.set_tuning(abi.TUNE_GATE_UP_BAND, bands[0])
+        abi.set_tuning(abi.TUNE_DOWN_BAND, bands[1])
+        abi.set_tuning(abi.TUNE_PAIR_INTERLEAVE, bands[2])
+        abi.set_tuning(abi.TUNE_PAIR_A_TRIM, bands[3])
+        abi.set_tuning(abi.TUNE_PAIR_SWAP_AB, bands[4])
+        for t in (b.h, b.y_perm, b.out):
+            t.zero_()
+        abi.run_steps(*args)
+        torch.cuda.synchronize()
+    finally:
+        abi.set_tuning(abi.TUNE_GATE_UP_BAND, 0)
+        abi.set_tuning(abi.TUNE_DOWN_BAND, 0)
+        abi.set_tuning(abi.TUNE_PAIR_INTERLEAVE, 0)
+        abi.set_tuning(abi.TUNE_PAIR_A_TRIM, 1)
+        abi.set_tuning(abi.TUNE_PAIR_SWAP_AB, 1)
+    assert abi.read_device_status(b.ws) == 0
+    same = [torch.equal(w_, g_) for w_, g_ in zip(want, [b.h[:R], b.y_perm[:R], b.out])]
+    if bands[4]:
+        assert all(same)
+    else:
+        # M = 128 tiles instead of swapped ones: other MMA shapes, so other fp32 summation
+        # orders in the tensor cores; both must stay within rounding of each other
+        for w_, g_ in zip(want, [b.h[:R], b.y_perm[:R], b.out]):
+            assert gh.row_rel_err(gh.host(g_), gh.host(w_)) < 1e-2
