@@ -151,6 +151,9 @@ uint64_t moe_launch_count(void);
  *                             the operands swapped: the expert's weights as the M = 256
  *                             side, the tile's rows (rounded up to 16, 32, 64 or 128) as
  *                             N; 0: such tiles run as M = 128 tiles.
+ *   MOE_TUNE_PAIR_STREAM_HINT 1 (default): the CTA-pair GEMMs load the weights of experts
+ *                             with at most 256 rows (read once) with an evict-first L2
+ *                             policy; 0: plain loads.
  * moe_set_tuning returns MOE_ERR_INVALID_ARG for an unknown switch or a value outside its
  * range. moe_get_tuning writes the current value. */
 typedef enum {
@@ -166,7 +169,8 @@ typedef enum {
   MOE_TUNE_DOWN_BAND = 9,
   MOE_TUNE_PAIR_INTERLEAVE = 10,
   MOE_TUNE_PAIR_A_TRIM = 11,
-  MOE_TUNE_PAIR_SWAP_AB = 12
+  MOE_TUNE_PAIR_SWAP_AB = 12,
+  MOE_TUNE_PAIR_STREAM_HINT = 13
 } moe_tune_t;
 
 int moe_set_tuning(int knob, int64_t value);

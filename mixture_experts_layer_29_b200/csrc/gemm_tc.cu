@@ -109,6 +109,7 @@ struct GemmArgs {
   int interleave;             // pair kernel: spread single-tile experts' tiles (see below)
   int a_trim;                 // pair kernel: load only the A rows of the group (a_box_rows)
   int swap_ab;                // pair kernel, forward: tiles of <= 128 rows run swapped (swap_npad)
+  int stream_hint;            // pair kernel: single-tile experts' weights loaded evict-first
 };
 
 // The testing hook of GemmArgs::test_stall: this (tile, k-block) is not loaded.
@@ -1002,6 +1003,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      const uint64_t policy = l2_evict_first_policy();
       for (int tile = cluster; tile < total_tiles && !*abort_flag; tile += nclusters) {
         const Tile t = decode_pair_tile(s, g, tile);
         const int npad = swap_npad(g, t);                  // swap tile: npad / 2 rows per CTA
@@ -1015,6 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    : t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM;
         // MN-major B (dgrad): this CTA's 128 N columns as two 64 x 64 boxes of K rows
         const int bcol = t.nt * BN + 128 * (int)rank;
+        const bool stream = g.stream_hint && !b_mn && t.row_end - s.offs[t.e] <= BMP;
         const int a_rows = npad ? npad / 2 : a_box_rows(g, t, half, (int)rank);
         const CUtensorMap* a_map = a_rows == 128 ? &tmA : a_rows == 64 ? &tmA64
                                  : a_rows == 32 ? &tmA32 : a_rows == 16 ? &tmA16 : &tmA8;
@@ -1038,6 +1041,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int y = t.e * g.b_rows + kb * BK;
             tma_load_2d_pair(s.b[stage], &tmB, bcol, y, full_leader);
             tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB, bcol + 64, y, full_leader);
+          } else if (stream) {
+            // an expert of one M tile: its weights are read once, so they leave L2 first
+            if (split_b) {
+              tma_load_2d_pair_hint(s.b[stage], &tmB64, kb * BK, brow, full_leader, policy);
+              tma_load_2d_pair_hint(s.b[stage] + P_B_BYTES / 2, &tmB64, kb * BK,
+                                    brow + g.b_second, full_leader, policy);
+            } else {
+              tma_load_2d_pair_hint(s.b[stage], &tmB, kb * BK, brow, full_leader, policy);
+            }
           } else if (split_b) {
             tma_load_2d_pair(s.b[stage], &tmB64, kb * BK, brow, full_leader);
             tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB64, kb * BK, brow + g.b_second,
@@ -1261,6 +1273,7 @@ int launch_pair(const AMaps& ma, const CUtensorMap& mb, const CUtensorMap& mb64,
   ga.a_trim = tuning(MOE_TUNE_PAIR_A_TRIM) != 0 ? 1 : 0;
   ga.swap_ab = (g.mode != kDgradDH && g.mode != kDgradDX && tuning(MOE_TUNE_PAIR_SWAP_AB) != 0)
                    ? 1 : 0;
+  ga.stream_hint = tuning(MOE_TUNE_PAIR_STREAM_HINT) != 0 ? 1 : 0;
   if (launch_kernel(kern, 2 * nclusters, kThreads, smem, st, 2, ma.m128, ma.m64, ma.m32, ma.m16,
                     ma.m8, mb, mb64, ga) != cudaSuccess) {
     cudaGetLastError();

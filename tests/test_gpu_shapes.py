@@ -129,13 +129,14 @@ def test_odd_fp32_shape_layer_matches_oracle(cuda_device, name, combine):
     assert err <= gh.TOL["fp32"], err
 
 
-@pytest.mark.parametrize("bands", [(3, 5, 1, 1, 1), (8, 1, 0, 0, 1), (64, 64, 1, 0, 1),
-                                   (1, 8, 0, 1, 1), (1, 1, 0, 0, 1), (1, 1, 0, 1, 0)])
+@pytest.mark.parametrize("bands", [(3, 5, 1, 1, 1, 1), (8, 1, 0, 0, 1, 0), (64, 64, 1, 0, 1, 1),
+                                   (1, 8, 0, 1, 1, 0), (1, 1, 0, 0, 1, 1), (1, 1, 0, 1, 0, 0)])
 def test_tile_order_changes_no_bits(cuda_device, bands):
     """The CTA-pair GEMMs visit an expert's M tiles in bands (MOE_TUNE_GATE_UP_BAND /
     MOE_TUNE_DOWN_BAND) and spread the tiles of single-tile experts among the others
-    (MOE_TUNE_PAIR_INTERLEAVE), and load only the A rows of the group (MOE_TUNE_PAIR_A_TRIM;
-    the MMA rows past the group see stale shared memory and are dropped). Every output
+    (MOE_TUNE_PAIR_INTERLEAVE), load only the A rows of the group (MOE_TUNE_PAIR_A_TRIM;
+    the MMA rows past the group see stale shared memory and are dropped), and may load
+    single-tile experts' weights evict-first (MOE_TUNE_PAIR_STREAM_HINT). Every output
     tile is still one cluster's, summed over K in the same order from the same rows, so
     any setting gives the same bits as the default one; with the largest expert holding
     thousands of rows (a dozen M tiles) and several experts of one tile, the settings here
@@ -159,6 +160,7 @@ def test_tile_order_changes_no_bits(cuda_device, bands):
         abi.set_tuning(abi.TUNE_PAIR_INTERLEAVE, bands[2])
         abi.set_tuning(abi.TUNE_PAIR_A_TRIM, bands[3])
         abi.set_tuning(abi.TUNE_PAIR_SWAP_AB, bands[4])
+        abi.set_tuning(abi.TUNE_PAIR_STREAM_HINT, bands[5])
         for t in (b.h, b.y_perm, b.out):
             t.zero_()
         abi.run_steps(*args)
@@ -169,6 +171,7 @@ def test_tile_order_changes_no_bits(cuda_device, bands):
         abi.set_tuning(abi.TUNE_PAIR_INTERLEAVE, 0)
         abi.set_tuning(abi.TUNE_PAIR_A_TRIM, 1)
         abi.set_tuning(abi.TUNE_PAIR_SWAP_AB, 1)
+        abi.set_tuning(abi.TUNE_PAIR_STREAM_HINT, 1)
     assert abi.read_device_status(b.ws) == 0
     same = [torch.equal(w_, g_) for w_, g_ in zip(want, [b.h[:R], b.y_perm[:R], b.out])]
     if bands[4]:
