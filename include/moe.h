@@ -154,6 +154,11 @@ uint64_t moe_launch_count(void);
  *   MOE_TUNE_PAIR_STREAM_HINT 1 (default): the CTA-pair GEMMs load the weights of experts
  *                             with at most 256 rows (read once) with an evict-first L2
  *                             policy; 0: plain loads.
+ *   MOE_TUNE_PAIR_TAILS       0 (default): the pair kernel takes every row; 1: where the
+ *                             forward's expert GEMMs use CTA pairs, each runs as two
+ *                             launches: the pair kernel takes every expert's whole 256-row
+ *                             tiles (and a last tile of more than 128 rows), the one-CTA
+ *                             kernel the rest (at most 128 rows per expert).
  * moe_set_tuning returns MOE_ERR_INVALID_ARG for an unknown switch or a value outside its
  * range. moe_get_tuning writes the current value. */
 typedef enum {
@@ -170,7 +175,8 @@ typedef enum {
   MOE_TUNE_PAIR_INTERLEAVE = 10,
   MOE_TUNE_PAIR_A_TRIM = 11,
   MOE_TUNE_PAIR_SWAP_AB = 12,
-  MOE_TUNE_PAIR_STREAM_HINT = 13
+  MOE_TUNE_PAIR_STREAM_HINT = 13,
+  MOE_TUNE_PAIR_TAILS = 14
 } moe_tune_t;
 
 int moe_set_tuning(int knob, int64_t value);

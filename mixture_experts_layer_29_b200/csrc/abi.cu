@@ -18,9 +18,9 @@ void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_r
 
 // Process-wide tuning switches (moe_set_tuning), each at its default until changed.
 namespace {
-constexpr int kTuneCount = MOE_TUNE_PAIR_STREAM_HINT + 1;
+constexpr int kTuneCount = MOE_TUNE_PAIR_TAILS + 1;
 std::atomic<int64_t> g_tune[kTuneCount] = {{1}, {-1}, {1}, {0}, {12}, {1}, {4}, {0}, {0}, {0}, {0}, {1},
-                                           {1}, {1}};
+                                           {1}, {1}, {0}};
 
 bool tune_value_ok(int knob, int64_t v) {
   switch (knob) {
@@ -31,6 +31,7 @@ bool tune_value_ok(int knob, int64_t v) {
     case MOE_TUNE_PAIR_A_TRIM:
     case MOE_TUNE_PAIR_SWAP_AB:
     case MOE_TUNE_PAIR_STREAM_HINT:
+    case MOE_TUNE_PAIR_TAILS:
     case MOE_TUNE_TEST_STALL: return v == 0 || v == 1;
     case MOE_TUNE_GEMM_PAIR: return v >= -1 && v <= 1;
     case MOE_TUNE_ROUTER_N: return v == 0 || v == 192 || v == 256;

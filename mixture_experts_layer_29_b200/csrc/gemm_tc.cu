@@ -110,7 +110,19 @@ struct GemmArgs {
   int a_trim;                 // pair kernel: load only the A rows of the group (a_box_rows)
   int swap_ab;                // pair kernel, forward: tiles of <= 128 rows run swapped (swap_npad)
   int stream_hint;            // pair kernel: single-tile experts' weights loaded evict-first
+  int row_split;              // 0: every row of each expert; 1: its pair rows only (pair
+                              // kernel); 2: the rest of them (one-CTA kernel): see pair_rows
 };
+
+// The rows of an expert's group that the CTA-pair GEMM takes when the forward is split
+// between the two kernels (GemmArgs::row_split): whole 256-row tiles, plus the last partial
+// tile when it holds more than 128 rows. The rest, at most 128 rows (a small expert, or a
+// large expert's tail), goes to the one-CTA kernel as one 128-row tile: a pair tile of few
+// rows holds two SMs for as long as a full one, the one-CTA tile holds one.
+__device__ __forceinline__ int pair_rows(int count) {
+  const int r = count & 255;
+  return r <= 128 ? count - r : count;
+}
 
 // The testing hook of GemmArgs::test_stall: this (tile, k-block) is not loaded.
 __device__ __forceinline__ bool stalled_stage(const GemmArgs& g, int tile, int kb, int kb0) {
@@ -137,7 +149,8 @@ __device__ __forceinline__ Tile decode_tile(const SharedStorage& s, const GemmAr
     if (s.toff[mid] <= mt) lo = mid; else hi = mid - 1;
   }
   t.e = lo;
-  t.row0 = s.offs[lo] + (mt - s.toff[lo]) * BM;
+  const int begin = g.row_split == 2 ? s.offs[lo] + pair_rows(s.offs[lo + 1] - s.offs[lo]) : s.offs[lo];
+  t.row0 = begin + (mt - s.toff[lo]) * BM;
   t.row_end = s.offs[lo + 1];
   return t;
 }
@@ -405,14 +418,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int per = (g.n_ffn + 31) / 32;
     const int b = lane * per;
     int local = 0;
+    // M tiles of expert e: all of its rows, or (row_split == 2) the rows the pair kernel leaves
+    auto tiles_of = [&](int e) {
+      int rows = s.offs[e + 1] - s.offs[e];
+      if (g.row_split == 2) rows -= pair_rows(rows);
+      return (rows + BM - 1) / BM;
+    };
     for (int i = 0; i < per; ++i)
-      if (b + i < g.n_ffn) local += (s.offs[b + i + 1] - s.offs[b + i] + BM - 1) / BM;
+      if (b + i < g.n_ffn) local += tiles_of(b + i);
     const int inc = warp_inclusive_scan(local);
     int run = inc - local;
     for (int i = 0; i < per; ++i)
       if (b + i < g.n_ffn) {
         s.toff[b + i] = run;
-        run += (s.offs[b + i + 1] - s.offs[b + i] + BM - 1) / BM;
+        run += tiles_of(b + i);
       }
     if (lane == 31) s.toff[g.n_ffn] = inc;
   }
@@ -670,6 +689,11 @@ static_assert(offsetof(PairStorage, epi_stage) % 16 == 0, "16-byte staging rows"
 static_assert(offsetof(PairStorage, a) % 1024 == 0 && offsetof(PairStorage, b) % 1024 == 0,
               "128-byte-swizzled TMA boxes need 1024-byte alignment");
 
+// End of expert e's rows in the CTA-pair kernel (its pair rows when the forward is split).
+__device__ __forceinline__ int pair_end(const PairStorage& s, const GemmArgs& g, int e) {
+  return g.row_split == 1 ? s.offs[e] + pair_rows(s.offs[e + 1] - s.offs[e]) : s.offs[e + 1];
+}
+
 // Tile order of the CTA-pair kernel. Tiles are handed out round-robin in this order, so
 // the order is also roughly the time at which a tile runs.
 //  * Experts of a single M tile (at most 256 rows; g.interleave) stream their whole weight
@@ -698,7 +722,7 @@ __device__ __forceinline__ Tile decode_pair_tile(const PairStorage& s, const Gem
       t.nt = ns0 - k * g.n_tiles;
       t.e = e;
       t.row0 = s.offs[e];
-      t.row_end = s.offs[e + 1];
+      t.row_end = pair_end(s, g, e);
       return t;
     }
     tile -= ns0;                                        // the tile-th L tile
@@ -724,7 +748,7 @@ __device__ __forceinline__ Tile decode_pair_tile(const PairStorage& s, const Gem
   }
   t.e = lo;
   t.row0 = s.offs[lo] + mt * BMP;
-  t.row_end = s.offs[lo + 1];
+  t.row_end = pair_end(s, g, lo);
   return t;
 }
 
@@ -970,9 +994,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int per = (g.n_ffn + 31) / 32;
     const int b = lane * per;
     int local = 0, nsingle = 0;
+    auto tiles_of = [&](int e) {
+      int rows = s.offs[e + 1] - s.offs[e];
+      if (g.row_split == 1) rows = pair_rows(rows);
+      return (rows + BMP - 1) / BMP;
+    };
     for (int i = 0; i < per; ++i)
       if (b + i < g.n_ffn) {
-        const int m = (s.offs[b + i + 1] - s.offs[b + i] + BMP - 1) / BMP;
+        const int m = tiles_of(b + i);
         if (g.interleave && m == 1) ++nsingle;
         else local += m;
       }
@@ -982,7 +1011,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < per; ++i)
       if (b + i < g.n_ffn) {
         s.toff[b + i] = run;
-        const int m = (s.offs[b + i + 1] - s.offs[b + i] + BMP - 1) / BMP;
+        const int m = tiles_of(b + i);
         if (g.interleave && m == 1) s.single[srun++] = (int16_t)(b + i);
         else run += m;
       }
@@ -1504,9 +1533,21 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g1.half_tiles = pair ? pair_half_tiles() : 0;
   g1.band = band_of(MOE_TUNE_GATE_UP_BAND);
   g1.test_stall = take_test_stall() ? 1 : 0;
-  if ((rc = pair ? launch_pair(ax, mwgu, mwgu64, g1, sm_count, st)
-                 : launch_one(mx, mwgu, g1, sm_count, st)) != MOE_OK)
+  // CTA pairs: an expert's whole 256-row tiles on the pair kernel, the rest of its rows
+  // (at most 128) on the one-CTA kernel (pair_rows), each GEMM as two launches
+  const bool split = pair && tuning(MOE_TUNE_PAIR_TAILS) != 0;
+  if (split) {
+    g1.row_split = 1;
+    if ((rc = launch_pair(ax, mwgu, mwgu64, g1, sm_count, st)) != MOE_OK) return rc;
+    GemmArgs t1 = g1;
+    t1.row_split = 2;
+    t1.half_tiles = 0;
+    t1.test_stall = 0;
+    if ((rc = launch_one(mx, mwgu, t1, sm_count, st)) != MOE_OK) return rc;
+  } else if ((rc = pair ? launch_pair(ax, mwgu, mwgu64, g1, sm_count, st)
+                        : launch_one(mx, mwgu, g1, sm_count, st)) != MOE_OK) {
     return rc;
+  }
 
   GemmArgs g2{};
   g2.mode = fused ? kDownAtomic : kDownStore;
@@ -1527,6 +1568,14 @@ int launch_grouped_ffn_tc(const void* x, const void* x_perm, const int32_t* offs
   g2.kb_per_split = g2.kblocks;
   g2.half_tiles = pair ? pair_half_tiles() : 0;
   g2.band = band_of(MOE_TUNE_DOWN_BAND);
+  if (split) {
+    g2.row_split = 1;
+    if ((rc = launch_pair(ah, mwd, mwd, g2, sm_count, st)) != MOE_OK) return rc;
+    GemmArgs t2 = g2;
+    t2.row_split = 2;
+    t2.half_tiles = 0;
+    return launch_one(mh, mwd, t2, sm_count, st);
+  }
   return pair ? launch_pair(ah, mwd, mwd, g2, sm_count, st)
               : launch_one(mh, mwd, g2, sm_count, st);
 }
@@ -1561,6 +1610,14 @@ int launch_gate_up_raw(const void* x_perm, const int32_t* offsets, const void* w
   g.ksplit = 1;
   g.kb_per_split = g.kblocks;
   g.half_tiles = pair ? pair_half_tiles() : 0;
+  // the same split as the forward, so that G | U come out with the forward's bits
+  if (pair && tuning(MOE_TUNE_PAIR_TAILS) != 0) {
+    g.row_split = 1;
+    if ((rc = launch_pair(ax, mwgu, mwgu64, g, sm_count, st)) != MOE_OK) return rc;
+    g.row_split = 2;
+    g.half_tiles = 0;
+    return launch_one(mx, mwgu, g, sm_count, st);
+  }
   return pair ? launch_pair(ax, mwgu, mwgu64, g, sm_count, st)
               : launch_one(mx, mwgu, g, sm_count, st);
 }

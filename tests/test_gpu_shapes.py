@@ -129,8 +129,10 @@ def test_odd_fp32_shape_layer_matches_oracle(cuda_device, name, combine):
     assert err <= gh.TOL["fp32"], err
 
 
-@pytest.mark.parametrize("bands", [(3, 5, 1, 1, 1, 1), (8, 1, 0, 0, 1, 0), (64, 64, 1, 0, 1, 1),
-                                   (1, 8, 0, 1, 1, 0), (1, 1, 0, 0, 1, 1), (1, 1, 0, 1, 0, 0)])
+@pytest.mark.parametrize("bands", [(3, 5, 1, 1, 1, 1, 0), (8, 1, 0, 0, 1, 0, 0),
+                                   (64, 64, 1, 0, 1, 1, 0), (1, 8, 0, 1, 1, 0, 0),
+                                   (1, 1, 0, 0, 1, 1, 0), (1, 1, 0, 1, 0, 0, 0),
+                                   (1, 1, 0, 1, 1, 1, 1)])
 def test_tile_order_changes_no_bits(cuda_device, bands):
     """The CTA-pair GEMMs visit an expert's M tiles in bands (MOE_TUNE_GATE_UP_BAND /
     MOE_TUNE_DOWN_BAND) and spread the tiles of single-tile experts among the others
@@ -141,8 +143,9 @@ def test_tile_order_changes_no_bits(cuda_device, bands):
     any setting gives the same bits as the default one; with the largest expert holding
     thousands of rows (a dozen M tiles) and several experts of one tile, the settings here
     cut it into full and partial bands, with and without the spread and the trim. Swapped
-    tiles of at most 128 rows (MOE_TUNE_PAIR_SWAP_AB) against M = 128 tiles are other MMA
-    shapes, so other fp32 summation orders: those two agree within rounding."""
+    tiles of at most 128 rows (MOE_TUNE_PAIR_SWAP_AB) against M = 128 tiles, and such rows
+    on the one-CTA kernel (MOE_TUNE_PAIR_TAILS), are other MMA shapes, so other fp32
+    summation orders: those agree within rounding."""
     cfg = wl.CONFIGS["proxy_bf16"].with_(T=3001)
     case = gh.Case(cfg, seed=21)
     b = case.buffers("deterministic")
@@ -161,6 +164,7 @@ def test_tile_order_changes_no_bits(cuda_device, bands):
         abi.set_tuning(abi.TUNE_PAIR_A_TRIM, bands[3])
         abi.set_tuning(abi.TUNE_PAIR_SWAP_AB, bands[4])
         abi.set_tuning(abi.TUNE_PAIR_STREAM_HINT, bands[5])
+        abi.set_tuning(abi.TUNE_PAIR_TAILS, bands[6])
         for t in (b.h, b.y_perm, b.out):
             t.zero_()
         abi.run_steps(*args)
@@ -172,9 +176,10 @@ def test_tile_order_changes_no_bits(cuda_device, bands):
         abi.set_tuning(abi.TUNE_PAIR_A_TRIM, 1)
         abi.set_tuning(abi.TUNE_PAIR_SWAP_AB, 1)
         abi.set_tuning(abi.TUNE_PAIR_STREAM_HINT, 1)
+        abi.set_tuning(abi.TUNE_PAIR_TAILS, 0)
     assert abi.read_device_status(b.ws) == 0
     same = [torch.equal(w_, g_) for w_, g_ in zip(want, [b.h[:R], b.y_perm[:R], b.out])]
-    if bands[4]:
+    if bands[4] and not bands[6]:
         assert all(same)
     else:
         # M = 128 tiles instead of swapped ones: other MMA shapes, so other fp32 summation
