@@ -159,6 +159,10 @@ uint64_t moe_launch_count(void);
  *                             launches: the pair kernel takes every expert's whole 256-row
  *                             tiles (and a last tile of more than 128 rows), the one-CTA
  *                             kernel the rest (at most 128 rows per expert).
+ *   MOE_TUNE_PAIR_PREFETCH    0 (default): no prefetch; 1 to 64: for the tiles of experts with
+ *                             at most 256 rows, the CTA-pair GEMMs' producer prefetches into
+ *                             L2 the weight boxes it will load this many k-blocks later
+ *                             (crossing into its next tile).
  * moe_set_tuning returns MOE_ERR_INVALID_ARG for an unknown switch or a value outside its
  * range. moe_get_tuning writes the current value. */
 typedef enum {
@@ -176,7 +180,8 @@ typedef enum {
   MOE_TUNE_PAIR_A_TRIM = 11,
   MOE_TUNE_PAIR_SWAP_AB = 12,
   MOE_TUNE_PAIR_STREAM_HINT = 13,
-  MOE_TUNE_PAIR_TAILS = 14
+  MOE_TUNE_PAIR_TAILS = 14,
+  MOE_TUNE_PAIR_PREFETCH = 15
 } moe_tune_t;
 
 int moe_set_tuning(int knob, int64_t value);

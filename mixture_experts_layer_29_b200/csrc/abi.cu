@@ -18,9 +18,9 @@ void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_r
 
 // Process-wide tuning switches (moe_set_tuning), each at its default until changed.
 namespace {
-constexpr int kTuneCount = MOE_TUNE_PAIR_TAILS + 1;
+constexpr int kTuneCount = MOE_TUNE_PAIR_PREFETCH + 1;
 std::atomic<int64_t> g_tune[kTuneCount] = {{1}, {-1}, {1}, {0}, {12}, {1}, {4}, {0}, {0}, {0}, {0}, {1},
-                                           {1}, {1}, {0}};
+                                           {1}, {1}, {0}, {0}};
 
 bool tune_value_ok(int knob, int64_t v) {
   switch (knob) {
@@ -38,7 +38,8 @@ bool tune_value_ok(int knob, int64_t v) {
     case MOE_TUNE_ROUTER_MIN_SPLIT: return v >= 1 && v <= 1024;
     case MOE_TUNE_BWD_DY_ROWS: return v == 1 || v == 4;
     case MOE_TUNE_GATE_UP_BAND:
-    case MOE_TUNE_DOWN_BAND: return v >= 0 && v <= 64;
+    case MOE_TUNE_DOWN_BAND:
+    case MOE_TUNE_PAIR_PREFETCH: return v >= 0 && v <= 64;
     default: return false;
   }
 }

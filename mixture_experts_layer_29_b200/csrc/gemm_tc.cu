@@ -110,6 +110,7 @@ struct GemmArgs {
   int a_trim;                 // pair kernel: load only the A rows of the group (a_box_rows)
   int swap_ab;                // pair kernel, forward: tiles of <= 128 rows run swapped (swap_npad)
   int stream_hint;            // pair kernel: single-tile experts' weights loaded evict-first
+  int prefetch;               // pair kernel: L2 prefetch of the boxes this many k-blocks ahead
   int row_split;              // 0: every row of each expert; 1: its pair rows only (pair
                               // kernel); 2: the rest of them (one-CTA kernel): see pair_rows
 };
@@ -936,6 +937,51 @@ __device__ __forceinline__ void epilogue_pair(const GemmArgs& g, const Tile& t, 
   }
 }
 
+// What the producer of CTA `rank` loads for a pair tile: its A box (rows and tensor map) and
+// its B half (rows or, MN-major, columns).
+struct PairPlan {
+  int arow, a_rows, brow, bcol;
+  bool split_b, stream;
+  const CUtensorMap* a_map;
+};
+
+__device__ __forceinline__ PairPlan pair_plan(const PairStorage& s, const GemmArgs& g,
+                                              const Tile& t, int rank, bool b_mn,
+                                              const CUtensorMap* mA, const CUtensorMap* mA64,
+                                              const CUtensorMap* mA32, const CUtensorMap* mA16,
+                                              const CUtensorMap* mA8) {
+  PairPlan p;
+  const int npad = swap_npad(g, t);                  // swap tile: npad / 2 rows per CTA
+  const bool half = !npad && half_tile(g, t);
+  p.split_b = (half || npad) && g.mode == kGateUp;   // 64 gate + 64 up rows
+  p.arow = npad ? t.row0 + (npad / 2) * rank : t.row0 + (half ? 64 : 128) * rank;
+  p.brow = g.mode != kGateUp ? t.e * g.b_rows + t.nt * BN + 128 * rank
+           : p.split_b ? t.e * g.b_rows + t.nt * BM + 64 * rank
+                       : t.e * g.b_rows + rank * g.b_second + t.nt * BM;
+  // MN-major B (dgrad): this CTA's 128 N columns as two 64 x 64 boxes of K rows
+  p.bcol = t.nt * BN + 128 * rank;
+  p.stream = g.stream_hint && !b_mn && s.offs[t.e + 1] - s.offs[t.e] <= BMP;
+  p.a_rows = npad ? npad / 2 : a_box_rows(g, t, half, rank);
+  p.a_map = p.a_rows == 128 ? mA : p.a_rows == 64 ? mA64 : p.a_rows == 32 ? mA32
+          : p.a_rows == 16 ? mA16 : mA8;
+  return p;
+}
+
+// The weight boxes pair_plan's loads read for k-block kb of a tile of a single-tile expert
+// (p.stream), brought into L2 g.prefetch k-blocks ahead of the loads. Such tiles stream their
+// weights from DRAM with six stages in flight and wait on DRAM latency; the other tiles find
+// their operands in L2 and keep the SM's TMA unit busy, so they prefetch nothing.
+__device__ __forceinline__ void pair_prefetch(const PairPlan& p, const GemmArgs& g, int kb,
+                                              const CUtensorMap* mB, const CUtensorMap* mB64) {
+  if (!p.stream) return;
+  if (p.split_b) {
+    tma_prefetch_2d(mB64, kb * BK, p.brow);
+    tma_prefetch_2d(mB64, kb * BK, p.brow + g.b_second);
+  } else {
+    tma_prefetch_2d(mB, kb * BK, p.brow);
+  }
+}
+
 // tmB64: the gate/up B tensor with 64-row boxes (half tiles); unused by the down GEMM.
 // KIND: kPairFwd, kPairFwdKeep or kPairDgrad (see epilogue_pair), so that the plain
 // forward carries none of the other kinds' code.
@@ -1033,27 +1079,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       const uint64_t policy = l2_evict_first_policy();
+      constexpr bool b_mn = KIND == kPairDgrad;
+      const int pf = g.prefetch;
       for (int tile = cluster; tile < total_tiles && !*abort_flag; tile += nclusters) {
         const Tile t = decode_pair_tile(s, g, tile);
-        const int npad = swap_npad(g, t);                  // swap tile: npad / 2 rows per CTA
+        const PairPlan p = pair_plan(s, g, t, (int)rank, b_mn, &tmA, &tmA64, &tmA32, &tmA16, &tmA8);
+        const int npad = swap_npad(g, t);
         const bool half = !npad && half_tile(g, t);
-        const bool split_b = (half || npad) && g.mode == kGateUp;   // 64 gate + 64 up rows
-        constexpr bool b_mn = KIND == kPairDgrad;
-        const int arow = npad ? t.row0 + (npad / 2) * (int)rank
-                              : t.row0 + (half ? 64 : 128) * (int)rank;
-        const int brow = g.mode != kGateUp ? t.e * g.b_rows + t.nt * BN + 128 * (int)rank
-                         : split_b ? t.e * g.b_rows + t.nt * BM + 64 * (int)rank
-                                   : t.e * g.b_rows + (int)rank * g.b_second + t.nt * BM;
-        // MN-major B (dgrad): this CTA's 128 N columns as two 64 x 64 boxes of K rows
-        const int bcol = t.nt * BN + 128 * (int)rank;
-        const bool stream = g.stream_hint && !b_mn && t.row_end - s.offs[t.e] <= BMP;
-        const int a_rows = npad ? npad / 2 : a_box_rows(g, t, half, (int)rank);
-        const CUtensorMap* a_map = a_rows == 128 ? &tmA : a_rows == 64 ? &tmA64
-                                 : a_rows == 32 ? &tmA32 : a_rows == 16 ? &tmA16 : &tmA8;
         // the leader expects both CTAs' bytes: B halves of 16 KB and the two A boxes
         const uint32_t tx = 2 * P_B_BYTES +
             (npad ? (uint32_t)npad * BK * 2
                   : (uint32_t)(a_box_rows(g, t, half, 0) + a_box_rows(g, t, half, 1)) * BK * 2);
+        // the cluster's next tile, for prefetches that run past this tile's last k-block
+        const bool has_next = pf > 0 && tile + nclusters < total_tiles;
+        Tile tn = t;
+        PairPlan pn = p;
+        if (has_next) {
+          tn = decode_pair_tile(s, g, tile + nclusters);
+          pn = pair_plan(s, g, tn, (int)rank, b_mn, &tmA, &tmA64, &tmA32, &tmA16, &tmA8);
+        }
+        if (pf > 0 && tile == cluster)
+          for (int kb = 0; kb < pf && kb < g.kblocks; ++kb) pair_prefetch(p, g, kb, &tmB, &tmB64);
         for (int kb = 0; kb < g.kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) break;
           if (stalled_stage(g, tile, kb, 0)) {   // neither CTA loads; nothing is expected
@@ -1065,26 +1111,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], tx);
-          if (a_rows > 0) tma_load_2d_pair(s.a[stage], a_map, kb * BK, arow, full_leader);
+          if (p.a_rows > 0) tma_load_2d_pair(s.a[stage], p.a_map, kb * BK, p.arow, full_leader);
           if (b_mn) {
             const int y = t.e * g.b_rows + kb * BK;
-            tma_load_2d_pair(s.b[stage], &tmB, bcol, y, full_leader);
-            tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB, bcol + 64, y, full_leader);
-          } else if (stream) {
+            tma_load_2d_pair(s.b[stage], &tmB, p.bcol, y, full_leader);
+            tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB, p.bcol + 64, y, full_leader);
+          } else if (p.stream) {
             // an expert of one M tile: its weights are read once, so they leave L2 first
-            if (split_b) {
-              tma_load_2d_pair_hint(s.b[stage], &tmB64, kb * BK, brow, full_leader, policy);
+            if (p.split_b) {
+              tma_load_2d_pair_hint(s.b[stage], &tmB64, kb * BK, p.brow, full_leader, policy);
               tma_load_2d_pair_hint(s.b[stage] + P_B_BYTES / 2, &tmB64, kb * BK,
-                                    brow + g.b_second, full_leader, policy);
+                                    p.brow + g.b_second, full_leader, policy);
             } else {
-              tma_load_2d_pair_hint(s.b[stage], &tmB, kb * BK, brow, full_leader, policy);
+              tma_load_2d_pair_hint(s.b[stage], &tmB, kb * BK, p.brow, full_leader, policy);
             }
-          } else if (split_b) {
-            tma_load_2d_pair(s.b[stage], &tmB64, kb * BK, brow, full_leader);
-            tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB64, kb * BK, brow + g.b_second,
+          } else if (p.split_b) {
+            tma_load_2d_pair(s.b[stage], &tmB64, kb * BK, p.brow, full_leader);
+            tma_load_2d_pair(s.b[stage] + P_B_BYTES / 2, &tmB64, kb * BK, p.brow + g.b_second,
                              full_leader);
           } else {
-            tma_load_2d_pair(s.b[stage], &tmB, kb * BK, brow, full_leader);
+            tma_load_2d_pair(s.b[stage], &tmB, kb * BK, p.brow, full_leader);
+          }
+          if (pf > 0) {
+            const int kp = kb + pf;
+            if (kp < g.kblocks) pair_prefetch(p, g, kp, &tmB, &tmB64);
+            else if (has_next && kp - g.kblocks < g.kblocks)
+              pair_prefetch(pn, g, kp - g.kblocks, &tmB, &tmB64);
           }
           if (++stage == PSTAGES) {
             stage = 0;
@@ -1303,6 +1355,7 @@ int launch_pair(const AMaps& ma, const CUtensorMap& mb, const CUtensorMap& mb64,
   ga.swap_ab = (g.mode != kDgradDH && g.mode != kDgradDX && tuning(MOE_TUNE_PAIR_SWAP_AB) != 0)
                    ? 1 : 0;
   ga.stream_hint = tuning(MOE_TUNE_PAIR_STREAM_HINT) != 0 ? 1 : 0;
+  ga.prefetch = (int)tuning(MOE_TUNE_PAIR_PREFETCH);
   if (launch_kernel(kern, 2 * nclusters, kThreads, smem, st, 2, ma.m128, ma.m64, ma.m32, ma.m16,
                     ma.m8, mb, mb64, ga) != cudaSuccess) {
     cudaGetLastError();

@@ -129,10 +129,10 @@ def test_odd_fp32_shape_layer_matches_oracle(cuda_device, name, combine):
     assert err <= gh.TOL["fp32"], err
 
 
-@pytest.mark.parametrize("bands", [(3, 5, 1, 1, 1, 1, 0), (8, 1, 0, 0, 1, 0, 0),
-                                   (64, 64, 1, 0, 1, 1, 0), (1, 8, 0, 1, 1, 0, 0),
-                                   (1, 1, 0, 0, 1, 1, 0), (1, 1, 0, 1, 0, 0, 0),
-                                   (1, 1, 0, 1, 1, 1, 1)])
+@pytest.mark.parametrize("bands", [(3, 5, 1, 1, 1, 1, 0, 0), (8, 1, 0, 0, 1, 0, 0, 8),
+                                   (64, 64, 1, 0, 1, 1, 0, 3), (1, 8, 0, 1, 1, 0, 0, 64),
+                                   (1, 1, 0, 0, 1, 1, 0, 1), (1, 1, 0, 1, 0, 0, 0, 0),
+                                   (1, 1, 0, 1, 1, 1, 1, 8)])
 def test_tile_order_changes_no_bits(cuda_device, bands):
     """The CTA-pair GEMMs visit an expert's M tiles in bands (MOE_TUNE_GATE_UP_BAND /
     MOE_TUNE_DOWN_BAND) and spread the tiles of single-tile experts among the others
@@ -142,7 +142,8 @@ def test_tile_order_changes_no_bits(cuda_device, bands):
     tile is still one cluster's, summed over K in the same order from the same rows, so
     any setting gives the same bits as the default one; with the largest expert holding
     thousands of rows (a dozen M tiles) and several experts of one tile, the settings here
-    cut it into full and partial bands, with and without the spread and the trim. Swapped
+    cut it into full and partial bands, with and without the spread, the trim and L2
+    prefetches ahead of the loads (MOE_TUNE_PAIR_PREFETCH). Swapped
     tiles of at most 128 rows (MOE_TUNE_PAIR_SWAP_AB) against M = 128 tiles, and such rows
     on the one-CTA kernel (MOE_TUNE_PAIR_TAILS), are other MMA shapes, so other fp32
     summation orders: those agree within rounding."""
@@ -165,6 +166,7 @@ def test_tile_order_changes_no_bits(cuda_device, bands):
         abi.set_tuning(abi.TUNE_PAIR_SWAP_AB, bands[4])
         abi.set_tuning(abi.TUNE_PAIR_STREAM_HINT, bands[5])
         abi.set_tuning(abi.TUNE_PAIR_TAILS, bands[6])
+        abi.set_tuning(abi.TUNE_PAIR_PREFETCH, bands[7])
         for t in (b.h, b.y_perm, b.out):
             t.zero_()
         abi.run_steps(*args)
@@ -177,6 +179,7 @@ def test_tile_order_changes_no_bits(cuda_device, bands):
         abi.set_tuning(abi.TUNE_PAIR_SWAP_AB, 1)
         abi.set_tuning(abi.TUNE_PAIR_STREAM_HINT, 1)
         abi.set_tuning(abi.TUNE_PAIR_TAILS, 0)
+        abi.set_tuning(abi.TUNE_PAIR_PREFETCH, 0)
     assert abi.read_device_status(b.ws) == 0
     same = [torch.equal(w_, g_) for w_, g_ in zip(want, [b.h[:R], b.y_perm[:R], b.out])]
     if bands[4] and not bands[6]:
