@@ -231,7 +231,8 @@ __device__ __forceinline__ void epi_gateup_chunk(const GemmArgs& g, const Tile& 
 // down: 32 columns of y from the accumulator columns at tbase + tcol; output columns
 // [oc, oc + 32) of the tile's 256. Deterministic store: through the warp's staging rows
 // stg (32 x 80 bytes), so that a warp store covers 8 rows x 64 bytes; fused: s * g * y
-// added to the token's fp32 accumulator (tok, sc of this row).
+// added to the token's fp32 accumulator (tok, sc of this row), through the same staging
+// rows. Every lane of the warp must call it (warp shuffles and syncs).
 __device__ __forceinline__ void epi_down_chunk(const GemmArgs& g, const Tile& t, uint32_t tbase,
                                                int row, int tcol, int oc, int tok, float sc,
                                                float (*stg)[20], int lane) {
@@ -267,14 +268,32 @@ __device__ __forceinline__ void epi_down_chunk(const GemmArgs& g, const Tile& t,
     __syncwarp();
     return;
   }
-  if (row >= t.row_end || col >= g.n_valid) return;
-  float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)tok * g.ld_out + col);
+  // fused: s * g * y of this lane's row into its token's fp32 accumulator, 16 columns at a
+  // time through the staging rows, so that an atomic instruction covers 8 rows x 64
+  // contiguous bytes (8 half lines) instead of 32 rows x 16 bytes (32 lines)
+  const int valid = row < t.row_end ? 1 : 0;
 #pragma unroll
-  for (int v = 0; v < 8; ++v)
-    atomicAdd(dst + v, make_float4(sc * __uint_as_float(yr[4 * v + 0]),
-                                   sc * __uint_as_float(yr[4 * v + 1]),
-                                   sc * __uint_as_float(yr[4 * v + 2]),
-                                   sc * __uint_as_float(yr[4 * v + 3])));
+  for (int h16 = 0; h16 < 2; ++h16) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      *reinterpret_cast<float4*>(&stg[lane][4 * v]) =
+          make_float4(sc * __uint_as_float(yr[16 * h16 + 4 * v + 0]),
+                      sc * __uint_as_float(yr[16 * h16 + 4 * v + 1]),
+                      sc * __uint_as_float(yr[16 * h16 + 4 * v + 2]),
+                      sc * __uint_as_float(yr[16 * h16 + 4 * v + 3]));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 8 * i + (lane >> 2), ch = lane & 3;
+      const int tok_r = __shfl_sync(0xffffffffu, tok, r);
+      const int ok_r = __shfl_sync(0xffffffffu, valid, r);
+      const int c = col + 16 * h16 + 4 * ch;
+      if (ok_r && c < g.n_valid)
+        atomicAdd(reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)tok_r * g.ld_out + c),
+                  *reinterpret_cast<const float4*>(&stg[r][4 * ch]));
+    }
+    __syncwarp();
+  }
 }
 
 __device__ __forceinline__ void row_scale(const GemmArgs& g, const Tile& t, int row, int& tok,
