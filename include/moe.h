@@ -127,7 +127,8 @@ uint64_t moe_launch_count(void);
  *   MOE_TUNE_ROUTER_MIN_SPLIT 12 (default): fewest k-blocks of 64 in one split-K slice of
  *                             the bf16 router GEMM; 1 to 1024.
  *   MOE_TUNE_BWD_PAIR         1 (default): moe_backward's dgrad GEMMs run on CTA pairs
- *                             wherever the forward does; 0: one CTA per tile.
+ *                             wherever the forward does, its weight-gradient GEMMs always;
+ *                             2: only the dgrad GEMMs; 0: one CTA per tile everywhere.
  *   MOE_TUNE_BWD_DY_ROWS      4 (default): y rows each thread of the backward's dy kernel
  *                             loads before using them; 1: one at a time.
  *   MOE_TUNE_TEST_STALL       testing hook, 0 (default). Set to 1, the next gate/up GEMM
@@ -163,6 +164,13 @@ uint64_t moe_launch_count(void);
  *                             at most 256 rows, the CTA-pair GEMMs' producer prefetches into
  *                             L2 the weight boxes it will load this many k-blocks later
  *                             (crossing into its next tile).
+ *   MOE_TUNE_BWD_WGRAD_GROUP  tile order of the backward's weight-gradient GEMMs within an
+ *                             expert: 16 (default), or 1 to 64: groups of this many M tiles,
+ *                             N tiles outer within a group (a wave of tiles then spans fewer
+ *                             operand columns); 0: M tiles outer, N tiles inner.
+ *   MOE_TUNE_BWD_WGRAD_MIX    0 (default), or 1 to 65536: on CTA pairs, the weight-gradient
+ *                             tiles of experts with at most this many rows alternate with
+ *                             those of the larger experts (measured slower).
  * moe_set_tuning returns MOE_ERR_INVALID_ARG for an unknown switch or a value outside its
  * range. moe_get_tuning writes the current value. */
 typedef enum {
@@ -181,7 +189,9 @@ typedef enum {
   MOE_TUNE_PAIR_SWAP_AB = 12,
   MOE_TUNE_PAIR_STREAM_HINT = 13,
   MOE_TUNE_PAIR_TAILS = 14,
-  MOE_TUNE_PAIR_PREFETCH = 15
+  MOE_TUNE_PAIR_PREFETCH = 15,
+  MOE_TUNE_BWD_WGRAD_GROUP = 16,
+  MOE_TUNE_BWD_WGRAD_MIX = 17
 } moe_tune_t;
 
 int moe_set_tuning(int knob, int64_t value);

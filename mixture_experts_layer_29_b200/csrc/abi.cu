@@ -18,15 +18,15 @@ void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_r
 
 // Process-wide tuning switches (moe_set_tuning), each at its default until changed.
 namespace {
-constexpr int kTuneCount = MOE_TUNE_PAIR_PREFETCH + 1;
+constexpr int kTuneCount = MOE_TUNE_BWD_WGRAD_MIX + 1;
 std::atomic<int64_t> g_tune[kTuneCount] = {{1}, {-1}, {1}, {0}, {12}, {1}, {4}, {0}, {0}, {0}, {0}, {1},
-                                           {1}, {1}, {0}, {0}};
+                                           {1}, {1}, {0}, {0}, {16}, {0}};
 
 bool tune_value_ok(int knob, int64_t v) {
   switch (knob) {
+    case MOE_TUNE_BWD_PAIR: return v >= 0 && v <= 2;
     case MOE_TUNE_PDL:
     case MOE_TUNE_PAIR_HALF:
-    case MOE_TUNE_BWD_PAIR:
     case MOE_TUNE_PAIR_INTERLEAVE:
     case MOE_TUNE_PAIR_A_TRIM:
     case MOE_TUNE_PAIR_SWAP_AB:
@@ -40,6 +40,8 @@ bool tune_value_ok(int knob, int64_t v) {
     case MOE_TUNE_GATE_UP_BAND:
     case MOE_TUNE_DOWN_BAND:
     case MOE_TUNE_PAIR_PREFETCH: return v >= 0 && v <= 64;
+    case MOE_TUNE_BWD_WGRAD_GROUP: return v >= 0 && v <= 64;
+    case MOE_TUNE_BWD_WGRAD_MIX: return v >= 0 && v <= 65536;
     default: return false;
   }
 }

@@ -239,6 +239,41 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
   return r;
 }
+// Arrive on an mbarrier of the peer CTA (cluster address) with release semantics at
+// cluster scope: this thread's earlier shared-memory writes are visible to a thread of the
+// peer that acquires the phase at cluster scope.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// mbar_wait with acquire semantics at cluster scope (for phases completed by the peer CTA).
+__device__ __forceinline__ uint32_t mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kTrySuspendNs)
+      : "memory");
+  return ok;
+}
+__device__ __forceinline__ bool mbar_wait_acq_cluster(uint64_t* bar, uint32_t parity,
+                                                      volatile int* abort_flag) {
+  const uint32_t a = smem_u32(bar);
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 4; ++i)
+      if (mbar_try_wait_acq_cluster(a, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
 // Arrive on an mbarrier of this CTA or of the peer (cluster address), release at CTA
 // scope: it hands over a TMEM accumulator (ordered by the tcgen05 fences around it), not
 // global data, so the arriving thread need not wait for its global stores to land.

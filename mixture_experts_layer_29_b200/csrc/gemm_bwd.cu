@@ -8,7 +8,9 @@
 //   kDW  d_down[e]    = dy_e^T  h_e       M = H,  K = rows of e, N = I
 //        d_gate_up[e] = dgu_e^T x_perm_e  M = 2I, K = rows of e, N = H
 //        A and B both MN-major (the row buffers read along their rows); fp32, written for
-//        the experts that have rows only.
+//        the experts that have rows only. The experts' kDW runs on CTA pairs
+//        (k_bwd_wgrad_pair, 256 x 256 tiles); k_bwd_gemm keeps the router's and serves
+//        when MOE_TUNE_BWD_PAIR is 0 or 2.
 // The forward's SwiGLU expert (LongCat-Flash Technical Report digest, Key claims, report
 // §2.4: per-expert intermediate 2048 at hidden 6144) differentiated with the selection held
 // fixed.
@@ -24,6 +26,9 @@
 // the producer warp zeroes the K-rows past the expert in shared memory, fences them to the
 // async proxy and only then releases the stage to the MMA.
 #include <cuda.h>
+
+#include <cstddef>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -50,7 +55,7 @@ struct BwdArgs {
   int mode;
   int n_ffn;
   int kblocks;            // kDH / kDX: K / 64
-  int m_tiles;            // kDW: M / 128
+  int m_tiles;            // kDW: M / 128 (256 on CTA pairs), rounded up
   int n_tiles;            // N / 256 (rounded up)
   int b_krows;            // kDH / kDX: K rows of B per expert in its 2-D view
   int n_valid;            // output columns N
@@ -59,6 +64,9 @@ struct BwdArgs {
   int I;                  // kDH: G at column c, U at column I + c of gu and dgu
   int m_valid;            // kDW: output rows M
   int b_kwrap;            // kDW: B's row is the K row modulo this (0: no wrap)
+  int m_group;            // kDW: 0, or M tiles per group (N tiles outer within a group)
+  int mix_rows;           // pair kDW: 0, or experts of at most this many rows take every
+                          // other tile (see decode_w)
   const int32_t* offsets;
   const __nv_bfloat16* gu;
   void* out;
@@ -81,18 +89,31 @@ struct alignas(1024) Smem {
   int abort_flag;
   int offs[kMaxExperts + 1];
   int toff[kMaxExperts + 1];    // kDH / kDX: prefix of ceil(count / 128); kDW: of (count > 0)
-  float stg[kEpiWarps][32][20];
+  alignas(16) float stg[kEpiWarps][32][20];   // read and written as float4
 };
+static_assert(offsetof(Smem, stg) % 16 == 0, "staging rows are accessed as float4");
 
-__device__ __forceinline__ Tile decode(const Smem& s, const BwdArgs& g, int tile) {
+template <class S>
+__device__ __forceinline__ Tile decode(const S& s, const BwdArgs& g, int tile) {
   Tile t;
   int unit;
   if (g.mode == kDW) {
     const int per = g.m_tiles * g.n_tiles;
     unit = tile / per;
     const int rem = tile - unit * per;
-    t.mt = rem / g.n_tiles;
-    t.nt = rem - t.mt * g.n_tiles;
+    if (g.m_group > 0) {
+      // groups of m_group M tiles (the last one may be short); within a group the M tile
+      // runs fastest, so a wave of consecutive tiles spans fewer B columns
+      const int grp = rem / (g.m_group * g.n_tiles);
+      const int m0 = grp * g.m_group;
+      const int gsz = min(g.m_group, g.m_tiles - m0);
+      const int r2 = rem - grp * g.m_group * g.n_tiles;
+      t.nt = r2 / gsz;
+      t.mt = m0 + (r2 - t.nt * gsz);
+    } else {
+      t.mt = rem / g.n_tiles;
+      t.nt = rem - t.mt * g.n_tiles;
+    }
   } else {
     unit = tile / g.n_tiles;
     t.nt = tile - unit * g.n_tiles;
@@ -412,6 +433,381 @@ int launch(const CUtensorMap& ma, const CUtensorMap& mb, const BwdArgs& g, int s
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// ---- weight gradients on CTA pairs ----------------------------------------------------------
+// d_down[e] = dy_e^T h_e and d_gate_up[e] = dgu_e^T x_perm_e as 256 x 256 tiles on a cluster
+// of two CTAs (tcgen05 cta_group::2). CTA r loads the weight rows [256 mt + 128 r, +128) of
+// A and the columns [256 nt + 128 r, +128) of B, both MN-major (two 64 x 64 boxes each, 8 KB
+// apart), and keeps its 128 rows of the fp32 accumulator in its own TMEM; the leader issues
+// the MMAs. Per SM and k-block that is 32 KB of operands against the one-CTA tile's 48 KB.
+// The last k-block of an expert whose row count is not a multiple of 16: each CTA lands its
+// four boxes on a barrier of its own, zeroes the K-rows past the expert and fences them to
+// the async proxy. The peer's fix warp then arrives on the leader's `pfix` barrier (release
+// at cluster scope); the leader's fix warp acquires it and releases the stage to the MMA.
+constexpr int WSTAGES = 6;
+constexpr int W_HALF_BYTES = 2 * BOX_BYTES;            // 128 MN elements x 64 K rows: 16 KB
+constexpr int WBM = 256;                               // weight rows of a pair tile
+
+struct alignas(1024) WSmem {
+  uint8_t a[WSTAGES][W_HALF_BYTES];
+  uint8_t b[WSTAGES][W_HALF_BYTES];
+  uint64_t full[WSTAGES];       // leader: both CTAs' TMA bytes, or its fix warp on fix blocks
+  uint64_t empty[WSTAGES];      // the leader's MMA commit, in both CTAs
+  uint64_t landed[WSTAGES];     // fix blocks: this CTA's TMA bytes
+  uint64_t pfix[WSTAGES];       // leader: the peer's fix warp is done with the stage
+  uint64_t tfull[2];
+  uint64_t tempty[2];           // leader: both CTAs' epilogue warps
+  uint32_t tmem_base;
+  int abort_flag;
+  int n_heavy, n_light;         // experts with rows, more / at most mix_rows of them
+  int offs[kMaxExperts + 1];
+  int16_t order[kMaxExperts];   // the heavy experts, then the light ones, each by index
+  alignas(16) float stg[kEpiWarps][32][20];   // read and written as float4
+};
+static_assert(offsetof(WSmem, stg) % 16 == 0, "staging rows are accessed as float4");
+static_assert(offsetof(WSmem, a) % 1024 == 0 && offsetof(WSmem, b) % 1024 == 0 &&
+                  W_HALF_BYTES % 1024 == 0, "128-byte swizzled boxes need 1024-byte alignment");
+
+// Tile `tile` of the pair kernel: per expert m_tiles x n_tiles tiles. With light experts
+// (mix_rows), tiles alternate between the heavy and the light ones while both last, so
+// that the store-bound tiles of experts with few rows run beside MMA-bound ones; then the
+// rest of the longer list.
+__device__ __forceinline__ Tile decode_w(const WSmem& s, const BwdArgs& g, int tile) {
+  const int per = g.m_tiles * g.n_tiles;
+  const int nh = s.n_heavy * per, nl = s.n_light * per;
+  const int m = min(nh, nl);
+  int j;
+  bool light;
+  if (tile < 2 * m) {
+    light = (tile & 1) != 0;
+    j = tile >> 1;
+  } else {
+    light = nl > nh;
+    j = tile - m;
+  }
+  const int unit = j / per;
+  const int rem = j - unit * per;
+  Tile t;
+  t.e = s.order[(light ? s.n_heavy : 0) + unit];
+  t.row0 = s.offs[t.e];
+  t.row_end = s.offs[t.e + 1];
+  if (g.m_group > 0) {
+    const int grp = rem / (g.m_group * g.n_tiles);
+    const int m0 = grp * g.m_group;
+    const int gsz = min(g.m_group, g.m_tiles - m0);
+    const int r2 = rem - grp * g.m_group * g.n_tiles;
+    t.nt = r2 / gsz;
+    t.mt = m0 + (r2 - t.nt * gsz);
+  } else {
+    t.mt = rem / g.n_tiles;
+    t.nt = rem - t.mt * g.n_tiles;
+  }
+  return t;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_bwd_wgrad_pair(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB, const BwdArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  WSmem& s = *reinterpret_cast<WSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                       ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();            // 0: leader, 1: peer
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < WSTAGES; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+      mbar_init(&s.landed[i], 1);
+      mbar_init(&s.pfix[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 2 * kEpiWarps);
+    }
+    s.abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  pdl_wait();
+  for (int i = threadIdx.x; i <= g.n_ffn; i += kThreads) s.offs[i] = g.offsets[i];
+  __syncthreads();
+  cluster_sync();                                     // both CTAs' barriers initialised
+  if (warp == 1) {
+    tmem_alloc_pair(&s.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == 2) {
+    // the experts with rows, heavy ones first, each list in index order; lane l takes a
+    // contiguous run of experts
+    const int per = (g.n_ffn + 31) / 32;
+    const int b = lane * per;
+    auto cls = [&](int e) {     // 0: no rows, 1: heavy, 2: light
+      const int c = s.offs[e + 1] - s.offs[e];
+      return c <= 0 ? 0 : (g.mix_rows > 0 && c <= g.mix_rows ? 2 : 1);
+    };
+    int nh = 0, nl = 0;
+    for (int i = 0; i < per; ++i)
+      if (b + i < g.n_ffn) {
+        const int c = cls(b + i);
+        nh += c == 1 ? 1 : 0;
+        nl += c == 2 ? 1 : 0;
+      }
+    const int hinc = warp_inclusive_scan(nh);
+    const int linc = warp_inclusive_scan(nl);
+    const int h_all = __shfl_sync(0xffffffffu, hinc, 31);
+    int hrun = hinc - nh, lrun = h_all + linc - nl;
+    for (int i = 0; i < per; ++i)
+      if (b + i < g.n_ffn) {
+        const int c = cls(b + i);
+        if (c == 1) s.order[hrun++] = static_cast<int16_t>(b + i);
+        else if (c == 2) s.order[lrun++] = static_cast<int16_t>(b + i);
+      }
+    if (lane == 31) {
+      s.n_heavy = hinc;
+      s.n_light = linc;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s.tmem_base;
+  const int total_tiles = (s.n_heavy + s.n_light) * g.m_tiles * g.n_tiles;
+  volatile int* abort_flag = &s.abort_flag;
+
+  if (warp == 0) {
+    // ---- TMA producer (both CTAs): this CTA's weight rows of A and its columns of B ------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
+        const Tile t = decode_w(s, g, tile);
+        const int nkb = kblocks_of(g, t);
+        const int ax = t.mt * WBM + static_cast<int>(rank) * 128;
+        const int bx = t.nt * BN + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int y = t.row0 + kb * BK;
+          if (fix_block(kvalid(g, t, kb))) {
+            uint64_t* bar = &s.landed[stage];
+            mbar_arrive_expect_tx(bar, 2 * W_HALF_BYTES);
+            tma_load_2d(s.a[stage], &tmA, ax, y, bar);
+            tma_load_2d(s.a[stage] + BOX_BYTES, &tmA, ax + 64, y, bar);
+            tma_load_2d(s.b[stage], &tmB, bx, y, bar);
+            tma_load_2d(s.b[stage] + BOX_BYTES, &tmB, bx + 64, y, bar);
+          } else {
+            // the leader expects both CTAs' bytes
+            const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 4 * W_HALF_BYTES);
+            tma_load_2d_pair(s.a[stage], &tmA, ax, y, full_leader);
+            tma_load_2d_pair(s.a[stage] + BOX_BYTES, &tmA, ax + 64, y, full_leader);
+            tma_load_2d_pair(s.b[stage], &tmB, bx, y, full_leader);
+            tma_load_2d_pair(s.b[stage] + BOX_BYTES, &tmB, bx + 64, y, full_leader);
+          }
+          if (++stage == WSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer (leader only) ---------------------------------------------------------
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32_major(WBM, BN, true, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
+        const Tile t = decode_w(s, g, tile);
+        const int nkb = kblocks_of(g, t);
+        if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(s.a[stage]);
+          const uint32_t b0 = smem_u32(s.b[stage]);
+          const int nk = (kvalid(g, t, kb) + 15) / 16;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            if (k >= nk) break;
+            umma_bf16_pair(d_tmem, sw128_mnmajor_desc(a0 + k * 2048, BOX_BYTES),
+                           sw128_mnmajor_desc(b0 + k * 2048, BOX_BYTES), idesc,
+                           (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          const uint32_t e_local = smem_u32(&s.empty[stage]);
+          umma_commit_pair(mapa_shared(e_local, 0));
+          umma_commit_pair(mapa_shared(e_local, 1));
+          if (++stage == WSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        const uint32_t f_local = smem_u32(&s.tfull[acc]);
+        umma_commit_pair(mapa_shared(f_local, 0));
+        umma_commit_pair(mapa_shared(f_local, 1));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else if (warp == kFixWarp) {
+    // ---- fix warp (both CTAs): zeroes the K-rows past the expert on fix blocks ------------
+    int stage = 0;
+    uint32_t landed_phase = 0;   // bit i: parity of the next completion of landed[i]
+    uint32_t pfix_phase = 0;     // leader, bit i: of pfix[i]
+    bool ok = true;
+    for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
+      const Tile t = decode_w(s, g, tile);
+      const int nkb = kblocks_of(g, t);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int valid = kvalid(g, t, kb);
+        if (fix_block(valid)) {
+          int w_ok = 1;
+          if (lane == 0)
+            w_ok = mbar_wait(&s.landed[stage], (landed_phase >> stage) & 1u, abort_flag) ? 1 : 0;
+          landed_phase ^= 1u << stage;
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+            ok = false;
+            break;
+          }
+          const int nrow = ((valid + 15) & ~15) - valid;
+          for (int i = lane; i < 4 * nrow * 8; i += 32) {
+            const int box = i / (nrow * 8), rem = i - box * nrow * 8;
+            const int r = valid + rem / 8, c16 = rem & 7;
+            uint8_t* base = box < 2 ? s.a[stage] + box * BOX_BYTES : s.b[stage] + (box - 2) * BOX_BYTES;
+            *reinterpret_cast<uint4*>(base + r * 128 + c16 * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (rank != 0) {
+              mbar_arrive_release_cluster(mapa_shared(smem_u32(&s.pfix[stage]), 0));
+            } else {
+              w_ok = mbar_wait_acq_cluster(&s.pfix[stage], (pfix_phase >> stage) & 1u, abort_flag)
+                         ? 1 : 0;
+              if (w_ok) mbar_arrive(&s.full[stage]);
+            }
+          }
+          pfix_phase ^= 1u << stage;
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+            ok = false;
+            break;
+          }
+        }
+        if (++stage == WSTAGES) stage = 0;
+      }
+    }
+  } else {
+    // ---- epilogue (both CTAs, warps 2..9): this CTA's 128 weight rows of the tile ---------
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
+    float (*stg)[20] = s.stg[warp - 2];
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster; tile < total_tiles; tile += nclusters) {
+      const Tile t = decode_w(s, g, tile);
+      int w_ok = 1;
+      if (lane == 0) w_ok = mbar_wait(&s.tfull[acc], acc_phase, abort_flag) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      const int row_base = t.mt * WBM + static_cast<int>(rank) * 128 + q * 32;
+      float* out = static_cast<float*>(g.out) + (size_t)t.e * g.out_expert;
+#pragma unroll 1
+      for (int c = 128 * h; c < 128 * h + 128; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + c, v);
+        tmem_ld_wait();
+        const int col = t.nt * BN + c;
+        float f[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+        store_f32_16(stg, lane, f, out, g.ld_out, row_base, g.m_valid, col, g.n_valid);
+        store_f32_16(stg, lane, f + 16, out, g.ld_out, row_base, g.m_valid, col + 16, g.n_valid);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  if (*abort_flag) {
+    set_status(g.status, MOE_ERR_TIMEOUT);
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();            // neither CTA leaves while the other may still signal it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+// Cluster-of-two launch: as many clusters as fit at once (cached per device).
+int launch_wgrad_pair(const CUtensorMap& ma, const CUtensorMap& mb, const BwdArgs& g,
+                      int sm_count, cudaStream_t st) {
+  constexpr size_t smem = sizeof(WSmem) + 1024;
+  static_assert(smem <= 227 * 1024, "shared memory budget");
+  static std::mutex mu;
+  static int clusters_of[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return MOE_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_bwd_wgrad_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int nclusters;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (clusters_of[dev] == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(sm_count & ~1);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k_bwd_wgrad_pair, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      clusters_of[dev] = n;
+    }
+    nclusters = clusters_of[dev];
+  }
+  if (nclusters > sm_count / 2) nclusters = sm_count / 2;
+  if (launch_kernel(k_bwd_wgrad_pair, 2 * nclusters, kThreads, smem, st, 2, ma, mb, g) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  count_launch();
+  return MOE_OK;
+}
+
 }  // namespace
 
 int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* x_perm,
@@ -463,25 +859,32 @@ int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* 
   g.ld_out = H;
   g.out = dx_perm;
   if (!pair && (rc = launch(m_dgu128, m_wgu, g, sm_count, st)) != MOE_OK) return rc;
-  // d_down[e] = dy^T h
+  // d_down[e] = dy^T h, then d_gate_up[e] = dgu^T x_perm: on CTA pairs (256 weight rows
+  // per tile) unless MOE_TUNE_BWD_PAIR is 0 or 2
+  const bool wpair = tuning(MOE_TUNE_BWD_PAIR) == 1 && sm_count >= 2;
+  const int bm = wpair ? WBM : BM;
   g.mode = kDW;
+  g.m_group = (int)tuning(MOE_TUNE_BWD_WGRAD_GROUP);
+  g.mix_rows = (int)tuning(MOE_TUNE_BWD_WGRAD_MIX);
   g.m_valid = H;
-  g.m_tiles = H / BM;
+  g.m_tiles = (H + bm - 1) / bm;
   g.n_tiles = (I + BN - 1) / BN;
   g.n_valid = I;
   g.ld_out = I;
   g.out_expert = (long long)H * I;
   g.out = d_down;
-  if ((rc = launch(m_dy64, m_h64, g, sm_count, st)) != MOE_OK) return rc;
-  // d_gate_up[e] = dgu^T x_perm
+  rc = wpair ? launch_wgrad_pair(m_dy64, m_h64, g, sm_count, st)
+             : launch(m_dy64, m_h64, g, sm_count, st);
+  if (rc != MOE_OK) return rc;
   g.m_valid = 2 * I;
-  g.m_tiles = 2 * I / BM;
+  g.m_tiles = (2 * I + bm - 1) / bm;
   g.n_tiles = (H + BN - 1) / BN;
   g.n_valid = H;
   g.ld_out = H;
   g.out_expert = 2LL * I * H;
   g.out = d_gate_up;
-  return launch(m_dgu64, m_x64, g, sm_count, st);
+  return wpair ? launch_wgrad_pair(m_dgu64, m_x64, g, sm_count, st)
+               : launch(m_dgu64, m_x64, g, sm_count, st);
 }
 
 int launch_bwd_router_gemms(const void* dl3, int Tp, const void* x, const void* wr16,

@@ -179,3 +179,31 @@ def test_backward_full_shape_prefill(cuda_device, parity_report):
     del d_gu, d_d, gu, ws, b, case
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("knobs", [(1, 3, 0), (1, 0, 256), (1, 16, 1), (1, 1, 65536),
+                                   (1, 8, 256), (1, 0, 0), (2, 16, 0), (2, 0, 0)])
+def test_weight_gradient_schedules_change_no_bits(cuda_device, knobs):
+    """The weight-gradient GEMMs on CTA pairs visit an expert's tiles in groups of M tiles
+    (MOE_TUNE_BWD_WGRAD_GROUP) and may alternate the tiles of experts with few rows with
+    those of the others (MOE_TUNE_BWD_WGRAD_MIX; here with some, none and all experts in
+    the light list). Each output tile is still summed over the expert's rows in the same
+    order, so every setting gives the bits of the default one. MOE_TUNE_BWD_PAIR = 2 runs
+    them on the one-CTA kernel (128-row tiles), whose per-element sums take the same
+    k-steps in the same order."""
+    cfg = wl.CONFIGS["proxy_bf16"].with_(T=3001)
+    want = _run(cfg, seed=21)
+    counts = gh.host(want[1].counts)[: cfg.n_ffn]
+    assert counts.max() > 1000
+    assert ((counts > 0) & (counts <= 256)).sum() >= 3
+    try:
+        abi.set_tuning(abi.TUNE_BWD_PAIR, knobs[0])
+        abi.set_tuning(abi.TUNE_BWD_WGRAD_GROUP, knobs[1])
+        abi.set_tuning(abi.TUNE_BWD_WGRAD_MIX, knobs[2])
+        got = _run(cfg, seed=21)
+    finally:
+        abi.set_tuning(abi.TUNE_BWD_PAIR, 1)
+        abi.set_tuning(abi.TUNE_BWD_WGRAD_GROUP, 16)
+        abi.set_tuning(abi.TUNE_BWD_WGRAD_MIX, 0)
+    for a, c in zip(want[3:], got[3:]):
+        assert torch.equal(a, c)
