@@ -89,7 +89,7 @@ struct alignas(1024) Smem {
   int abort_flag;
   int offs[kMaxExperts + 1];
   int toff[kMaxExperts + 1];    // kDH / kDX: prefix of ceil(count / 128); kDW: of (count > 0)
-  alignas(16) float stg[kEpiWarps][32][20];   // read and written as float4
+  alignas(16) float stg[kEpiWarps][32][16];   // read and written as float4
 };
 static_assert(offsetof(Smem, stg) % 16 == 0, "staging rows are accessed as float4");
 
@@ -144,13 +144,18 @@ __device__ __forceinline__ int kvalid(const BwdArgs& g, const Tile& t, int kb) {
 __device__ __forceinline__ bool fix_block(int valid) { return (valid & 15) != 0; }
 
 // fp32 row stores through the warp's staging block: this thread's row holds 16 values at
-// output columns [col, col + 16); a warp store then covers 8 rows x 64 bytes.
-__device__ __forceinline__ void store_f32_16(float (*stg)[20], int lane, const float* v,
+// output columns [col, col + 16); a warp store then covers 8 rows x 64 bytes. A staging row
+// is 16 floats, and its 16-byte chunk ch sits at chunk ch ^ ((row >> 1) & 3): each group of 8
+// lanes then touches 32 distinct banks, both when a lane writes its row and when 8 lanes
+// read two rows.
+__device__ __forceinline__ int stg_chunk(int row, int ch) { return 4 * (ch ^ ((row >> 1) & 3)); }
+
+__device__ __forceinline__ void store_f32_16(float (*stg)[16], int lane, const float* v,
                                              float* out, long long ld, int row_base,
                                              int row_end, int col, int n_valid) {
 #pragma unroll
   for (int i = 0; i < 4; ++i)
-    *reinterpret_cast<float4*>(&stg[lane][4 * i]) =
+    *reinterpret_cast<float4*>(&stg[lane][stg_chunk(lane, i)]) =
         make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
   __syncwarp();
 #pragma unroll
@@ -159,7 +164,7 @@ __device__ __forceinline__ void store_f32_16(float (*stg)[20], int lane, const f
     const int grow = row_base + r;
     if (grow < row_end && c < n_valid)
       *reinterpret_cast<float4*>(out + (size_t)grow * ld + c) =
-          *reinterpret_cast<const float4*>(&stg[r][4 * (lane & 3)]);
+          *reinterpret_cast<const float4*>(&stg[r][stg_chunk(r, lane & 3)]);
   }
   __syncwarp();
 }
@@ -346,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- epilogue: TMEM lane quarter q = warp % 4, column half h = (warp - 2) / 4 ---------
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
-    float (*stg)[20] = s.stg[warp - 2];
+    float (*stg)[16] = s.stg[warp - 2];
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
@@ -461,7 +466,7 @@ struct alignas(1024) WSmem {
   int n_heavy, n_light;         // experts with rows, more / at most mix_rows of them
   int offs[kMaxExperts + 1];
   int16_t order[kMaxExperts];   // the heavy experts, then the light ones, each by index
-  alignas(16) float stg[kEpiWarps][32][20];   // read and written as float4
+  alignas(16) float stg[kEpiWarps][32][16];   // read and written as float4
 };
 static_assert(offsetof(WSmem, stg) % 16 == 0, "staging rows are accessed as float4");
 static_assert(offsetof(WSmem, a) % 1024 == 0 && offsetof(WSmem, b) % 1024 == 0 &&
@@ -714,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- epilogue (both CTAs, warps 2..9): this CTA's 128 weight rows of the tile ---------
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
-    float (*stg)[20] = s.stg[warp - 2];
+    float (*stg)[16] = s.stg[warp - 2];
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cluster; tile < total_tiles; tile += nclusters) {
@@ -724,24 +729,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
-      const int row_base = t.mt * WBM + static_cast<int>(rank) * 128 + q * 32;
-      float* out = static_cast<float*>(g.out) + (size_t)t.e * g.out_expert;
-#pragma unroll 1
-      for (int c = 128 * h; c < 128 * h + 128; c += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tbase + c, v);
-        tmem_ld_wait();
-        const int col = t.nt * BN + c;
-        float f[32];
+                             static_cast<uint32_t>(acc * BN + 128 * h);
+      // the warp's 128 columns in flight at once and one wait; the accumulator then goes
+      // back to the MMA before the stores
+      uint32_t v[4][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
-        store_f32_16(stg, lane, f, out, g.ld_out, row_base, g.m_valid, col, g.n_valid);
-        store_f32_16(stg, lane, f + 16, out, g.ld_out, row_base, g.m_valid, col + 16, g.n_valid);
-      }
+      for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(tbase + 32 * i, v[i]);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
+      const int row_base = t.mt * WBM + static_cast<int>(rank) * 128 + q * 32;
+      float* out = static_cast<float*>(g.out) + (size_t)t.e * g.out_expert;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = t.nt * BN + 128 * h + 32 * i;
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[i][j]);
+        store_f32_16(stg, lane, f, out, g.ld_out, row_base, g.m_valid, col, g.n_valid);
+        store_f32_16(stg, lane, f + 16, out, g.ld_out, row_base, g.m_valid, col + 16, g.n_valid);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
