@@ -84,6 +84,16 @@ def test_backward_without_zero_experts(cuda_device):
     _check(wl.CONFIGS["proxy_bf16"].with_(T=512, n_zero=0))
 
 
+@pytest.mark.parametrize("T", [300, 2048])
+def test_backward_widths_off_the_pair_tile(cuda_device, T):
+    """H = 640 and I = 384: the weight-gradient tiles on CTA pairs are 256 x 256, so dW_d's
+    last tile has its peer CTA's 128 weight rows past H, and the last tile of dW_gu (N = H)
+    and of dW_d (N = I) has the peer's 128 columns past the matrix: those rows and columns
+    load as zeros and are never stored. T = 300 runs the dgrad GEMMs on one CTA, T = 2048 on
+    CTA pairs."""
+    _check(wl.CONFIGS["proxy_bf16"].with_(T=T, H=640, I=384))
+
+
 def test_backward_full_width(cuda_device):
     """Hidden 6144, intermediate 2048 with 16 + 8 experts (the oracle evaluates every row)."""
     _check(wl.CONFIGS["prefill_bf16"].with_(T=64, n_ffn=16, n_zero=8))
