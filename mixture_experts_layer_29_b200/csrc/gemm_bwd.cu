@@ -169,6 +169,35 @@ __device__ __forceinline__ void store_f32_16(float (*stg)[16], int lane, const f
   __syncwarp();
 }
 
+// fp32 stores of 32 columns [col, col + 32) of this warp's 32 rows (this thread's row holds
+// them in v) as full 128-byte lines: two passes of 16 rows through a 16 x 32 staging block,
+// whose 16-byte chunk c of row r sits at chunk c ^ (r & 7). The lanes of a pass write their
+// rows, then each warp store covers 4 rows x 128 bytes.
+__device__ __forceinline__ void store_f32_32(float (*stg)[32], int lane, const uint32_t* v,
+                                             float* out, long long ld, int row_base,
+                                             int row_end, int col, int n_valid) {
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    if ((lane >> 4) == p) {
+      const int r = lane & 15;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(&stg[r][4 * (c ^ (r & 7))]) =
+            make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 4 * i + (lane >> 3), ch = lane & 7;
+      const int grow = row_base + 16 * p + r, c = col + 4 * ch;
+      if (grow < row_end && c < n_valid)
+        *reinterpret_cast<float4*>(out + (size_t)grow * ld + c) =
+            *reinterpret_cast<const float4*>(&stg[r][4 * (ch ^ (r & 7))]);
+    }
+    __syncwarp();
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const BwdArgs g) {
@@ -466,7 +495,7 @@ struct alignas(1024) WSmem {
   int n_heavy, n_light;         // experts with rows, more / at most mix_rows of them
   int offs[kMaxExperts + 1];
   int16_t order[kMaxExperts];   // the heavy experts, then the light ones, each by index
-  alignas(16) float stg[kEpiWarps][32][16];   // read and written as float4
+  alignas(16) float stg[kEpiWarps][16][32];   // read and written as float4
 };
 static_assert(offsetof(WSmem, stg) % 16 == 0, "staging rows are accessed as float4");
 static_assert(offsetof(WSmem, a) % 1024 == 0 && offsetof(WSmem, b) % 1024 == 0 &&
@@ -719,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- epilogue (both CTAs, warps 2..9): this CTA's 128 weight rows of the tile ---------
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
-    float (*stg)[16] = s.stg[warp - 2];
+    float (*stg)[32] = s.stg[warp - 2];
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cluster; tile < total_tiles; tile += nclusters) {
@@ -730,25 +759,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + 128 * h);
-      // the warp's 128 columns in flight at once and one wait; the accumulator then goes
-      // back to the MMA before the stores
-      uint32_t v[4][32];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(tbase + 32 * i, v[i]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
+      // the warp's 128 columns in two batches of 64, each in flight at once with one wait;
+      // the accumulator goes back to the MMA before the second batch's stores
       const int row_base = t.mt * WBM + static_cast<int>(rank) * 128 + q * 32;
       float* out = static_cast<float*>(g.out) + (size_t)t.e * g.out_expert;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int col = t.nt * BN + 128 * h + 32 * i;
-        float f[32];
+      for (int b = 0; b < 2; ++b) {
+        uint32_t v[2][32];
+        tmem_ld_32x32b_x32(tbase + 64 * b, v[0]);
+        tmem_ld_32x32b_x32(tbase + 64 * b + 32, v[1]);
+        tmem_ld_wait();
+        if (b == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
+        }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[i][j]);
-        store_f32_16(stg, lane, f, out, g.ld_out, row_base, g.m_valid, col, g.n_valid);
-        store_f32_16(stg, lane, f + 16, out, g.ld_out, row_base, g.m_valid, col + 16, g.n_valid);
+        for (int i = 0; i < 2; ++i)
+          store_f32_32(stg, lane, v[i], out, g.ld_out, row_base, g.m_valid,
+                       t.nt * BN + 128 * h + 64 * b + 32 * i, g.n_valid);
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
