@@ -171,6 +171,9 @@ uint64_t moe_launch_count(void);
  *   MOE_TUNE_BWD_WGRAD_MIX    0 (default), or 1 to 65536: on CTA pairs, the weight-gradient
  *                             tiles of experts with at most this many rows alternate with
  *                             those of the larger experts (measured slower).
+ *   MOE_TUNE_BWD_WGRAD_BK     64 (default) or 128: K rows (expert rows) per pipeline stage of
+ *                             the CTA-pair weight-gradient GEMMs: six stages of 64-row
+ *                             operand boxes, or three of 128-row ones.
  * moe_set_tuning returns MOE_ERR_INVALID_ARG for an unknown switch or a value outside its
  * range. moe_get_tuning writes the current value. */
 typedef enum {
@@ -191,7 +194,8 @@ typedef enum {
   MOE_TUNE_PAIR_TAILS = 14,
   MOE_TUNE_PAIR_PREFETCH = 15,
   MOE_TUNE_BWD_WGRAD_GROUP = 16,
-  MOE_TUNE_BWD_WGRAD_MIX = 17
+  MOE_TUNE_BWD_WGRAD_MIX = 17,
+  MOE_TUNE_BWD_WGRAD_BK = 18
 } moe_tune_t;
 
 int moe_set_tuning(int knob, int64_t value);

@@ -175,7 +175,7 @@ TUNE_PDL, TUNE_GEMM_PAIR, TUNE_PAIR_HALF, TUNE_ROUTER_N = 0, 1, 2, 3
 TUNE_ROUTER_MIN_SPLIT, TUNE_BWD_PAIR, TUNE_BWD_DY_ROWS, TUNE_TEST_STALL = 4, 5, 6, 7
 TUNE_GATE_UP_BAND, TUNE_DOWN_BAND, TUNE_PAIR_INTERLEAVE, TUNE_PAIR_A_TRIM = 8, 9, 10, 11
 TUNE_PAIR_SWAP_AB, TUNE_PAIR_STREAM_HINT, TUNE_PAIR_TAILS, TUNE_PAIR_PREFETCH = 12, 13, 14, 15
-TUNE_BWD_WGRAD_GROUP, TUNE_BWD_WGRAD_MIX = 16, 17
+TUNE_BWD_WGRAD_GROUP, TUNE_BWD_WGRAD_MIX, TUNE_BWD_WGRAD_BK = 16, 17, 18
 
 
 def set_tuning(knob: int, value: int):

@@ -18,9 +18,9 @@ void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_r
 
 // Process-wide tuning switches (moe_set_tuning), each at its default until changed.
 namespace {
-constexpr int kTuneCount = MOE_TUNE_BWD_WGRAD_MIX + 1;
+constexpr int kTuneCount = MOE_TUNE_BWD_WGRAD_BK + 1;
 std::atomic<int64_t> g_tune[kTuneCount] = {{1}, {-1}, {1}, {0}, {12}, {1}, {4}, {0}, {0}, {0}, {0}, {1},
-                                           {1}, {1}, {0}, {0}, {16}, {0}};
+                                           {1}, {1}, {0}, {0}, {16}, {0}, {64}};
 
 bool tune_value_ok(int knob, int64_t v) {
   switch (knob) {
@@ -42,6 +42,7 @@ bool tune_value_ok(int knob, int64_t v) {
     case MOE_TUNE_PAIR_PREFETCH: return v >= 0 && v <= 64;
     case MOE_TUNE_BWD_WGRAD_GROUP: return v >= 0 && v <= 64;
     case MOE_TUNE_BWD_WGRAD_MIX: return v >= 0 && v <= 65536;
+    case MOE_TUNE_BWD_WGRAD_BK: return v == 64 || v == 128;
     default: return false;
   }
 }

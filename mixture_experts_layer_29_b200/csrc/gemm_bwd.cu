@@ -477,17 +477,27 @@ int launch(const CUtensorMap& ma, const CUtensorMap& mb, const BwdArgs& g, int s
 // four boxes on a barrier of its own, zeroes the K-rows past the expert and fences them to
 // the async proxy. The peer's fix warp then arrives on the leader's `pfix` barrier (release
 // at cluster scope); the leader's fix warp acquires it and releases the stage to the MMA.
-constexpr int WSTAGES = 6;
-constexpr int W_HALF_BYTES = 2 * BOX_BYTES;            // 128 MN elements x 64 K rows: 16 KB
 constexpr int WBM = 256;                               // weight rows of a pair tile
 
+// K rows per stage WK (64 or 128; MOE_TUNE_BWD_WGRAD_BK): each operand half of a CTA is two
+// boxes of WK K-rows x 64 MN elements (the 128-byte swizzle caps an MN-major box at 64
+// elements), so a stage holds 32 KB (WK = 64, six stages) or 64 KB (WK = 128, three).
+template <int WK>
+struct WCfg {
+  static constexpr int STAGES = 6 * 64 / WK;
+  static constexpr int BOX = WK * 128;                 // one box: WK rows of 128 bytes
+  static constexpr int HALF = 2 * BOX;                 // 128 MN elements
+};
+
+template <int WK>
 struct alignas(1024) WSmem {
-  uint8_t a[WSTAGES][W_HALF_BYTES];
-  uint8_t b[WSTAGES][W_HALF_BYTES];
-  uint64_t full[WSTAGES];       // leader: both CTAs' TMA bytes, or its fix warp on fix blocks
-  uint64_t empty[WSTAGES];      // the leader's MMA commit, in both CTAs
-  uint64_t landed[WSTAGES];     // fix blocks: this CTA's TMA bytes
-  uint64_t pfix[WSTAGES];       // leader: the peer's fix warp is done with the stage
+  static constexpr int STAGES = WCfg<WK>::STAGES;
+  uint8_t a[STAGES][WCfg<WK>::HALF];
+  uint8_t b[STAGES][WCfg<WK>::HALF];
+  uint64_t full[STAGES];        // leader: both CTAs' TMA bytes, or its fix warp on fix blocks
+  uint64_t empty[STAGES];       // the leader's MMA commit, in both CTAs
+  uint64_t landed[STAGES];      // fix blocks: this CTA's TMA bytes
+  uint64_t pfix[STAGES];        // leader: the peer's fix warp is done with the stage
   uint64_t tfull[2];
   uint64_t tempty[2];           // leader: both CTAs' epilogue warps
   uint32_t tmem_base;
@@ -497,15 +507,25 @@ struct alignas(1024) WSmem {
   int16_t order[kMaxExperts];   // the heavy experts, then the light ones, each by index
   alignas(16) float stg[kEpiWarps][16][32];   // read and written as float4
 };
-static_assert(offsetof(WSmem, stg) % 16 == 0, "staging rows are accessed as float4");
-static_assert(offsetof(WSmem, a) % 1024 == 0 && offsetof(WSmem, b) % 1024 == 0 &&
-                  W_HALF_BYTES % 1024 == 0, "128-byte swizzled boxes need 1024-byte alignment");
+static_assert(offsetof(WSmem<64>, stg) % 16 == 0 && offsetof(WSmem<128>, stg) % 16 == 0,
+              "staging rows are accessed as float4");
+static_assert(offsetof(WSmem<64>, b) % 1024 == 0 && offsetof(WSmem<128>, b) % 1024 == 0 &&
+                  WCfg<64>::HALF % 1024 == 0, "128-byte swizzled boxes need 1024-byte alignment");
+
+// k-blocks of WK rows of a tile's expert, and the rows of k-block kb that belong to it
+template <int WK>
+__device__ __forceinline__ int w_kblocks(const Tile& t) { return (t.row_end - t.row0 + WK - 1) / WK; }
+template <int WK>
+__device__ __forceinline__ int w_kvalid(const Tile& t, int kb) {
+  return min(WK, t.row_end - (t.row0 + kb * WK));
+}
 
 // Tile `tile` of the pair kernel: per expert m_tiles x n_tiles tiles. With light experts
 // (mix_rows), tiles alternate between the heavy and the light ones while both last, so
 // that the store-bound tiles of experts with few rows run beside MMA-bound ones; then the
 // rest of the longer list.
-__device__ __forceinline__ Tile decode_w(const WSmem& s, const BwdArgs& g, int tile) {
+template <class S>
+__device__ __forceinline__ Tile decode_w(const S& s, const BwdArgs& g, int tile) {
   const int per = g.m_tiles * g.n_tiles;
   const int nh = s.n_heavy * per, nl = s.n_light * per;
   const int m = min(nh, nl);
@@ -538,18 +558,20 @@ __device__ __forceinline__ Tile decode_w(const WSmem& s, const BwdArgs& g, int t
   return t;
 }
 
+template <int WK>
 __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_wgrad_pair(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, const BwdArgs g) {
+  constexpr int STAGES = WCfg<WK>::STAGES, WBOX = WCfg<WK>::BOX, WHALF = WCfg<WK>::HALF;
   extern __shared__ uint8_t smem_raw[];
-  WSmem& s = *reinterpret_cast<WSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                       ~static_cast<uintptr_t>(1023));
+  WSmem<WK>& s = *reinterpret_cast<WSmem<WK>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();            // 0: leader, 1: peer
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < WSTAGES; ++i) {
+    for (int i = 0; i < STAGES; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
       mbar_init(&s.landed[i], 1);
@@ -618,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
         const Tile t = decode_w(s, g, tile);
-        const int nkb = kblocks_of(g, t);
+        const int nkb = w_kblocks<WK>(t);
         const int ax = t.mt * WBM + static_cast<int>(rank) * 128;
         const int bx = t.nt * BN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -626,24 +648,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const int y = t.row0 + kb * BK;
-          if (fix_block(kvalid(g, t, kb))) {
+          const int y = t.row0 + kb * WK;
+          if (fix_block(w_kvalid<WK>(t, kb))) {
             uint64_t* bar = &s.landed[stage];
-            mbar_arrive_expect_tx(bar, 2 * W_HALF_BYTES);
+            mbar_arrive_expect_tx(bar, 2 * WHALF);
             tma_load_2d(s.a[stage], &tmA, ax, y, bar);
-            tma_load_2d(s.a[stage] + BOX_BYTES, &tmA, ax + 64, y, bar);
+            tma_load_2d(s.a[stage] + WBOX, &tmA, ax + 64, y, bar);
             tma_load_2d(s.b[stage], &tmB, bx, y, bar);
-            tma_load_2d(s.b[stage] + BOX_BYTES, &tmB, bx + 64, y, bar);
+            tma_load_2d(s.b[stage] + WBOX, &tmB, bx + 64, y, bar);
           } else {
             // the leader expects both CTAs' bytes
             const uint32_t full_leader = mapa_shared(smem_u32(&s.full[stage]), 0);
-            if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 4 * W_HALF_BYTES);
+            if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 4 * WHALF);
             tma_load_2d_pair(s.a[stage], &tmA, ax, y, full_leader);
-            tma_load_2d_pair(s.a[stage] + BOX_BYTES, &tmA, ax + 64, y, full_leader);
+            tma_load_2d_pair(s.a[stage] + WBOX, &tmA, ax + 64, y, full_leader);
             tma_load_2d_pair(s.b[stage], &tmB, bx, y, full_leader);
-            tma_load_2d_pair(s.b[stage] + BOX_BYTES, &tmB, bx + 64, y, full_leader);
+            tma_load_2d_pair(s.b[stage] + WBOX, &tmB, bx + 64, y, full_leader);
           }
-          if (++stage == WSTAGES) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -661,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
         const Tile t = decode_w(s, g, tile);
-        const int nkb = kblocks_of(g, t);
+        const int nkb = w_kblocks<WK>(t);
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -673,18 +695,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(s.a[stage]);
           const uint32_t b0 = smem_u32(s.b[stage]);
-          const int nk = (kvalid(g, t, kb) + 15) / 16;
+          const int nk = (w_kvalid<WK>(t, kb) + 15) / 16;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
+          for (int k = 0; k < WK / 16; ++k) {
             if (k >= nk) break;
-            umma_bf16_pair(d_tmem, sw128_mnmajor_desc(a0 + k * 2048, BOX_BYTES),
-                           sw128_mnmajor_desc(b0 + k * 2048, BOX_BYTES), idesc,
+            umma_bf16_pair(d_tmem, sw128_mnmajor_desc(a0 + k * 2048, WBOX),
+                           sw128_mnmajor_desc(b0 + k * 2048, WBOX), idesc,
                            (kb > 0 || k > 0) ? 1u : 0u);
           }
           const uint32_t e_local = smem_u32(&s.empty[stage]);
           umma_commit_pair(mapa_shared(e_local, 0));
           umma_commit_pair(mapa_shared(e_local, 1));
-          if (++stage == WSTAGES) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -705,9 +727,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int tile = cluster; ok && tile < total_tiles && !*abort_flag; tile += nclusters) {
       const Tile t = decode_w(s, g, tile);
-      const int nkb = kblocks_of(g, t);
+      const int nkb = w_kblocks<WK>(t);
       for (int kb = 0; kb < nkb; ++kb) {
-        const int valid = kvalid(g, t, kb);
+        const int valid = w_kvalid<WK>(t, kb);
         if (fix_block(valid)) {
           int w_ok = 1;
           if (lane == 0)
@@ -721,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = lane; i < 4 * nrow * 8; i += 32) {
             const int box = i / (nrow * 8), rem = i - box * nrow * 8;
             const int r = valid + rem / 8, c16 = rem & 7;
-            uint8_t* base = box < 2 ? s.a[stage] + box * BOX_BYTES : s.b[stage] + (box - 2) * BOX_BYTES;
+            uint8_t* base = box < 2 ? s.a[stage] + box * WBOX : s.b[stage] + (box - 2) * WBOX;
             *reinterpret_cast<uint4*>(base + r * 128 + c16 * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
           fence_proxy_async_smem();
@@ -741,7 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        if (++stage == WSTAGES) stage = 0;
+        if (++stage == STAGES) stage = 0;
       }
     }
   } else {
@@ -799,15 +821,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Cluster-of-two launch: as many clusters as fit at once (cached per device).
+template <int WK>
 int launch_wgrad_pair(const CUtensorMap& ma, const CUtensorMap& mb, const BwdArgs& g,
                       int sm_count, cudaStream_t st) {
-  constexpr size_t smem = sizeof(WSmem) + 1024;
+  constexpr size_t smem = sizeof(WSmem<WK>) + 1024;
   static_assert(smem <= 227 * 1024, "shared memory budget");
   static std::mutex mu;
   static int clusters_of[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return MOE_ERR_CUDA;
-  if (cudaFuncSetAttribute(k_bwd_wgrad_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(k_bwd_wgrad_pair<WK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
   int nclusters;
@@ -827,7 +850,7 @@ int launch_wgrad_pair(const CUtensorMap& ma, const CUtensorMap& mb, const BwdArg
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, k_bwd_wgrad_pair, &cfg) != cudaSuccess || n < 1) {
+      if (cudaOccupancyMaxActiveClusters(&n, k_bwd_wgrad_pair<WK>, &cfg) != cudaSuccess || n < 1) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
       }
@@ -836,7 +859,7 @@ int launch_wgrad_pair(const CUtensorMap& ma, const CUtensorMap& mb, const BwdArg
     nclusters = clusters_of[dev];
   }
   if (nclusters > sm_count / 2) nclusters = sm_count / 2;
-  if (launch_kernel(k_bwd_wgrad_pair, 2 * nclusters, kThreads, smem, st, 2, ma, mb, g) !=
+  if (launch_kernel(k_bwd_wgrad_pair<WK>, 2 * nclusters, kThreads, smem, st, 2, ma, mb, g) !=
       cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -910,8 +933,15 @@ int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* 
   g.ld_out = I;
   g.out_expert = (long long)H * I;
   g.out = d_down;
-  rc = wpair ? launch_wgrad_pair(m_dy64, m_h64, g, sm_count, st)
-             : launch(m_dy64, m_h64, g, sm_count, st);
+  // K rows per stage of the pair kernel: 64 (boxes of 64 rows) or 128
+  const bool wk128 = wpair && tuning(MOE_TUNE_BWD_WGRAD_BK) == 128;
+  CUtensorMap m_h128, m_x128;
+  if (wk128 && ((rc = make_tma_map_bf16(&m_h128, h, rows, I, 128)) != MOE_OK ||
+                (rc = make_tma_map_bf16(&m_x128, x_perm, rows, H, 128)) != MOE_OK))
+    return rc;
+  rc = wk128  ? launch_wgrad_pair<128>(m_dy128, m_h128, g, sm_count, st)
+       : wpair ? launch_wgrad_pair<64>(m_dy64, m_h64, g, sm_count, st)
+               : launch(m_dy64, m_h64, g, sm_count, st);
   if (rc != MOE_OK) return rc;
   g.m_valid = 2 * I;
   g.m_tiles = (2 * I + bm - 1) / bm;
@@ -920,8 +950,9 @@ int launch_bwd_gemms(const void* dy, const void* gu, const void* h, const void* 
   g.ld_out = H;
   g.out_expert = 2LL * I * H;
   g.out = d_gate_up;
-  return wpair ? launch_wgrad_pair(m_dgu64, m_x64, g, sm_count, st)
-               : launch(m_dgu64, m_x64, g, sm_count, st);
+  return wk128  ? launch_wgrad_pair<128>(m_dgu128, m_x128, g, sm_count, st)
+         : wpair ? launch_wgrad_pair<64>(m_dgu64, m_x64, g, sm_count, st)
+                 : launch(m_dgu64, m_x64, g, sm_count, st);
 }
 
 int launch_bwd_router_gemms(const void* dl3, int Tp, const void* x, const void* wr16,

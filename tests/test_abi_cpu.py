@@ -31,17 +31,18 @@ def test_tuning_switches_defaults_ranges_and_round_trip(L):
                 abi.TUNE_DOWN_BAND: 0, abi.TUNE_PAIR_INTERLEAVE: 0, abi.TUNE_PAIR_A_TRIM: 1,
                 abi.TUNE_PAIR_SWAP_AB: 1, abi.TUNE_PAIR_STREAM_HINT: 1,
                 abi.TUNE_PAIR_TAILS: 0, abi.TUNE_PAIR_PREFETCH: 0,
-                abi.TUNE_BWD_WGRAD_GROUP: 16, abi.TUNE_BWD_WGRAD_MIX: 0}
+                abi.TUNE_BWD_WGRAD_GROUP: 16, abi.TUNE_BWD_WGRAD_MIX: 0,
+                abi.TUNE_BWD_WGRAD_BK: 64}
     for k, v in defaults.items():
         assert abi.get_tuning(k) == v, k
     bad = [(abi.TUNE_PDL, 2), (abi.TUNE_GEMM_PAIR, -2), (abi.TUNE_ROUTER_N, 128),
            (abi.TUNE_ROUTER_MIN_SPLIT, 0), (abi.TUNE_ROUTER_MIN_SPLIT, 1025),
            (abi.TUNE_BWD_DY_ROWS, 2), (abi.TUNE_BWD_PAIR, 3), (abi.TUNE_TEST_STALL, -1), (abi.TUNE_GATE_UP_BAND, 65),
-           (abi.TUNE_DOWN_BAND, -1), (abi.TUNE_PAIR_INTERLEAVE, 2), (abi.TUNE_PAIR_A_TRIM, 3), (abi.TUNE_PAIR_SWAP_AB, 2), (abi.TUNE_PAIR_STREAM_HINT, 5), (abi.TUNE_PAIR_TAILS, 2), (abi.TUNE_PAIR_PREFETCH, 65), (abi.TUNE_BWD_WGRAD_GROUP, 65), (abi.TUNE_BWD_WGRAD_MIX, 65537), (18, 0), (-1, 0)]
+           (abi.TUNE_DOWN_BAND, -1), (abi.TUNE_PAIR_INTERLEAVE, 2), (abi.TUNE_PAIR_A_TRIM, 3), (abi.TUNE_PAIR_SWAP_AB, 2), (abi.TUNE_PAIR_STREAM_HINT, 5), (abi.TUNE_PAIR_TAILS, 2), (abi.TUNE_PAIR_PREFETCH, 65), (abi.TUNE_BWD_WGRAD_GROUP, 65), (abi.TUNE_BWD_WGRAD_MIX, 65537), (abi.TUNE_BWD_WGRAD_BK, 96), (19, 0), (-1, 0)]
     for k, v in bad:
         assert L.moe_set_tuning(k, v) == -1, (k, v)
     v = ctypes.c_int64(0)
-    assert L.moe_get_tuning(18, ctypes.byref(v)) == -1
+    assert L.moe_get_tuning(19, ctypes.byref(v)) == -1
     assert L.moe_get_tuning(0, None) == -1
     try:
         for k, v in [(abi.TUNE_PDL, 0), (abi.TUNE_GEMM_PAIR, 1), (abi.TUNE_ROUTER_N, 192),
@@ -49,7 +50,8 @@ def test_tuning_switches_defaults_ranges_and_round_trip(L):
                      (abi.TUNE_GATE_UP_BAND, 8), (abi.TUNE_DOWN_BAND, 64),
                      (abi.TUNE_PAIR_INTERLEAVE, 1), (abi.TUNE_PAIR_A_TRIM, 0),
                      (abi.TUNE_PAIR_SWAP_AB, 0), (abi.TUNE_PAIR_STREAM_HINT, 0), (abi.TUNE_PAIR_TAILS, 1),
-                     (abi.TUNE_PAIR_PREFETCH, 6), (abi.TUNE_BWD_WGRAD_GROUP, 0), (abi.TUNE_BWD_WGRAD_MIX, 512)]:
+                     (abi.TUNE_PAIR_PREFETCH, 6), (abi.TUNE_BWD_WGRAD_GROUP, 0), (abi.TUNE_BWD_WGRAD_MIX, 512),
+                     (abi.TUNE_BWD_WGRAD_BK, 128)]:
             abi.set_tuning(k, v)
             assert abi.get_tuning(k) == v
     finally:

@@ -191,13 +191,16 @@ def test_backward_full_shape_prefill(cuda_device, parity_report):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("knobs", [(1, 3, 0), (1, 0, 256), (1, 16, 1), (1, 1, 65536),
-                                   (1, 8, 256), (1, 0, 0), (2, 16, 0), (2, 0, 0)])
+@pytest.mark.parametrize("knobs", [(1, 3, 0, 64), (1, 0, 256, 64), (1, 16, 1, 64),
+                                   (1, 1, 65536, 64), (1, 8, 256, 64), (1, 0, 0, 64),
+                                   (2, 16, 0, 64), (2, 0, 0, 64), (1, 16, 0, 128),
+                                   (1, 0, 256, 128)])
 def test_weight_gradient_schedules_change_no_bits(cuda_device, knobs):
     """The weight-gradient GEMMs on CTA pairs visit an expert's tiles in groups of M tiles
     (MOE_TUNE_BWD_WGRAD_GROUP) and may alternate the tiles of experts with few rows with
     those of the others (MOE_TUNE_BWD_WGRAD_MIX; here with some, none and all experts in
-    the light list). Each output tile is still summed over the expert's rows in the same
+    the light list), with 64 or 128 expert rows per pipeline stage (MOE_TUNE_BWD_WGRAD_BK;
+    the MMA takes the same K = 16 steps in the same order). Each output tile is still summed over the expert's rows in the same
     order, so every setting gives the bits of the default one. MOE_TUNE_BWD_PAIR = 2 runs
     them on the one-CTA kernel (128-row tiles), whose per-element sums take the same
     k-steps in the same order."""
@@ -210,10 +213,12 @@ def test_weight_gradient_schedules_change_no_bits(cuda_device, knobs):
         abi.set_tuning(abi.TUNE_BWD_PAIR, knobs[0])
         abi.set_tuning(abi.TUNE_BWD_WGRAD_GROUP, knobs[1])
         abi.set_tuning(abi.TUNE_BWD_WGRAD_MIX, knobs[2])
+        abi.set_tuning(abi.TUNE_BWD_WGRAD_BK, knobs[3])
         got = _run(cfg, seed=21)
     finally:
         abi.set_tuning(abi.TUNE_BWD_PAIR, 1)
         abi.set_tuning(abi.TUNE_BWD_WGRAD_GROUP, 16)
         abi.set_tuning(abi.TUNE_BWD_WGRAD_MIX, 0)
+        abi.set_tuning(abi.TUNE_BWD_WGRAD_BK, 64)
     for a, c in zip(want[3:], got[3:]):
         assert torch.equal(a, c)
