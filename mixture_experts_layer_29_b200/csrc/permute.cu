@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(256) k_perm_scan(const uint32_t* masks, int n_
   if (lane == 0) ecount[e] = run;
 }
 
-// 8 tokens per CTA (one warp each). VEC = 16-byte vectors per row of x.
+// 8 tokens per CTA (one warp each).
+constexpr int kPermVec = 4;   // 16-byte vectors of x each lane loads before storing them
 template <bool XBF16>
 __global__ void __launch_bounds__(256) k_perm_scatter(
     const int32_t* topk_idx, const float* topk_gate,
@@ -150,32 +151,41 @@ __global__ void __launch_bounds__(256) k_perm_scatter(
   }
   __syncwarp();
 
-  // copy x[t] into every FFN row of the token, 16 bytes per lane per step
+  // copy x[t] into every FFN row of the token: each lane loads kPermVec 16-byte vectors of
+  // the row (32 apart) before storing them, so that more loads are in flight per warp
   const float zg = out_acc ? zgate[t] : 0.f;
   constexpr int esz = XBF16 ? 2 : 4;
   const int nvec = H * esz / 16;
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + (size_t)t * H * esz);
   if (!x_perm && !out_acc) return;
-  for (int v = lane; v < nvec; v += 32) {
-    const uint4 q = src[v];
-    if (x_perm) {
-      for (int k = 0; k < K; ++k) {
-        const int r = s_rows[warp][k];
-        if (r >= 0)
-          reinterpret_cast<uint4*>(static_cast<char*>(x_perm) + (size_t)r * H * esz)[v] = q;
+  for (int v0 = lane; v0 < nvec; v0 += 32 * kPermVec) {
+    uint4 q[kPermVec];
+#pragma unroll
+    for (int u = 0; u < kPermVec; ++u)
+      if (v0 + 32 * u < nvec) q[u] = src[v0 + 32 * u];
+#pragma unroll
+    for (int u = 0; u < kPermVec; ++u) {
+      const int v = v0 + 32 * u;
+      if (v >= nvec) break;
+      if (x_perm) {
+        for (int k = 0; k < K; ++k) {
+          const int r = s_rows[warp][k];
+          if (r >= 0)
+            reinterpret_cast<uint4*>(static_cast<char*>(x_perm) + (size_t)r * H * esz)[v] = q[u];
+        }
       }
-    }
-    if (out_acc) {
-      float* o = out_acc + (size_t)t * H + (size_t)v * (16 / esz);
-      if (XBF16) {
-        const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&q);
-        reinterpret_cast<float4*>(o)[0] =
-            make_float4(zg * to_f32(b[0]), zg * to_f32(b[1]), zg * to_f32(b[2]), zg * to_f32(b[3]));
-        reinterpret_cast<float4*>(o)[1] =
-            make_float4(zg * to_f32(b[4]), zg * to_f32(b[5]), zg * to_f32(b[6]), zg * to_f32(b[7]));
-      } else {
-        const float* f = reinterpret_cast<const float*>(&q);
-        reinterpret_cast<float4*>(o)[0] = make_float4(zg * f[0], zg * f[1], zg * f[2], zg * f[3]);
+      if (out_acc) {
+        float* o = out_acc + (size_t)t * H + (size_t)v * (16 / esz);
+        if (XBF16) {
+          const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&q[u]);
+          reinterpret_cast<float4*>(o)[0] = make_float4(zg * to_f32(b[0]), zg * to_f32(b[1]),
+                                                        zg * to_f32(b[2]), zg * to_f32(b[3]));
+          reinterpret_cast<float4*>(o)[1] = make_float4(zg * to_f32(b[4]), zg * to_f32(b[5]),
+                                                        zg * to_f32(b[6]), zg * to_f32(b[7]));
+        } else {
+          const float* f = reinterpret_cast<const float*>(&q[u]);
+          reinterpret_cast<float4*>(o)[0] = make_float4(zg * f[0], zg * f[1], zg * f[2], zg * f[3]);
+        }
       }
     }
   }
