@@ -102,6 +102,7 @@ FP32_SHAPES = {
     "f_odd":   (50, 112, 36, 5, 3, 2),
     "f_prime": (301, 272, 129, 9, 0, 4),
     "f_k1":    (97, 64, 1, 2, 5, 1),
+    "f_t700":  (700, 144, 40, 6, 2, 3),
 }
 
 
@@ -109,7 +110,9 @@ FP32_SHAPES = {
 @pytest.mark.parametrize("combine", ["deterministic", "fused"])
 def test_odd_fp32_shape_layer_matches_oracle(cuda_device, name, combine):
     """fp32 layers (the CUDA-core FFN) take any I >= 1 and H % 16 == 0: I = 1, 36, 129 and
-    H = 112, 272 (not multiples of 32), against the oracle within 1e-5."""
+    H = 112, 272 (not multiples of 32), against the oracle within 1e-5. T = 700 takes the
+    large-batch permutation (H = 144: 36 16-byte vectors per row, so the copy's second
+    vector round covers four lanes only)."""
     T, H, I, N, Z, K = FP32_SHAPES[name]
     cfg = wl.CONFIGS["tiny_fp32"].with_(name=f"shape_{name}", T=T, H=H, I=I, n_ffn=N,
                                         n_zero=Z, K=K)
